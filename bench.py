@@ -1,0 +1,408 @@
+"""Benchmark of the streaming KV hot path (one JSON line on rank 0).
+
+One step = one streamed chunk through every DiT layer: for each layer,
+sdv2_kv_append then sdv2_chunk_attention over the sink + window cache; then
+sdv2_sink_refresh and sdv2_motion_noise_rate.  Default workload: the
+Wan-1.3B-shaped stack at 512x512 (30 layers, 12 heads x 128, 32x32 tokens per
+latent frame, chunk of 1 frame, 1 sink + 6 window frames, batch 1), with the
+ring already wrapped (steady state), sink refresh on 1536-wide hidden states
+and motion on 16x64x64 latents.  Inputs are seeded synthetic N(0,1) data.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+Under torchrun each rank runs an independent replica (the path has no
+cross-GPU exchange); value = frames of all ranks / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "chunk-attn TFLOP/s + KV HBM GB/s vs roofline; latent frames/s (1.3B/14B shape)"
+UNIT = "latent frames/s"
+
+WORKLOADS = {
+    # name: cache config + refresh/motion shapes
+    "wan1.3b-512x512": dict(batch=1, layers=30, heads=12, head_dim=128, frame_h=32, frame_w=32, chunk_frames=1,
+                            sink_frames=1, window_frames=6, embed_dim=1536, motion=(16, 64, 64)),
+    "wan1.3b-480x832-b4": dict(batch=4, layers=30, heads=12, head_dim=128, frame_h=30, frame_w=52, chunk_frames=2,
+                               sink_frames=1, window_frames=8, embed_dim=1536, motion=(16, 60, 104)),
+    "wan14b-512x512-b1": dict(batch=1, layers=40, heads=40, head_dim=128, frame_h=32, frame_w=32, chunk_frames=1,
+                              sink_frames=1, window_frames=6, embed_dim=5120, motion=(16, 64, 64)),
+    "wan14b-512x512-b8": dict(batch=8, layers=40, heads=40, head_dim=128, frame_h=32, frame_w=32, chunk_frames=1,
+                              sink_frames=1, window_frames=6, embed_dim=5120, motion=(16, 64, 64)),
+}
+DEFAULT_WORKLOAD = "wan1.3b-512x512"
+TAU = 0.9
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            pk = json.load(fh)
+        return pk, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def attn_flops(w, keys):
+    lq = w["chunk_frames"] * w["frame_h"] * w["frame_w"]
+    return sum(4.0 * w["heads"] * lq * k * w["head_dim"] for k in keys)
+
+
+def attn_bytes(w, keys):
+    lq = w["chunk_frames"] * w["frame_h"] * w["frame_w"]
+    hd = w["heads"] * w["head_dim"]
+    return sum(2.0 * 2 * k * hd + 2.0 * 2 * lq * hd for k in keys)   # K+V read once, Q read, O written
+
+
+def steady_keys(w):
+    n = w["frame_h"] * w["frame_w"]
+    return [(w["sink_frames"] + w["window_frames"]) * n] * w["batch"]
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        out = {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        if not self.path or not os.path.exists(self.path):
+            return out
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx.append(float(f[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, f[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        os.unlink(self.path)
+        if sm:
+            out.update(sm_mhz=statistics.median(sm), sm_max_mhz=max(mx), reasons=sorted(reasons), samples=len(sm))
+        return out
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args, w, name):
+    import datetime
+
+    import torch
+
+    import synth
+    from causal_dit_kv_b200 import KVCache, MotionState, binding
+
+    world, rank, local = dist_setup(args)
+    torch.cuda.set_device(local)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    B, L, H, D = w["batch"], w["layers"], w["heads"], w["head_dim"]
+    N = w["frame_h"] * w["frame_w"]
+    Tp = w["chunk_frames"]
+    Lq = Tp * N
+    E = w["embed_dim"]
+    C, MH, MW = w["motion"]
+    cache = KVCache(B, L, H, D, w["frame_h"], w["frame_w"], Tp, w["sink_frames"], w["window_frames"], embed_dim=E)
+    mot = MotionState(B, Tp, C, MH, MW, window=4, sigma=2.0, lam=0.9)
+    scale = 1.0 / math.sqrt(D)
+    dev = torch.device("cuda", local)
+
+    # Input pool: two distinct steps' worth of Q/K/V for every layer, hidden states and latents.
+    pool = []
+    seed = 2000 + rank
+    for p in range(2):
+        qkv = [synth.chunk_qkv(seed, B, Lq, H, D, p, l) for l in range(L)]
+        hid = next(synth.drifting_hidden(seed + p, B, Lq, E, 1, drift=0.05))
+        lat = next(synth.motion_latents(seed + p, B, Tp, C, MH, MW, 1))
+        pool.append(dict(qkv=qkv, hid=hid, lat=lat))
+    dev_pool = [dict(q=[t[0].to(dev) for t in p["qkv"]], k=[t[1].to(dev) for t in p["qkv"]],
+                     v=[t[2].to(dev) for t in p["qkv"]], hid=p["hid"].to(dev), lat=p["lat"].to(dev)) for p in pool]
+    out = torch.empty((B, Lq, H, D), dtype=torch.bfloat16, device=dev)
+    out_slot = torch.empty(B, dtype=torch.int32, device=dev)
+    rate = torch.empty(B, dtype=torch.float32, device=dev)
+    frame = [0]
+    stream = torch.cuda.current_stream(dev)
+
+    def step(inp, attn_events=None):
+        f0 = [frame[0]] * B
+        for l in range(L):
+            cache.kv_append(l, inp["k"][l], inp["v"][l], f0)
+            if attn_events is not None:
+                attn_events[l][0].record(stream)
+            cache.chunk_attention(l, inp["q"][l], out, f0, scale)
+            if attn_events is not None:
+                attn_events[l][1].record(stream)
+        cache.sink_refresh(inp["hid"], TAU, f0, out_slot)
+        mot.noise_rate(inp["lat"], rate)
+        frame[0] += Tp
+
+    # Pre-roll to steady state (ring wrapped, every slot valid), then warm up.
+    for i in range(w["sink_frames"] + w["window_frames"] + 1):
+        step(dev_pool[i % 2])
+    for i in range(args.warmup):
+        step(dev_pool[i % 2])
+    torch.cuda.synchronize()
+
+    # ---- device-resident timing
+    events = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
+              for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = binding.sdv2_launch_count()
+    with ClockSampler(local) as clocks:
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for i in range(args.steps):
+            step(dev_pool[i % 2], events[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+        if pg:
+            pg.barrier()
+    launches = binding.sdv2_launch_count() - launches0
+    ms = t0.elapsed_time(t1)
+    attn_ms = [a.elapsed_time(b) for ev in events for (a, b) in ev]
+    assert cache.check() == 0 and mot.check() == 0, "device status word set"
+
+    # ---- end to end: pinned host inputs copied in, results copied out, every step
+    host_pool = []
+    for p in pool:
+        host_pool.append(dict(q=[t[0].pin_memory() for t in p["qkv"]], k=[t[1].pin_memory() for t in p["qkv"]],
+                              v=[t[2].pin_memory() for t in p["qkv"]], hid=p["hid"].pin_memory(),
+                              lat=p["lat"].pin_memory()))
+    stage = dict(q=[torch.empty_like(t) for t in dev_pool[0]["q"]], k=[torch.empty_like(t) for t in dev_pool[0]["k"]],
+                 v=[torch.empty_like(t) for t in dev_pool[0]["v"]], hid=torch.empty_like(dev_pool[0]["hid"]),
+                 lat=torch.empty_like(dev_pool[0]["lat"]))
+    res_out = torch.empty((B, Lq, H, D), dtype=torch.bfloat16).pin_memory()
+    res_rate = torch.empty(B, dtype=torch.float32).pin_memory()
+    res_slot = torch.empty(B, dtype=torch.int32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_pool[0]["q"] + host_pool[0]["k"] + host_pool[0]["v"])
+    h2d += host_pool[0]["hid"].numel() * 2 + host_pool[0]["lat"].numel() * 4
+    d2h = res_out.numel() * 2 + B * 8
+
+    def e2e_step(hp):
+        for key in ("q", "k", "v"):
+            for l in range(L):
+                stage[key][l].copy_(hp[key][l], non_blocking=True)
+        stage["hid"].copy_(hp["hid"], non_blocking=True)
+        stage["lat"].copy_(hp["lat"], non_blocking=True)
+        step(stage)
+        res_out.copy_(out, non_blocking=True)
+        res_rate.copy_(rate, non_blocking=True)
+        res_slot.copy_(out_slot, non_blocking=True)
+
+    e2e_step(host_pool[0])
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if pg:
+        pg.barrier()
+    e0.record(stream)
+    for i in range(args.steps):
+        e2e_step(host_pool[i % 2])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+
+    if pg:
+        t = torch.tensor([ms, e2e_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms, e2e_ms = float(t[0]), float(t[1])
+    frames = world * args.steps * B * Tp
+    value = frames / (ms / 1e3)
+    e2e_value = frames / (e2e_ms / 1e3)
+
+    keys = steady_keys(w)
+    flops = attn_flops(w, keys)
+    abytes = attn_bytes(w, keys)
+    attn_avg_s = statistics.mean(attn_ms) / 1e3
+    peaks, peak_src = load_peaks()
+    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    achieved = flops / attn_avg_s / 1e12
+    result = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": name, "batch": B, "layers": L, "heads": H, "head_dim": D,
+                   "tokens_per_frame": N, "chunk_frames": Tp, "sink_frames": w["sink_frames"],
+                   "window_frames": w["window_frames"], "keys_per_stream": keys[0], "queries_per_stream": Lq,
+                   "refresh_embed_dim": E, "motion_latent": [C, MH, MW],
+                   "l2": "inputs larger than L2 (per-step caches %.0f MB over %d layers)" % (
+                       2 * cache.layout.layer_stride * L / 1e6, L),
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"kernel": "sdv2_chunk_attention (attention + split-KV combine)", "bound": "tensor",
+                     "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained",
+                     "algorithmic_flops_per_launch": flops, "avg_launch_us": round(attn_avg_s * 1e6, 3),
+                     "kv_gbs": round(abytes / attn_avg_s / 1e9, 1)},
+        "attention": {"tflops": round(achieved, 2), "kv_hbm_gbs": round(abytes / attn_avg_s / 1e9, 1),
+                      "us_per_layer": round(attn_avg_s * 1e6, 3),
+                      "frac_of_burst_peak": round(achieved / peaks["bf16_tflops"], 4)},
+        "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": int(launches),
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result))
+
+
+# ----------------------------------------------------------------------------- oracle arms
+
+def oracle_sample(w, threads=None):
+    """Time the fp64 oracle on one layer of the workload's step (append + attention of
+    every query of every stream) plus the refresh and motion of the step; returns
+    the step time extrapolated to all layers."""
+    import numpy as np
+
+    import oracle as O
+    import synth
+
+    B, H, D = w["batch"], w["heads"], w["head_dim"]
+    N = w["frame_h"] * w["frame_w"]
+    Tp = w["chunk_frames"]
+    Lq = Tp * N
+    cfg = O.CacheConfig(batch=B, layers=1, heads=H, head_dim=D, frame_h=w["frame_h"], frame_w=w["frame_w"],
+                        chunk_frames=Tp, sink_frames=w["sink_frames"], window_frames=w["window_frames"],
+                        embed_dim=w["embed_dim"])
+    cache = O.OracleCache(cfg)
+    # fill to steady state (not timed)
+    pre = (w["sink_frames"] + w["window_frames"] + Tp - 1) // Tp + 1
+    for s in range(pre):
+        _, k, v = synth.chunk_qkv(5, B, Lq, H, D, s, 0)
+        O.kv_append(cache, 0, synth.bf16_bits(k), synth.bf16_bits(v), [s * Tp] * B)
+    mcfg = O.MotionConfig(batch=B, channels=w["motion"][0], height=w["motion"][1], width=w["motion"][2])
+    mstate = O.MotionState(mcfg)
+    lat = synth.motion_latents(5, B, Tp, *w["motion"], n_chunks=2)
+    O.motion_noise_rate(mstate, next(lat).numpy())
+    hid = next(synth.drifting_hidden(5, B, Lq, w["embed_dim"], 1))
+    q, k, v = synth.chunk_qkv(5, B, Lq, H, D, pre, 0)
+    f0 = [pre * Tp] * B
+    x = next(lat).numpy()
+    t0 = time.perf_counter()
+    O.kv_append(cache, 0, synth.bf16_bits(k), synth.bf16_bits(v), f0)
+    O.chunk_attention(cache, 0, synth.bf16_bits(q), f0, 1.0 / math.sqrt(D))
+    t1 = time.perf_counter()
+    O.sink_refresh(cache, synth.bf16_bits(hid), TAU, f0)
+    O.motion_noise_rate(mstate, x)
+    t2 = time.perf_counter()
+    layer_s = t1 - t0
+    step_s = layer_s * w["layers"] + (t2 - t1)
+    return step_s, layer_s, t2 - t1
+
+
+def cpu_baseline(w):
+    import torch
+    step_s, layer_s, rest_s = oracle_sample(w)
+    frames = w["batch"] * w["chunk_frames"]
+    return {"value": round(frames / step_s, 5), "unit": UNIT, "cores": torch.get_num_threads(), "kind": "oracle",
+            "sample": f"1 of {w['layers']} layers (append + attention of all queries, fp64 numpy, "
+                      f"{layer_s:.2f} s) + sink refresh and motion ({rest_s:.2f} s); step time = "
+                      f"{w['layers']} x layer + refresh + motion"}
+
+
+def run_reference(args, w, name):
+    world, rank, _ = dist_setup(args)
+    if rank != 0:
+        return
+    import torch
+    times = []
+    for i in range(args.warmup + args.steps):
+        step_s, layer_s, rest_s = oracle_sample(w)
+        if i >= args.warmup:
+            times.append(step_s)
+    mean_step = statistics.mean(times)
+    frames = w["batch"] * w["chunk_frames"]
+    value = frames / mean_step
+    cores = torch.get_num_threads()
+    sample = (f"per step: 1 of {w['layers']} layers (append + attention, fp64 numpy oracle) + refresh + motion, "
+              f"extrapolated to {w['layers']} layers")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(mean_step * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": name}, "gpu_launches": 0,
+        "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w, args.workload)
+    else:
+        run_ours(args, w, args.workload)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,517 @@
+// Chunk attention over the sink + rolling-window KV cache on the sm_100a
+// tensor cores (tcgen05 MMA, accumulators in TMEM, K/V tiles by TMA).
+//
+// Sources: admirer.cn article on StreamDiffusionV2, "深入分析：內存帶寬約束
+// 導致的性能受限" (each chunk loads the long KV cache while computing only on
+// the current input); qq8o.cn walkthrough, "Adaptive sink and RoPE refresh"
+// (sink tokens, RoPE); agentlens page "chenfengxu714/StreamDiffusionV2"
+// (ring-buffer KV cache with sliding-window attention).
+//
+// out = softmax(scale * RoPE(q) K^T) V over the valid slots of the stream.
+// The valid slots are always the prefix 0..n_valid-1 of the ring (sinks fill
+// first, window slots after), and attention is invariant to the order of the
+// keys, so the kernel reads keys 0..lk-1 of the slot-major cache directly,
+// without unrolling the ring.
+//
+// One CTA = one (stream, head, pair of 128-row query tiles, KV split):
+//   warp 0      TMA producer: K and V tiles (128 keys x d) into a 2-stage ring
+//   warp 1      MMA issuer (one thread): S_t = Q_t K^T and O_t += P_t V
+//   warps 4..7  softmax + epilogue of query tile 0 (thread i owns row i)
+//   warps 8..11 softmax + epilogue of query tile 1
+// TMEM (512 columns): S_0 | S_1 | O_0 | O_1, 128 columns each; P_t (bf16)
+// is written over the first 64 columns of S_t and fed to the PV MMA from
+// TMEM.  The MMA order PV(0,j), QK(0,j+1), PV(1,j), QK(1,j+1) lets one tile's
+// softmax run while the tensor core works on the other tile.
+// Online softmax in base 2 with lazy rescaling: the running max only moves
+// (and O is rescaled in TMEM) when a tile's max exceeds it by more than 8,
+// so P stays <= 256.
+// Q is rotated on load (fp32 RoPE, rounded to bf16) by the softmax threads
+// and written into the 128-byte-swizzled K-major layout the MMA reads.
+// Every wait is bounded (2 s), after which the CTA records an error in the
+// device status word and unwinds; TMEM is always released.
+#include <cmath>
+
+#include "ptx.cuh"
+
+namespace sdv2 {
+
+template <int D>
+struct AttnLayout {
+    static constexpr int kQTile = kBlockM * D * 2;    // bytes of one Q tile
+    static constexpr int kKVTile = kBlockN * D * 2;   // bytes of one K (or V) tile
+    static constexpr int kSub = kBlockM * 128;        // one 64-column (128-byte) sub-tile
+    static constexpr int kStages = 2;
+    static constexpr int kQ = 0;
+    static constexpr int kK = kQ + kQTilesPerCta * kQTile;
+    static constexpr int kV = kK + kStages * kKVTile;
+    static constexpr int kBar = kV + kStages * kKVTile;
+    // barriers
+    static constexpr int kQFull = 0;
+    static constexpr int kKFull = 1;
+    static constexpr int kKEmpty = kKFull + kStages;
+    static constexpr int kVFull = kKEmpty + kStages;
+    static constexpr int kVEmpty = kVFull + kStages;
+    static constexpr int kSFull = kVEmpty + kStages;
+    static constexpr int kPFull = kSFull + 2;
+    static constexpr int kOFull = kPFull + 2;
+    static constexpr int kDrain = kOFull + 2;
+    static constexpr int kNumBars = kDrain + 1;
+    static constexpr int kMisc = kBar + kNumBars * 8;
+    static constexpr int kBytes = kMisc + 16;
+    static constexpr int kAlloc = kBytes + 1024;      // room to align the base to 1024 bytes
+};
+
+int attention_smem_bytes(int head_dim) {
+    return head_dim == 64 ? AttnLayout<64>::kAlloc : AttnLayout<128>::kAlloc;
+}
+
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale only when the max grows by > 2^8
+
+// fp32 (cos, sin) of rotation pair j for a query token.
+__device__ __forceinline__ float2 q_cos_sin(const AttnParams &p, int bl, int fi, int row, int col, int j) {
+    if (j < p.n_t) {
+        const int e = (bl * p.chunk_frames + fi) * p.n_t + j;
+        return make_float2(p.tab_t[e][0], p.tab_t[e][1]);
+    }
+    if (j < p.n_t + p.n_h) {
+        const float *t = p.rope_h + 2 * (row * p.n_h + (j - p.n_t));
+        return make_float2(t[0], t[1]);
+    }
+    const float *t = p.rope_w + 2 * (col * p.n_w + (j - p.n_t - p.n_h));
+    return make_float2(t[0], t[1]);
+}
+
+// All 32 lanes wait; the warp proceeds only if every lane saw the phase
+// complete, so the .sync.aligned tcgen05 ops that follow stay warp-uniform.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile uint32_t *abort, uint32_t *status,
+                                          uint32_t code) {
+    const bool ok = mbar_wait(bar, parity, abort, status, code);
+    return __all_sync(0xffffffffu, ok);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    chunk_attention_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmap_k,
+                           const __grid_constant__ CUtensorMap tmap_v) {
+    using L = AttnLayout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBar);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
+    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + L::kMisc + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int qpair = blockIdx.x / p.n_split;
+    const int split = blockIdx.x - qpair * p.n_split;
+    const int h = blockIdx.y;
+    const int bl = blockIdx.z;                  // stream within this launch
+    const int bg = p.b_offset + bl;             // stream index in the cache
+    const int lk = p.lk[bl];
+    if (lk <= 0) return;                        // stream not part of this call (uniform per CTA)
+
+    const int n_kv = (lk + kBlockN - 1) / kBlockN;
+    const int per = (n_kv + p.n_split - 1) / p.n_split;
+    const int kv_begin = split * per;
+    const int kv_end = min(n_kv, kv_begin + per);
+    const int n_local = kv_end > kv_begin ? kv_end - kv_begin : 0;
+    const int q_row0 = qpair * (kBlockM * kQTilesPerCta);
+    const int n_qt = (q_row0 + kBlockM < p.lq) ? 2 : 1;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars[L::kQFull], kBlockM * n_qt);
+        for (int s = 0; s < L::kStages; ++s) {
+            mbar_init(&bars[L::kKFull + s], 1);
+            mbar_init(&bars[L::kKEmpty + s], 1);
+            mbar_init(&bars[L::kVFull + s], 1);
+            mbar_init(&bars[L::kVEmpty + s], 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&bars[L::kSFull + t], 1);
+            mbar_init(&bars[L::kPFull + t], kBlockM);
+            mbar_init(&bars[L::kOFull + t], 1);
+        }
+        mbar_init(&bars[L::kDrain], 1);
+        *abort_flag = 0u;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmap_k);
+        tma_prefetch_desc(&tmap_v);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0 && n_local > 0) {
+            int issued[L::kStages] = {0, 0};
+            for (int it = 0; it < n_local; ++it) {
+                const int st = it % L::kStages;
+                const uint32_t ph = (it / L::kStages) & 1;
+                const int kv0 = (kv_begin + it) * kBlockN;
+                if (!mbar_wait(&bars[L::kKEmpty + st], ph ^ 1u, abort_flag, p.status, kStatusTmaWait)) break;
+                mbar_arrive_expect_tx(&bars[L::kKFull + st], L::kKVTile);
+#pragma unroll
+                for (int kb = 0; kb < D / 64; ++kb)
+                    tma_load_4d(smem + L::kK + st * L::kKVTile + kb * L::kSub, &tmap_k, &bars[L::kKFull + st], kb * 64,
+                                h, kv0, bg);
+                if (!mbar_wait(&bars[L::kVEmpty + st], ph ^ 1u, abort_flag, p.status, kStatusTmaWait)) {
+                    issued[st] = it + 1;
+                    break;
+                }
+                mbar_arrive_expect_tx(&bars[L::kVFull + st], L::kKVTile);
+#pragma unroll
+                for (int kb = 0; kb < D / 64; ++kb)
+                    tma_load_4d(smem + L::kV + st * L::kKVTile + kb * L::kSub, &tmap_v, &bars[L::kVFull + st], kb * 64,
+                                h, kv0, bg);
+                issued[st] = it + 1;
+            }
+            if (*abort_flag) {
+                // Let every copy already in flight land before the CTA leaves.
+                for (int st = 0; st < L::kStages; ++st) {
+                    if (issued[st] == 0) continue;
+                    const uint32_t ph = ((issued[st] - 1) / L::kStages) & 1;
+                    const uint64_t t0 = global_timer_ns();
+                    while (!(mbar_try_wait(&bars[L::kKFull + st], ph) && mbar_try_wait(&bars[L::kVFull + st], ph))) {
+                        if (global_timer_ns() - t0 > kWaitLimitNs) break;
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0 && n_local > 0) {
+            constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kBlockN, 0, 0);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, D, 0, 1);
+            const uint32_t q_base = smem_addr(smem + L::kQ);
+            const uint32_t k_base = smem_addr(smem + L::kK);
+            const uint32_t v_base = smem_addr(smem + L::kV);
+            auto issue_qk = [&](int t, int st) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * L::kSub + (kk & 3) * 32;
+                    const uint64_t a = smem_desc_sw128(q_base + t * L::kQTile + off, 16, 1024);
+                    const uint64_t b = smem_desc_sw128(k_base + st * L::kKVTile + off, 16, 1024);
+                    umma_ss(tmem + t * 128, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+                }
+            };
+            auto issue_pv = [&](int t, int st, bool acc) {
+#pragma unroll
+                for (int kk = 0; kk < kBlockN / 16; ++kk) {
+                    const uint64_t b = smem_desc_sw128(v_base + st * L::kKVTile + kk * 2048, L::kSub, 1024);
+                    umma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, b, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+                }
+            };
+            bool ok = mbar_wait(&bars[L::kQFull], 0, abort_flag, p.status, kStatusMmaWait);
+            if (ok) {
+                tc_fence_after();
+                ok = mbar_wait(&bars[L::kKFull + 0], 0, abort_flag, p.status, kStatusMmaWait);
+            }
+            if (ok) {
+                tc_fence_after();
+                for (int t = 0; t < n_qt; ++t) {
+                    issue_qk(t, 0);
+                    umma_commit(&bars[L::kSFull + t]);
+                }
+                umma_commit(&bars[L::kKEmpty + 0]);
+            }
+            for (int it = 0; ok && it < n_local; ++it) {
+                const int st = it % L::kStages;
+                const uint32_t ph = (it / L::kStages) & 1;
+                const int nst = (it + 1) % L::kStages;
+                const uint32_t nph = ((it + 1) / L::kStages) & 1;
+                const bool more = it + 1 < n_local;
+                if (!mbar_wait(&bars[L::kVFull + st], ph, abort_flag, p.status, kStatusMmaWait)) break;
+                tc_fence_after();
+                for (int t = 0; t < n_qt; ++t) {
+                    if (!mbar_wait(&bars[L::kPFull + t], it & 1, abort_flag, p.status, kStatusMmaWait)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    issue_pv(t, st, it > 0);
+                    if (more) {
+                        if (t == 0) {
+                            if (!mbar_wait(&bars[L::kKFull + nst], nph, abort_flag, p.status, kStatusMmaWait)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                        }
+                        issue_qk(t, nst);
+                        umma_commit(&bars[L::kSFull + t]);
+                    } else {
+                        umma_commit(&bars[L::kOFull + t]);
+                    }
+                }
+                if (!ok) break;
+                umma_commit(&bars[L::kVEmpty + st]);
+                if (more) umma_commit(&bars[L::kKEmpty + nst]);
+            }
+            // Drain: every MMA issued so far has finished before TMEM is released.
+            umma_commit(&bars[L::kDrain]);
+            const uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait(&bars[L::kDrain], 0)) {
+                if (global_timer_ns() - t0 > kWaitLimitNs) {
+                    atomicOr(p.status, kStatusMmaWait);
+                    break;
+                }
+            }
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------ softmax / epilogue
+        const int t = (warp - 4) >> 2;               // query tile of this warpgroup
+        const int row = ((warp & 3) << 5) + lane;    // TMEM lane == query row in the tile
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) << 5) << 16;
+        if (t < n_qt) {
+            const int token = q_row0 + t * kBlockM + row;
+            const bool valid = token < p.lq;
+            // ---- Q load + RoPE (fp32) into the swizzled K-major tile
+            uint8_t *qtile = smem + L::kQ + t * L::kQTile;
+            if (n_local > 0) {
+                const int fi = valid ? token / p.tokens_per_frame : 0;
+                const int n = valid ? token - fi * p.tokens_per_frame : 0;
+                const int prow = n / p.frame_w;
+                const int pcol = n - prow * p.frame_w;
+                const uint16_t *qrow =
+                    p.q + ((static_cast<int64_t>(bg) * p.lq + (valid ? token : 0)) * p.heads + h) * D;
+#pragma unroll 4
+                for (int c = 0; c < D / 8; ++c) {
+                    uint4 w = make_uint4(0, 0, 0, 0);
+                    if (valid) {
+                        const uint4 x = *reinterpret_cast<const uint4 *>(qrow + c * 8);
+                        uint32_t in[4] = {x.x, x.y, x.z, x.w};
+                        uint32_t o[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float2 cs = q_cos_sin(p, bl, fi, prow, pcol, c * 4 + q);
+                            const float x0 = bf16_lo(in[q]), x1 = bf16_hi(in[q]);
+                            o[q] = pack_bf16x2(x0 * cs.x - x1 * cs.y, x0 * cs.y + x1 * cs.x);
+                        }
+                        w = make_uint4(o[0], o[1], o[2], o[3]);
+                    }
+                    const int kb = c >> 3, c16 = c & 7;
+                    *reinterpret_cast<uint4 *>(qtile + kb * L::kSub + row * 128 + ((c16 ^ (row & 7)) << 4)) = w;
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&bars[L::kQFull]);
+            }
+
+            float m_run = -INFINITY;   // running max of scale*log2(e)*s
+            float l_run = 0.0f;
+            bool ok = true;
+            const uint32_t s_tmem = tmem + lane_base + t * 128;
+            const uint32_t o_tmem = tmem + lane_base + 256 + t * 128;
+            for (int it = 0; it < n_local; ++it) {
+                if (!warp_wait(&bars[L::kSFull + t], it & 1, abort_flag, p.status, kStatusSoftmaxWait)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t sr[kBlockN / 32][32];
+#pragma unroll
+                for (int cb = 0; cb < kBlockN / 32; ++cb) tmem_ld32(s_tmem + cb * 32, sr[cb]);
+                tmem_wait_ld_bind(sr[0]);
+#pragma unroll
+                for (int cb = 1; cb < kBlockN / 32; ++cb) reg_bind(sr[cb]);
+                float s[kBlockN];
+#pragma unroll
+                for (int cb = 0; cb < kBlockN / 32; ++cb)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) s[cb * 32 + i] = __uint_as_float(sr[cb][i]);
+                const int valid_cols = lk - (kv_begin + it) * kBlockN;
+                if (valid_cols < kBlockN) {
+#pragma unroll
+                    for (int i = 0; i < kBlockN; ++i)
+                        if (i >= valid_cols) s[i] = -INFINITY;
+                }
+                float mx = s[0];
+#pragma unroll
+                for (int i = 1; i < kBlockN; ++i) mx = fmaxf(mx, s[i]);
+                const float m_tile = mx * p.scale_log2;
+                bool rescale = false;
+                float alpha = 1.0f;
+                if (it == 0) {
+                    m_run = m_tile;
+                } else if (m_tile > m_run + kRescaleThreshold) {
+                    rescale = true;
+                    alpha = ex2_approx(m_run - m_tile);
+                    l_run *= alpha;
+                    m_run = m_tile;
+                }
+                if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+                    for (int cb = 0; cb < D / 32; ++cb) {
+                        uint32_t r[32];
+                        tmem_ld32(o_tmem + cb * 32, r);
+                        tmem_wait_ld_bind(r);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                        tmem_st32(o_tmem + cb * 32, r);
+                    }
+                    tmem_wait_st();
+                }
+                const float neg_m = -m_run;
+                float sum = 0.0f;
+#pragma unroll
+                for (int cb = 0; cb < 2; ++cb) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const float p0 = ex2_approx(fmaf(s[cb * 64 + 2 * i], p.scale_log2, neg_m));
+                        const float p1 = ex2_approx(fmaf(s[cb * 64 + 2 * i + 1], p.scale_log2, neg_m));
+                        sum += p0 + p1;
+                        pk[i] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st32(s_tmem + cb * 32, pk);
+                }
+                l_run += sum;
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&bars[L::kPFull + t]);
+            }
+
+            // ---- epilogue
+            if (ok && n_local > 0) ok = warp_wait(&bars[L::kOFull + t], 0, abort_flag, p.status, kStatusSoftmaxWait);
+            if (ok) {
+                tc_fence_after();
+                if (p.n_split == 1) {
+                    const float inv = 1.0f / l_run;
+                    uint16_t *orow = p.out + ((static_cast<int64_t>(bg) * p.lq + token) * p.heads + h) * D;
+#pragma unroll
+                    for (int cb = 0; cb < D / 32; ++cb) {
+                        uint32_t r[32];
+                        tmem_ld32(o_tmem + cb * 32, r);
+                        tmem_wait_ld_bind(r);
+                        if (valid) {
+#pragma unroll
+                            for (int v = 0; v < 4; ++v) {
+                                uint4 w;
+                                w.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]) * inv, __uint_as_float(r[8 * v + 1]) * inv);
+                                w.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]) * inv, __uint_as_float(r[8 * v + 3]) * inv);
+                                w.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]) * inv, __uint_as_float(r[8 * v + 5]) * inv);
+                                w.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]) * inv, __uint_as_float(r[8 * v + 7]) * inv);
+                                *reinterpret_cast<uint4 *>(orow + cb * 32 + v * 8) = w;
+                            }
+                        }
+                    }
+                } else {
+                    const int64_t prow_idx =
+                        ((static_cast<int64_t>(split) * p.batch + bg) * p.heads + h) * p.lq_pad + q_row0 + t * kBlockM + row;
+                    if (n_local > 0) {
+                        float *po = p.part_o + prow_idx * D;
+#pragma unroll
+                        for (int cb = 0; cb < D / 32; ++cb) {
+                            uint32_t r[32];
+                            tmem_ld32(o_tmem + cb * 32, r);
+                            tmem_wait_ld_bind(r);
+                            if (valid) {
+#pragma unroll
+                                for (int v = 0; v < 8; ++v)
+                                    *reinterpret_cast<uint4 *>(po + cb * 32 + v * 4) =
+                                        make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+                            }
+                        }
+                    }
+                    if (valid) {
+                        p.part_ml[prow_idx * 2 + 0] = n_local > 0 ? m_run : -INFINITY;
+                        p.part_ml[prow_idx * 2 + 1] = l_run;
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// One warp per (stream, head, query row): merges the split partials.
+template <int D>
+__global__ void __launch_bounds__(256) attention_combine_kernel(const __grid_constant__ CombineParams p) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row = blockIdx.x * 8 + warp;
+    const int h = blockIdx.y;
+    const int bl = blockIdx.z;
+    const int bg = p.b_offset + bl;
+    if (p.lk[bl] <= 0 || row >= p.lq) return;
+    constexpr int kPer = D / 32;   // columns per lane
+    float m = -INFINITY;
+    for (int s = 0; s < p.n_split; ++s) {
+        const int64_t idx = ((static_cast<int64_t>(s) * p.batch + bg) * p.heads + h) * p.lq_pad + row;
+        m = fmaxf(m, p.part_ml[idx * 2]);
+    }
+    float acc[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) acc[i] = 0.0f;
+    float l = 0.0f;
+    for (int s = 0; s < p.n_split; ++s) {
+        const int64_t idx = ((static_cast<int64_t>(s) * p.batch + bg) * p.heads + h) * p.lq_pad + row;
+        const float ms = p.part_ml[idx * 2];
+        if (ms == -INFINITY) continue;            // empty split: no keys, no partial
+        const float w = exp2f(ms - m);
+        l += w * p.part_ml[idx * 2 + 1];
+        const float *po = p.part_o + idx * D + lane * kPer;
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) acc[i] += w * po[i];
+    }
+    const float inv = 1.0f / l;
+    uint16_t *orow = p.out + ((static_cast<int64_t>(bg) * p.lq + row) * p.heads + h) * D + lane * kPer;
+#pragma unroll
+    for (int i = 0; i < kPer; i += 2) {
+        *reinterpret_cast<uint32_t *>(orow + i) = pack_bf16x2(acc[i] * inv, acc[i + 1] * inv);
+    }
+}
+
+template <int D>
+static cudaError_t launch_attention_d(const AttnParams &p, const CUtensorMap &tk, const CUtensorMap &tv,
+                                      cudaStream_t s) {
+    static bool configured = false;
+    const int smem = AttnLayout<D>::kAlloc;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(chunk_attention_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    int nb = 0;
+    for (int i = 0; i < kMaxBatch; ++i)
+        if (p.lk[i] > 0) nb = i + 1;
+    if (nb == 0) return cudaSuccess;
+    dim3 grid(static_cast<unsigned>(p.n_qpairs * p.n_split), static_cast<unsigned>(p.heads), static_cast<unsigned>(nb));
+    chunk_attention_kernel<D><<<grid, kAttnThreads, smem, s>>>(p, tk, tv);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attention(const AttnParams &p, const CUtensorMap &tk, const CUtensorMap &tv, int head_dim,
+                             cudaStream_t s) {
+    if (head_dim == 64) return launch_attention_d<64>(p, tk, tv, s);
+    return launch_attention_d<128>(p, tk, tv, s);
+}
+
+cudaError_t launch_combine(const CombineParams &p, cudaStream_t s) {
+    int nb = 0;
+    for (int i = 0; i < kMaxBatch; ++i)
+        if (p.lk[i] > 0) nb = i + 1;
+    if (nb == 0) return cudaSuccess;
+    dim3 grid(static_cast<unsigned>((p.lq + 7) / 8), static_cast<unsigned>(p.heads), static_cast<unsigned>(nb));
+    if (p.head_dim == 64)
+        attention_combine_kernel<64><<<grid, 256, 0, s>>>(p);
+    else
+        attention_combine_kernel<128><<<grid, 256, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace sdv2

@@ -1,0 +1,805 @@
+// libsdv2 host layer: config validation, buffer layout, the ring/phase
+// bookkeeping of every stream, RoPE tables, TMA descriptors and kernel
+// launches on the caller's stream.  Implements include/sdv2.h.
+//
+// Ring and phase rules (admirer.cn article on StreamDiffusionV2, method item
+// 1; agentlens page "chenfengxu714/StreamDiffusionV2", component table;
+// qq8o.cn walkthrough, "Adaptive sink and RoPE refresh"): frame f < S goes to
+// sink slot f, later frames to S + (f - S) mod W; the temporal RoPE phase is
+// f mod T_reset; the valid slots after frames 0..f_end-1 are the prefix of
+// length min(f_end, S) + min(max(f_end - S, 0), W).
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <atomic>
+#include <string>
+#include <vector>
+
+#include <cudaTypedefs.h>
+
+#include "sdv2.h"
+#include "sdv2_internal.h"
+
+using namespace sdv2;
+
+namespace {
+
+thread_local std::string g_err;
+std::atomic<uint64_t> g_launches{0};
+
+sdv2_status fail(sdv2_status st, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return st;
+}
+
+sdv2_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(SDV2_E_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+inline uint64_t align_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int32_t slot_of(int64_t f, int32_t S, int32_t W) {
+    if (f < 0) return -1;
+    if (f < S) return static_cast<int32_t>(f);
+    return S + static_cast<int32_t>((f - S) % W);
+}
+
+int64_t phase_of(int64_t f, int32_t reset) { return reset > 0 ? f % reset : f; }
+
+void valid_counts(int64_t f_end, int32_t S, int32_t W, int32_t *sv, int32_t *wv) {
+    const int64_t s = f_end < S ? f_end : S;
+    int64_t w = f_end - S;
+    if (w < 0) w = 0;
+    if (w > W) w = W;
+    *sv = static_cast<int32_t>(s < 0 ? 0 : s);
+    *wv = static_cast<int32_t>(w);
+}
+
+// Angle of pair j on an axis with n pairs at integer position pos.  Same
+// expression as the definition: pos * base^(-j/n), in fp64 with the C library.
+double rope_angle(double base, int j, int n, int64_t pos) {
+    const double omega = std::pow(base, -static_cast<double>(j) / static_cast<double>(n));
+    return static_cast<double>(pos) * omega;
+}
+
+struct Geometry {
+    int64_t N, slots, lq, frame_elems, layer_elems;
+    int n_qpairs, lq_pad;
+    int64_t part_rows;  // capacity of the split-KV partial buffer, rows of d floats
+    // region offsets
+    uint64_t rope_h64, rope_w64, rope_h32, rope_w32;
+    uint64_t sink_embed, sink_frame, status;
+    uint64_t scratch, refresh_mean, refresh_counter, part_ml, part_o, scratch_end;
+    uint64_t k, v, layer_stride, total;
+};
+
+constexpr int64_t kPartRowsCap = 196608;  // split-KV partial rows (~100 MB at d = 128)
+
+sdv2_status check_config(const sdv2_cache_config *c, sdv2_cache_config *norm) {
+    if (!c) return fail(SDV2_E_ARG, "config is NULL");
+    sdv2_cache_config n = *c;
+    if (n.batch < 1 || n.batch > kMaxBatch) return fail(SDV2_E_SHAPE, "batch must be in 1..%d", kMaxBatch);
+    if (n.layers < 1 || n.heads < 1) return fail(SDV2_E_SHAPE, "layers and heads must be >= 1");
+    if (n.head_dim != 64 && n.head_dim != 128) return fail(SDV2_E_SHAPE, "head_dim must be 64 or 128");
+    if (n.frame_h < 1 || n.frame_w < 1) return fail(SDV2_E_SHAPE, "frame_h and frame_w must be >= 1");
+    if (n.chunk_frames < 1 || n.sink_frames < 1 || n.window_frames < 1)
+        return fail(SDV2_E_SHAPE, "chunk_frames, sink_frames and window_frames must be >= 1");
+    if (n.window_frames < n.chunk_frames) return fail(SDV2_E_SHAPE, "window_frames must be >= chunk_frames");
+    if (n.rope_reset_period < 0) return fail(SDV2_E_SHAPE, "rope_reset_period must be >= 0");
+    if (n.embed_dim < 0 || (n.embed_dim & 1)) return fail(SDV2_E_SHAPE, "embed_dim must be even and >= 0");
+    if (!(n.rope_base > 0.0)) n.rope_base = 10000.0;
+    const int c2 = n.head_dim / 2;
+    if (n.rope_pairs[0] == 0 && n.rope_pairs[1] == 0 && n.rope_pairs[2] == 0) {
+        n.rope_pairs[1] = c2 / 3;
+        n.rope_pairs[2] = c2 / 3;
+        n.rope_pairs[0] = c2 - 2 * (c2 / 3);
+    }
+    if (n.rope_pairs[0] < 0 || n.rope_pairs[1] < 0 || n.rope_pairs[2] < 0 ||
+        n.rope_pairs[0] + n.rope_pairs[1] + n.rope_pairs[2] != c2)
+        return fail(SDV2_E_SHAPE, "rope_pairs must be >= 0 and sum to head_dim/2");
+    if (n.rope_pairs[0] < 1 || n.rope_pairs[0] > 64)
+        return fail(SDV2_E_SHAPE, "the temporal axis needs 1..64 rotation pairs");
+    if (n.rope_pairs[0] * n.chunk_frames > kAttnTabEntries)
+        return fail(SDV2_E_SHAPE, "chunk_frames * temporal pairs exceeds %d", kAttnTabEntries);
+    const int64_t N = static_cast<int64_t>(n.frame_h) * n.frame_w;
+    const int64_t slots = n.sink_frames + n.window_frames;
+    const int64_t fe = N * n.heads * n.head_dim;
+    if (slots * N >= (1ll << 31) || fe * kAppendMaxFrames * 2 / 8 >= (1ll << 31) ||
+        N * n.chunk_frames >= (1ll << 30))
+        return fail(SDV2_E_SHAPE, "cache dimensions exceed the supported 32-bit index range");
+    *norm = n;
+    return SDV2_OK;
+}
+
+Geometry geometry(const sdv2_cache_config &c) {
+    Geometry g{};
+    g.N = static_cast<int64_t>(c.frame_h) * c.frame_w;
+    g.slots = c.sink_frames + c.window_frames;
+    g.lq = g.N * c.chunk_frames;
+    g.frame_elems = g.N * c.heads * c.head_dim;
+    g.layer_elems = static_cast<int64_t>(c.batch) * g.slots * g.frame_elems;
+    g.n_qpairs = static_cast<int>((g.lq + kBlockM * kQTilesPerCta - 1) / (kBlockM * kQTilesPerCta));
+    g.lq_pad = g.n_qpairs * kBlockM * kQTilesPerCta;
+    const int64_t rows_one = static_cast<int64_t>(c.batch) * c.heads * g.lq_pad;
+    g.part_rows = rows_one * kMaxSplits;
+    if (g.part_rows > kPartRowsCap) g.part_rows = (kPartRowsCap / rows_one) * rows_one;
+    uint64_t off = 0;
+    g.k = off;
+    g.layer_stride = static_cast<uint64_t>(g.layer_elems) * 2;
+    off = align_up(off + g.layer_stride * c.layers, 256);
+    g.v = off;
+    off = align_up(off + g.layer_stride * c.layers, 256);
+    g.rope_h64 = off;
+    off = align_up(off + 16ull * c.frame_h * c.rope_pairs[1], 256);
+    g.rope_w64 = off;
+    off = align_up(off + 16ull * c.frame_w * c.rope_pairs[2], 256);
+    g.rope_h32 = off;
+    off = align_up(off + 8ull * c.frame_h * c.rope_pairs[1], 256);
+    g.rope_w32 = off;
+    off = align_up(off + 8ull * c.frame_w * c.rope_pairs[2], 256);
+    g.sink_embed = off;
+    off = align_up(off + 8ull * c.batch * c.sink_frames * (c.embed_dim > 0 ? c.embed_dim : 1), 256);
+    g.sink_frame = off;
+    off = align_up(off + 8ull * c.batch * c.sink_frames, 256);
+    g.status = off;
+    off = align_up(off + 4, 256);
+    g.scratch = off;
+    g.refresh_mean = off;
+    off = align_up(off + 8ull * c.batch * (c.embed_dim > 0 ? c.embed_dim : 1), 256);
+    g.refresh_counter = off;
+    off = align_up(off + 4ull * c.batch, 256);
+    g.part_ml = off;
+    off = align_up(off + 8ull * g.part_rows, 256);
+    g.part_o = off;
+    off = align_up(off + 4ull * c.head_dim * g.part_rows, 256);
+    g.scratch_end = off;
+    g.total = off;
+    return g;
+}
+
+// Split-KV partition count for one attention call: minimises an estimate of
+// the makespan (waves x KV tiles per CTA) plus the cost of writing and
+// merging partials, within the partial buffer's capacity.
+int plan_splits(const sdv2_cache_config &c, const Geometry &g, const int64_t *keys, int sm_count) {
+    int64_t max_tiles = 0;
+    int active = 0;
+    for (int b = 0; b < c.batch; ++b) {
+        if (keys[b] <= 0) continue;
+        ++active;
+        const int64_t t = (keys[b] + kBlockN - 1) / kBlockN;
+        if (t > max_tiles) max_tiles = t;
+    }
+    if (active == 0 || max_tiles <= 1 || sm_count <= 0) return 1;
+    const int64_t ctas1 = static_cast<int64_t>(c.batch) * c.heads * g.n_qpairs;
+    const int64_t rows_one = static_cast<int64_t>(c.batch) * c.heads * g.lq_pad;
+    // Cost units: one KV tile of one CTA (~2.5 us on a B200 SM at these sizes).
+    // Partial traffic per split: rows * (d + 2) floats written and read back.
+    const double tile_us = 2.5;
+    const double bytes_per_us = 6.0e6;   // ~6 TB/s
+    double best_cost = 1e300;
+    int best = 1;
+    for (int s = 1; s <= kMaxSplits; ++s) {
+        if (s > 1 && rows_one * s > g.part_rows) break;
+        const int64_t per = (max_tiles + s - 1) / s;
+        const int64_t ctas = ctas1 * s;
+        const int64_t waves = (ctas + sm_count - 1) / sm_count;
+        double cost = static_cast<double>(waves * per) * tile_us;
+        if (s > 1) cost += 3.0 + static_cast<double>(s) * rows_one * (c.head_dim + 2) * 8.0 / bytes_per_us;
+        if (cost < best_cost - 1e-9) {
+            best_cost = cost;
+            best = s;
+        }
+        if (per <= 1) break;
+    }
+    return best;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+}  // namespace
+
+struct sdv2_cache {
+    sdv2_cache_config cfg;
+    Geometry g;
+    uint8_t *base;
+    int device;
+    int sm_count;
+    std::vector<int64_t> next_frame;  // [B][L]
+    std::vector<CUtensorMap> tk, tv;  // [L]
+};
+
+struct sdv2_motion {
+    sdv2_motion_config cfg;
+    uint8_t *base;
+    int device;
+    int n_blocks;
+    int64_t frame_elems;
+    uint64_t off_prev, off_has_prev, off_hist, off_hist_len, off_hist_pos, off_rate, off_partial, off_counter,
+        off_status, total;
+};
+
+namespace {
+
+sdv2_status check_device(int device) {
+    int cur = -1;
+    cudaError_t e = cudaGetDevice(&cur);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (cur != device) return fail(SDV2_E_ARG, "current device %d is not the handle's device %d", cur, device);
+    return SDV2_OK;
+}
+
+sdv2_status check_stream_frames(const sdv2_cache *c, int32_t layer, const int64_t *f0, bool after_append,
+                                int *active_out) {
+    if (!f0) return fail(SDV2_E_ARG, "chunk_first_frame is NULL");
+    int active = 0;
+    for (int b = 0; b < c->cfg.batch; ++b) {
+        if (f0[b] < 0) continue;
+        ++active;
+        const int64_t expect = c->next_frame[static_cast<size_t>(b) * c->cfg.layers + layer];
+        const int64_t want = after_append ? f0[b] + c->cfg.chunk_frames : f0[b];
+        if (want != expect) {
+            if (after_append)
+                return fail(SDV2_E_STATE, "stream %d layer %d: chunk at frame %lld is not the last appended chunk", b,
+                            layer, static_cast<long long>(f0[b]));
+            return fail(SDV2_E_STATE, "stream %d layer %d: expected chunk at frame %lld, got %lld", b, layer,
+                        static_cast<long long>(expect), static_cast<long long>(f0[b]));
+        }
+    }
+    *active_out = active;
+    return SDV2_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sdv2_cache_bytes(const sdv2_cache_config *cfg) {
+    sdv2_cache_config n;
+    if (check_config(cfg, &n) != SDV2_OK) return 0;
+    return static_cast<size_t>(geometry(n).total);
+}
+
+static void fill_layout(const sdv2_cache_config &n, const Geometry &g, sdv2_cache_layout *out) {
+    out->k_offset = g.k;
+    out->v_offset = g.v;
+    out->layer_stride = g.layer_stride;
+    out->sink_embed_offset = g.sink_embed;
+    out->sink_frame_offset = g.sink_frame;
+    out->status_offset = g.status;
+    out->scratch_offset = g.scratch;
+    out->scratch_bytes = g.scratch_end - g.scratch;
+    out->total_bytes = g.total;
+    (void)n;
+}
+
+sdv2_status sdv2_cache_layout_of(const sdv2_cache_config *cfg, sdv2_cache_layout *out) {
+    if (!out) return fail(SDV2_E_ARG, "out is NULL");
+    sdv2_cache_config n;
+    sdv2_status st = check_config(cfg, &n);
+    if (st != SDV2_OK) return st;
+    fill_layout(n, geometry(n), out);
+    return SDV2_OK;
+}
+
+sdv2_status sdv2_cache_create(const sdv2_cache_config *cfg, void *dev_buf, size_t bytes, sdv2_cache **out) {
+    if (!out) return fail(SDV2_E_ARG, "out is NULL");
+    *out = nullptr;
+    sdv2_cache_config n;
+    sdv2_status st = check_config(cfg, &n);
+    if (st != SDV2_OK) return st;
+    if (!dev_buf) return fail(SDV2_E_ARG, "dev_buf is NULL");
+    if ((reinterpret_cast<uintptr_t>(dev_buf) & 255u) != 0) return fail(SDV2_E_ALIGN, "dev_buf must be 256-byte aligned");
+    const Geometry g = geometry(n);
+    if (bytes < g.total)
+        return fail(SDV2_E_ALIGN, "buffer of %zu bytes is smaller than the %llu bytes required", bytes,
+                    static_cast<unsigned long long>(g.total));
+    PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode_fn();
+    if (!encode) return fail(SDV2_E_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+
+    sdv2_cache *c = new sdv2_cache();
+    c->cfg = n;
+    c->g = g;
+    c->base = static_cast<uint8_t *>(dev_buf);
+    cudaError_t e = cudaGetDevice(&c->device);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, c->device);
+    if (e == cudaSuccess) e = cudaMemset(dev_buf, 0, g.total);
+    if (e != cudaSuccess) {
+        delete c;
+        return cuda_fail(e, "cache_create");
+    }
+    // RoPE row / column tables (fp64 for the bit-exact key rotation, fp32 for queries).
+    const int nh = n.rope_pairs[1], nw = n.rope_pairs[2];
+    std::vector<double> h64(2ull * n.frame_h * nh), w64(2ull * n.frame_w * nw);
+    std::vector<float> h32(h64.size()), w32(w64.size());
+    for (int r = 0; r < n.frame_h; ++r)
+        for (int j = 0; j < nh; ++j) {
+            const double a = rope_angle(n.rope_base, j, nh, r);
+            h64[2 * (r * nh + j)] = std::cos(a);
+            h64[2 * (r * nh + j) + 1] = std::sin(a);
+        }
+    for (int col = 0; col < n.frame_w; ++col)
+        for (int j = 0; j < nw; ++j) {
+            const double a = rope_angle(n.rope_base, j, nw, col);
+            w64[2 * (col * nw + j)] = std::cos(a);
+            w64[2 * (col * nw + j) + 1] = std::sin(a);
+        }
+    for (size_t i = 0; i < h64.size(); ++i) h32[i] = static_cast<float>(h64[i]);
+    for (size_t i = 0; i < w64.size(); ++i) w32[i] = static_cast<float>(w64[i]);
+    std::vector<int64_t> sink_frames(static_cast<size_t>(n.batch) * n.sink_frames, -1);
+    struct Up { uint64_t off; const void *src; size_t bytes; } ups[] = {
+        {g.rope_h64, h64.data(), h64.size() * 8}, {g.rope_w64, w64.data(), w64.size() * 8},
+        {g.rope_h32, h32.data(), h32.size() * 4}, {g.rope_w32, w32.data(), w32.size() * 4},
+        {g.sink_frame, sink_frames.data(), sink_frames.size() * 8}};
+    for (const Up &u : ups) {
+        if (u.bytes == 0) continue;
+        e = cudaMemcpy(c->base + u.off, u.src, u.bytes, cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) {
+            delete c;
+            return cuda_fail(e, "cache_create upload");
+        }
+    }
+    // One TMA descriptor per layer for K and for V: dims (d, H, slots*N, B).
+    c->tk.resize(n.layers);
+    c->tv.resize(n.layers);
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(n.head_dim), static_cast<cuuint64_t>(n.heads),
+                                static_cast<cuuint64_t>(g.slots * g.N), static_cast<cuuint64_t>(n.batch)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(n.head_dim) * 2,
+                                   static_cast<cuuint64_t>(n.heads) * n.head_dim * 2,
+                                   static_cast<cuuint64_t>(g.slots * g.frame_elems) * 2};
+    const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kBlockN), 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    for (int l = 0; l < n.layers; ++l) {
+        for (int kv = 0; kv < 2; ++kv) {
+            void *ptr = c->base + (kv ? g.v : g.k) + g.layer_stride * l;
+            CUresult r = encode(kv ? &c->tv[l] : &c->tk[l], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, ptr, dims, strides,
+                                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+            if (r != CUDA_SUCCESS) {
+                delete c;
+                return fail(SDV2_E_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+            }
+        }
+    }
+    c->next_frame.assign(static_cast<size_t>(n.batch) * n.layers, 0);
+    *out = c;
+    return SDV2_OK;
+}
+
+sdv2_status sdv2_cache_destroy(sdv2_cache *cache) {
+    delete cache;
+    return SDV2_OK;
+}
+
+sdv2_status sdv2_kv_append(sdv2_cache *c, int32_t layer, const void *k, const void *v,
+                           const int64_t *chunk_first_frame, sdv2_stream stream) {
+    if (!c || !k || !v) return fail(SDV2_E_ARG, "NULL argument");
+    if (layer < 0 || layer >= c->cfg.layers) return fail(SDV2_E_ARG, "layer %d out of range", layer);
+    if (!aligned16(k) || !aligned16(v)) return fail(SDV2_E_ALIGN, "k and v must be 16-byte aligned");
+    int active = 0;
+    sdv2_status st = check_stream_frames(c, layer, chunk_first_frame, false, &active);
+    if (st != SDV2_OK) return st;
+    if ((st = check_device(c->device)) != SDV2_OK) return st;
+    const sdv2_cache_config &n = c->cfg;
+    const int n_t = n.rope_pairs[0];
+    const int per_launch = std::min(kAppendMaxFrames, kAppendTabEntries / n_t);
+    AppendParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.k_in = static_cast<const uint16_t *>(k);
+    p.v_in = static_cast<const uint16_t *>(v);
+    p.k_layer = reinterpret_cast<uint16_t *>(c->base + c->g.k + c->g.layer_stride * layer);
+    p.v_layer = reinterpret_cast<uint16_t *>(c->base + c->g.v + c->g.layer_stride * layer);
+    p.rope_h = reinterpret_cast<const double *>(c->base + c->g.rope_h64);
+    p.rope_w = reinterpret_cast<const double *>(c->base + c->g.rope_w64);
+    p.frame_elems = c->g.frame_elems;
+    p.chunk_tokens = static_cast<int32_t>(c->g.lq);
+    p.heads = n.heads;
+    p.head_dim = n.head_dim;
+    p.frame_w = n.frame_w;
+    p.n_t = n_t;
+    p.n_h = n.rope_pairs[1];
+    p.n_w = n.rope_pairs[2];
+    p.slots = static_cast<int32_t>(c->g.slots);
+    auto flush = [&]() -> sdv2_status {
+        if (p.n_frames == 0) return SDV2_OK;
+        cudaError_t e = launch_append(p, c->sm_count, reinterpret_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return cuda_fail(e, "kv_append launch");
+        g_launches.fetch_add(1);
+        p.n_frames = 0;
+        return SDV2_OK;
+    };
+    for (int b = 0; b < n.batch; ++b) {
+        const int64_t f0 = chunk_first_frame[b];
+        if (f0 < 0) continue;
+        for (int i = 0; i < n.chunk_frames; ++i) {
+            const int64_t f = f0 + i;
+            const int fi = p.n_frames;
+            p.src_b[fi] = b;
+            p.src_i[fi] = i;
+            p.dst_slot[fi] = slot_of(f, n.sink_frames, n.window_frames);
+            const int64_t ph = phase_of(f, n.rope_reset_period);
+            for (int j = 0; j < n_t; ++j) {
+                const double a = rope_angle(n.rope_base, j, n_t, ph);
+                p.tab_t[fi * n_t + j][0] = std::cos(a);
+                p.tab_t[fi * n_t + j][1] = std::sin(a);
+            }
+            ++p.n_frames;
+            if (p.n_frames == per_launch && (st = flush()) != SDV2_OK) return st;
+        }
+    }
+    if ((st = flush()) != SDV2_OK) return st;
+    for (int b = 0; b < n.batch; ++b)
+        if (chunk_first_frame[b] >= 0) c->next_frame[static_cast<size_t>(b) * n.layers + layer] += n.chunk_frames;
+    return SDV2_OK;
+}
+
+sdv2_status sdv2_chunk_attention(sdv2_cache *c, int32_t layer, const void *q, void *out,
+                                 const int64_t *chunk_first_frame, float softmax_scale, sdv2_stream stream) {
+    if (!c || !q || !out) return fail(SDV2_E_ARG, "NULL argument");
+    if (layer < 0 || layer >= c->cfg.layers) return fail(SDV2_E_ARG, "layer %d out of range", layer);
+    if (!(softmax_scale > 0.0f) || !std::isfinite(softmax_scale)) return fail(SDV2_E_ARG, "softmax_scale must be > 0");
+    if (!aligned16(q) || !aligned16(out)) return fail(SDV2_E_ALIGN, "q and out must be 16-byte aligned");
+    int active = 0;
+    sdv2_status st = check_stream_frames(c, layer, chunk_first_frame, true, &active);
+    if (st != SDV2_OK) return st;
+    if ((st = check_device(c->device)) != SDV2_OK) return st;
+    if (active == 0) return SDV2_OK;
+    const sdv2_cache_config &n = c->cfg;
+    const Geometry &g = c->g;
+    std::vector<int64_t> keys(n.batch, 0);
+    for (int b = 0; b < n.batch; ++b) {
+        if (chunk_first_frame[b] < 0) continue;
+        int32_t sv, wv;
+        valid_counts(chunk_first_frame[b] + n.chunk_frames, n.sink_frames, n.window_frames, &sv, &wv);
+        keys[b] = static_cast<int64_t>(sv + wv) * g.N;
+    }
+    const int n_split = plan_splits(n, g, keys.data(), c->sm_count);
+    const int n_t = n.rope_pairs[0];
+    const int streams_per_launch = std::min(kMaxBatch, kAttnTabEntries / (n_t * n.chunk_frames));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    AttnParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.q = static_cast<const uint16_t *>(q);
+    p.out = static_cast<uint16_t *>(out);
+    p.part_o = reinterpret_cast<float *>(c->base + g.part_o);
+    p.part_ml = reinterpret_cast<float *>(c->base + g.part_ml);
+    p.rope_h = reinterpret_cast<const float *>(c->base + g.rope_h32);
+    p.rope_w = reinterpret_cast<const float *>(c->base + g.rope_w32);
+    p.status = reinterpret_cast<uint32_t *>(c->base + g.status);
+    p.batch = n.batch;
+    p.heads = n.heads;
+    p.lq = static_cast<int32_t>(g.lq);
+    p.lq_pad = g.lq_pad;
+    p.tokens_per_frame = static_cast<int32_t>(g.N);
+    p.frame_w = n.frame_w;
+    p.chunk_frames = n.chunk_frames;
+    p.n_t = n_t;
+    p.n_h = n.rope_pairs[1];
+    p.n_w = n.rope_pairs[2];
+    p.n_qpairs = g.n_qpairs;
+    p.n_split = n_split;
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    for (int b0 = 0; b0 < n.batch; b0 += streams_per_launch) {
+        const int nb = std::min(streams_per_launch, n.batch - b0);
+        p.b_offset = b0;
+        bool any = false;
+        for (int bl = 0; bl < kMaxBatch; ++bl) p.lk[bl] = 0;
+        for (int bl = 0; bl < nb; ++bl) {
+            const int b = b0 + bl;
+            p.lk[bl] = static_cast<int32_t>(keys[b]);
+            if (keys[b] <= 0) continue;
+            any = true;
+            const int64_t f0 = chunk_first_frame[b];
+            for (int fi = 0; fi < n.chunk_frames; ++fi) {
+                const int64_t ph = phase_of(f0 + fi, n.rope_reset_period);
+                for (int j = 0; j < n_t; ++j) {
+                    const double a = rope_angle(n.rope_base, j, n_t, ph);
+                    p.tab_t[(bl * n.chunk_frames + fi) * n_t + j][0] = static_cast<float>(std::cos(a));
+                    p.tab_t[(bl * n.chunk_frames + fi) * n_t + j][1] = static_cast<float>(std::sin(a));
+                }
+            }
+        }
+        if (!any) continue;
+        cudaError_t e = launch_attention(p, c->tk[layer], c->tv[layer], n.head_dim, s);
+        if (e != cudaSuccess) return cuda_fail(e, "chunk_attention launch");
+        g_launches.fetch_add(1);
+        if (n_split > 1) {
+            CombineParams cp;
+            std::memset(&cp, 0, sizeof(cp));
+            cp.part_o = p.part_o;
+            cp.part_ml = p.part_ml;
+            cp.out = p.out;
+            cp.batch = n.batch;
+            cp.heads = n.heads;
+            cp.lq = p.lq;
+            cp.lq_pad = p.lq_pad;
+            cp.head_dim = n.head_dim;
+            cp.n_split = n_split;
+            cp.b_offset = b0;
+            for (int bl = 0; bl < kMaxBatch; ++bl) cp.lk[bl] = p.lk[bl];
+            e = launch_combine(cp, s);
+            if (e != cudaSuccess) return cuda_fail(e, "attention combine launch");
+            g_launches.fetch_add(1);
+        }
+    }
+    return SDV2_OK;
+}
+
+sdv2_status sdv2_sink_refresh(sdv2_cache *c, const void *hidden, float tau, const int64_t *chunk_first_frame,
+                              int32_t *out_slot_dev, sdv2_stream stream) {
+    if (!c || !hidden || !out_slot_dev) return fail(SDV2_E_ARG, "NULL argument");
+    if (c->cfg.embed_dim <= 0) return fail(SDV2_E_SHAPE, "the cache was created with embed_dim 0");
+    if (!aligned16(hidden) || (reinterpret_cast<uintptr_t>(out_slot_dev) & 3u))
+        return fail(SDV2_E_ALIGN, "hidden must be 16-byte aligned and out_slot_dev 4-byte aligned");
+    if (!std::isfinite(tau)) return fail(SDV2_E_ARG, "tau must be finite");
+    if (!chunk_first_frame) return fail(SDV2_E_ARG, "chunk_first_frame is NULL");
+    const sdv2_cache_config &n = c->cfg;
+    for (int l = 0; l < n.layers; ++l) {
+        int active = 0;
+        sdv2_status st = check_stream_frames(c, l, chunk_first_frame, true, &active);
+        if (st != SDV2_OK) return st;
+    }
+    sdv2_status st = check_device(c->device);
+    if (st != SDV2_OK) return st;
+    const Geometry &g = c->g;
+    RefreshParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.hidden = static_cast<const uint16_t *>(hidden);
+    p.mean = reinterpret_cast<double *>(c->base + g.refresh_mean);
+    p.counter = reinterpret_cast<uint32_t *>(c->base + g.refresh_counter);
+    p.sink_embed = reinterpret_cast<double *>(c->base + g.sink_embed);
+    p.sink_frame = reinterpret_cast<int64_t *>(c->base + g.sink_frame);
+    p.out_slot = out_slot_dev;
+    p.k_cache = reinterpret_cast<uint16_t *>(c->base + g.k);
+    p.v_cache = reinterpret_cast<uint16_t *>(c->base + g.v);
+    p.layer_stride_elems = static_cast<int64_t>(g.layer_stride / 2);
+    p.frame_elems = g.frame_elems;
+    p.batch = n.batch;
+    p.lq = static_cast<int32_t>(g.lq);
+    p.dim = n.embed_dim;
+    p.sinks = n.sink_frames;
+    p.slots = static_cast<int32_t>(g.slots);
+    p.layers = n.layers;
+    p.tau = static_cast<double>(tau);
+    for (int b = 0; b < n.batch; ++b) {
+        const int64_t f0 = chunk_first_frame[b];
+        p.fill_first[b] = -1;
+        if (f0 < 0) continue;
+        p.active[b] = 1;
+        if (f0 < n.sink_frames) {
+            p.fill_first[b] = static_cast<int32_t>(f0);
+            const int64_t end = std::min<int64_t>(n.sink_frames, f0 + n.chunk_frames);
+            p.fill_count[b] = static_cast<int32_t>(end - f0);
+        }
+        p.last_frame[b] = f0 + n.chunk_frames - 1;
+        p.last_slot[b] = slot_of(p.last_frame[b], n.sink_frames, n.window_frames);
+    }
+    int launches = 0;
+    cudaError_t e = launch_refresh(p, c->sm_count, reinterpret_cast<cudaStream_t>(stream), &launches);
+    g_launches.fetch_add(static_cast<uint64_t>(launches));
+    if (e != cudaSuccess) return cuda_fail(e, "sink_refresh launch");
+    return SDV2_OK;
+}
+
+sdv2_status sdv2_cache_query(const sdv2_cache *c, int32_t b, int32_t layer, int64_t *slot_frame, int32_t *slot_phase,
+                             int32_t *valid_slots) {
+    if (!c) return fail(SDV2_E_ARG, "cache is NULL");
+    const sdv2_cache_config &n = c->cfg;
+    if (b < 0 || b >= n.batch || layer < 0 || layer >= n.layers) return fail(SDV2_E_ARG, "stream or layer out of range");
+    const int64_t f_end = c->next_frame[static_cast<size_t>(b) * n.layers + layer];
+    const int slots = n.sink_frames + n.window_frames;
+    for (int s = 0; s < slots; ++s) {
+        if (slot_frame) slot_frame[s] = -1;
+        if (slot_phase) slot_phase[s] = -1;
+    }
+    for (int64_t f = f_end - n.window_frames - n.sink_frames; f < f_end; ++f) {
+        if (f < 0) continue;
+        const int s = slot_of(f, n.sink_frames, n.window_frames);
+        if (slot_frame) slot_frame[s] = f;
+        if (slot_phase) slot_phase[s] = static_cast<int32_t>(phase_of(f, n.rope_reset_period));
+    }
+    for (int s = 0; s < n.sink_frames && s < f_end; ++s) {
+        if (slot_frame) slot_frame[s] = s;
+        if (slot_phase) slot_phase[s] = static_cast<int32_t>(phase_of(s, n.rope_reset_period));
+    }
+    int32_t sv, wv;
+    valid_counts(f_end, n.sink_frames, n.window_frames, &sv, &wv);
+    if (valid_slots) *valid_slots = sv + wv;
+    return SDV2_OK;
+}
+
+sdv2_status sdv2_cache_layout_get(const sdv2_cache *c, sdv2_cache_layout *out) {
+    if (!c || !out) return fail(SDV2_E_ARG, "NULL argument");
+    fill_layout(c->cfg, c->g, out);
+    return SDV2_OK;
+}
+
+sdv2_status sdv2_cache_check(sdv2_cache *c) {
+    if (!c) return fail(SDV2_E_ARG, "cache is NULL");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cache_check");
+    uint32_t word = 0;
+    e = cudaMemcpy(&word, c->base + c->g.status, 4, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "cache_check");
+    if (word != 0) {
+        const uint32_t zero = 0;
+        cudaMemcpy(c->base + c->g.status, &zero, 4, cudaMemcpyHostToDevice);
+        return fail(SDV2_E_DEVICE, "device status 0x%x (a kernel gave up on a bounded wait)", word);
+    }
+    return SDV2_OK;
+}
+
+// ------------------------------------------------------------------ motion
+
+static sdv2_status check_motion(const sdv2_motion_config *m) {
+    if (!m) return fail(SDV2_E_ARG, "config is NULL");
+    if (m->batch < 1 || m->batch > kMaxBatch) return fail(SDV2_E_SHAPE, "batch must be in 1..%d", kMaxBatch);
+    if (m->chunk_frames < 1 || m->chunk_frames > 64) return fail(SDV2_E_SHAPE, "chunk_frames must be in 1..64");
+    if (m->channels < 1 || m->height < 1 || m->width < 1) return fail(SDV2_E_SHAPE, "latent shape must be >= 1");
+    if (m->window < 1 || m->window > 64) return fail(SDV2_E_SHAPE, "window must be in 1..64");
+    if (!(m->sigma > 0.0) || !(m->lambda > 0.0) || !(m->lambda <= 1.0))
+        return fail(SDV2_E_ARG, "need sigma > 0 and 0 < lambda <= 1");
+    if (!std::isfinite(m->s_min) || !std::isfinite(m->s_max) || !std::isfinite(m->s_init))
+        return fail(SDV2_E_ARG, "noise-rate bounds must be finite");
+    return SDV2_OK;
+}
+
+static void motion_layout(const sdv2_motion_config &m, sdv2_motion *h) {
+    h->frame_elems = static_cast<int64_t>(m.channels) * m.height * m.width;
+    h->n_blocks = static_cast<int>((h->frame_elems + kMotionBlockElems - 1) / kMotionBlockElems);
+    uint64_t off = 0;
+    h->off_prev = off;
+    off = align_up(off + 4ull * m.batch * h->frame_elems, 256);
+    h->off_has_prev = off;
+    off = align_up(off + 4ull * m.batch, 256);
+    h->off_hist = off;
+    off = align_up(off + 8ull * m.batch * m.window, 256);
+    h->off_hist_len = off;
+    off = align_up(off + 4ull * m.batch, 256);
+    h->off_hist_pos = off;
+    off = align_up(off + 4ull * m.batch, 256);
+    h->off_rate = off;
+    off = align_up(off + 8ull * m.batch, 256);
+    h->off_status = off;
+    off = align_up(off + 4, 256);
+    h->off_partial = off;
+    off = align_up(off + 8ull * m.batch * m.chunk_frames * h->n_blocks, 256);
+    h->off_counter = off;
+    off = align_up(off + 4ull * m.batch, 256);
+    h->total = off;
+}
+
+size_t sdv2_motion_bytes(const sdv2_motion_config *cfg) {
+    if (check_motion(cfg) != SDV2_OK) return 0;
+    sdv2_motion h{};
+    motion_layout(*cfg, &h);
+    return static_cast<size_t>(h.total);
+}
+
+sdv2_status sdv2_motion_create(const sdv2_motion_config *cfg, void *dev_buf, size_t bytes, sdv2_motion **out) {
+    if (!out) return fail(SDV2_E_ARG, "out is NULL");
+    *out = nullptr;
+    sdv2_status st = check_motion(cfg);
+    if (st != SDV2_OK) return st;
+    if (!dev_buf) return fail(SDV2_E_ARG, "dev_buf is NULL");
+    if ((reinterpret_cast<uintptr_t>(dev_buf) & 255u) != 0) return fail(SDV2_E_ALIGN, "dev_buf must be 256-byte aligned");
+    sdv2_motion *h = new sdv2_motion();
+    h->cfg = *cfg;
+    motion_layout(*cfg, h);
+    if (bytes < h->total) {
+        const unsigned long long need = h->total;
+        delete h;
+        return fail(SDV2_E_ALIGN, "buffer of %zu bytes is smaller than the %llu bytes required", bytes, need);
+    }
+    h->base = static_cast<uint8_t *>(dev_buf);
+    cudaError_t e = cudaGetDevice(&h->device);
+    if (e == cudaSuccess) e = cudaMemset(dev_buf, 0, h->total);
+    std::vector<double> rate(cfg->batch, cfg->s_init);
+    if (e == cudaSuccess) e = cudaMemcpy(h->base + h->off_rate, rate.data(), 8ull * cfg->batch, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+        delete h;
+        return cuda_fail(e, "motion_create");
+    }
+    *out = h;
+    return SDV2_OK;
+}
+
+sdv2_status sdv2_motion_destroy(sdv2_motion *m) {
+    delete m;
+    return SDV2_OK;
+}
+
+sdv2_status sdv2_motion_noise_rate(sdv2_motion *m, const float *latents, float *out_rate_dev, float *out_d_dev,
+                                   sdv2_stream stream) {
+    if (!m || !latents || !out_rate_dev) return fail(SDV2_E_ARG, "NULL argument");
+    if (!aligned16(latents) || (reinterpret_cast<uintptr_t>(out_rate_dev) & 3u) ||
+        (reinterpret_cast<uintptr_t>(out_d_dev) & 3u))
+        return fail(SDV2_E_ALIGN, "latents must be 16-byte aligned, outputs 4-byte aligned");
+    sdv2_status st = check_device(m->device);
+    if (st != SDV2_OK) return st;
+    MotionParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.latents = latents;
+    p.prev = reinterpret_cast<float *>(m->base + m->off_prev);
+    p.has_prev = reinterpret_cast<int32_t *>(m->base + m->off_has_prev);
+    p.hist = reinterpret_cast<double *>(m->base + m->off_hist);
+    p.hist_len = reinterpret_cast<int32_t *>(m->base + m->off_hist_len);
+    p.hist_pos = reinterpret_cast<int32_t *>(m->base + m->off_hist_pos);
+    p.rate = reinterpret_cast<double *>(m->base + m->off_rate);
+    p.partial = reinterpret_cast<double *>(m->base + m->off_partial);
+    p.counter = reinterpret_cast<uint32_t *>(m->base + m->off_counter);
+    p.out_rate = out_rate_dev;
+    p.out_d = out_d_dev;
+    p.frame_elems = m->frame_elems;
+    p.batch = m->cfg.batch;
+    p.chunk_frames = m->cfg.chunk_frames;
+    p.window = m->cfg.window;
+    p.n_blocks = m->n_blocks;
+    p.sigma = m->cfg.sigma;
+    p.lambda = m->cfg.lambda;
+    p.s_min = m->cfg.s_min;
+    p.s_max = m->cfg.s_max;
+    cudaError_t e = launch_motion(p, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "motion launch");
+    g_launches.fetch_add(1);
+    return SDV2_OK;
+}
+
+sdv2_status sdv2_motion_check(sdv2_motion *m) {
+    if (!m) return fail(SDV2_E_ARG, "motion is NULL");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "motion_check");
+    uint32_t word = 0;
+    e = cudaMemcpy(&word, m->base + m->off_status, 4, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "motion_check");
+    if (word != 0) return fail(SDV2_E_DEVICE, "device status 0x%x", word);
+    return SDV2_OK;
+}
+
+// ------------------------------------------------------------------ host-only helpers
+
+int32_t sdv2_slot_of_frame(int64_t f, int32_t sink_frames, int32_t window_frames) {
+    if (sink_frames < 1 || window_frames < 1) return -1;
+    return slot_of(f, sink_frames, window_frames);
+}
+
+int64_t sdv2_rope_phase(int64_t f, int32_t rope_reset_period) { return phase_of(f, rope_reset_period); }
+
+void sdv2_valid_slots(int64_t frame_end, int32_t sink_frames, int32_t window_frames, int32_t *sink_valid,
+                      int32_t *window_valid) {
+    int32_t sv = 0, wv = 0;
+    valid_counts(frame_end, sink_frames, window_frames, &sv, &wv);
+    if (sink_valid) *sink_valid = sv;
+    if (window_valid) *window_valid = wv;
+}
+
+int32_t sdv2_attention_splits(const sdv2_cache_config *cfg, const int64_t *keys, int32_t sm_count) {
+    sdv2_cache_config n;
+    if (!keys || check_config(cfg, &n) != SDV2_OK) return -1;
+    return plan_splits(n, geometry(n), keys, sm_count);
+}
+
+uint64_t sdv2_launch_count(void) { return g_launches.load(); }
+
+const char *sdv2_last_error(void) { return g_err.c_str(); }
+
+const char *sdv2_version(void) { return "sdv2 0.1.0 (sm_100a)"; }
+
+}  // extern "C"

@@ -1,0 +1,110 @@
+// Motion-aware noise rate: frame-difference RMS, k-frame maximum, clip and EMA.
+//
+// Sources: admirer.cn article on StreamDiffusionV2, method item 2 (motion
+// strength from the L2 distance of adjacent frames; more motion -> less
+// noise); qq8o.cn walkthrough, "Motion-aware noise scheduler" (normalise by
+// a statistical scale over a short k-frame window, clip to [0, 1], EMA with
+// 0 < lambda < 1 between s_min and s_max).
+//
+// One launch per call.  Block (x, b) owns a contiguous slice of the latent
+// frame of stream b: it sums squared differences of that slice for every
+// frame of the chunk in fp64, writes one partial per frame, then overwrites
+// the slice of the stored previous frame with the chunk's last frame (only
+// this block touches that slice, so no ordering across blocks is needed).
+// The last block of a stream to finish (counted with an atomic ticket) sums
+// the partials in block order and runs the recurrence in fp64.
+#include <cmath>
+
+#include "ptx.cuh"
+
+namespace sdv2 {
+
+__global__ void __launch_bounds__(kMotionThreads) motion_kernel(const __grid_constant__ MotionParams p) {
+    const int b = blockIdx.y;
+    const int blk = blockIdx.x;
+    const int tid = threadIdx.x;
+    const int64_t n = p.frame_elems;
+    const int64_t begin = static_cast<int64_t>(blk) * kMotionBlockElems;
+    const int64_t end = begin + kMotionBlockElems < n ? begin + kMotionBlockElems : n;
+    const float *x = p.latents + static_cast<int64_t>(b) * p.chunk_frames * n;
+    float *prev = p.prev + static_cast<int64_t>(b) * n;
+    const bool had_prev = p.has_prev[b] != 0;
+
+    __shared__ double red[kMotionThreads / 32];
+    __shared__ int is_last;
+
+    for (int t = 0; t < p.chunk_frames; ++t) {
+        double acc = 0.0;
+        if (t > 0 || had_prev) {
+            const float *cur = x + static_cast<int64_t>(t) * n;
+            const float *before = t == 0 ? prev : x + static_cast<int64_t>(t - 1) * n;
+            for (int64_t e = begin + tid; e < end; e += kMotionThreads) {
+                const double dlt = static_cast<double>(cur[e]) - static_cast<double>(before[e]);
+                acc += dlt * dlt;
+            }
+        }
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if ((tid & 31) == 0) red[tid >> 5] = acc;
+        __syncthreads();
+        if (tid == 0) {
+            double s = 0.0;
+            for (int w = 0; w < kMotionThreads / 32; ++w) s += red[w];
+            p.partial[(static_cast<int64_t>(b) * p.chunk_frames + t) * p.n_blocks + blk] = s;
+        }
+        __syncthreads();
+    }
+    // This block's slice of the previous frame is no longer needed: replace it.
+    const float *last = x + static_cast<int64_t>(p.chunk_frames - 1) * n;
+    for (int64_t e = begin + tid; e < end; e += kMotionThreads) prev[e] = last[e];
+
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        const unsigned ticket = atomicAdd(p.counter + b, 1u);
+        is_last = ticket == static_cast<unsigned>(p.n_blocks - 1);
+    }
+    __syncthreads();
+    if (!is_last || tid != 0) return;
+    __threadfence();
+
+    double rate = p.rate[b];
+    int len = p.hist_len[b];
+    int pos = p.hist_pos[b];
+    double *hist = p.hist + static_cast<int64_t>(b) * p.window;
+    bool have = had_prev;
+    for (int t = 0; t < p.chunk_frames; ++t) {
+        float d_out = -1.0f;
+        if (have) {
+            double ss = 0.0;
+            const double *part = p.partial + (static_cast<int64_t>(b) * p.chunk_frames + t) * p.n_blocks;
+            for (int i = 0; i < p.n_blocks; ++i) ss += __ldcg(part + i);
+            const double d = sqrt(ss / static_cast<double>(n));
+            hist[pos] = d;
+            pos = (pos + 1) % p.window;
+            if (len < p.window) ++len;
+            double dbar = hist[0];
+            for (int i = 1; i < len; ++i) dbar = fmax(dbar, hist[i]);
+            double dhat = dbar / p.sigma;
+            dhat = dhat < 0.0 ? 0.0 : (dhat > 1.0 ? 1.0 : dhat);
+            const double target = p.s_max - (p.s_max - p.s_min) * dhat;
+            rate = p.lambda * target + (1.0 - p.lambda) * rate;
+            d_out = static_cast<float>(d);
+        }
+        have = true;
+        if (p.out_d) p.out_d[static_cast<int64_t>(b) * p.chunk_frames + t] = d_out;
+    }
+    p.rate[b] = rate;
+    p.hist_len[b] = len;
+    p.hist_pos[b] = pos;
+    p.has_prev[b] = 1;
+    p.out_rate[b] = static_cast<float>(rate);
+    p.counter[b] = 0u;
+}
+
+cudaError_t launch_motion(const MotionParams &p, cudaStream_t s) {
+    dim3 grid(static_cast<unsigned>(p.n_blocks), static_cast<unsigned>(p.batch));
+    motion_kernel<<<grid, kMotionThreads, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace sdv2

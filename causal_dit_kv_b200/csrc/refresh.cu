@@ -1,0 +1,160 @@
+// Adaptive sink refresh: chunk-mean embedding, cosine against the sink set,
+// device-side decision, predicated copy of the chunk's last frame K/V.
+//
+// Source: qq8o.cn walkthrough of StreamDiffusionV2, "Adaptive sink and RoPE
+// refresh" (compare the new chunk embedding with the sink set by cosine
+// similarity; replace the least similar sink when the similarity falls
+// below the threshold tau).
+//
+// Kernel 1, grid (column blocks, B): block (x, b) averages 64 columns of the
+// hidden states over all tokens in fp64 (warp w takes tokens w, w+8, ...;
+// lane l takes columns 2l, 2l+1), fixed-order reduction across warps.  The
+// last block of stream b (atomic ticket) computes the dot products and
+// norms in fp64, takes the decision, updates the sink embedding and the
+// sink-frame record, and writes out_slot[b].
+// Kernel 2, grid (blocks, B): if out_slot[b] >= 0, copies slot last_slot[b]
+// to slot out_slot[b] in every layer, K and V, as 16-byte vectors; otherwise
+// the blocks return at once.
+#include <cmath>
+
+#include "ptx.cuh"
+
+namespace sdv2 {
+
+constexpr int kRefreshThreads = 256;
+constexpr int kRefreshCols = 64;
+
+__device__ __forceinline__ double block_sum_fixed(double v, double *red) {
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    double s = 0.0;
+    for (int w = 0; w < kRefreshThreads / 32; ++w) s += red[w];
+    return s;
+}
+
+__global__ void __launch_bounds__(kRefreshThreads) refresh_decide_kernel(const __grid_constant__ RefreshParams p) {
+    const int b = blockIdx.y;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (!p.active[b]) {
+        if (blockIdx.x == 0 && tid == 0) p.out_slot[b] = -1;
+        return;
+    }
+    __shared__ double part[kRefreshThreads / 32][kRefreshCols];
+    __shared__ double red[kRefreshThreads / 32];
+    __shared__ int is_last;
+
+    const int col0 = blockIdx.x * kRefreshCols + 2 * lane;
+    const uint16_t *hb = p.hidden + static_cast<int64_t>(b) * p.lq * p.dim;
+    double a0 = 0.0, a1 = 0.0;
+    if (col0 < p.dim) {
+        for (int t = warp; t < p.lq; t += kRefreshThreads / 32) {
+            const uint32_t w = *reinterpret_cast<const uint32_t *>(hb + static_cast<int64_t>(t) * p.dim + col0);
+            a0 += static_cast<double>(bf16_lo(w));
+            a1 += static_cast<double>(bf16_hi(w));
+        }
+    }
+    part[warp][2 * lane] = a0;
+    part[warp][2 * lane + 1] = a1;
+    __syncthreads();
+    if (tid < kRefreshCols) {
+        const int c = blockIdx.x * kRefreshCols + tid;
+        if (c < p.dim) {
+            double s = 0.0;
+            for (int w = 0; w < kRefreshThreads / 32; ++w) s += part[w][tid];
+            p.mean[static_cast<int64_t>(b) * p.dim + c] = s / static_cast<double>(p.lq);
+        }
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) is_last = atomicAdd(p.counter + b, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+
+    const double *h = p.mean + static_cast<int64_t>(b) * p.dim;
+    double *emb = p.sink_embed + static_cast<int64_t>(b) * p.sinks * p.dim;
+    if (p.fill_count[b] > 0) {
+        // The chunk fills sink slots itself: record their embedding only.
+        for (int j = p.fill_first[b]; j < p.fill_first[b] + p.fill_count[b]; ++j) {
+            for (int c = tid; c < p.dim; c += kRefreshThreads) emb[static_cast<int64_t>(j) * p.dim + c] = __ldcg(h + c);
+            if (tid == 0) p.sink_frame[static_cast<int64_t>(b) * p.sinks + j] = j;
+        }
+        if (tid == 0) {
+            p.out_slot[b] = -1;
+            p.counter[b] = 0u;
+        }
+        return;
+    }
+    double hh = 0.0;
+    for (int c = tid; c < p.dim; c += kRefreshThreads) {
+        const double v = __ldcg(h + c);
+        hh += v * v;
+    }
+    hh = block_sum_fixed(hh, red);
+    double best = 0.0;
+    int best_j = -1;
+    for (int j = 0; j < p.sinks; ++j) {
+        double he = 0.0, ee = 0.0;
+        for (int c = tid; c < p.dim; c += kRefreshThreads) {
+            const double v = __ldcg(h + c);
+            const double e = emb[static_cast<int64_t>(j) * p.dim + c];
+            he += v * e;
+            ee += e * e;
+        }
+        he = block_sum_fixed(he, red);
+        ee = block_sum_fixed(ee, red);
+        const double cj = (hh == 0.0 || ee == 0.0) ? 1.0 : he / (sqrt(hh) * sqrt(ee));
+        if (best_j < 0 || cj < best) {   // strict: the lowest index wins ties
+            best = cj;
+            best_j = j;
+        }
+    }
+    const bool fire = best < p.tau;
+    __syncthreads();
+    if (fire) {
+        for (int c = tid; c < p.dim; c += kRefreshThreads) emb[static_cast<int64_t>(best_j) * p.dim + c] = __ldcg(h + c);
+    }
+    if (tid == 0) {
+        if (fire) p.sink_frame[static_cast<int64_t>(b) * p.sinks + best_j] = p.last_frame[b];
+        p.out_slot[b] = fire ? best_j : -1;
+        p.counter[b] = 0u;
+    }
+}
+
+__global__ void __launch_bounds__(256) refresh_copy_kernel(const __grid_constant__ RefreshParams p) {
+    const int b = blockIdx.y;
+    if (!p.active[b] || p.fill_count[b] > 0) return;
+    const int dst_slot = *reinterpret_cast<volatile const int32_t *>(p.out_slot + b);
+    if (dst_slot < 0) return;
+    const int src_slot = p.last_slot[b];
+    const int64_t vec_per_frame = p.frame_elems / 8;
+    const int64_t total = 2ll * p.layers * vec_per_frame;
+    for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < total;
+         g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t per_kv = p.layers * vec_per_frame;
+        uint16_t *base = g < per_kv ? p.k_cache : p.v_cache;
+        const int64_t r = g < per_kv ? g : g - per_kv;
+        const int64_t layer = r / vec_per_frame;
+        const int64_t vec = r - layer * vec_per_frame;
+        uint16_t *lb = base + layer * p.layer_stride_elems + static_cast<int64_t>(b) * p.slots * p.frame_elems;
+        const uint4 x = *reinterpret_cast<const uint4 *>(lb + static_cast<int64_t>(src_slot) * p.frame_elems + vec * 8);
+        *reinterpret_cast<uint4 *>(lb + static_cast<int64_t>(dst_slot) * p.frame_elems + vec * 8) = x;
+    }
+}
+
+cudaError_t launch_refresh(const RefreshParams &p, int sm_count, cudaStream_t s, int *launches) {
+    dim3 g1(static_cast<unsigned>((p.dim + kRefreshCols - 1) / kRefreshCols), static_cast<unsigned>(p.batch));
+    refresh_decide_kernel<<<g1, kRefreshThreads, 0, s>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    unsigned blocks = static_cast<unsigned>(sm_count) * 2u / static_cast<unsigned>(p.batch);
+    if (blocks < 4) blocks = 4;
+    dim3 g2(blocks, static_cast<unsigned>(p.batch));
+    refresh_copy_kernel<<<g2, 256, 0, s>>>(p);
+    *launches = 2;
+    return cudaGetLastError();
+}
+
+}  // namespace sdv2

@@ -1,0 +1,127 @@
+// Internal declarations shared by the host library (host.cpp) and the
+// kernel translation units.  Nothing here is part of the public C ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda.h>           // CUtensorMap (type only; the driver is reached at run time)
+#include <cuda_runtime.h>
+
+namespace sdv2 {
+
+constexpr int kMaxBatch = 64;
+// fp64 (cos, sin) entries of the temporal axis carried in one append launch.
+constexpr int kAppendTabEntries = 1536;   // 24 KB of kernel parameters
+constexpr int kAppendMaxFrames = 64;
+// fp32 (cos, sin) entries of the temporal axis carried in one attention launch.
+constexpr int kAttnTabEntries = 2048;     // 16 KB of kernel parameters
+constexpr int kMaxSplits = 8;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits give up after 2 s
+
+// Device status word bits (set with atomicOr, never cleared by kernels).
+enum : uint32_t {
+    kStatusTmaWait = 1u << 0,
+    kStatusMmaWait = 1u << 1,
+    kStatusSoftmaxWait = 1u << 2,
+    kStatusBadArgs = 1u << 3,
+};
+
+struct AppendParams {
+    const uint16_t *k_in;       // [B][T'N][H][d]
+    const uint16_t *v_in;
+    uint16_t *k_layer;          // [B][slots][N][H][d] of this layer
+    uint16_t *v_layer;
+    const double *rope_h;       // [frame_h][n_h][2] fp64 (cos, sin)
+    const double *rope_w;       // [frame_w][n_w][2]
+    int64_t frame_elems;        // N*H*d
+    int32_t chunk_tokens;       // T'N
+    int32_t heads, head_dim, frame_w, n_t, n_h, n_w, slots;
+    int32_t n_frames;           // frames handled by this launch
+    int32_t src_b[kAppendMaxFrames];     // stream of each frame
+    int32_t src_i[kAppendMaxFrames];     // index of the frame in the chunk
+    int32_t dst_slot[kAppendMaxFrames];  // ring slot it goes to
+    double tab_t[kAppendTabEntries][2];  // [frame][n_t] temporal cos, sin
+};
+
+struct AttnParams {
+    const uint16_t *q;          // [B][Lq][H][d]
+    uint16_t *out;              // [B][Lq][H][d]
+    float *part_o;              // [split][B][H][Lq_pad][d] (split > 1)
+    float *part_ml;             // [split][B][H][Lq_pad][2]  (row max in log2 units, row sum)
+    const float *rope_h;        // [frame_h][n_h][2] fp32
+    const float *rope_w;        // [frame_w][n_w][2]
+    uint32_t *status;
+    int32_t batch, heads, lq, lq_pad, tokens_per_frame, frame_w, chunk_frames;
+    int32_t n_t, n_h, n_w;
+    int32_t n_qpairs, n_split, b_offset;
+    float scale_log2;           // softmax_scale * log2(e)
+    int32_t lk[kMaxBatch];      // valid keys per stream of this launch (0 = skip)
+    float tab_t[kAttnTabEntries][2];     // [b][frame in chunk][n_t] temporal cos, sin
+};
+
+struct CombineParams {
+    const float *part_o;
+    const float *part_ml;
+    uint16_t *out;
+    int32_t batch, heads, lq, lq_pad, head_dim, n_split, b_offset;
+    int32_t lk[kMaxBatch];
+};
+
+struct RefreshParams {
+    const uint16_t *hidden;     // [B][Lq][D]
+    double *mean;               // scratch [B][D]
+    uint32_t *counter;          // scratch [B]
+    double *sink_embed;         // [B][S][D]
+    int64_t *sink_frame;        // [B][S]
+    int32_t *out_slot;          // [B] (caller's)
+    uint16_t *k_cache;          // all layers [L][B][slots][N][H][d]
+    uint16_t *v_cache;
+    int64_t layer_stride_elems; // elements between layers
+    int64_t frame_elems;        // N*H*d
+    int32_t batch, lq, dim, sinks, slots, layers;
+    double tau;
+    int32_t active[kMaxBatch];  // 1 if stream takes part in this call
+    int32_t fill_first[kMaxBatch];  // first sink slot this chunk fills itself (-1 none)
+    int32_t fill_count[kMaxBatch];  // number of sink slots it fills
+    int32_t last_slot[kMaxBatch];   // ring slot of the chunk's last frame
+    int64_t last_frame[kMaxBatch];  // frame index of the chunk's last frame
+};
+
+struct MotionParams {
+    const float *latents;       // [B][T'][CHW]
+    float *prev;                // [B][CHW] state: last frame seen
+    int32_t *has_prev;          // [B]
+    double *hist;               // [B][window] ring of motion values
+    int32_t *hist_len;          // [B]
+    int32_t *hist_pos;          // [B]
+    double *rate;               // [B]
+    double *partial;            // scratch [B][T'][n_blocks]
+    uint32_t *counter;          // scratch [B]
+    float *out_rate;            // [B]
+    float *out_d;               // [B][T'] or null
+    int64_t frame_elems;        // CHW
+    int32_t batch, chunk_frames, window, n_blocks;
+    double sigma, lambda, s_min, s_max;
+};
+
+// Launchers (defined next to their kernels).  Each returns the CUDA error
+// of the launch; the host layer turns it into an sdv2_status.
+cudaError_t launch_append(const AppendParams &p, int sm_count, cudaStream_t s);
+cudaError_t launch_attention(const AttnParams &p, const CUtensorMap &tk, const CUtensorMap &tv,
+                             int head_dim, cudaStream_t s);
+cudaError_t launch_combine(const CombineParams &p, cudaStream_t s);
+cudaError_t launch_refresh(const RefreshParams &p, int sm_count, cudaStream_t s, int *launches);
+cudaError_t launch_motion(const MotionParams &p, cudaStream_t s);
+
+// Attention tiling shared by host planning and kernels.
+constexpr int kBlockM = 128;      // query rows per tile (one TMEM lane each)
+constexpr int kBlockN = 128;      // keys per KV tile
+constexpr int kQTilesPerCta = 2;  // two query tiles ping-pong over the tensor core
+constexpr int kAttnThreads = 384;
+int attention_smem_bytes(int head_dim);
+
+constexpr int kMotionBlockElems = 2048;   // latent elements per motion block
+constexpr int kMotionThreads = 256;
+
+}  // namespace sdv2
