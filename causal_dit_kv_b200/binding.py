@@ -63,6 +63,7 @@ _SIGNATURES = [
     ("sdv2_motion_destroy", c_int32, [c_void_p]),
     ("sdv2_motion_noise_rate", c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     ("sdv2_motion_check", c_int32, [c_void_p]),
+    ("sdv2_motion_noise_rate_noalloc", c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     ("sdv2_slot_of_frame", c_int32, [c_int64, c_int32, c_int32]),
     ("sdv2_rope_phase", c_int64, [c_int64, c_int32]),
     ("sdv2_valid_slots", None, [c_int64, c_int32, c_int32, POINTER(c_int32), POINTER(c_int32)]),
@@ -220,6 +221,12 @@ def sdv2_motion_destroy(motion: int) -> None:
 def sdv2_motion_noise_rate(motion: int, latents, out_rate, out_d=None, stream=None) -> None:
     _check(lib().sdv2_motion_noise_rate(motion, _ptr(latents), _ptr(out_rate), _ptr(out_d), _stream(stream)),
            "sdv2_motion_noise_rate")
+
+
+def sdv2_motion_noise_rate_noalloc(motion: int, latents, out_rate, out_d=None, stream=None) -> None:
+    """Same as sdv2_motion_noise_rate with the library's fixed scratch (no caller scratch)."""
+    _check(lib().sdv2_motion_noise_rate_noalloc(motion, _ptr(latents), _ptr(out_rate), _ptr(out_d),
+                                                _stream(stream)), "sdv2_motion_noise_rate_noalloc")
 
 
 def sdv2_motion_check(motion: int) -> int:

@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsdv2.so")
-SOURCES = ["host.cpp", "append.cu", "attention.cu", "refresh.cu", "motion.cu"]
+SOURCES = ["host.cpp", "append.cu", "attention.cu", "refresh.cu", "motion.cu", "motion_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

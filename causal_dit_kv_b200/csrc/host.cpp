@@ -773,6 +773,46 @@ sdv2_status sdv2_motion_check(sdv2_motion *m) {
     return SDV2_OK;
 }
 
+sdv2_status sdv2_motion_noise_rate_noalloc(sdv2_motion *m, const float *latents, float *out_rate_dev,
+                                           float *out_d_dev, sdv2_stream stream) {
+    if (!m || !latents || !out_rate_dev) return fail(SDV2_E_ARG, "NULL argument");
+    if (!aligned16(latents) || (reinterpret_cast<uintptr_t>(out_rate_dev) & 3u) ||
+        (reinterpret_cast<uintptr_t>(out_d_dev) & 3u))
+        return fail(SDV2_E_ALIGN, "latents must be 16-byte aligned, outputs 4-byte aligned");
+    const int64_t partials = static_cast<int64_t>(m->cfg.batch) * m->cfg.chunk_frames * m->n_blocks;
+    if (partials > motion_noalloc_max_partials())
+        return fail(SDV2_E_SHAPE,
+                    "batch * chunk_frames * ceil(C*H*W / %d) = %lld exceeds the %d partial sums of the "
+                    "library's fixed scratch; use sdv2_motion_noise_rate",
+                    kMotionBlockElems, static_cast<long long>(partials), motion_noalloc_max_partials());
+    sdv2_status st = check_device(m->device);
+    if (st != SDV2_OK) return st;
+    MotionParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.latents = latents;
+    p.prev = reinterpret_cast<float *>(m->base + m->off_prev);
+    p.has_prev = reinterpret_cast<int32_t *>(m->base + m->off_has_prev);
+    p.hist = reinterpret_cast<double *>(m->base + m->off_hist);
+    p.hist_len = reinterpret_cast<int32_t *>(m->base + m->off_hist_len);
+    p.hist_pos = reinterpret_cast<int32_t *>(m->base + m->off_hist_pos);
+    p.rate = reinterpret_cast<double *>(m->base + m->off_rate);
+    p.out_rate = out_rate_dev;
+    p.out_d = out_d_dev;
+    p.frame_elems = m->frame_elems;
+    p.batch = m->cfg.batch;
+    p.chunk_frames = m->cfg.chunk_frames;
+    p.window = m->cfg.window;
+    p.n_blocks = m->n_blocks;
+    p.sigma = m->cfg.sigma;
+    p.lambda = m->cfg.lambda;
+    p.s_min = m->cfg.s_min;
+    p.s_max = m->cfg.s_max;
+    cudaError_t e = launch_motion_noalloc(p, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "motion (no-alloc) launch");
+    g_launches.fetch_add(1);
+    return SDV2_OK;
+}
+
 // ------------------------------------------------------------------ host-only helpers
 
 int32_t sdv2_slot_of_frame(int64_t f, int32_t sink_frames, int32_t window_frames) {

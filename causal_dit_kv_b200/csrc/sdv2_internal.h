@@ -113,6 +113,9 @@ cudaError_t launch_attention(const AttnParams &p, const CUtensorMap &tk, const C
 cudaError_t launch_combine(const CombineParams &p, cudaStream_t s);
 cudaError_t launch_refresh(const RefreshParams &p, int sm_count, cudaStream_t s, int *launches);
 cudaError_t launch_motion(const MotionParams &p, cudaStream_t s);
+// Same kernel with partial/counter in the library's static device array.
+cudaError_t launch_motion_noalloc(MotionParams p, cudaStream_t s);
+int motion_noalloc_max_partials();
 
 // Attention tiling shared by host planning and kernels.
 constexpr int kBlockM = 128;      // query rows per tile (one TMEM lane each)

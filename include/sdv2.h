@@ -235,6 +235,24 @@ sdv2_status sdv2_motion_destroy(sdv2_motion *motion);
 sdv2_status sdv2_motion_noise_rate(sdv2_motion *motion, const float *latents, float *out_rate_dev,
                                    float *out_d_dev, sdv2_stream stream);
 
+/* Allocation-free variant of sdv2_motion_noise_rate.  The pages have no
+ * counterpart: this is a deployment convenience of this library.
+ * Same arguments, state and results as sdv2_motion_noise_rate, but the
+ * per-call scratch (one fp64 partial sum per 2048-element block of each
+ * frame, one ticket counter per stream) lives in a fixed 128 KB device array
+ * that the library holds on every GPU that loads it, until the process exits.
+ * For callers that cannot call cudaMalloc where they run the step: a host
+ * framework that owns all device memory and hands out only fixed buffers, or
+ * a real-time loop that must not allocate.  The array's device address is
+ * looked up the first time the call runs on a device, so make that first
+ * call before any stream capture.  Every call shares the one array: calls
+ * whose work overlaps on the GPU (other streams, other threads) race and must
+ * be serialised by the caller.  Limit: batch * chunk_frames *
+ * ceil(C*H*W / 2048) <= 16384, else SDV2_E_SHAPE.  Allocates nothing.
+ * Errors: SDV2_E_ARG, SDV2_E_SHAPE, SDV2_E_ALIGN, SDV2_E_CUDA. */
+sdv2_status sdv2_motion_noise_rate_noalloc(sdv2_motion *motion, const float *latents, float *out_rate_dev,
+                                           float *out_d_dev, sdv2_stream stream);
+
 /* Synchronise and read the motion status word (as sdv2_cache_check). */
 sdv2_status sdv2_motion_check(sdv2_motion *motion);
 
