@@ -283,7 +283,7 @@ def run_ours(args, w, name):
                    "l2": "inputs larger than L2 (per-step caches %.0f MB over %d layers)" % (
                        2 * cache.layout.layer_stride * L / 1e6, L),
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"kernel": "sdv2_chunk_attention (attention + split-KV combine)", "bound": "tensor",
+        "roofline": {"kernel": "chunk_attention_kernel (one launch per layer, split merge in-kernel)", "bound": "tensor",
                      "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": None,
                      "peak_source": f"{peak_src} bf16_tflops_sustained",

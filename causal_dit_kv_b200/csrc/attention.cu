@@ -18,15 +18,24 @@
 //   warp 1      MMA issuer (one thread): S_t = Q_t K^T and O_t += P_t V
 //   warps 4..7  softmax + epilogue of query tile 0 (thread i owns row i)
 //   warps 8..11 softmax + epilogue of query tile 1
+// The producer/MMA warpgroup gives registers to the two softmax warpgroups
+// (setmaxnreg 80 / 208).
 // TMEM (512 columns): S_0 | S_1 | O_0 | O_1, 128 columns each; P_t (bf16)
 // is written over the first 64 columns of S_t and fed to the PV MMA from
 // TMEM.  The MMA order PV(0,j), QK(0,j+1), PV(1,j), QK(1,j+1) lets one tile's
 // softmax run while the tensor core works on the other tile.
 // Online softmax in base 2 with lazy rescaling: the running max only moves
 // (and O is rescaled in TMEM) when a tile's max exceeds it by more than 8,
-// so P stays <= 256.
-// Q is rotated on load (fp32 RoPE, rounded to bf16) by the softmax threads
-// and written into the 128-byte-swizzled K-major layout the MMA reads.
+// so P stays <= 256.  Half of the exponentials run as a polynomial on
+// the FMA pipe (exp2_poly2) to relieve the MUFU pipe; the exponent
+// arguments and row sums use packed f32x2 arithmetic.
+// Q: rope_q_kernel rotates the chunk's queries once per call (fp32 RoPE,
+// rounded to bf16) into a scratch buffer; the producer warp TMA-loads the
+// rotated tiles straight into the 128-byte-swizzled K-major layout the MMA
+// reads.
+// KV splits: each split CTA writes an unnormalised partial (O, row max, row
+// sum); the last CTA of a tile to finish (atomic ticket) merges them and
+// writes the output, so no second launch is needed.
 // Every wait is bounded (2 s), after which the CTA records an error in the
 // device status word and unwinds; TMEM is always released.
 #include <cmath>
@@ -56,7 +65,7 @@ struct AttnLayout {
     static constexpr int kOFull = kPFull + 2;
     static constexpr int kDrain = kOFull + 2;
     static constexpr int kNumBars = kDrain + 1;
-    static constexpr int kMisc = kBar + kNumBars * 8;
+    static constexpr int kMisc = kBar + kNumBars * 8;   // tmem base, abort flag, merge flag
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;      // room to align the base to 1024 bytes
 };
@@ -67,6 +76,7 @@ int attention_smem_bytes(int head_dim) {
 
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale only when the max grows by > 2^8
+constexpr uint32_t kSoftmaxBarrier = 1;     // named barrier of the softmax warpgroups
 
 // fp32 (cos, sin) of rotation pair j for a query token.
 __device__ __forceinline__ float2 q_cos_sin(const AttnParams &p, int bl, int fi, int row, int col, int j) {
@@ -90,16 +100,88 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return __all_sync(0xffffffffu, ok);
 }
 
+// RoPE of the chunk's queries: q_rot = rotate(q) at (phase(frame), row, col),
+// fp32 arithmetic, bf16 result.  One thread per 16-byte vector (4 pairs).
+__global__ void __launch_bounds__(256) rope_q_kernel(const __grid_constant__ AttnParams p, int head_dim) {
+    const uint32_t vec_per_token = static_cast<uint32_t>(p.heads * head_dim / 8);
+    const uint32_t vec_per_stream = static_cast<uint32_t>(p.lq) * vec_per_token;
+    int nb = 0;
+    for (int i = 0; i < kMaxBatch; ++i)
+        if (p.lk[i] > 0) nb = i + 1;
+    const uint32_t total = static_cast<uint32_t>(nb) * vec_per_stream;
+    for (uint32_t g = blockIdx.x * blockDim.x + threadIdx.x; g < total; g += gridDim.x * blockDim.x) {
+        const int bl = static_cast<int>(g / vec_per_stream);
+        if (p.lk[bl] <= 0) continue;
+        const uint32_t r = g - static_cast<uint32_t>(bl) * vec_per_stream;
+        const int token = static_cast<int>(r / vec_per_token);
+        const uint32_t cv = r - static_cast<uint32_t>(token) * vec_per_token;   // vector within the token
+        const int j0 = static_cast<int>((cv * 8) % static_cast<uint32_t>(head_dim)) >> 1;
+        const int fi = token / p.tokens_per_frame;
+        const int n = token - fi * p.tokens_per_frame;
+        const int prow = n / p.frame_w;
+        const int pcol = n - prow * p.frame_w;
+        const int64_t off = (static_cast<int64_t>(p.b_offset + bl) * p.lq + token) * p.heads * head_dim + cv * 8;
+        const uint4 x = *reinterpret_cast<const uint4 *>(p.q + off);
+        const uint32_t in[4] = {x.x, x.y, x.z, x.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float2 cs = q_cos_sin(p, bl, fi, prow, pcol, j0 + q);
+            const float x0 = bf16_lo(in[q]), x1 = bf16_hi(in[q]);
+            o[q] = pack_bf16x2(x0 * cs.x - x1 * cs.y, x0 * cs.y + x1 * cs.x);
+        }
+        *reinterpret_cast<uint4 *>(p.q_rot + off) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+// P = 2^(s*scale_log2 - m) for one row of 128 scores (raw fp32 bits in sr),
+// packed to bf16 into TMEM columns [0, 64) of the row's S region; returns
+// the row sum (fp32).  Columns 16..31 of every 32 use the FMA-pipe
+// polynomial, the rest the MUFU ex2.  Pairs of columns share one f32x2 FMA
+// for the exponent argument and one f32x2 add for the sum.
+__device__ __forceinline__ float softmax_exp_store(const uint32_t (&sr)[kBlockN / 32][32], float scale_log2,
+                                                   float neg_m, uint32_t s_tmem) {
+    const uint64_t scale2 = f2_pack(scale_log2, scale_log2);
+    const uint64_t negm2 = f2_pack(neg_m, neg_m);
+    uint64_t acc[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i] = 0ull;
+#pragma unroll
+    for (int cb = 0; cb < kBlockN / 32; ++cb) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const uint64_t x = f2_fma(f2_pack(__uint_as_float(sr[cb][2 * i]), __uint_as_float(sr[cb][2 * i + 1])),
+                                      scale2, negm2);
+            float x0, x1, p0, p1;
+            f2_unpack(x, x0, x1);
+            if (i >= 8) {
+                exp2_poly2(x0, x1, p0, p1);
+            } else {
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+            }
+            acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
+            pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(s_tmem + cb * 16, pk);
+    }
+    float a0, a1;
+    f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
+    return a0 + a1;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
-    chunk_attention_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmap_k,
-                           const __grid_constant__ CUtensorMap tmap_v) {
+    chunk_attention_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
+                           const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v) {
     using L = AttnLayout<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBar);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + L::kMisc + 4);
+    volatile uint32_t *merge_flag = reinterpret_cast<volatile uint32_t *>(smem + L::kMisc + 8);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -120,7 +202,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int n_qt = (q_row0 + kBlockM < p.lq) ? 2 : 1;
 
     if (threadIdx.x == 0) {
-        mbar_init(&bars[L::kQFull], kBlockM * n_qt);
+        mbar_init(&bars[L::kQFull], 1);
         for (int s = 0; s < L::kStages; ++s) {
             mbar_init(&bars[L::kKFull + s], 1);
             mbar_init(&bars[L::kKEmpty + s], 1);
@@ -134,9 +216,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         mbar_init(&bars[L::kDrain], 1);
         *abort_flag = 0u;
+        *merge_flag = 0u;
         fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmap_q);
         tma_prefetch_desc(&tmap_k);
         tma_prefetch_desc(&tmap_v);
     }
@@ -149,10 +233,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
+    if (warp < 4) {
+      regs_dec<80>();
+      if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0 && n_local > 0) {
-            int issued[L::kStages] = {0, 0};
+            // rotated query tiles of this CTA (rows past lq are filled with zeros)
+            mbar_arrive_expect_tx(&bars[L::kQFull], n_qt * L::kQTile);
+            for (int t = 0; t < n_qt; ++t)
+#pragma unroll
+                for (int kb = 0; kb < D / 64; ++kb)
+                    tma_load_4d(smem + L::kQ + t * L::kQTile + kb * L::kSub, &tmap_q, &bars[L::kQFull], kb * 64, h,
+                                q_row0 + t * kBlockM, bg);
+            int issued = 0;   // tiles whose loads were issued
             for (int it = 0; it < n_local; ++it) {
                 const int st = it % L::kStages;
                 const uint32_t ph = (it / L::kStages) & 1;
@@ -164,7 +257,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     tma_load_4d(smem + L::kK + st * L::kKVTile + kb * L::kSub, &tmap_k, &bars[L::kKFull + st], kb * 64,
                                 h, kv0, bg);
                 if (!mbar_wait(&bars[L::kVEmpty + st], ph ^ 1u, abort_flag, p.status, kStatusTmaWait)) {
-                    issued[st] = it + 1;
+                    issued = it + 1;
                     break;
                 }
                 mbar_arrive_expect_tx(&bars[L::kVFull + st], L::kKVTile);
@@ -172,13 +265,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 for (int kb = 0; kb < D / 64; ++kb)
                     tma_load_4d(smem + L::kV + st * L::kKVTile + kb * L::kSub, &tmap_v, &bars[L::kVFull + st], kb * 64,
                                 h, kv0, bg);
-                issued[st] = it + 1;
+                issued = it + 1;
             }
             if (*abort_flag) {
                 // Let every copy already in flight land before the CTA leaves.
-                for (int st = 0; st < L::kStages; ++st) {
-                    if (issued[st] == 0) continue;
-                    const uint32_t ph = ((issued[st] - 1) / L::kStages) & 1;
+                for (int it = issued - L::kStages; it < issued; ++it) {
+                    if (it < 0) continue;
+                    const int st = it % L::kStages;
+                    const uint32_t ph = (it / L::kStages) & 1;
                     const uint64_t t0 = global_timer_ns();
                     while (!(mbar_try_wait(&bars[L::kKFull + st], ph) && mbar_try_wait(&bars[L::kVFull + st], ph))) {
                         if (global_timer_ns() - t0 > kWaitLimitNs) break;
@@ -266,7 +360,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
             }
         }
-    } else if (warp >= 4) {
+      }
+    } else {
+        regs_inc<208>();
         // ------------------------------------------------ softmax / epilogue
         const int t = (warp - 4) >> 2;               // query tile of this warpgroup
         const int row = ((warp & 3) << 5) + lane;    // TMEM lane == query row in the tile
@@ -274,37 +370,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (t < n_qt) {
             const int token = q_row0 + t * kBlockM + row;
             const bool valid = token < p.lq;
-            // ---- Q load + RoPE (fp32) into the swizzled K-major tile
-            uint8_t *qtile = smem + L::kQ + t * L::kQTile;
-            if (n_local > 0) {
-                const int fi = valid ? token / p.tokens_per_frame : 0;
-                const int n = valid ? token - fi * p.tokens_per_frame : 0;
-                const int prow = n / p.frame_w;
-                const int pcol = n - prow * p.frame_w;
-                const uint16_t *qrow =
-                    p.q + ((static_cast<int64_t>(bg) * p.lq + (valid ? token : 0)) * p.heads + h) * D;
-#pragma unroll 4
-                for (int c = 0; c < D / 8; ++c) {
-                    uint4 w = make_uint4(0, 0, 0, 0);
-                    if (valid) {
-                        const uint4 x = *reinterpret_cast<const uint4 *>(qrow + c * 8);
-                        uint32_t in[4] = {x.x, x.y, x.z, x.w};
-                        uint32_t o[4];
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const float2 cs = q_cos_sin(p, bl, fi, prow, pcol, c * 4 + q);
-                            const float x0 = bf16_lo(in[q]), x1 = bf16_hi(in[q]);
-                            o[q] = pack_bf16x2(x0 * cs.x - x1 * cs.y, x0 * cs.y + x1 * cs.x);
-                        }
-                        w = make_uint4(o[0], o[1], o[2], o[3]);
-                    }
-                    const int kb = c >> 3, c16 = c & 7;
-                    *reinterpret_cast<uint4 *>(qtile + kb * L::kSub + row * 128 + ((c16 ^ (row & 7)) << 4)) = w;
-                }
-                fence_proxy_async_smem();
-                mbar_arrive(&bars[L::kQFull]);
-            }
-
             float m_run = -INFINITY;   // running max of scale*log2(e)*s
             float l_run = 0.0f;
             bool ok = true;
@@ -322,20 +387,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 tmem_wait_ld_bind(sr[0]);
 #pragma unroll
                 for (int cb = 1; cb < kBlockN / 32; ++cb) reg_bind(sr[cb]);
-                float s[kBlockN];
-#pragma unroll
-                for (int cb = 0; cb < kBlockN / 32; ++cb)
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) s[cb * 32 + i] = __uint_as_float(sr[cb][i]);
                 const int valid_cols = lk - (kv_begin + it) * kBlockN;
                 if (valid_cols < kBlockN) {
 #pragma unroll
-                    for (int i = 0; i < kBlockN; ++i)
-                        if (i >= valid_cols) s[i] = -INFINITY;
-                }
-                float mx = s[0];
+                    for (int cb = 0; cb < kBlockN / 32; ++cb)
 #pragma unroll
-                for (int i = 1; i < kBlockN; ++i) mx = fmaxf(mx, s[i]);
+                        for (int i = 0; i < 32; ++i)
+                            if (cb * 32 + i >= valid_cols) sr[cb][i] = 0xff800000u;   // -inf
+                }
+                // row max: four 3-input max chains, then combine
+                float m4[4];
+#pragma unroll
+                for (int cb = 0; cb < 4; ++cb) {
+                    float m = __uint_as_float(sr[cb][0]);
+#pragma unroll
+                    for (int i = 1; i < 31; i += 2)
+                        m = fmax3(m, __uint_as_float(sr[cb][i]), __uint_as_float(sr[cb][i + 1]));
+                    m4[cb] = fmaxf(m, __uint_as_float(sr[cb][31]));
+                }
+                const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
                 const float m_tile = mx * p.scale_log2;
                 bool rescale = false;
                 float alpha = 1.0f;
@@ -359,20 +429,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     }
                     tmem_wait_st();
                 }
-                const float neg_m = -m_run;
-                float sum = 0.0f;
-#pragma unroll
-                for (int cb = 0; cb < 2; ++cb) {
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float p0 = ex2_approx(fmaf(s[cb * 64 + 2 * i], p.scale_log2, neg_m));
-                        const float p1 = ex2_approx(fmaf(s[cb * 64 + 2 * i + 1], p.scale_log2, neg_m));
-                        sum += p0 + p1;
-                        pk[i] = pack_bf16x2(p0, p1);
-                    }
-                    tmem_st32(s_tmem + cb * 32, pk);
-                }
+                const float sum = softmax_exp_store(sr, p.scale_log2, -m_run, s_tmem);
                 l_run += sum;
                 tmem_wait_st();
                 tc_fence_before();
@@ -381,6 +438,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
             // ---- epilogue
             if (ok && n_local > 0) ok = warp_wait(&bars[L::kOFull + t], 0, abort_flag, p.status, kStatusSoftmaxWait);
+            const int prow_local = q_row0 + t * kBlockM + row;     // row index within the padded query range
             if (ok) {
                 tc_fence_after();
                 if (p.n_split == 1) {
@@ -404,10 +462,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         }
                     }
                 } else {
-                    const int64_t prow_idx =
-                        ((static_cast<int64_t>(split) * p.batch + bg) * p.heads + h) * p.lq_pad + q_row0 + t * kBlockM + row;
+                    // Partial of this split, column-major in float4 units so that a warp's
+                    // 32 rows write (and the merge reads) 512 contiguous bytes per access:
+                    // part_o[((split*B + b)*H + h)][D/4][lq_pad] float4, part_ml[...][lq_pad] float2.
+                    const int64_t head_idx = (static_cast<int64_t>(split) * p.batch + bg) * p.heads + h;
+                    float4 *po = reinterpret_cast<float4 *>(p.part_o) + head_idx * (D / 4) * p.lq_pad + prow_local;
                     if (n_local > 0) {
-                        float *po = p.part_o + prow_idx * D;
 #pragma unroll
                         for (int cb = 0; cb < D / 32; ++cb) {
                             uint32_t r[32];
@@ -416,14 +476,85 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                             if (valid) {
 #pragma unroll
                                 for (int v = 0; v < 8; ++v)
-                                    *reinterpret_cast<uint4 *>(po + cb * 32 + v * 4) =
-                                        make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+                                    po[static_cast<int64_t>(cb * 8 + v) * p.lq_pad] =
+                                        make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                                    __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
                             }
                         }
                     }
-                    if (valid) {
-                        p.part_ml[prow_idx * 2 + 0] = n_local > 0 ? m_run : -INFINITY;
-                        p.part_ml[prow_idx * 2 + 1] = l_run;
+                    if (valid)
+                        reinterpret_cast<float2 *>(p.part_ml)[head_idx * p.lq_pad + prow_local] =
+                            make_float2(n_local > 0 ? m_run : -INFINITY, l_run);
+                }
+            }
+            // ---- split merge: the last split CTA of this tile combines the partials
+            if (p.n_split > 1) {
+                const uint32_t nthreads = kBlockM * static_cast<uint32_t>(n_qt);
+                __threadfence();
+                named_bar_sync(kSoftmaxBarrier, nthreads);
+                if (threadIdx.x == 128) {
+                    uint32_t *ticket = p.tickets + (static_cast<int64_t>(bg) * p.heads + h) * p.n_qpairs + qpair;
+                    const uint32_t prev = atomicAdd(ticket, 1u);
+                    const bool last = prev == static_cast<uint32_t>(p.n_split - 1);
+                    if (last) *ticket = 0u;                    // every split has arrived: re-arm for the next call
+                    *merge_flag = (last && !*abort_flag) ? 1u : 0u;
+                }
+                named_bar_sync(kSoftmaxBarrier, nthreads);
+                if (*merge_flag && valid) {
+                    __threadfence();
+                    const int64_t head0 = static_cast<int64_t>(bg) * p.heads + h;
+                    const int64_t stride_s = static_cast<int64_t>(p.batch) * p.heads;
+                    const float2 *mlp = reinterpret_cast<const float2 *>(p.part_ml);
+                    float2 ml[kMaxSplits];
+                    float m = -INFINITY;
+#pragma unroll
+                    for (int s = 0; s < kMaxSplits; ++s) {
+                        ml[s] = make_float2(-INFINITY, 0.0f);
+                        if (s < p.n_split) ml[s] = __ldcg(mlp + (s * stride_s + head0) * p.lq_pad + prow_local);
+                        m = fmaxf(m, ml[s].x);
+                    }
+                    float wgt[kMaxSplits];
+                    float l = 0.0f;
+#pragma unroll
+                    for (int s = 0; s < kMaxSplits; ++s) {
+                        wgt[s] = ml[s].x == -INFINITY ? 0.0f : exp2f(ml[s].x - m);
+                        l += wgt[s] * ml[s].y;
+                    }
+                    const float inv = 1.0f / l;
+                    uint16_t *orow = p.out + ((static_cast<int64_t>(bg) * p.lq + token) * p.heads + h) * D;
+                    // two passes of D/2 columns; each split's loads of a pass are issued together
+#pragma unroll 1
+                    for (int half = 0; half < 2; ++half) {
+                        float4 acc[D / 8];
+#pragma unroll
+                        for (int i = 0; i < D / 8; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+                        for (int s = 0; s < p.n_split; ++s) {
+                            if (wgt[s] == 0.0f) continue;
+                            const float4 *po = reinterpret_cast<const float4 *>(p.part_o) +
+                                               (s * stride_s + head0) * (D / 4) * p.lq_pad + prow_local;
+                            float4 u[D / 8];
+#pragma unroll
+                            for (int i = 0; i < D / 8; ++i)
+                                u[i] = __ldcg(po + static_cast<int64_t>(half * (D / 8) + i) * p.lq_pad);
+                            const float w = wgt[s];
+#pragma unroll
+                            for (int i = 0; i < D / 8; ++i) {
+                                acc[i].x += w * u[i].x;
+                                acc[i].y += w * u[i].y;
+                                acc[i].z += w * u[i].z;
+                                acc[i].w += w * u[i].w;
+                            }
+                        }
+#pragma unroll
+                        for (int i = 0; i < D / 8; i += 2) {
+                            uint4 w;
+                            w.x = pack_bf16x2(acc[i].x * inv, acc[i].y * inv);
+                            w.y = pack_bf16x2(acc[i].z * inv, acc[i].w * inv);
+                            w.z = pack_bf16x2(acc[i + 1].x * inv, acc[i + 1].y * inv);
+                            w.w = pack_bf16x2(acc[i + 1].z * inv, acc[i + 1].w * inv);
+                            *reinterpret_cast<uint4 *>(orow + half * (D / 2) + i * 4) = w;
+                        }
                     }
                 }
             }
@@ -439,46 +570,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
 }
 
-// One warp per (stream, head, query row): merges the split partials.
 template <int D>
-__global__ void __launch_bounds__(256) attention_combine_kernel(const __grid_constant__ CombineParams p) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int row = blockIdx.x * 8 + warp;
-    const int h = blockIdx.y;
-    const int bl = blockIdx.z;
-    const int bg = p.b_offset + bl;
-    if (p.lk[bl] <= 0 || row >= p.lq) return;
-    constexpr int kPer = D / 32;   // columns per lane
-    float m = -INFINITY;
-    for (int s = 0; s < p.n_split; ++s) {
-        const int64_t idx = ((static_cast<int64_t>(s) * p.batch + bg) * p.heads + h) * p.lq_pad + row;
-        m = fmaxf(m, p.part_ml[idx * 2]);
-    }
-    float acc[kPer];
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) acc[i] = 0.0f;
-    float l = 0.0f;
-    for (int s = 0; s < p.n_split; ++s) {
-        const int64_t idx = ((static_cast<int64_t>(s) * p.batch + bg) * p.heads + h) * p.lq_pad + row;
-        const float ms = p.part_ml[idx * 2];
-        if (ms == -INFINITY) continue;            // empty split: no keys, no partial
-        const float w = exp2f(ms - m);
-        l += w * p.part_ml[idx * 2 + 1];
-        const float *po = p.part_o + idx * D + lane * kPer;
-#pragma unroll
-        for (int i = 0; i < kPer; ++i) acc[i] += w * po[i];
-    }
-    const float inv = 1.0f / l;
-    uint16_t *orow = p.out + ((static_cast<int64_t>(bg) * p.lq + row) * p.heads + h) * D + lane * kPer;
-#pragma unroll
-    for (int i = 0; i < kPer; i += 2) {
-        *reinterpret_cast<uint32_t *>(orow + i) = pack_bf16x2(acc[i] * inv, acc[i + 1] * inv);
-    }
-}
-
-template <int D>
-static cudaError_t launch_attention_d(const AttnParams &p, const CUtensorMap &tk, const CUtensorMap &tv,
-                                      cudaStream_t s) {
+static cudaError_t launch_attention_d(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
+                                      const CUtensorMap &tv, cudaStream_t s) {
     static bool configured = false;
     const int smem = AttnLayout<D>::kAlloc;
     if (!configured) {
@@ -491,26 +585,26 @@ static cudaError_t launch_attention_d(const AttnParams &p, const CUtensorMap &tk
         if (p.lk[i] > 0) nb = i + 1;
     if (nb == 0) return cudaSuccess;
     dim3 grid(static_cast<unsigned>(p.n_qpairs * p.n_split), static_cast<unsigned>(p.heads), static_cast<unsigned>(nb));
-    chunk_attention_kernel<D><<<grid, kAttnThreads, smem, s>>>(p, tk, tv);
+    chunk_attention_kernel<D><<<grid, kAttnThreads, smem, s>>>(p, tq, tk, tv);
     return cudaGetLastError();
 }
 
-cudaError_t launch_attention(const AttnParams &p, const CUtensorMap &tk, const CUtensorMap &tv, int head_dim,
-                             cudaStream_t s) {
-    if (head_dim == 64) return launch_attention_d<64>(p, tk, tv, s);
-    return launch_attention_d<128>(p, tk, tv, s);
+cudaError_t launch_attention(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
+                             const CUtensorMap &tv, int head_dim, cudaStream_t s) {
+    if (head_dim == 64) return launch_attention_d<64>(p, tq, tk, tv, s);
+    return launch_attention_d<128>(p, tq, tk, tv, s);
 }
 
-cudaError_t launch_combine(const CombineParams &p, cudaStream_t s) {
+cudaError_t launch_rope_q(const AttnParams &p, int sm_count, cudaStream_t s) {
     int nb = 0;
     for (int i = 0; i < kMaxBatch; ++i)
         if (p.lk[i] > 0) nb = i + 1;
-    if (nb == 0) return cudaSuccess;
-    dim3 grid(static_cast<unsigned>((p.lq + 7) / 8), static_cast<unsigned>(p.heads), static_cast<unsigned>(nb));
-    if (p.head_dim == 64)
-        attention_combine_kernel<64><<<grid, 256, 0, s>>>(p);
-    else
-        attention_combine_kernel<128><<<grid, 256, 0, s>>>(p);
+    const int head_dim = p.heads > 0 ? static_cast<int>(p.n_t + p.n_h + p.n_w) * 2 : 0;
+    const uint64_t total = static_cast<uint64_t>(nb) * p.lq * p.heads * head_dim / 8;
+    if (total == 0) return cudaSuccess;
+    uint64_t blocks = (total + 255) / 256;
+    if (blocks > static_cast<uint64_t>(sm_count) * 8) blocks = static_cast<uint64_t>(sm_count) * 8;
+    rope_q_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(p, head_dim);
     return cudaGetLastError();
 }
 

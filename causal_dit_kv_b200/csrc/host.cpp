@@ -77,7 +77,7 @@ struct Geometry {
     // region offsets
     uint64_t rope_h64, rope_w64, rope_h32, rope_w32;
     uint64_t sink_embed, sink_frame, status;
-    uint64_t scratch, refresh_mean, refresh_counter, part_ml, part_o, scratch_end;
+    uint64_t scratch, refresh_mean, refresh_counter, tickets, tickets_bytes, q_rot, part_ml, part_o, scratch_end;
     uint64_t k, v, layer_stride, total;
 };
 
@@ -156,6 +156,11 @@ Geometry geometry(const sdv2_cache_config &c) {
     off = align_up(off + 8ull * c.batch * (c.embed_dim > 0 ? c.embed_dim : 1), 256);
     g.refresh_counter = off;
     off = align_up(off + 4ull * c.batch, 256);
+    g.tickets = off;
+    g.tickets_bytes = 4ull * c.batch * c.heads * g.n_qpairs;
+    off = align_up(off + g.tickets_bytes, 256);
+    g.q_rot = off;
+    off = align_up(off + 2ull * c.batch * g.lq * c.heads * c.head_dim, 1024);
     g.part_ml = off;
     off = align_up(off + 8ull * g.part_rows, 256);
     g.part_o = off;
@@ -224,6 +229,7 @@ struct sdv2_cache {
     int sm_count;
     std::vector<int64_t> next_frame;  // [B][L]
     std::vector<CUtensorMap> tk, tv;  // [L]
+    CUtensorMap tq;                   // rotated queries in scratch: (d, H, Lq, B)
 };
 
 struct sdv2_motion {
@@ -378,6 +384,21 @@ sdv2_status sdv2_cache_create(const sdv2_cache_config *cfg, void *dev_buf, size_
             }
         }
     }
+    {
+        const cuuint64_t qdims[4] = {static_cast<cuuint64_t>(n.head_dim), static_cast<cuuint64_t>(n.heads),
+                                     static_cast<cuuint64_t>(g.lq), static_cast<cuuint64_t>(n.batch)};
+        const cuuint64_t qstrides[3] = {static_cast<cuuint64_t>(n.head_dim) * 2,
+                                        static_cast<cuuint64_t>(n.heads) * n.head_dim * 2,
+                                        static_cast<cuuint64_t>(g.lq) * n.heads * n.head_dim * 2};
+        const cuuint32_t qbox[4] = {64, 1, static_cast<cuuint32_t>(kBlockM), 1};
+        CUresult r = encode(&c->tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, c->base + g.q_rot, qdims, qstrides, qbox,
+                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) {
+            delete c;
+            return fail(SDV2_E_CUDA, "cuTensorMapEncodeTiled (queries) failed (%d)", static_cast<int>(r));
+        }
+    }
     c->next_frame.assign(static_cast<size_t>(n.batch) * n.layers, 0);
     *out = c;
     return SDV2_OK;
@@ -477,9 +498,11 @@ sdv2_status sdv2_chunk_attention(sdv2_cache *c, int32_t layer, const void *q, vo
     AttnParams p;
     std::memset(&p, 0, sizeof(p));
     p.q = static_cast<const uint16_t *>(q);
+    p.q_rot = reinterpret_cast<uint16_t *>(c->base + g.q_rot);
     p.out = static_cast<uint16_t *>(out);
     p.part_o = reinterpret_cast<float *>(c->base + g.part_o);
     p.part_ml = reinterpret_cast<float *>(c->base + g.part_ml);
+    p.tickets = reinterpret_cast<uint32_t *>(c->base + g.tickets);
     p.rope_h = reinterpret_cast<const float *>(c->base + g.rope_h32);
     p.rope_w = reinterpret_cast<const float *>(c->base + g.rope_w32);
     p.status = reinterpret_cast<uint32_t *>(c->base + g.status);
@@ -517,27 +540,11 @@ sdv2_status sdv2_chunk_attention(sdv2_cache *c, int32_t layer, const void *q, vo
             }
         }
         if (!any) continue;
-        cudaError_t e = launch_attention(p, c->tk[layer], c->tv[layer], n.head_dim, s);
+        cudaError_t e = launch_rope_q(p, c->sm_count, s);
+        if (e != cudaSuccess) return cuda_fail(e, "rope_q launch");
+        e = launch_attention(p, c->tq, c->tk[layer], c->tv[layer], n.head_dim, s);
         if (e != cudaSuccess) return cuda_fail(e, "chunk_attention launch");
-        g_launches.fetch_add(1);
-        if (n_split > 1) {
-            CombineParams cp;
-            std::memset(&cp, 0, sizeof(cp));
-            cp.part_o = p.part_o;
-            cp.part_ml = p.part_ml;
-            cp.out = p.out;
-            cp.batch = n.batch;
-            cp.heads = n.heads;
-            cp.lq = p.lq;
-            cp.lq_pad = p.lq_pad;
-            cp.head_dim = n.head_dim;
-            cp.n_split = n_split;
-            cp.b_offset = b0;
-            for (int bl = 0; bl < kMaxBatch; ++bl) cp.lk[bl] = p.lk[bl];
-            e = launch_combine(cp, s);
-            if (e != cudaSuccess) return cuda_fail(e, "attention combine launch");
-            g_launches.fetch_add(1);
-        }
+        g_launches.fetch_add(2);
     }
     return SDV2_OK;
 }
@@ -639,8 +646,11 @@ sdv2_status sdv2_cache_check(sdv2_cache *c) {
     e = cudaMemcpy(&word, c->base + c->g.status, 4, cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(e, "cache_check");
     if (word != 0) {
-        const uint32_t zero = 0;
-        cudaMemcpy(c->base + c->g.status, &zero, 4, cudaMemcpyHostToDevice);
+        // A CTA that gave up may have left split tickets half counted: re-arm them.
+        cudaMemset(c->base + c->g.status, 0, 4);
+        cudaMemset(c->base + c->g.tickets, 0, c->g.tickets_bytes);
+        cudaMemset(c->base + c->g.refresh_counter, 0, 4ull * c->cfg.batch);
+        cudaDeviceSynchronize();
         return fail(SDV2_E_DEVICE, "device status 0x%x (a kernel gave up on a bounded wait)", word);
     }
     return SDV2_OK;

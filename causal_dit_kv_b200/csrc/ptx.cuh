@@ -185,6 +185,10 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]) : "memory");
+}
+
 // ---------------------------------------------------------------- descriptors
 
 // Shared-memory matrix descriptor, 128-byte swizzle (tcgen05 format):
@@ -214,6 +218,79 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n, int a_mn, in
 }
 
 // ---------------------------------------------------------------- misc
+
+// Barrier over `count` threads (a multiple of 32) on hardware barrier `id` (1..15).
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+template <uint32_t kRegs>
+__device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+
+template <uint32_t kRegs>
+__device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+
+// ---- packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction, two lanes of work)
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t r, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// Two lanes of exp2_poly (below) with the arithmetic in f32x2 form.
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float &y0, float &y1) {
+    const uint64_t x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+    const uint64_t t = f2_add(x, f2_pack(12582912.0f, 12582912.0f));
+    const uint64_t j = f2_add(t, f2_pack(-12582912.0f, -12582912.0f));
+    const uint64_t f = f2_fma(j, f2_pack(-1.0f, -1.0f), x);
+    uint64_t p = f2_fma(f2_pack(5.517166853e-02f, 5.517166853e-02f), f, f2_pack(2.426111251e-01f, 2.426111251e-01f));
+    p = f2_fma(p, f, f2_pack(6.932609677e-01f, 6.932609677e-01f));
+    p = f2_fma(p, f, f2_pack(9.999280572e-01f, 9.999280572e-01f));
+    float p0, p1, t0, t1;
+    f2_unpack(p, p0, p1);
+    f2_unpack(t, t0, t1);
+    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
+// 2^x on the FMA pipe (no MUFU), for -inf <= x <= 64.  Cody-Waite style
+// reduction x = j + f, j = round(x) (the 1.5 * 2^23 shift leaves j in the low
+// mantissa bits of t), f in [-1/2, 1/2]; 2^f from the degree-3 minimax
+// polynomial of gen_exp2_poly.py (max relative error 7.5e-5 in fp32); 2^j is
+// added to the exponent field.  x is clamped at -125 so the exponent stays
+// normal: the result there is 2^-125 instead of 0.
+__device__ __forceinline__ float exp2_poly(float x) {
+    x = fmaxf(x, -125.0f);
+    const float t = x + 12582912.0f;
+    const float j = t - 12582912.0f;
+    const float f = x - j;
+    float p = fmaf(5.517166853e-02f, f, 2.426111251e-01f);
+    p = fmaf(p, f, 6.932609677e-01f);
+    p = fmaf(p, f, 9.999280572e-01f);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
 
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;

@@ -45,10 +45,12 @@ struct AppendParams {
 };
 
 struct AttnParams {
-    const uint16_t *q;          // [B][Lq][H][d]
+    const uint16_t *q;          // [B][Lq][H][d] as given (not rotated)
+    uint16_t *q_rot;            // [B][Lq][H][d] RoPE(q) in bf16, scratch (read by TMA)
     uint16_t *out;              // [B][Lq][H][d]
-    float *part_o;              // [split][B][H][Lq_pad][d] (split > 1)
-    float *part_ml;             // [split][B][H][Lq_pad][2]  (row max in log2 units, row sum)
+    float *part_o;              // [split][B][H][d/4][Lq_pad] float4 (split > 1)
+    float *part_ml;             // [split][B][H][Lq_pad] float2 (row max in log2 units, row sum)
+    uint32_t *tickets;          // [B][H][n_qpairs] arrival counters of the split CTAs (0 between calls)
     const float *rope_h;        // [frame_h][n_h][2] fp32
     const float *rope_w;        // [frame_w][n_w][2]
     uint32_t *status;
@@ -58,14 +60,6 @@ struct AttnParams {
     float scale_log2;           // softmax_scale * log2(e)
     int32_t lk[kMaxBatch];      // valid keys per stream of this launch (0 = skip)
     float tab_t[kAttnTabEntries][2];     // [b][frame in chunk][n_t] temporal cos, sin
-};
-
-struct CombineParams {
-    const float *part_o;
-    const float *part_ml;
-    uint16_t *out;
-    int32_t batch, heads, lq, lq_pad, head_dim, n_split, b_offset;
-    int32_t lk[kMaxBatch];
 };
 
 struct RefreshParams {
@@ -108,9 +102,10 @@ struct MotionParams {
 // Launchers (defined next to their kernels).  Each returns the CUDA error
 // of the launch; the host layer turns it into an sdv2_status.
 cudaError_t launch_append(const AppendParams &p, int sm_count, cudaStream_t s);
-cudaError_t launch_attention(const AttnParams &p, const CUtensorMap &tk, const CUtensorMap &tv,
-                             int head_dim, cudaStream_t s);
-cudaError_t launch_combine(const CombineParams &p, cudaStream_t s);
+// RoPE(q) -> q_rot for the streams of the launch (lk > 0), then the attention kernel.
+cudaError_t launch_rope_q(const AttnParams &p, int sm_count, cudaStream_t s);
+cudaError_t launch_attention(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
+                             const CUtensorMap &tv, int head_dim, cudaStream_t s);
 cudaError_t launch_refresh(const RefreshParams &p, int sm_count, cudaStream_t s, int *launches);
 cudaError_t launch_motion(const MotionParams &p, cudaStream_t s);
 // Same kernel with partial/counter in the library's static device array.
