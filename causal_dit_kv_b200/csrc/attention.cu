@@ -14,7 +14,8 @@
 // without unrolling the ring.
 //
 // One CTA = one (stream, head, pair of 128-row query tiles, KV split):
-//   warp 0      TMA producer: K and V tiles (128 keys x d) into a 2-stage ring
+//   warp 0      TMA producer: K tiles (128 keys x d) into a 2-slot ring, V tiles
+//               into a 3-slot ring
 //   warp 1      MMA issuer (one thread): S_t = Q_t K^T and O_t += P_t V
 //   warps 4..7  softmax + epilogue of query tile 0 (thread i owns row i)
 //   warps 8..11 softmax + epilogue of query tile 1
@@ -26,9 +27,8 @@
 // softmax run while the tensor core works on the other tile.
 // Online softmax in base 2 with lazy rescaling: the running max only moves
 // (and O is rescaled in TMEM) when a tile's max exceeds it by more than 8,
-// so P stays <= 256.  Half of the exponentials run as a polynomial on
-// the FMA pipe (exp2_poly2) to relieve the MUFU pipe; the exponent
-// arguments and row sums use packed f32x2 arithmetic.
+// so P stays <= 256.  The exponent arguments and row sums use packed f32x2
+// arithmetic.
 // Q: rope_q_kernel rotates the chunk's queries once per call (fp32 RoPE,
 // rounded to bf16) into a scratch buffer; the producer warp TMA-loads the
 // rotated tiles straight into the 128-byte-swizzled K-major layout the MMA
@@ -49,18 +49,19 @@ struct AttnLayout {
     static constexpr int kQTile = kBlockM * D * 2;    // bytes of one Q tile
     static constexpr int kKVTile = kBlockN * D * 2;   // bytes of one K (or V) tile
     static constexpr int kSub = kBlockM * 128;        // one 64-column (128-byte) sub-tile
-    static constexpr int kStages = 2;
+    static constexpr int kKStages = 2;                // K tile i is needed one half-iteration before V tile i,
+    static constexpr int kVStages = 3;                // so V gets the deeper ring to hide its load latency
     static constexpr int kQ = 0;
     static constexpr int kK = kQ + kQTilesPerCta * kQTile;
-    static constexpr int kV = kK + kStages * kKVTile;
-    static constexpr int kBar = kV + kStages * kKVTile;
+    static constexpr int kV = kK + kKStages * kKVTile;
+    static constexpr int kBar = kV + kVStages * kKVTile;
     // barriers
     static constexpr int kQFull = 0;
     static constexpr int kKFull = 1;
-    static constexpr int kKEmpty = kKFull + kStages;
-    static constexpr int kVFull = kKEmpty + kStages;
-    static constexpr int kVEmpty = kVFull + kStages;
-    static constexpr int kSFull = kVEmpty + kStages;
+    static constexpr int kKEmpty = kKFull + kKStages;
+    static constexpr int kVFull = kKEmpty + kKStages;
+    static constexpr int kVEmpty = kVFull + kVStages;
+    static constexpr int kSFull = kVEmpty + kVStages;
     static constexpr int kPFull = kSFull + 2;
     static constexpr int kOFull = kPFull + 2;
     static constexpr int kDrain = kOFull + 2;
@@ -136,9 +137,8 @@ __global__ void __launch_bounds__(256) rope_q_kernel(const __grid_constant__ Att
 
 // P = 2^(s*scale_log2 - m) for one row of 128 scores (raw fp32 bits in sr),
 // packed to bf16 into TMEM columns [0, 64) of the row's S region; returns
-// the row sum (fp32).  Columns 16..31 of every 32 use the FMA-pipe
-// polynomial, the rest the MUFU ex2.  Pairs of columns share one f32x2 FMA
-// for the exponent argument and one f32x2 add for the sum.
+// the row sum (fp32).  Exponentials on the MUFU ex2; pairs of columns share
+// one f32x2 FMA for the exponent argument and one f32x2 add for the sum.
 __device__ __forceinline__ float softmax_exp_store(const uint32_t (&sr)[kBlockN / 32][32], float scale_log2,
                                                    float neg_m, uint32_t s_tmem) {
     const uint64_t scale2 = f2_pack(scale_log2, scale_log2);
@@ -155,12 +155,8 @@ __device__ __forceinline__ float softmax_exp_store(const uint32_t (&sr)[kBlockN 
                                       scale2, negm2);
             float x0, x1, p0, p1;
             f2_unpack(x, x0, x1);
-            if (i >= 8) {
-                exp2_poly2(x0, x1, p0, p1);
-            } else {
-                p0 = ex2_approx(x0);
-                p1 = ex2_approx(x1);
-            }
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
             acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
             pk[i] = pack_bf16x2(p0, p1);
         }
@@ -203,9 +199,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(&bars[L::kQFull], 1);
-        for (int s = 0; s < L::kStages; ++s) {
+        for (int s = 0; s < L::kKStages; ++s) {
             mbar_init(&bars[L::kKFull + s], 1);
             mbar_init(&bars[L::kKEmpty + s], 1);
+        }
+        for (int s = 0; s < L::kVStages; ++s) {
             mbar_init(&bars[L::kVFull + s], 1);
             mbar_init(&bars[L::kVEmpty + s], 1);
         }
@@ -245,38 +243,49 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 for (int kb = 0; kb < D / 64; ++kb)
                     tma_load_4d(smem + L::kQ + t * L::kQTile + kb * L::kSub, &tmap_q, &bars[L::kQFull], kb * 64, h,
                                 q_row0 + t * kBlockM, bg);
-            int issued = 0;   // tiles whose loads were issued
-            for (int it = 0; it < n_local; ++it) {
-                const int st = it % L::kStages;
-                const uint32_t ph = (it / L::kStages) & 1;
-                const int kv0 = (kv_begin + it) * kBlockN;
-                if (!mbar_wait(&bars[L::kKEmpty + st], ph ^ 1u, abort_flag, p.status, kStatusTmaWait)) break;
-                mbar_arrive_expect_tx(&bars[L::kKFull + st], L::kKVTile);
+            // K tile `it` and V tile `it` are issued as soon as their own ring slot is free.
+            int k_issued = 0, v_issued = 0;
+            bool ok = true;
+            while (ok && v_issued < n_local) {
+                if (k_issued < n_local && k_issued <= v_issued + 1) {
+                    const int st = k_issued % L::kKStages;
+                    const uint32_t ph = (k_issued / L::kKStages) & 1;
+                    if (!mbar_wait(&bars[L::kKEmpty + st], ph ^ 1u, abort_flag, p.status, kStatusTmaWait)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&bars[L::kKFull + st], L::kKVTile);
 #pragma unroll
-                for (int kb = 0; kb < D / 64; ++kb)
-                    tma_load_4d(smem + L::kK + st * L::kKVTile + kb * L::kSub, &tmap_k, &bars[L::kKFull + st], kb * 64,
-                                h, kv0, bg);
+                    for (int kb = 0; kb < D / 64; ++kb)
+                        tma_load_4d(smem + L::kK + st * L::kKVTile + kb * L::kSub, &tmap_k, &bars[L::kKFull + st],
+                                    kb * 64, h, (kv_begin + k_issued) * kBlockN, bg);
+                    ++k_issued;
+                }
+                const int st = v_issued % L::kVStages;
+                const uint32_t ph = (v_issued / L::kVStages) & 1;
                 if (!mbar_wait(&bars[L::kVEmpty + st], ph ^ 1u, abort_flag, p.status, kStatusTmaWait)) {
-                    issued = it + 1;
+                    ok = false;
                     break;
                 }
                 mbar_arrive_expect_tx(&bars[L::kVFull + st], L::kKVTile);
 #pragma unroll
                 for (int kb = 0; kb < D / 64; ++kb)
-                    tma_load_4d(smem + L::kV + st * L::kKVTile + kb * L::kSub, &tmap_v, &bars[L::kVFull + st], kb * 64,
-                                h, kv0, bg);
-                issued = it + 1;
+                    tma_load_4d(smem + L::kV + st * L::kKVTile + kb * L::kSub, &tmap_v, &bars[L::kVFull + st],
+                                kb * 64, h, (kv_begin + v_issued) * kBlockN, bg);
+                ++v_issued;
             }
-            if (*abort_flag) {
+            if (!ok) {
                 // Let every copy already in flight land before the CTA leaves.
-                for (int it = issued - L::kStages; it < issued; ++it) {
-                    if (it < 0) continue;
-                    const int st = it % L::kStages;
-                    const uint32_t ph = (it / L::kStages) & 1;
-                    const uint64_t t0 = global_timer_ns();
-                    while (!(mbar_try_wait(&bars[L::kKFull + st], ph) && mbar_try_wait(&bars[L::kVFull + st], ph))) {
+                const uint64_t t0 = global_timer_ns();
+                for (int i = k_issued - L::kKStages; i < k_issued; ++i) {
+                    if (i < 0) continue;
+                    while (!mbar_try_wait(&bars[L::kKFull + i % L::kKStages], (i / L::kKStages) & 1))
                         if (global_timer_ns() - t0 > kWaitLimitNs) break;
-                    }
+                }
+                for (int i = v_issued - L::kVStages; i < v_issued; ++i) {
+                    if (i < 0) continue;
+                    while (!mbar_try_wait(&bars[L::kVFull + i % L::kVStages], (i / L::kVStages) & 1))
+                        if (global_timer_ns() - t0 > kWaitLimitNs) break;
                 }
             }
         }
@@ -318,10 +327,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 umma_commit(&bars[L::kKEmpty + 0]);
             }
             for (int it = 0; ok && it < n_local; ++it) {
-                const int st = it % L::kStages;
-                const uint32_t ph = (it / L::kStages) & 1;
-                const int nst = (it + 1) % L::kStages;
-                const uint32_t nph = ((it + 1) / L::kStages) & 1;
+                const int st = it % L::kVStages;            // V slot of tile it
+                const uint32_t ph = (it / L::kVStages) & 1;
+                const int nst = (it + 1) % L::kKStages;     // K slot of tile it+1
+                const uint32_t nph = ((it + 1) / L::kKStages) & 1;
                 const bool more = it + 1 < n_local;
                 if (!mbar_wait(&bars[L::kVFull + st], ph, abort_flag, p.status, kStatusMmaWait)) break;
                 tc_fence_after();
@@ -417,6 +426,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     l_run *= alpha;
                     m_run = m_tile;
                 }
+                l_run += softmax_exp_store(sr, p.scale_log2, -m_run, s_tmem);
+                // O_t is idle here (PV(t, it-1) completed before S(t, it) was signalled and
+                // PV(t, it) waits for this thread's arrival below), so it can be rescaled now.
                 if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
                     for (int cb = 0; cb < D / 32; ++cb) {
@@ -427,10 +439,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
                         tmem_st32(o_tmem + cb * 32, r);
                     }
-                    tmem_wait_st();
                 }
-                const float sum = softmax_exp_store(sr, p.scale_log2, -m_run, s_tmem);
-                l_run += sum;
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&bars[L::kPFull + t]);

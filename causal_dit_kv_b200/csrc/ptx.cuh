@@ -259,39 +259,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return d;
 }
 
-// Two lanes of exp2_poly (below) with the arithmetic in f32x2 form.
-__device__ __forceinline__ void exp2_poly2(float x0, float x1, float &y0, float &y1) {
-    const uint64_t x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-    const uint64_t t = f2_add(x, f2_pack(12582912.0f, 12582912.0f));
-    const uint64_t j = f2_add(t, f2_pack(-12582912.0f, -12582912.0f));
-    const uint64_t f = f2_fma(j, f2_pack(-1.0f, -1.0f), x);
-    uint64_t p = f2_fma(f2_pack(5.517166853e-02f, 5.517166853e-02f), f, f2_pack(2.426111251e-01f, 2.426111251e-01f));
-    p = f2_fma(p, f, f2_pack(6.932609677e-01f, 6.932609677e-01f));
-    p = f2_fma(p, f, f2_pack(9.999280572e-01f, 9.999280572e-01f));
-    float p0, p1, t0, t1;
-    f2_unpack(p, p0, p1);
-    f2_unpack(t, t0, t1);
-    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-}
-
-// 2^x on the FMA pipe (no MUFU), for -inf <= x <= 64.  Cody-Waite style
-// reduction x = j + f, j = round(x) (the 1.5 * 2^23 shift leaves j in the low
-// mantissa bits of t), f in [-1/2, 1/2]; 2^f from the degree-3 minimax
-// polynomial of gen_exp2_poly.py (max relative error 7.5e-5 in fp32); 2^j is
-// added to the exponent field.  x is clamped at -125 so the exponent stays
-// normal: the result there is 2^-125 instead of 0.
-__device__ __forceinline__ float exp2_poly(float x) {
-    x = fmaxf(x, -125.0f);
-    const float t = x + 12582912.0f;
-    const float j = t - 12582912.0f;
-    const float f = x - j;
-    float p = fmaf(5.517166853e-02f, f, 2.426111251e-01f);
-    p = fmaf(p, f, 6.932609677e-01f);
-    p = fmaf(p, f, 9.999280572e-01f);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
