@@ -6,8 +6,8 @@
 // walkthrough, "Adaptive sink and RoPE refresh" (periodic RoPE phase reset).
 //
 // Each frame of the chunk is a contiguous N*H*d block in both the input and
-// its ring slot, so the kernel is a flat 16-byte-vector stream over
-// (K frames, V frames).  K vectors are rotated pair by pair in fp64 with
+// its ring slot, so the kernel is a 16-byte-vector stream over (K frames,
+// V frames).  K vectors are rotated pair by pair in fp64 with
 // separately rounded products and sums (no FMA) and rounded once to bf16 by
 // cvt.rn.bf16.f64; V vectors are copied.  The temporal cos/sin of each frame
 // arrive in the kernel parameters (computed on the host per call); the row
@@ -43,64 +43,78 @@ __device__ __forceinline__ uint32_t rotate_pair(uint32_t w, double c, double s) 
     return static_cast<uint32_t>(bf16_from_f64_rn(r0)) | (static_cast<uint32_t>(bf16_from_f64_rn(r1)) << 16);
 }
 
+// Block = 64 (token, head) rows of one frame, 4 threads per row; each thread
+// moves every 4th 16-byte vector of its row (4 vectors for d = 128), all
+// loads issued before the rotations and stores.  grid = (row blocks, frames
+// of the launch, {K, V}).
+constexpr int kAppendRowsPerBlock = 64;
+
 __global__ void __launch_bounds__(256) kv_append_kernel(const __grid_constant__ AppendParams p) {
-    const uint32_t vec_per_frame = static_cast<uint32_t>(p.frame_elems / 8);
-    const uint32_t k_vectors = static_cast<uint32_t>(p.n_frames) * vec_per_frame;
-    const uint32_t total = 2u * k_vectors;
-    const uint32_t hd = static_cast<uint32_t>(p.heads * p.head_dim);
-    for (uint32_t g = blockIdx.x * blockDim.x + threadIdx.x; g < total; g += gridDim.x * blockDim.x) {
-        const bool is_v = g >= k_vectors;
-        const uint32_t r = is_v ? g - k_vectors : g;
-        const uint32_t fi = r / vec_per_frame;
-        const uint32_t vec = r - fi * vec_per_frame;
-        const int b = p.src_b[fi];
-        const int64_t src = static_cast<int64_t>(b) * p.chunk_tokens * hd +
-                            static_cast<int64_t>(p.src_i[fi]) * p.frame_elems + static_cast<int64_t>(vec) * 8;
-        const int64_t dst = (static_cast<int64_t>(b) * p.slots + p.dst_slot[fi]) * p.frame_elems +
-                            static_cast<int64_t>(vec) * 8;
-        if (is_v) {
-            const uint4 x = ld_nc_v4(p.v_in + src);
-            *reinterpret_cast<uint4 *>(p.v_layer + dst) = x;
-            continue;
-        }
-        uint4 x = ld_nc_v4(p.k_in + src);
-        const uint32_t e = vec * 8;
-        const uint32_t n = e / hd;                       // token in the frame
-        const uint32_t dd = e - n * hd;
-        const uint32_t j0 = (dd % static_cast<uint32_t>(p.head_dim)) >> 1;   // first pair of the vector
-        const uint32_t row = n / static_cast<uint32_t>(p.frame_w);
-        const uint32_t col = n - row * static_cast<uint32_t>(p.frame_w);
-        uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    // The previous kernel in the stream may still be running (dependent launch):
+    // wait for it, then let the next one (the queries' RoPE) start alongside.
+    grid_dependency_wait();
+    grid_launch_dependents();
+    const int fi = blockIdx.y;
+    const bool is_v = blockIdx.z != 0;
+    const int rows = static_cast<int>(p.frame_elems / p.head_dim);     // N * H
+    const int row = blockIdx.x * kAppendRowsPerBlock + (threadIdx.x >> 2);
+    const int sub = threadIdx.x & 3;
+    if (row >= rows) return;
+    const int b = p.src_b[fi];
+    const int64_t src = static_cast<int64_t>(b) * p.chunk_tokens * p.heads * p.head_dim +
+                        static_cast<int64_t>(p.src_i[fi]) * p.frame_elems + static_cast<int64_t>(row) * p.head_dim;
+    const int64_t dst = (static_cast<int64_t>(b) * p.slots + p.dst_slot[fi]) * p.frame_elems +
+                        static_cast<int64_t>(row) * p.head_dim;
+    constexpr int kMaxVec = 4;                       // d = 128: 16 vectors per row / 4 threads
+    const int nvec = p.head_dim / 32;                // vectors per thread: 4 (d = 128) or 2 (d = 64)
+    uint4 x[kMaxVec];
+    const uint16_t *in = is_v ? p.v_in : p.k_in;
+#pragma unroll
+    for (int i = 0; i < kMaxVec; ++i)
+        if (i < nvec) x[i] = ld_nc_v4(in + src + (sub + 4 * i) * 8);
+    if (is_v) {
+#pragma unroll
+        for (int i = 0; i < kMaxVec; ++i)
+            if (i < nvec) *reinterpret_cast<uint4 *>(p.v_layer + dst + (sub + 4 * i) * 8) = x[i];
+        return;
+    }
+    const int n = row / p.heads;                     // token in the frame
+    const int prow = n / p.frame_w;
+    const int pcol = n - prow * p.frame_w;
+#pragma unroll
+    for (int i = 0; i < kMaxVec; ++i) {
+        if (i >= nvec) break;
+        const int j0 = (sub + 4 * i) * 4;            // first rotation pair of the vector
+        uint32_t w[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const int j = static_cast<int>(j0) + q;
+            const int j = j0 + q;
             double c, s;
             if (j < p.n_t) {
                 c = p.tab_t[fi * p.n_t + j][0];
                 s = p.tab_t[fi * p.n_t + j][1];
             } else if (j < p.n_t + p.n_h) {
-                const double *t = p.rope_h + 2 * (static_cast<int64_t>(row) * p.n_h + (j - p.n_t));
+                const double *t = p.rope_h + 2 * (static_cast<int64_t>(prow) * p.n_h + (j - p.n_t));
                 c = t[0];
                 s = t[1];
             } else {
-                const double *t = p.rope_w + 2 * (static_cast<int64_t>(col) * p.n_w + (j - p.n_t - p.n_h));
+                const double *t = p.rope_w + 2 * (static_cast<int64_t>(pcol) * p.n_w + (j - p.n_t - p.n_h));
                 c = t[0];
                 s = t[1];
             }
             w[q] = rotate_pair(w[q], c, s);
         }
-        *reinterpret_cast<uint4 *>(p.k_layer + dst) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4 *>(p.k_layer + dst + (sub + 4 * i) * 8) = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
 
 cudaError_t launch_append(const AppendParams &p, int sm_count, cudaStream_t s) {
-    const uint64_t total = 2ull * static_cast<uint64_t>(p.n_frames) * static_cast<uint64_t>(p.frame_elems / 8);
-    if (total == 0) return cudaSuccess;
-    uint64_t blocks = (total + 255) / 256;
-    const uint64_t cap = static_cast<uint64_t>(sm_count) * 8;
-    if (blocks > cap) blocks = cap;
-    kv_append_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
-    return cudaGetLastError();
+    (void)sm_count;
+    if (p.n_frames == 0) return cudaSuccess;
+    const int rows = static_cast<int>(p.frame_elems / p.head_dim);
+    dim3 grid(static_cast<unsigned>((rows + kAppendRowsPerBlock - 1) / kAppendRowsPerBlock),
+              static_cast<unsigned>(p.n_frames), 2u);
+    return launch_dependent(kv_append_kernel, grid, dim3(256), 0, s, p);
 }
 
 }  // namespace sdv2

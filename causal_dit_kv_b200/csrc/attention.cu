@@ -33,9 +33,10 @@
 // rounded to bf16) into a scratch buffer; the producer warp TMA-loads the
 // rotated tiles straight into the 128-byte-swizzled K-major layout the MMA
 // reads.
-// KV splits: each split CTA writes an unnormalised partial (O, row max, row
-// sum); the last CTA of a tile to finish (atomic ticket) merges them and
-// writes the output, so no second launch is needed.
+// KV splits: the split CTAs of a tile take atomic tickets as they finish;
+// all but the last write an unnormalised partial (O, row max, row sum); the
+// last merges them with its own O straight from TMEM and writes the output,
+// so no second launch is needed.
 // Every wait is bounded (2 s), after which the CTA records an error in the
 // device status word and unwinds; TMEM is always released.
 #include <cmath>
@@ -102,28 +103,39 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
 }
 
 // RoPE of the chunk's queries: q_rot = rotate(q) at (phase(frame), row, col),
-// fp32 arithmetic, bf16 result.  One thread per 16-byte vector (4 pairs).
+// fp32 arithmetic, bf16 result.  Block = 64 (token, head) rows of one stream,
+// 4 threads per row, every 4th 16-byte vector of the row per thread (loads
+// first).  grid = (row blocks, streams of the launch).
 __global__ void __launch_bounds__(256) rope_q_kernel(const __grid_constant__ AttnParams p, int head_dim) {
-    const uint32_t vec_per_token = static_cast<uint32_t>(p.heads * head_dim / 8);
-    const uint32_t vec_per_stream = static_cast<uint32_t>(p.lq) * vec_per_token;
-    int nb = 0;
-    for (int i = 0; i < kMaxBatch; ++i)
-        if (p.lk[i] > 0) nb = i + 1;
-    const uint32_t total = static_cast<uint32_t>(nb) * vec_per_stream;
-    for (uint32_t g = blockIdx.x * blockDim.x + threadIdx.x; g < total; g += gridDim.x * blockDim.x) {
-        const int bl = static_cast<int>(g / vec_per_stream);
-        if (p.lk[bl] <= 0) continue;
-        const uint32_t r = g - static_cast<uint32_t>(bl) * vec_per_stream;
-        const int token = static_cast<int>(r / vec_per_token);
-        const uint32_t cv = r - static_cast<uint32_t>(token) * vec_per_token;   // vector within the token
-        const int j0 = static_cast<int>((cv * 8) % static_cast<uint32_t>(head_dim)) >> 1;
-        const int fi = token / p.tokens_per_frame;
-        const int n = token - fi * p.tokens_per_frame;
-        const int prow = n / p.frame_w;
-        const int pcol = n - prow * p.frame_w;
-        const int64_t off = (static_cast<int64_t>(p.b_offset + bl) * p.lq + token) * p.heads * head_dim + cv * 8;
-        const uint4 x = *reinterpret_cast<const uint4 *>(p.q + off);
-        const uint32_t in[4] = {x.x, x.y, x.z, x.w};
+    // Launched right behind the KV append, whose own wait already ordered it after
+    // the producer of q: q can be read at once.  Completing only after the append
+    // (wait at the end) lets the attention kernel wait on this kernel alone.
+    grid_launch_dependents();
+    const int bl = blockIdx.y;
+    const int rows = p.lq * p.heads;
+    const int row = blockIdx.x * 64 + (threadIdx.x >> 2);
+    const int sub = threadIdx.x & 3;
+    if (p.lk[bl] <= 0 || row >= rows) {
+        grid_dependency_wait();
+        return;
+    }
+    const int token = row / p.heads;
+    const int fi = token / p.tokens_per_frame;
+    const int n = token - fi * p.tokens_per_frame;
+    const int prow = n / p.frame_w;
+    const int pcol = n - prow * p.frame_w;
+    const int64_t off = (static_cast<int64_t>(p.b_offset + bl) * rows + row) * head_dim;
+    constexpr int kMaxVec = 4;
+    const int nvec = head_dim / 32;
+    uint4 x[kMaxVec];
+#pragma unroll
+    for (int i = 0; i < kMaxVec; ++i)
+        if (i < nvec) x[i] = *reinterpret_cast<const uint4 *>(p.q + off + (sub + 4 * i) * 8);
+#pragma unroll
+    for (int i = 0; i < kMaxVec; ++i) {
+        if (i >= nvec) break;
+        const int j0 = (sub + 4 * i) * 4;
+        const uint32_t in[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
         uint32_t o[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -131,8 +143,9 @@ __global__ void __launch_bounds__(256) rope_q_kernel(const __grid_constant__ Att
             const float x0 = bf16_lo(in[q]), x1 = bf16_hi(in[q]);
             o[q] = pack_bf16x2(x0 * cs.x - x1 * cs.y, x0 * cs.y + x1 * cs.x);
         }
-        *reinterpret_cast<uint4 *>(p.q_rot + off) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4 *>(p.q_rot + off + (sub + 4 * i) * 8) = make_uint4(o[0], o[1], o[2], o[3]);
     }
+    grid_dependency_wait();
 }
 
 // P = 2^(s*scale_log2 - m) for one row of 128 scores (raw fp32 bits in sr),
@@ -230,6 +243,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // Everything above overlaps the previous kernels (dependent launch); the
+    // rotated queries, the cache and the split tickets are only touched below.
+    grid_dependency_wait();
+    grid_launch_dependents();
 
     if (warp < 4) {
       regs_dec<80>();
@@ -448,9 +465,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             // ---- epilogue
             if (ok && n_local > 0) ok = warp_wait(&bars[L::kOFull + t], 0, abort_flag, p.status, kStatusSoftmaxWait);
             const int prow_local = q_row0 + t * kBlockM + row;     // row index within the padded query range
-            if (ok) {
-                tc_fence_after();
-                if (p.n_split == 1) {
+            if (ok) tc_fence_after();
+            if (p.n_split == 1) {
+                if (ok) {
                     const float inv = 1.0f / l_run;
                     uint16_t *orow = p.out + ((static_cast<int64_t>(bg) * p.lq + token) * p.heads + h) * D;
 #pragma unroll
@@ -470,60 +487,84 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                             }
                         }
                     }
-                } else {
-                    // Partial of this split, column-major in float4 units so that a warp's
-                    // 32 rows write (and the merge reads) 512 contiguous bytes per access:
-                    // part_o[((split*B + b)*H + h)][D/4][lq_pad] float4, part_ml[...][lq_pad] float2.
-                    const int64_t head_idx = (static_cast<int64_t>(split) * p.batch + bg) * p.heads + h;
-                    float4 *po = reinterpret_cast<float4 *>(p.part_o) + head_idx * (D / 4) * p.lq_pad + prow_local;
-                    if (n_local > 0) {
+                }
+            } else {
+                // ---- KV split: the split CTAs of a tile take tickets as they finish; all but
+                // the last write an unnormalised partial (O, row max, row sum) and count it
+                // written; the last one merges those partials with its own O, read from TMEM.
+                const uint32_t nthreads = kBlockM * static_cast<uint32_t>(n_qt);
+                const int64_t group = (static_cast<int64_t>(bg) * p.heads + h) * p.n_qpairs + qpair;
+                uint32_t *ticket = p.tickets + group;
+                uint32_t *written = p.tickets + static_cast<int64_t>(p.batch) * p.heads * p.n_qpairs + group;
+                named_bar_sync(kSoftmaxBarrier, nthreads);
+                if (threadIdx.x == 128) {
+                    const uint32_t prev = atomicAdd(ticket, 1u);
+                    const bool last = prev == static_cast<uint32_t>(p.n_split - 1);
+                    if (last) *ticket = 0u;                    // every split has arrived: re-arm
+                    *merge_flag = last ? 1u : 0u;
+                }
+                named_bar_sync(kSoftmaxBarrier, nthreads);
+                const bool last = *merge_flag != 0u;
+                const float m_own = n_local > 0 ? m_run : -INFINITY;
+                // partial layout: part_o[((split*B + b)*H + h)][D/4][lq_pad] float4 (a warp's 32 rows
+                // are 512 contiguous bytes), part_ml[...][lq_pad] float2 (row max in log2 units, row sum)
+                const int64_t stride_s = static_cast<int64_t>(p.batch) * p.heads;
+                const int64_t head0 = static_cast<int64_t>(bg) * p.heads + h;
+                if (!last) {
+                    const int64_t hs = split * stride_s + head0;
+                    if (ok && n_local > 0) {               // warp-uniform: every lane takes part in tcgen05.ld
+                        float4 *po = reinterpret_cast<float4 *>(p.part_o) + hs * (D / 4) * p.lq_pad + prow_local;
+                        uint32_t r[D / 32][32];
 #pragma unroll
-                        for (int cb = 0; cb < D / 32; ++cb) {
-                            uint32_t r[32];
-                            tmem_ld32(o_tmem + cb * 32, r);
-                            tmem_wait_ld_bind(r);
-                            if (valid) {
+                        for (int cb = 0; cb < D / 32; ++cb) tmem_ld32(o_tmem + cb * 32, r[cb]);
+                        tmem_wait_ld_bind(r[0]);
+#pragma unroll
+                        for (int cb = 1; cb < D / 32; ++cb) reg_bind(r[cb]);
+                        if (valid) {
+#pragma unroll
+                            for (int cb = 0; cb < D / 32; ++cb)
 #pragma unroll
                                 for (int v = 0; v < 8; ++v)
                                     po[static_cast<int64_t>(cb * 8 + v) * p.lq_pad] =
-                                        make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                                    __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
-                            }
+                                        make_float4(__uint_as_float(r[cb][4 * v]), __uint_as_float(r[cb][4 * v + 1]),
+                                                    __uint_as_float(r[cb][4 * v + 2]), __uint_as_float(r[cb][4 * v + 3]));
                         }
                     }
-                    if (valid)
-                        reinterpret_cast<float2 *>(p.part_ml)[head_idx * p.lq_pad + prow_local] =
-                            make_float2(n_local > 0 ? m_run : -INFINITY, l_run);
-                }
-            }
-            // ---- split merge: the last split CTA of this tile combines the partials
-            if (p.n_split > 1) {
-                const uint32_t nthreads = kBlockM * static_cast<uint32_t>(n_qt);
-                __threadfence();
-                named_bar_sync(kSoftmaxBarrier, nthreads);
-                if (threadIdx.x == 128) {
-                    uint32_t *ticket = p.tickets + (static_cast<int64_t>(bg) * p.heads + h) * p.n_qpairs + qpair;
-                    const uint32_t prev = atomicAdd(ticket, 1u);
-                    const bool last = prev == static_cast<uint32_t>(p.n_split - 1);
-                    if (last) *ticket = 0u;                    // every split has arrived: re-arm for the next call
-                    *merge_flag = (last && !*abort_flag) ? 1u : 0u;
-                }
-                named_bar_sync(kSoftmaxBarrier, nthreads);
-                if (*merge_flag && valid) {
+                    if (ok && valid)
+                        reinterpret_cast<float2 *>(p.part_ml)[hs * p.lq_pad + prow_local] = make_float2(m_own, l_run);
                     __threadfence();
-                    const int64_t head0 = static_cast<int64_t>(bg) * p.heads + h;
-                    const int64_t stride_s = static_cast<int64_t>(p.batch) * p.heads;
-                    const float2 *mlp = reinterpret_cast<const float2 *>(p.part_ml);
+                    named_bar_sync(kSoftmaxBarrier, nthreads);
+                    if (threadIdx.x == 128) atomicAdd(written, 1u);
+                } else {
+                    if (threadIdx.x == 128) {
+                        // The other splits took their tickets first, so they are running and only
+                        // have their stores left: wait (bounded) until all of them count as written.
+                        const uint64_t t0 = global_timer_ns();
+                        while (*reinterpret_cast<volatile uint32_t *>(written) < static_cast<uint32_t>(p.n_split - 1)) {
+                            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                                atomicOr(p.status, kStatusSoftmaxWait);
+                                *abort_flag = 1u;
+                                break;
+                            }
+                        }
+                        *written = 0u;
+                        __threadfence();
+                    }
+                    named_bar_sync(kSoftmaxBarrier, nthreads);
+                    const bool merge = ok && !*abort_flag;
                     float2 ml[kMaxSplits];
-                    float m = -INFINITY;
+                    float m = m_own;
 #pragma unroll
                     for (int s = 0; s < kMaxSplits; ++s) {
                         ml[s] = make_float2(-INFINITY, 0.0f);
-                        if (s < p.n_split) ml[s] = __ldcg(mlp + (s * stride_s + head0) * p.lq_pad + prow_local);
+                        if (merge && valid && s < p.n_split && s != split)
+                            ml[s] = __ldcg(reinterpret_cast<const float2 *>(p.part_ml) + (s * stride_s + head0) * p.lq_pad +
+                                           prow_local);
                         m = fmaxf(m, ml[s].x);
                     }
+                    const float w_own = m_own == -INFINITY ? 0.0f : exp2f(m_own - m);
                     float wgt[kMaxSplits];
-                    float l = 0.0f;
+                    float l = w_own * l_run;
 #pragma unroll
                     for (int s = 0; s < kMaxSplits; ++s) {
                         wgt[s] = ml[s].x == -INFINITY ? 0.0f : exp2f(ml[s].x - m);
@@ -531,38 +572,52 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     }
                     const float inv = 1.0f / l;
                     uint16_t *orow = p.out + ((static_cast<int64_t>(bg) * p.lq + token) * p.heads + h) * D;
-                    // two passes of D/2 columns; each split's loads of a pass are issued together
 #pragma unroll 1
-                    for (int half = 0; half < 2; ++half) {
-                        float4 acc[D / 8];
+                    for (int cb = 0; cb < D / 32; ++cb) {
+                        // own 32 columns from TMEM, the other splits' from L2, all loads in flight together
+                        uint32_t r[32];
+                        if (n_local > 0) tmem_ld32(o_tmem + cb * 32, r);
+                        float4 u[kMaxSplits][8];
 #pragma unroll
-                        for (int i = 0; i < D / 8; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 1
-                        for (int s = 0; s < p.n_split; ++s) {
-                            if (wgt[s] == 0.0f) continue;
-                            const float4 *po = reinterpret_cast<const float4 *>(p.part_o) +
-                                               (s * stride_s + head0) * (D / 4) * p.lq_pad + prow_local;
-                            float4 u[D / 8];
+                        for (int s = 0; s < kMaxSplits; ++s) {
+                            if (wgt[s] != 0.0f) {
+                                const float4 *po = reinterpret_cast<const float4 *>(p.part_o) +
+                                                   ((s * stride_s + head0) * (D / 4) + cb * 8) * p.lq_pad + prow_local;
 #pragma unroll
-                            for (int i = 0; i < D / 8; ++i)
-                                u[i] = __ldcg(po + static_cast<int64_t>(half * (D / 8) + i) * p.lq_pad);
-                            const float w = wgt[s];
-#pragma unroll
-                            for (int i = 0; i < D / 8; ++i) {
-                                acc[i].x += w * u[i].x;
-                                acc[i].y += w * u[i].y;
-                                acc[i].z += w * u[i].z;
-                                acc[i].w += w * u[i].w;
+                                for (int i = 0; i < 8; ++i) u[s][i] = __ldcg(po + static_cast<int64_t>(i) * p.lq_pad);
                             }
                         }
+                        if (n_local > 0) {
+                            tmem_wait_ld_bind(r);
+                        } else {
 #pragma unroll
-                        for (int i = 0; i < D / 8; i += 2) {
-                            uint4 w;
-                            w.x = pack_bf16x2(acc[i].x * inv, acc[i].y * inv);
-                            w.y = pack_bf16x2(acc[i].z * inv, acc[i].w * inv);
-                            w.z = pack_bf16x2(acc[i + 1].x * inv, acc[i + 1].y * inv);
-                            w.w = pack_bf16x2(acc[i + 1].z * inv, acc[i + 1].w * inv);
-                            *reinterpret_cast<uint4 *>(orow + half * (D / 2) + i * 4) = w;
+                            for (int i = 0; i < 32; ++i) r[i] = 0u;
+                        }
+                        float a[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) a[i] = w_own * __uint_as_float(r[i]);
+#pragma unroll
+                        for (int s = 0; s < kMaxSplits; ++s) {
+                            if (wgt[s] != 0.0f) {
+#pragma unroll
+                                for (int i = 0; i < 8; ++i) {
+                                    a[4 * i] += wgt[s] * u[s][i].x;
+                                    a[4 * i + 1] += wgt[s] * u[s][i].y;
+                                    a[4 * i + 2] += wgt[s] * u[s][i].z;
+                                    a[4 * i + 3] += wgt[s] * u[s][i].w;
+                                }
+                            }
+                        }
+                        if (merge && valid) {
+#pragma unroll
+                            for (int v = 0; v < 4; ++v) {
+                                uint4 w;
+                                w.x = pack_bf16x2(a[8 * v + 0] * inv, a[8 * v + 1] * inv);
+                                w.y = pack_bf16x2(a[8 * v + 2] * inv, a[8 * v + 3] * inv);
+                                w.z = pack_bf16x2(a[8 * v + 4] * inv, a[8 * v + 5] * inv);
+                                w.w = pack_bf16x2(a[8 * v + 6] * inv, a[8 * v + 7] * inv);
+                                *reinterpret_cast<uint4 *>(orow + cb * 32 + v * 8) = w;
+                            }
                         }
                     }
                 }
@@ -594,8 +649,7 @@ static cudaError_t launch_attention_d(const AttnParams &p, const CUtensorMap &tq
         if (p.lk[i] > 0) nb = i + 1;
     if (nb == 0) return cudaSuccess;
     dim3 grid(static_cast<unsigned>(p.n_qpairs * p.n_split), static_cast<unsigned>(p.heads), static_cast<unsigned>(nb));
-    chunk_attention_kernel<D><<<grid, kAttnThreads, smem, s>>>(p, tq, tk, tv);
-    return cudaGetLastError();
+    return launch_dependent(chunk_attention_kernel<D>, grid, dim3(kAttnThreads), static_cast<size_t>(smem), s, p, tq, tk, tv);
 }
 
 cudaError_t launch_attention(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
@@ -605,16 +659,15 @@ cudaError_t launch_attention(const AttnParams &p, const CUtensorMap &tq, const C
 }
 
 cudaError_t launch_rope_q(const AttnParams &p, int sm_count, cudaStream_t s) {
+    (void)sm_count;
     int nb = 0;
     for (int i = 0; i < kMaxBatch; ++i)
         if (p.lk[i] > 0) nb = i + 1;
-    const int head_dim = p.heads > 0 ? static_cast<int>(p.n_t + p.n_h + p.n_w) * 2 : 0;
-    const uint64_t total = static_cast<uint64_t>(nb) * p.lq * p.heads * head_dim / 8;
-    if (total == 0) return cudaSuccess;
-    uint64_t blocks = (total + 255) / 256;
-    if (blocks > static_cast<uint64_t>(sm_count) * 8) blocks = static_cast<uint64_t>(sm_count) * 8;
-    rope_q_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(p, head_dim);
-    return cudaGetLastError();
+    if (nb == 0) return cudaSuccess;
+    const int head_dim = static_cast<int>(p.n_t + p.n_h + p.n_w) * 2;
+    const int rows = p.lq * p.heads;
+    dim3 grid(static_cast<unsigned>((rows + 63) / 64), static_cast<unsigned>(nb));
+    return launch_dependent(rope_q_kernel, grid, dim3(256), 0, s, p, head_dim);
 }
 
 }  // namespace sdv2

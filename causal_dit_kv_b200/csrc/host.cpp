@@ -157,7 +157,7 @@ Geometry geometry(const sdv2_cache_config &c) {
     g.refresh_counter = off;
     off = align_up(off + 4ull * c.batch, 256);
     g.tickets = off;
-    g.tickets_bytes = 4ull * c.batch * c.heads * g.n_qpairs;
+    g.tickets_bytes = 2 * 4ull * c.batch * c.heads * g.n_qpairs;   // tickets + written counts
     off = align_up(off + g.tickets_bytes, 256);
     g.q_rot = off;
     off = align_up(off + 2ull * c.batch * g.lq * c.heads * c.head_dim, 1024);

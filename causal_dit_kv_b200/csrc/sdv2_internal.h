@@ -4,6 +4,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 
 #include <cuda.h>           // CUtensorMap (type only; the driver is reached at run time)
 #include <cuda_runtime.h>
@@ -12,11 +13,11 @@ namespace sdv2 {
 
 constexpr int kMaxBatch = 64;
 // fp64 (cos, sin) entries of the temporal axis carried in one append launch.
-constexpr int kAppendTabEntries = 1536;   // 24 KB of kernel parameters
-constexpr int kAppendMaxFrames = 64;
+constexpr int kAppendTabEntries = 256;    // 4 KB of kernel parameters
+constexpr int kAppendMaxFrames = 16;
 // fp32 (cos, sin) entries of the temporal axis carried in one attention launch.
-constexpr int kAttnTabEntries = 2048;     // 16 KB of kernel parameters
-constexpr int kMaxSplits = 8;
+constexpr int kAttnTabEntries = 256;      // 2 KB of kernel parameters
+constexpr int kMaxSplits = 4;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits give up after 2 s
 
 // Device status word bits (set with atomicOr, never cleared by kernels).
@@ -50,7 +51,8 @@ struct AttnParams {
     uint16_t *out;              // [B][Lq][H][d]
     float *part_o;              // [split][B][H][d/4][Lq_pad] float4 (split > 1)
     float *part_ml;             // [split][B][H][Lq_pad] float2 (row max in log2 units, row sum)
-    uint32_t *tickets;          // [B][H][n_qpairs] arrival counters of the split CTAs (0 between calls)
+    uint32_t *tickets;          // [2][B][H][n_qpairs]: arrival tickets, then "partial written" counts
+                                //   of the split CTAs (both 0 between calls)
     const float *rope_h;        // [frame_h][n_h][2] fp32
     const float *rope_w;        // [frame_w][n_w][2]
     uint32_t *status;
@@ -98,6 +100,25 @@ struct MotionParams {
     int32_t batch, chunk_frames, window, n_blocks;
     double sigma, lambda, s_min, s_max;
 };
+
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel in the stream finishes; it calls grid_dependency_wait()
+// before touching anything that kernel may write.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                    Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Launchers (defined next to their kernels).  Each returns the CUDA error
 // of the launch; the host layer turns it into an sdv2_status.
