@@ -42,6 +42,8 @@ WORKLOADS = {
     "wan14b-512x512-b8": dict(batch=8, layers=40, heads=40, head_dim=128, frame_h=32, frame_w=32, chunk_frames=1,
                               sink_frames=1, window_frames=6, embed_dim=5120, motion=(16, 64, 64)),
 }
+WORKLOADS["tiny-stream"] = dict(batch=1, layers=1, heads=2, head_dim=64, frame_h=4, frame_w=4, chunk_frames=1,
+                                sink_frames=1, window_frames=2, embed_dim=64, motion=(16, 4, 4))
 DEFAULT_WORKLOAD = "wan1.3b-512x512"
 TAU = 0.9
 
@@ -53,6 +55,28 @@ def load_peaks():
             pk = json.load(fh)
         return pk, "measured"
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per attention launch from the committed ncu summary, if it was
+    taken on the current kernel source (else None)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"chunk_attention_{workload}.md")
+    src = os.path.join(ROOT, "causal_dit_kv_b200", "csrc", "attention.cu")
+    if not os.path.exists(path):
+        return None
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    fields = {}
+    for line in open(path):
+        if ":" in line and line.split(":")[0].strip() in ("traffic_bytes_per_launch", "source_sha256_prefix"):
+            k, v = line.split(":", 1)
+            fields[k.strip()] = v.strip()
+    if fields.get("source_sha256_prefix") != digest:
+        return None
+    try:
+        return int(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
 
 
 def attn_flops(w, keys):
@@ -126,6 +150,14 @@ class ClockSampler:
         return out
 
 
+def max_over_ranks(values, dist, device):
+    """Element-wise maximum of per-rank timings (every rank calls it once)."""
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -161,34 +193,56 @@ def run_ours(args, w, name):
     scale = 1.0 / math.sqrt(D)
     dev = torch.device("cuda", local)
 
-    # Input pool: two distinct steps' worth of Q/K/V for every layer, hidden states and latents.
+    # Input pool: two distinct steps' worth of Q/K/V for every layer.  Hidden states and
+    # latents form one continuous stream per step (a slowly drifting chunk embedding
+    # with rare scene cuts, latents with segment-wise motion), as in a live stream.
     pool = []
     seed = 2000 + rank
+    n_total = (w["sink_frames"] + w["window_frames"] + 1) + args.warmup + 3 * args.steps + 2
     for p in range(2):
         qkv = [synth.chunk_qkv(seed, B, Lq, H, D, p, l) for l in range(L)]
-        hid = next(synth.drifting_hidden(seed + p, B, Lq, E, 1, drift=0.05))
-        lat = next(synth.motion_latents(seed + p, B, Tp, C, MH, MW, 1))
-        pool.append(dict(qkv=qkv, hid=hid, lat=lat))
+        pool.append(dict(qkv=qkv))
+    hid_seq = [h.to(dev) for h in synth.drifting_hidden(seed, B, Lq, E, n_total, drift=0.02, cut_prob=0.01)]
+    lat_seq = [x.to(dev) for x in synth.motion_latents(seed, B, Tp, C, MH, MW, n_total)]
     dev_pool = [dict(q=[t[0].to(dev) for t in p["qkv"]], k=[t[1].to(dev) for t in p["qkv"]],
-                     v=[t[2].to(dev) for t in p["qkv"]], hid=p["hid"].to(dev), lat=p["lat"].to(dev)) for p in pool]
+                     v=[t[2].to(dev) for t in p["qkv"]]) for p in pool]
     out = torch.empty((B, Lq, H, D), dtype=torch.bfloat16, device=dev)
     out_slot = torch.empty(B, dtype=torch.int32, device=dev)
     rate = torch.empty(B, dtype=torch.float32, device=dev)
     frame = [0]
+    n_step = [0]
     stream = torch.cuda.current_stream(dev)
 
-    def step(inp, attn_events=None):
+    def step(inp, ev=None):
+        """One streamed chunk through every layer; ev (optional) collects event pairs per call."""
         f0 = [frame[0]] * B
         for l in range(L):
+            if ev is not None:
+                ev["append"].append([rec()])
             cache.kv_append(l, inp["k"][l], inp["v"][l], f0)
-            if attn_events is not None:
-                attn_events[l][0].record(stream)
+            if ev is not None:
+                ev["append"][-1].append(rec())
+                ev["attention"].append([rec()])
             cache.chunk_attention(l, inp["q"][l], out, f0, scale)
-            if attn_events is not None:
-                attn_events[l][1].record(stream)
-        cache.sink_refresh(inp["hid"], TAU, f0, out_slot)
-        mot.noise_rate(inp["lat"], rate)
+            if ev is not None:
+                ev["attention"][-1].append(rec())
+        if ev is not None:
+            ev["refresh"].append([rec()])
+        hid, lat = (inp["hid"], inp["lat"]) if "hid" in inp else (hid_seq[n_step[0] % n_total], lat_seq[n_step[0] % n_total])
+        cache.sink_refresh(hid, TAU, f0, out_slot)
+        if ev is not None:
+            ev["refresh"][-1].append(rec())
+            ev["motion"].append([rec()])
+        mot.noise_rate(lat, rate)
+        if ev is not None:
+            ev["motion"][-1].append(rec())
         frame[0] += Tp
+        n_step[0] += 1
+
+    def rec():
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)
+        return e
 
     # Pre-roll to steady state (ring wrapped, every slot valid), then warm up.
     for i in range(w["sink_frames"] + w["window_frames"] + 1):
@@ -197,9 +251,8 @@ def run_ours(args, w, name):
         step(dev_pool[i % 2])
     torch.cuda.synchronize()
 
-    # ---- device-resident timing
-    events = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
-              for _ in range(args.steps)]
+    # ---- device-resident timing of whole steps (no per-call events: they would
+    # break the overlap of dependent launches)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches0 = binding.sdv2_launch_count()
     with ClockSampler(local) as clocks:
@@ -208,25 +261,33 @@ def run_ours(args, w, name):
         torch.cuda.synchronize()
         t0.record(stream)
         for i in range(args.steps):
-            step(dev_pool[i % 2], events[i])
+            step(dev_pool[i % 2])
         t1.record(stream)
         torch.cuda.synchronize()
         if pg:
             pg.barrier()
     launches = binding.sdv2_launch_count() - launches0
     ms = t0.elapsed_time(t1)
-    attn_ms = [a.elapsed_time(b) for ev in events for (a, b) in ev]
+
+    # ---- per-call timing: the same steps again with events around every call
+    ev = {k: [] for k in ("append", "attention", "refresh", "motion")}
+    for i in range(args.steps):
+        step(dev_pool[i % 2], ev)
+    torch.cuda.synchronize()
+    call_us = {}
+    for k, pairs in ev.items():
+        call_us[k] = statistics.mean(a.elapsed_time(b) for a, b in pairs) * 1e3
     assert cache.check() == 0 and mot.check() == 0, "device status word set"
 
     # ---- end to end: pinned host inputs copied in, results copied out, every step
     host_pool = []
-    for p in pool:
+    for i, p in enumerate(pool):
         host_pool.append(dict(q=[t[0].pin_memory() for t in p["qkv"]], k=[t[1].pin_memory() for t in p["qkv"]],
-                              v=[t[2].pin_memory() for t in p["qkv"]], hid=p["hid"].pin_memory(),
-                              lat=p["lat"].pin_memory()))
+                              v=[t[2].pin_memory() for t in p["qkv"]], hid=hid_seq[i].cpu().pin_memory(),
+                              lat=lat_seq[i].cpu().pin_memory()))
     stage = dict(q=[torch.empty_like(t) for t in dev_pool[0]["q"]], k=[torch.empty_like(t) for t in dev_pool[0]["k"]],
-                 v=[torch.empty_like(t) for t in dev_pool[0]["v"]], hid=torch.empty_like(dev_pool[0]["hid"]),
-                 lat=torch.empty_like(dev_pool[0]["lat"]))
+                 v=[torch.empty_like(t) for t in dev_pool[0]["v"]], hid=torch.empty_like(hid_seq[0]),
+                 lat=torch.empty_like(lat_seq[0]))
     res_out = torch.empty((B, Lq, H, D), dtype=torch.bfloat16).pin_memory()
     res_rate = torch.empty(B, dtype=torch.float32).pin_memory()
     res_slot = torch.empty(B, dtype=torch.int32).pin_memory()
@@ -258,9 +319,7 @@ def run_ours(args, w, name):
     e2e_ms = e0.elapsed_time(e1)
 
     if pg:
-        t = torch.tensor([ms, e2e_ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms, e2e_ms = float(t[0]), float(t[1])
+        ms, e2e_ms = max_over_ranks([ms, e2e_ms], pg, dev)
     frames = world * args.steps * B * Tp
     value = frames / (ms / 1e3)
     e2e_value = frames / (e2e_ms / 1e3)
@@ -268,10 +327,16 @@ def run_ours(args, w, name):
     keys = steady_keys(w)
     flops = attn_flops(w, keys)
     abytes = attn_bytes(w, keys)
-    attn_avg_s = statistics.mean(attn_ms) / 1e3
+    attn_avg_s = call_us["attention"] / 1e6
     peaks, peak_src = load_peaks()
     peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    hbm = peaks["hbm_gbs"]
     achieved = flops / attn_avg_s / 1e12
+    kv_chunk = 2.0 * B * Lq * H * D * 2                      # K + V of the chunk, bf16
+    append_bytes = 2 * kv_chunk                               # read + written
+    refresh_bytes = B * Lq * E * 2 + B * E * 8 * (w["sink_frames"] + 1)
+    motion_bytes = B * (Tp + 2) * C * MH * MW * 4             # chunk + previous frame read, last frame written
+    traffic = profiled_traffic(name)
     result = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4), "higher_is_better": True,
@@ -283,15 +348,25 @@ def run_ours(args, w, name):
                    "l2": "inputs larger than L2 (per-step caches %.0f MB over %d layers)" % (
                        2 * cache.layout.layer_stride * L / 1e6, L),
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"kernel": "chunk_attention_kernel (one launch per layer, split merge in-kernel)", "bound": "tensor",
+        "roofline": {"kernel": "chunk_attention_kernel + rope_q (one sdv2_chunk_attention call)", "bound": "tensor",
                      "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_source": f"{peak_src} bf16_tflops_sustained",
-                     "algorithmic_flops_per_launch": flops, "avg_launch_us": round(attn_avg_s * 1e6, 3),
-                     "kv_gbs": round(abytes / attn_avg_s / 1e9, 1)},
-        "attention": {"tflops": round(achieved, 2), "kv_hbm_gbs": round(abytes / attn_avg_s / 1e9, 1),
-                      "us_per_layer": round(attn_avg_s * 1e6, 3),
-                      "frac_of_burst_peak": round(achieved / peaks["bf16_tflops"], 4)},
+                     "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": abytes,
+                     "avg_launch_us": round(attn_avg_s * 1e6, 3)},
+        "rows": {
+            "kv_append": {"us": round(call_us["append"], 3), "bytes": append_bytes,
+                          "gbs": round(append_bytes / call_us["append"] / 1e3, 1),
+                          "frac_hbm": round(append_bytes / call_us["append"] / 1e3 / hbm, 4)},
+            "chunk_attention": {"us": round(call_us["attention"], 3), "tflops": round(achieved, 2),
+                                "frac_tensor": round(achieved / peak, 4),
+                                "kv_gbs": round(abytes / attn_avg_s / 1e9, 1)},
+            "sink_refresh": {"us": round(call_us["refresh"], 3), "bytes_without_copy": refresh_bytes,
+                             "gbs": round(refresh_bytes / call_us["refresh"] / 1e3, 1)},
+            "motion_noise_rate": {"us": round(call_us["motion"], 3), "bytes": motion_bytes,
+                                  "gbs": round(motion_bytes / call_us["motion"] / 1e3, 1)},
+            "note": "per-call times from a second pass with events around each call (events serialise "
+                    "the dependent launches, so these are upper bounds of the in-step cost)"},
         "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": int(launches),

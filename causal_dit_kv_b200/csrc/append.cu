@@ -43,19 +43,25 @@ __device__ __forceinline__ uint32_t rotate_pair(uint32_t w, double c, double s) 
     return static_cast<uint32_t>(bf16_from_f64_rn(r0)) | (static_cast<uint32_t>(bf16_from_f64_rn(r1)) << 16);
 }
 
-// Block = 64 (token, head) rows of one frame, 4 threads per row; each thread
+// Block = 32 (token, head) rows of one frame, 4 threads per row; each thread
 // moves every 4th 16-byte vector of its row (4 vectors for d = 128), all
 // loads issued before the rotations and stores.  grid = (row blocks, frames
 // of the launch, {K, V}).
-constexpr int kAppendRowsPerBlock = 64;
+constexpr int kAppendRowsPerBlock = 32;
 
-__global__ void __launch_bounds__(256) kv_append_kernel(const __grid_constant__ AppendParams p) {
+__global__ void __launch_bounds__(128) kv_append_kernel(const __grid_constant__ AppendParams p) {
     // The previous kernel in the stream may still be running (dependent launch):
     // wait for it, then let the next one (the queries' RoPE) start alongside.
     grid_dependency_wait();
     grid_launch_dependents();
     const int fi = blockIdx.y;
     const bool is_v = blockIdx.z != 0;
+    __shared__ double2 s_tab[64];                    // temporal (cos, sin) of this block's frame
+    if (!is_v) {
+        if (threadIdx.x < p.n_t)
+            s_tab[threadIdx.x] = make_double2(p.tab_t[fi * p.n_t + threadIdx.x][0], p.tab_t[fi * p.n_t + threadIdx.x][1]);
+        __syncthreads();
+    }
     const int rows = static_cast<int>(p.frame_elems / p.head_dim);     // N * H
     const int row = blockIdx.x * kAppendRowsPerBlock + (threadIdx.x >> 2);
     const int sub = threadIdx.x & 3;
@@ -81,29 +87,28 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const __grid_constant__ 
     const int n = row / p.heads;                     // token in the frame
     const int prow = n / p.frame_w;
     const int pcol = n - prow * p.frame_w;
+    // (cos, sin) of every pair of this thread's vectors: branch-free addresses so
+    // all table loads issue together (the temporal entries come from shared memory)
+    const double2 *tab_h = reinterpret_cast<const double2 *>(p.rope_h) + static_cast<int64_t>(prow) * p.n_h - p.n_t;
+    const double2 *tab_w =
+        reinterpret_cast<const double2 *>(p.rope_w) + static_cast<int64_t>(pcol) * p.n_w - p.n_t - p.n_h;
+    double2 cs[kMaxVec][4];
 #pragma unroll
     for (int i = 0; i < kMaxVec; ++i) {
         if (i >= nvec) break;
-        const int j0 = (sub + 4 * i) * 4;            // first rotation pair of the vector
-        uint32_t w[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const int j = j0 + q;
-            double c, s;
-            if (j < p.n_t) {
-                c = p.tab_t[fi * p.n_t + j][0];
-                s = p.tab_t[fi * p.n_t + j][1];
-            } else if (j < p.n_t + p.n_h) {
-                const double *t = p.rope_h + 2 * (static_cast<int64_t>(prow) * p.n_h + (j - p.n_t));
-                c = t[0];
-                s = t[1];
-            } else {
-                const double *t = p.rope_w + 2 * (static_cast<int64_t>(pcol) * p.n_w + (j - p.n_t - p.n_h));
-                c = t[0];
-                s = t[1];
-            }
-            w[q] = rotate_pair(w[q], c, s);
+            const int j = (sub + 4 * i) * 4 + q;
+            const double2 *t = j < p.n_t ? &s_tab[j] : (j < p.n_t + p.n_h ? tab_h + j : tab_w + j);
+            cs[i][q] = *t;
         }
+    }
+#pragma unroll
+    for (int i = 0; i < kMaxVec; ++i) {
+        if (i >= nvec) break;
+        uint32_t w[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) w[q] = rotate_pair(w[q], cs[i][q].x, cs[i][q].y);
         *reinterpret_cast<uint4 *>(p.k_layer + dst + (sub + 4 * i) * 8) = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
@@ -114,7 +119,7 @@ cudaError_t launch_append(const AppendParams &p, int sm_count, cudaStream_t s) {
     const int rows = static_cast<int>(p.frame_elems / p.head_dim);
     dim3 grid(static_cast<unsigned>((rows + kAppendRowsPerBlock - 1) / kAppendRowsPerBlock),
               static_cast<unsigned>(p.n_frames), 2u);
-    return launch_dependent(kv_append_kernel, grid, dim3(256), 0, s, p);
+    return launch_dependent(kv_append_kernel, grid, dim3(4 * kAppendRowsPerBlock), 0, s, p);
 }
 
 }  // namespace sdv2

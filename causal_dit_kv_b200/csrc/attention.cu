@@ -112,6 +112,12 @@ __global__ void __launch_bounds__(256) rope_q_kernel(const __grid_constant__ Att
     // (wait at the end) lets the attention kernel wait on this kernel alone.
     grid_launch_dependents();
     const int bl = blockIdx.y;
+    __shared__ float2 s_tab[kAttnTabEntries];        // temporal (cos, sin) of this stream's frames
+    for (int e = threadIdx.x; e < p.chunk_frames * p.n_t; e += blockDim.x) {
+        const int src = bl * p.chunk_frames * p.n_t + e;
+        s_tab[e] = make_float2(p.tab_t[src][0], p.tab_t[src][1]);
+    }
+    __syncthreads();
     const int rows = p.lq * p.heads;
     const int row = blockIdx.x * 64 + (threadIdx.x >> 2);
     const int sub = threadIdx.x & 3;
@@ -131,17 +137,28 @@ __global__ void __launch_bounds__(256) rope_q_kernel(const __grid_constant__ Att
 #pragma unroll
     for (int i = 0; i < kMaxVec; ++i)
         if (i < nvec) x[i] = *reinterpret_cast<const uint4 *>(p.q + off + (sub + 4 * i) * 8);
+    const float2 *tab_t = s_tab + fi * p.n_t;
+    const float2 *tab_h = reinterpret_cast<const float2 *>(p.rope_h) + prow * p.n_h - p.n_t;
+    const float2 *tab_w = reinterpret_cast<const float2 *>(p.rope_w) + pcol * p.n_w - p.n_t - p.n_h;
+    float2 cs[kMaxVec][4];
 #pragma unroll
     for (int i = 0; i < kMaxVec; ++i) {
         if (i >= nvec) break;
-        const int j0 = (sub + 4 * i) * 4;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int j = (sub + 4 * i) * 4 + q;
+            cs[i][q] = *(j < p.n_t ? tab_t + j : (j < p.n_t + p.n_h ? tab_h + j : tab_w + j));
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < kMaxVec; ++i) {
+        if (i >= nvec) break;
         const uint32_t in[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
         uint32_t o[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const float2 cs = q_cos_sin(p, bl, fi, prow, pcol, j0 + q);
             const float x0 = bf16_lo(in[q]), x1 = bf16_hi(in[q]);
-            o[q] = pack_bf16x2(x0 * cs.x - x1 * cs.y, x0 * cs.y + x1 * cs.x);
+            o[q] = pack_bf16x2(x0 * cs[i][q].x - x1 * cs[i][q].y, x0 * cs[i][q].y + x1 * cs[i][q].x);
         }
         *reinterpret_cast<uint4 *>(p.q_rot + off + (sub + 4 * i) * 8) = make_uint4(o[0], o[1], o[2], o[3]);
     }

@@ -94,7 +94,8 @@ sdv2_status check_config(const sdv2_cache_config *c, sdv2_cache_config *norm) {
         return fail(SDV2_E_SHAPE, "chunk_frames, sink_frames and window_frames must be >= 1");
     if (n.window_frames < n.chunk_frames) return fail(SDV2_E_SHAPE, "window_frames must be >= chunk_frames");
     if (n.rope_reset_period < 0) return fail(SDV2_E_SHAPE, "rope_reset_period must be >= 0");
-    if (n.embed_dim < 0 || (n.embed_dim & 1)) return fail(SDV2_E_SHAPE, "embed_dim must be even and >= 0");
+    if (n.embed_dim < 0 || (n.embed_dim & 1) || n.embed_dim > 16384)
+        return fail(SDV2_E_SHAPE, "embed_dim must be even and in 0..16384");
     if (!(n.rope_base > 0.0)) n.rope_base = 10000.0;
     const int c2 = n.head_dim / 2;
     if (n.rope_pairs[0] == 0 && n.rope_pairs[1] == 0 && n.rope_pairs[2] == 0) {
@@ -153,7 +154,7 @@ Geometry geometry(const sdv2_cache_config &c) {
     off = align_up(off + 4, 256);
     g.scratch = off;
     g.refresh_mean = off;
-    off = align_up(off + 8ull * c.batch * (c.embed_dim > 0 ? c.embed_dim : 1), 256);
+    off = align_up(off + 8ull * c.batch * kRefreshRowChunks * (c.embed_dim > 0 ? c.embed_dim : 1), 256);
     g.refresh_counter = off;
     off = align_up(off + 4ull * c.batch, 256);
     g.tickets = off;
@@ -569,7 +570,7 @@ sdv2_status sdv2_sink_refresh(sdv2_cache *c, const void *hidden, float tau, cons
     RefreshParams p;
     std::memset(&p, 0, sizeof(p));
     p.hidden = static_cast<const uint16_t *>(hidden);
-    p.mean = reinterpret_cast<double *>(c->base + g.refresh_mean);
+    p.partial = reinterpret_cast<double *>(c->base + g.refresh_mean);
     p.counter = reinterpret_cast<uint32_t *>(c->base + g.refresh_counter);
     p.sink_embed = reinterpret_cast<double *>(c->base + g.sink_embed);
     p.sink_frame = reinterpret_cast<int64_t *>(c->base + g.sink_frame);

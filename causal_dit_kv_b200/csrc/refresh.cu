@@ -6,11 +6,12 @@
 // similarity; replace the least similar sink when the similarity falls
 // below the threshold tau).
 //
-// Kernel 1, grid (column blocks, B): block (x, b) averages 64 columns of the
-// hidden states over all tokens in fp64 (warp w takes tokens w, w+8, ...;
-// lane l takes columns 2l, 2l+1), fixed-order reduction across warps.  The
-// last block of stream b (atomic ticket) computes the dot products and
-// norms in fp64, takes the decision, updates the sink embedding and the
+// Kernel 1, grid (column blocks, token chunks, B): block (x, r, b) sums 64
+// columns of the hidden states over token chunk r in fp64 (warp w takes
+// tokens w, w+8, ...; lane l takes columns 2l, 2l+1; fixed-order reduction
+// across warps).  The last block of stream b (atomic ticket) adds the chunk
+// sums in chunk order, divides by the token count, computes the dot products
+// and norms in fp64, takes the decision, updates the sink embedding and the
 // sink-frame record, and writes out_slot[b].
 // Kernel 2, grid (blocks, B): if out_slot[b] >= 0, copies slot last_slot[b]
 // to slot out_slot[b] in every layer, K and V, as 16-byte vectors; otherwise
@@ -35,21 +36,25 @@ __device__ __forceinline__ double block_sum_fixed(double v, double *red) {
 }
 
 __global__ void __launch_bounds__(kRefreshThreads) refresh_decide_kernel(const __grid_constant__ RefreshParams p) {
-    const int b = blockIdx.y;
+    const int b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (!p.active[b]) {
-        if (blockIdx.x == 0 && tid == 0) p.out_slot[b] = -1;
+        if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) p.out_slot[b] = -1;
         return;
     }
     __shared__ double part[kRefreshThreads / 32][kRefreshCols];
     __shared__ double red[kRefreshThreads / 32];
     __shared__ int is_last;
 
+    // column sums of this block's 64 columns over its chunk of tokens
     const int col0 = blockIdx.x * kRefreshCols + 2 * lane;
+    const int t_begin = static_cast<int>((static_cast<int64_t>(p.lq) * blockIdx.y) / kRefreshRowChunks);
+    const int t_end = static_cast<int>((static_cast<int64_t>(p.lq) * (blockIdx.y + 1)) / kRefreshRowChunks);
     const uint16_t *hb = p.hidden + static_cast<int64_t>(b) * p.lq * p.dim;
     double a0 = 0.0, a1 = 0.0;
     if (col0 < p.dim) {
-        for (int t = warp; t < p.lq; t += kRefreshThreads / 32) {
+#pragma unroll 4
+        for (int t = t_begin + warp; t < t_end; t += kRefreshThreads / 32) {
             const uint32_t w = *reinterpret_cast<const uint32_t *>(hb + static_cast<int64_t>(t) * p.dim + col0);
             a0 += static_cast<double>(bf16_lo(w));
             a1 += static_cast<double>(bf16_hi(w));
@@ -63,44 +68,57 @@ __global__ void __launch_bounds__(kRefreshThreads) refresh_decide_kernel(const _
         if (c < p.dim) {
             double s = 0.0;
             for (int w = 0; w < kRefreshThreads / 32; ++w) s += part[w][tid];
-            p.mean[static_cast<int64_t>(b) * p.dim + c] = s / static_cast<double>(p.lq);
+            p.partial[(static_cast<int64_t>(b) * kRefreshRowChunks + blockIdx.y) * p.dim + c] = s;
         }
     }
     __threadfence();
     __syncthreads();
-    if (tid == 0) is_last = atomicAdd(p.counter + b, 1u) == gridDim.x - 1;
+    if (tid == 0) is_last = atomicAdd(p.counter + b, 1u) == gridDim.x * gridDim.y - 1;
     __syncthreads();
     if (!is_last) return;
     __threadfence();
 
-    const double *h = p.mean + static_cast<int64_t>(b) * p.dim;
+    // last block of stream b: chunk mean h (row chunks summed in order), then the decision
+    const double *pb = p.partial + static_cast<int64_t>(b) * kRefreshRowChunks * p.dim;
+    auto mean_at = [&](int c) {
+        double s = 0.0;
+        for (int r = 0; r < kRefreshRowChunks; ++r) s += __ldcg(pb + static_cast<int64_t>(r) * p.dim + c);
+        return s / static_cast<double>(p.lq);
+    };
     double *emb = p.sink_embed + static_cast<int64_t>(b) * p.sinks * p.dim;
     if (p.fill_count[b] > 0) {
         // The chunk fills sink slots itself: record their embedding only.
-        for (int j = p.fill_first[b]; j < p.fill_first[b] + p.fill_count[b]; ++j) {
-            for (int c = tid; c < p.dim; c += kRefreshThreads) emb[static_cast<int64_t>(j) * p.dim + c] = __ldcg(h + c);
-            if (tid == 0) p.sink_frame[static_cast<int64_t>(b) * p.sinks + j] = j;
+        for (int c = tid; c < p.dim; c += kRefreshThreads) {
+            const double h = mean_at(c);
+            for (int j = p.fill_first[b]; j < p.fill_first[b] + p.fill_count[b]; ++j)
+                emb[static_cast<int64_t>(j) * p.dim + c] = h;
         }
         if (tid == 0) {
+            for (int j = p.fill_first[b]; j < p.fill_first[b] + p.fill_count[b]; ++j)
+                p.sink_frame[static_cast<int64_t>(b) * p.sinks + j] = j;
             p.out_slot[b] = -1;
             p.counter[b] = 0u;
         }
         return;
     }
+    // h is consumed column by column; each thread keeps its columns' values
+    constexpr int kMaxColsPerThread = 64;          // embed_dim <= 16384
+    double hv[kMaxColsPerThread];
     double hh = 0.0;
-    for (int c = tid; c < p.dim; c += kRefreshThreads) {
-        const double v = __ldcg(h + c);
-        hh += v * v;
+    int k = 0;
+    for (int c = tid; c < p.dim && k < kMaxColsPerThread; c += kRefreshThreads, ++k) {
+        hv[k] = mean_at(c);
+        hh += hv[k] * hv[k];
     }
     hh = block_sum_fixed(hh, red);
     double best = 0.0;
     int best_j = -1;
     for (int j = 0; j < p.sinks; ++j) {
         double he = 0.0, ee = 0.0;
-        for (int c = tid; c < p.dim; c += kRefreshThreads) {
-            const double v = __ldcg(h + c);
+        k = 0;
+        for (int c = tid; c < p.dim && k < kMaxColsPerThread; c += kRefreshThreads, ++k) {
             const double e = emb[static_cast<int64_t>(j) * p.dim + c];
-            he += v * e;
+            he += hv[k] * e;
             ee += e * e;
         }
         he = block_sum_fixed(he, red);
@@ -114,7 +132,9 @@ __global__ void __launch_bounds__(kRefreshThreads) refresh_decide_kernel(const _
     const bool fire = best < p.tau;
     __syncthreads();
     if (fire) {
-        for (int c = tid; c < p.dim; c += kRefreshThreads) emb[static_cast<int64_t>(best_j) * p.dim + c] = __ldcg(h + c);
+        k = 0;
+        for (int c = tid; c < p.dim && k < kMaxColsPerThread; c += kRefreshThreads, ++k)
+            emb[static_cast<int64_t>(best_j) * p.dim + c] = hv[k];
     }
     if (tid == 0) {
         if (fire) p.sink_frame[static_cast<int64_t>(b) * p.sinks + best_j] = p.last_frame[b];
@@ -145,7 +165,8 @@ __global__ void __launch_bounds__(256) refresh_copy_kernel(const __grid_constant
 }
 
 cudaError_t launch_refresh(const RefreshParams &p, int sm_count, cudaStream_t s, int *launches) {
-    dim3 g1(static_cast<unsigned>((p.dim + kRefreshCols - 1) / kRefreshCols), static_cast<unsigned>(p.batch));
+    dim3 g1(static_cast<unsigned>((p.dim + kRefreshCols - 1) / kRefreshCols), kRefreshRowChunks,
+            static_cast<unsigned>(p.batch));
     refresh_decide_kernel<<<g1, kRefreshThreads, 0, s>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

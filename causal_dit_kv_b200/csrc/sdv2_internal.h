@@ -66,7 +66,7 @@ struct AttnParams {
 
 struct RefreshParams {
     const uint16_t *hidden;     // [B][Lq][D]
-    double *mean;               // scratch [B][D]
+    double *partial;            // scratch [B][kRefreshRowChunks][D]: column sums of each row chunk
     uint32_t *counter;          // scratch [B]
     double *sink_embed;         // [B][S][D]
     int64_t *sink_frame;        // [B][S]
@@ -140,6 +140,7 @@ constexpr int kQTilesPerCta = 2;  // two query tiles ping-pong over the tensor c
 constexpr int kAttnThreads = 384;
 int attention_smem_bytes(int head_dim);
 
+constexpr int kRefreshRowChunks = 8;      // token chunks the chunk-mean reduction is split into
 constexpr int kMotionBlockElems = 2048;   // latent elements per motion block
 constexpr int kMotionThreads = 256;
 

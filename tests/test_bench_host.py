@@ -1,0 +1,73 @@
+"""Host-side logic of bench.py, no GPU: the max-over-ranks timing reduction with
+two gloo ranks, the reference (oracle) arm's JSON line, and the ncu-traffic
+guard that only reports traffic for the kernel source it was measured on."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+def _rank_main(rank, world, port, out_q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import bench
+    got = bench.max_over_ranks([10.0 + rank, 5.0 - rank], dist, "cpu")
+    out_q.put((rank, got))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_max_over_ranks_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29500 + os.getpid() % 1000
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = dict(q.get(timeout=5) for _ in range(2))
+    assert res[0] == res[1] == [11.0, 5.0]
+
+
+def test_reference_arm_prints_one_line():
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny-stream",
+           "--steps", "2", "--warmup", "3"]
+    out = subprocess.run(cmd, capture_output=True, text=True, timeout=300, check=True).stdout.strip().splitlines()
+    assert len(out) == 1
+    line = json.loads(out[0])
+    assert line["impl"] == "reference" and line["unit"] == "latent frames/s" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny-stream",
+           "--steps", "1", "--warmup", "3"]
+    res = subprocess.run(cmd, capture_output=True, text=True, timeout=300, env=env)
+    assert res.returncode == 0 and res.stdout.strip() == ""
+
+
+def test_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
+    import bench
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    (tmp_path / "profiles").mkdir()
+    csrc = tmp_path / "causal_dit_kv_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "attention.cu").write_bytes(b"kernel v1")
+    import hashlib
+    h = hashlib.sha256(b"kernel v1").hexdigest()[:16]
+    (tmp_path / "profiles" / "chunk_attention_w.md").write_text(
+        f"traffic_bytes_per_launch: 123\nsource_sha256_prefix: {h}\n")
+    assert bench.profiled_traffic("w") == 123
+    (csrc / "attention.cu").write_bytes(b"kernel v2")
+    assert bench.profiled_traffic("w") is None
