@@ -33,10 +33,9 @@
 // rounded to bf16) into a scratch buffer; the producer warp TMA-loads the
 // rotated tiles straight into the 128-byte-swizzled K-major layout the MMA
 // reads.
-// KV splits: the split CTAs of a tile take atomic tickets as they finish;
-// all but the last write an unnormalised partial (O, row max, row sum); the
-// last merges them with its own O straight from TMEM and writes the output,
-// so no second launch is needed.
+// KV splits: each split CTA writes its unnormalised O, row max and row sum;
+// attention_combine_kernel (a dependent launch) merges them over the whole
+// GPU.
 // Every wait is bounded (2 s), after which the CTA records an error in the
 // device status word and unwinds; TMEM is always released.
 #include <cmath>
@@ -67,7 +66,7 @@ struct AttnLayout {
     static constexpr int kOFull = kPFull + 2;
     static constexpr int kDrain = kOFull + 2;
     static constexpr int kNumBars = kDrain + 1;
-    static constexpr int kMisc = kBar + kNumBars * 8;   // tmem base, abort flag, merge flag
+    static constexpr int kMisc = kBar + kNumBars * 8;   // tmem base, abort flag
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;      // room to align the base to 1024 bytes
 };
@@ -78,7 +77,6 @@ int attention_smem_bytes(int head_dim) {
 
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale only when the max grows by > 2^8
-constexpr uint32_t kSoftmaxBarrier = 1;     // named barrier of the softmax warpgroups
 
 // fp32 (cos, sin) of rotation pair j for a query token.
 __device__ __forceinline__ float2 q_cos_sin(const AttnParams &p, int bl, int fi, int row, int col, int j) {
@@ -207,7 +205,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBar);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + L::kMisc + 4);
-    volatile uint32_t *merge_flag = reinterpret_cast<volatile uint32_t *>(smem + L::kMisc + 8);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -244,7 +241,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         mbar_init(&bars[L::kDrain], 1);
         *abort_flag = 0u;
-        *merge_flag = 0u;
         fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {
@@ -261,7 +257,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     // Everything above overlaps the previous kernels (dependent launch); the
-    // rotated queries, the cache and the split tickets are only touched below.
+    // rotated queries, the cache and the split partials are only touched below.
     grid_dependency_wait();
     grid_launch_dependents();
 
@@ -505,139 +501,36 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         }
                     }
                 }
-            } else {
-                // ---- KV split: the split CTAs of a tile take tickets as they finish; all but
-                // the last write an unnormalised partial (O, row max, row sum) and count it
-                // written; the last one merges those partials with its own O, read from TMEM.
-                const uint32_t nthreads = kBlockM * static_cast<uint32_t>(n_qt);
+            } else if (ok) {
+                // ---- KV split: write this split's unnormalised partial for attention_combine_kernel.
+                // part_o: one block per (split, stream, head, query-tile pair) of [D/4 float4
+                // columns][256 rows] (rows t*128 + lane; a warp's 32 rows are 512 contiguous
+                // bytes); part_ml[(split*B + b)*H + h][lq_pad] float2 = (row max in log2 units, sum).
                 const int64_t group = (static_cast<int64_t>(bg) * p.heads + h) * p.n_qpairs + qpair;
-                uint32_t *ticket = p.tickets + group;
-                uint32_t *written = p.tickets + static_cast<int64_t>(p.batch) * p.heads * p.n_qpairs + group;
-                named_bar_sync(kSoftmaxBarrier, nthreads);
-                if (threadIdx.x == 128) {
-                    const uint32_t prev = atomicAdd(ticket, 1u);
-                    const bool last = prev == static_cast<uint32_t>(p.n_split - 1);
-                    if (last) *ticket = 0u;                    // every split has arrived: re-arm
-                    *merge_flag = last ? 1u : 0u;
-                }
-                named_bar_sync(kSoftmaxBarrier, nthreads);
-                const bool last = *merge_flag != 0u;
-                const float m_own = n_local > 0 ? m_run : -INFINITY;
-                // partial layout: part_o[((split*B + b)*H + h)][D/4][lq_pad] float4 (a warp's 32 rows
-                // are 512 contiguous bytes), part_ml[...][lq_pad] float2 (row max in log2 units, row sum)
-                const int64_t stride_s = static_cast<int64_t>(p.batch) * p.heads;
-                const int64_t head0 = static_cast<int64_t>(bg) * p.heads + h;
-                if (!last) {
-                    const int64_t hs = split * stride_s + head0;
-                    if (ok && n_local > 0) {               // warp-uniform: every lane takes part in tcgen05.ld
-                        float4 *po = reinterpret_cast<float4 *>(p.part_o) + hs * (D / 4) * p.lq_pad + prow_local;
-                        uint32_t r[D / 32][32];
+                const int64_t n_groups = static_cast<int64_t>(p.batch) * p.heads * p.n_qpairs;
+                const int srow = t * kBlockM + row;
+                if (n_local > 0) {                         // warp-uniform: every lane takes part in tcgen05.ld
+                    float4 *po = reinterpret_cast<float4 *>(p.part_o) + (split * n_groups + group) * (D / 4) * 256 + srow;
+                    uint32_t r[D / 32][32];
 #pragma unroll
-                        for (int cb = 0; cb < D / 32; ++cb) tmem_ld32(o_tmem + cb * 32, r[cb]);
-                        tmem_wait_ld_bind(r[0]);
+                    for (int cb = 0; cb < D / 32; ++cb) tmem_ld32(o_tmem + cb * 32, r[cb]);
+                    tmem_wait_ld_bind(r[0]);
 #pragma unroll
-                        for (int cb = 1; cb < D / 32; ++cb) reg_bind(r[cb]);
-                        if (valid) {
+                    for (int cb = 1; cb < D / 32; ++cb) reg_bind(r[cb]);
+                    if (valid) {
 #pragma unroll
-                            for (int cb = 0; cb < D / 32; ++cb)
+                        for (int cb = 0; cb < D / 32; ++cb)
 #pragma unroll
-                                for (int v = 0; v < 8; ++v)
-                                    po[static_cast<int64_t>(cb * 8 + v) * p.lq_pad] =
-                                        make_float4(__uint_as_float(r[cb][4 * v]), __uint_as_float(r[cb][4 * v + 1]),
-                                                    __uint_as_float(r[cb][4 * v + 2]), __uint_as_float(r[cb][4 * v + 3]));
-                        }
-                    }
-                    if (ok && valid)
-                        reinterpret_cast<float2 *>(p.part_ml)[hs * p.lq_pad + prow_local] = make_float2(m_own, l_run);
-                    __threadfence();
-                    named_bar_sync(kSoftmaxBarrier, nthreads);
-                    if (threadIdx.x == 128) atomicAdd(written, 1u);
-                } else {
-                    if (threadIdx.x == 128) {
-                        // The other splits took their tickets first, so they are running and only
-                        // have their stores left: wait (bounded) until all of them count as written.
-                        const uint64_t t0 = global_timer_ns();
-                        while (*reinterpret_cast<volatile uint32_t *>(written) < static_cast<uint32_t>(p.n_split - 1)) {
-                            if (global_timer_ns() - t0 > kWaitLimitNs) {
-                                atomicOr(p.status, kStatusSoftmaxWait);
-                                *abort_flag = 1u;
-                                break;
-                            }
-                        }
-                        *written = 0u;
-                        __threadfence();
-                    }
-                    named_bar_sync(kSoftmaxBarrier, nthreads);
-                    const bool merge = ok && !*abort_flag;
-                    float2 ml[kMaxSplits];
-                    float m = m_own;
-#pragma unroll
-                    for (int s = 0; s < kMaxSplits; ++s) {
-                        ml[s] = make_float2(-INFINITY, 0.0f);
-                        if (merge && valid && s < p.n_split && s != split)
-                            ml[s] = __ldcg(reinterpret_cast<const float2 *>(p.part_ml) + (s * stride_s + head0) * p.lq_pad +
-                                           prow_local);
-                        m = fmaxf(m, ml[s].x);
-                    }
-                    const float w_own = m_own == -INFINITY ? 0.0f : exp2f(m_own - m);
-                    float wgt[kMaxSplits];
-                    float l = w_own * l_run;
-#pragma unroll
-                    for (int s = 0; s < kMaxSplits; ++s) {
-                        wgt[s] = ml[s].x == -INFINITY ? 0.0f : exp2f(ml[s].x - m);
-                        l += wgt[s] * ml[s].y;
-                    }
-                    const float inv = 1.0f / l;
-                    uint16_t *orow = p.out + ((static_cast<int64_t>(bg) * p.lq + token) * p.heads + h) * D;
-#pragma unroll 1
-                    for (int cb = 0; cb < D / 32; ++cb) {
-                        // own 32 columns from TMEM, the other splits' from L2, all loads in flight together
-                        uint32_t r[32];
-                        if (n_local > 0) tmem_ld32(o_tmem + cb * 32, r);
-                        float4 u[kMaxSplits][8];
-#pragma unroll
-                        for (int s = 0; s < kMaxSplits; ++s) {
-                            if (wgt[s] != 0.0f) {
-                                const float4 *po = reinterpret_cast<const float4 *>(p.part_o) +
-                                                   ((s * stride_s + head0) * (D / 4) + cb * 8) * p.lq_pad + prow_local;
-#pragma unroll
-                                for (int i = 0; i < 8; ++i) u[s][i] = __ldcg(po + static_cast<int64_t>(i) * p.lq_pad);
-                            }
-                        }
-                        if (n_local > 0) {
-                            tmem_wait_ld_bind(r);
-                        } else {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) r[i] = 0u;
-                        }
-                        float a[32];
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) a[i] = w_own * __uint_as_float(r[i]);
-#pragma unroll
-                        for (int s = 0; s < kMaxSplits; ++s) {
-                            if (wgt[s] != 0.0f) {
-#pragma unroll
-                                for (int i = 0; i < 8; ++i) {
-                                    a[4 * i] += wgt[s] * u[s][i].x;
-                                    a[4 * i + 1] += wgt[s] * u[s][i].y;
-                                    a[4 * i + 2] += wgt[s] * u[s][i].z;
-                                    a[4 * i + 3] += wgt[s] * u[s][i].w;
-                                }
-                            }
-                        }
-                        if (merge && valid) {
-#pragma unroll
-                            for (int v = 0; v < 4; ++v) {
-                                uint4 w;
-                                w.x = pack_bf16x2(a[8 * v + 0] * inv, a[8 * v + 1] * inv);
-                                w.y = pack_bf16x2(a[8 * v + 2] * inv, a[8 * v + 3] * inv);
-                                w.z = pack_bf16x2(a[8 * v + 4] * inv, a[8 * v + 5] * inv);
-                                w.w = pack_bf16x2(a[8 * v + 6] * inv, a[8 * v + 7] * inv);
-                                *reinterpret_cast<uint4 *>(orow + cb * 32 + v * 8) = w;
-                            }
-                        }
+                            for (int v = 0; v < 8; ++v)
+                                po[(cb * 8 + v) * 256] =
+                                    make_float4(__uint_as_float(r[cb][4 * v]), __uint_as_float(r[cb][4 * v + 1]),
+                                                __uint_as_float(r[cb][4 * v + 2]), __uint_as_float(r[cb][4 * v + 3]));
                     }
                 }
+                if (valid)
+                    reinterpret_cast<float2 *>(p.part_ml)[((static_cast<int64_t>(split) * p.batch + bg) * p.heads + h) *
+                                                              p.lq_pad + prow_local] =
+                        make_float2(n_local > 0 ? m_run : -INFINITY, l_run);
             }
         }
     }
@@ -648,6 +541,81 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// Merge of the KV-split partials: out = sum_s 2^(m_s - m) O_s / sum_s 2^(m_s - m) l_s.
+// Thread = (row, 8 float4 columns) of one (stream, head, query-tile pair) block:
+// consecutive threads take consecutive rows, so every load of a split's column
+// is coalesced, and all splits' loads of a thread are in flight together.
+template <int D>
+__global__ void __launch_bounds__(256) attention_combine_kernel(const __grid_constant__ AttnParams p) {
+    grid_dependency_wait();                         // the split CTAs' partials
+    grid_launch_dependents();
+    constexpr int kC8 = D / 32;                     // 8-column chunks per row
+    const int64_t n_groups = static_cast<int64_t>(p.batch) * p.heads * p.n_qpairs;
+    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int srow = static_cast<int>(idx & 255);
+    const int64_t rest = idx >> 8;
+    const int c8 = static_cast<int>(rest % kC8);
+    const int64_t gl = rest / kC8;                  // group within this launch's streams
+    const int64_t per_stream = static_cast<int64_t>(p.heads) * p.n_qpairs;
+    const int bl = static_cast<int>(gl / per_stream);
+    if (bl >= kMaxBatch || p.lk[bl] <= 0) return;
+    const int bg = p.b_offset + bl;
+    const int h = static_cast<int>((gl % per_stream) / p.n_qpairs);
+    const int qpair = static_cast<int>(gl % p.n_qpairs);
+    const int token = qpair * 256 + srow;
+    if (token >= p.lq) return;
+    const int64_t group = (static_cast<int64_t>(bg) * p.heads + h) * p.n_qpairs + qpair;
+    float2 ml[kMaxSplits];
+    float m = -INFINITY;
+#pragma unroll
+    for (int s = 0; s < kMaxSplits; ++s) {
+        ml[s] = make_float2(-INFINITY, 0.0f);
+        if (s < p.n_split)
+            ml[s] = reinterpret_cast<const float2 *>(p.part_ml)[((static_cast<int64_t>(s) * p.batch + bg) * p.heads + h) *
+                                                                     p.lq_pad + token];
+        m = fmaxf(m, ml[s].x);
+    }
+    float4 u[kMaxSplits][8];
+#pragma unroll
+    for (int s = 0; s < kMaxSplits; ++s) {
+        if (s < p.n_split && ml[s].x != -INFINITY) {
+            const float4 *po = reinterpret_cast<const float4 *>(p.part_o) + (s * n_groups + group) * (D / 4) * 256 +
+                               (c8 * 8) * 256 + srow;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) u[s][i] = po[i * 256];
+        }
+    }
+    float a[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) a[i] = 0.0f;
+    float l = 0.0f;
+#pragma unroll
+    for (int s = 0; s < kMaxSplits; ++s) {
+        if (s < p.n_split && ml[s].x != -INFINITY) {
+            const float w = exp2f(ml[s].x - m);
+            l += w * ml[s].y;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                a[4 * i] += w * u[s][i].x;
+                a[4 * i + 1] += w * u[s][i].y;
+                a[4 * i + 2] += w * u[s][i].z;
+                a[4 * i + 3] += w * u[s][i].w;
+            }
+        }
+    }
+    const float inv = 1.0f / l;
+    uint16_t *orow = p.out + ((static_cast<int64_t>(bg) * p.lq + token) * p.heads + h) * D + c8 * 32;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+        uint4 w;
+        w.x = pack_bf16x2(a[8 * v + 0] * inv, a[8 * v + 1] * inv);
+        w.y = pack_bf16x2(a[8 * v + 2] * inv, a[8 * v + 3] * inv);
+        w.z = pack_bf16x2(a[8 * v + 4] * inv, a[8 * v + 5] * inv);
+        w.w = pack_bf16x2(a[8 * v + 6] * inv, a[8 * v + 7] * inv);
+        *reinterpret_cast<uint4 *>(orow + v * 8) = w;
     }
 }
 
@@ -673,6 +641,17 @@ cudaError_t launch_attention(const AttnParams &p, const CUtensorMap &tq, const C
                              const CUtensorMap &tv, int head_dim, cudaStream_t s) {
     if (head_dim == 64) return launch_attention_d<64>(p, tq, tk, tv, s);
     return launch_attention_d<128>(p, tq, tk, tv, s);
+}
+
+cudaError_t launch_combine(const AttnParams &p, int head_dim, cudaStream_t s) {
+    int nb = 0;
+    for (int i = 0; i < kMaxBatch; ++i)
+        if (p.lk[i] > 0) nb = i + 1;
+    if (nb == 0 || p.n_split <= 1) return cudaSuccess;
+    const int64_t threads = static_cast<int64_t>(nb) * p.heads * p.n_qpairs * (head_dim / 32) * 256;
+    const dim3 grid(static_cast<unsigned>((threads + 255) / 256));
+    if (head_dim == 64) return launch_dependent(attention_combine_kernel<64>, grid, dim3(256), 0, s, p);
+    return launch_dependent(attention_combine_kernel<128>, grid, dim3(256), 0, s, p);
 }
 
 cudaError_t launch_rope_q(const AttnParams &p, int sm_count, cudaStream_t s) {

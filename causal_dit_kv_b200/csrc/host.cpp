@@ -77,7 +77,7 @@ struct Geometry {
     // region offsets
     uint64_t rope_h64, rope_w64, rope_h32, rope_w32;
     uint64_t sink_embed, sink_frame, status;
-    uint64_t scratch, refresh_mean, refresh_counter, tickets, tickets_bytes, q_rot, part_ml, part_o, scratch_end;
+    uint64_t scratch, refresh_mean, refresh_counter, q_rot, q_rot_bytes, part_ml, part_o, scratch_end;
     uint64_t k, v, layer_stride, total;
 };
 
@@ -157,11 +157,11 @@ Geometry geometry(const sdv2_cache_config &c) {
     off = align_up(off + 8ull * c.batch * kRefreshRowChunks * (c.embed_dim > 0 ? c.embed_dim : 1), 256);
     g.refresh_counter = off;
     off = align_up(off + 4ull * c.batch, 256);
-    g.tickets = off;
-    g.tickets_bytes = 2 * 4ull * c.batch * c.heads * g.n_qpairs;   // tickets + written counts
-    off = align_up(off + g.tickets_bytes, 256);
+    // two buffers of rotated queries, used by alternate attention calls: a call's RoPE
+    // pass may then start before the previous call's attention kernel has finished
     g.q_rot = off;
-    off = align_up(off + 2ull * c.batch * g.lq * c.heads * c.head_dim, 1024);
+    g.q_rot_bytes = align_up(2ull * c.batch * g.lq * c.heads * c.head_dim, 1024);
+    off = align_up(off + 2 * g.q_rot_bytes, 1024);
     g.part_ml = off;
     off = align_up(off + 8ull * g.part_rows, 256);
     g.part_o = off;
@@ -230,7 +230,8 @@ struct sdv2_cache {
     int sm_count;
     std::vector<int64_t> next_frame;  // [B][L]
     std::vector<CUtensorMap> tk, tv;  // [L]
-    CUtensorMap tq;                   // rotated queries in scratch: (d, H, Lq, B)
+    CUtensorMap tq[2];                // the two rotated-query buffers in scratch: (d, H, Lq, B)
+    uint64_t attention_calls = 0;     // selects the rotated-query buffer
 };
 
 struct sdv2_motion {
@@ -392,12 +393,14 @@ sdv2_status sdv2_cache_create(const sdv2_cache_config *cfg, void *dev_buf, size_
                                         static_cast<cuuint64_t>(n.heads) * n.head_dim * 2,
                                         static_cast<cuuint64_t>(g.lq) * n.heads * n.head_dim * 2};
         const cuuint32_t qbox[4] = {64, 1, static_cast<cuuint32_t>(kBlockM), 1};
-        CUresult r = encode(&c->tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, c->base + g.q_rot, qdims, qstrides, qbox,
-                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) {
-            delete c;
-            return fail(SDV2_E_CUDA, "cuTensorMapEncodeTiled (queries) failed (%d)", static_cast<int>(r));
+        for (int buf = 0; buf < 2; ++buf) {
+            CUresult r = encode(&c->tq[buf], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, c->base + g.q_rot + buf * g.q_rot_bytes,
+                                qdims, qstrides, qbox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+            if (r != CUDA_SUCCESS) {
+                delete c;
+                return fail(SDV2_E_CUDA, "cuTensorMapEncodeTiled (queries) failed (%d)", static_cast<int>(r));
+            }
         }
     }
     c->next_frame.assign(static_cast<size_t>(n.batch) * n.layers, 0);
@@ -499,11 +502,11 @@ sdv2_status sdv2_chunk_attention(sdv2_cache *c, int32_t layer, const void *q, vo
     AttnParams p;
     std::memset(&p, 0, sizeof(p));
     p.q = static_cast<const uint16_t *>(q);
-    p.q_rot = reinterpret_cast<uint16_t *>(c->base + g.q_rot);
+    const int qbuf = static_cast<int>(c->attention_calls & 1);
+    p.q_rot = reinterpret_cast<uint16_t *>(c->base + g.q_rot + qbuf * g.q_rot_bytes);
     p.out = static_cast<uint16_t *>(out);
     p.part_o = reinterpret_cast<float *>(c->base + g.part_o);
     p.part_ml = reinterpret_cast<float *>(c->base + g.part_ml);
-    p.tickets = reinterpret_cast<uint32_t *>(c->base + g.tickets);
     p.rope_h = reinterpret_cast<const float *>(c->base + g.rope_h32);
     p.rope_w = reinterpret_cast<const float *>(c->base + g.rope_w32);
     p.status = reinterpret_cast<uint32_t *>(c->base + g.status);
@@ -543,10 +546,16 @@ sdv2_status sdv2_chunk_attention(sdv2_cache *c, int32_t layer, const void *q, vo
         if (!any) continue;
         cudaError_t e = launch_rope_q(p, c->sm_count, s);
         if (e != cudaSuccess) return cuda_fail(e, "rope_q launch");
-        e = launch_attention(p, c->tq, c->tk[layer], c->tv[layer], n.head_dim, s);
+        e = launch_attention(p, c->tq[qbuf], c->tk[layer], c->tv[layer], n.head_dim, s);
         if (e != cudaSuccess) return cuda_fail(e, "chunk_attention launch");
         g_launches.fetch_add(2);
+        if (n_split > 1) {
+            e = launch_combine(p, n.head_dim, s);
+            if (e != cudaSuccess) return cuda_fail(e, "attention combine launch");
+            g_launches.fetch_add(1);
+        }
     }
+    ++c->attention_calls;
     return SDV2_OK;
 }
 
@@ -647,9 +656,8 @@ sdv2_status sdv2_cache_check(sdv2_cache *c) {
     e = cudaMemcpy(&word, c->base + c->g.status, 4, cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(e, "cache_check");
     if (word != 0) {
-        // A CTA that gave up may have left split tickets half counted: re-arm them.
+        // A block that gave up may have left the refresh ticket half counted: re-arm it.
         cudaMemset(c->base + c->g.status, 0, 4);
-        cudaMemset(c->base + c->g.tickets, 0, c->g.tickets_bytes);
         cudaMemset(c->base + c->g.refresh_counter, 0, 4ull * c->cfg.batch);
         cudaDeviceSynchronize();
         return fail(SDV2_E_DEVICE, "device status 0x%x (a kernel gave up on a bounded wait)", word);

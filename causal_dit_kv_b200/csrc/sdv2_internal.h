@@ -51,8 +51,6 @@ struct AttnParams {
     uint16_t *out;              // [B][Lq][H][d]
     float *part_o;              // [split][B][H][d/4][Lq_pad] float4 (split > 1)
     float *part_ml;             // [split][B][H][Lq_pad] float2 (row max in log2 units, row sum)
-    uint32_t *tickets;          // [2][B][H][n_qpairs]: arrival tickets, then "partial written" counts
-                                //   of the split CTAs (both 0 between calls)
     const float *rope_h;        // [frame_h][n_h][2] fp32
     const float *rope_w;        // [frame_w][n_w][2]
     uint32_t *status;
@@ -125,6 +123,8 @@ inline cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 bl
 cudaError_t launch_append(const AppendParams &p, int sm_count, cudaStream_t s);
 // RoPE(q) -> q_rot for the streams of the launch (lk > 0), then the attention kernel.
 cudaError_t launch_rope_q(const AttnParams &p, int sm_count, cudaStream_t s);
+// Merge of the KV-split partials into out (a dependent launch after the attention kernel).
+cudaError_t launch_combine(const AttnParams &p, int head_dim, cudaStream_t s);
 cudaError_t launch_attention(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
                              const CUtensorMap &tv, int head_dim, cudaStream_t s);
 cudaError_t launch_refresh(const RefreshParams &p, int sm_count, cudaStream_t s, int *launches);
