@@ -58,6 +58,7 @@ _SIGNATURES = [
     ("sdv2_cache_query", c_int32, [c_void_p, c_int32, c_int32, POINTER(c_int64), POINTER(c_int32), POINTER(c_int32)]),
     ("sdv2_cache_layout_get", c_int32, [c_void_p, POINTER(sdv2_cache_layout)]),
     ("sdv2_cache_check", c_int32, [c_void_p]),
+    ("sdv2_cache_selftest_wait", c_int32, [c_void_p, c_uint64, c_void_p]),
     ("sdv2_motion_bytes", c_size_t, [POINTER(sdv2_motion_config)]),
     ("sdv2_motion_create", c_int32, [POINTER(sdv2_motion_config), c_void_p, c_size_t, POINTER(c_void_p)]),
     ("sdv2_motion_destroy", c_int32, [c_void_p]),
@@ -199,6 +200,10 @@ def sdv2_cache_layout_get(cache: int) -> sdv2_cache_layout:
 
 def sdv2_cache_check(cache: int) -> int:
     return int(lib().sdv2_cache_check(cache))
+
+
+def sdv2_cache_selftest_wait(cache: int, limit_ns: int, stream=None) -> None:
+    _check(lib().sdv2_cache_selftest_wait(cache, int(limit_ns), _stream(stream)), "sdv2_cache_selftest_wait")
 
 
 def sdv2_motion_bytes(cfg: sdv2_motion_config) -> int:

@@ -619,6 +619,28 @@ __global__ void __launch_bounds__(256) attention_combine_kernel(const __grid_con
     }
 }
 
+// Failure-detection self-test: one thread waits on an mbarrier that nothing
+// arrives on, with the given bound; the bounded wait gives up, records
+// kStatusSelfTest in the status word and the kernel returns normally.
+__global__ void bounded_wait_selftest_kernel(uint32_t *status, uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(&bar, 0)) {
+        if (global_timer_ns() - t0 > limit_ns) {
+            atomicOr(status, kStatusSelfTest);
+            return;
+        }
+    }
+}
+
+cudaError_t launch_wait_selftest(uint32_t *status, uint64_t limit_ns, cudaStream_t s) {
+    bounded_wait_selftest_kernel<<<1, 32, 0, s>>>(status, limit_ns);
+    return cudaGetLastError();
+}
+
 template <int D>
 static cudaError_t launch_attention_d(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
                                       const CUtensorMap &tv, cudaStream_t s) {

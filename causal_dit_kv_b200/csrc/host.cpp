@@ -665,6 +665,19 @@ sdv2_status sdv2_cache_check(sdv2_cache *c) {
     return SDV2_OK;
 }
 
+sdv2_status sdv2_cache_selftest_wait(sdv2_cache *c, uint64_t limit_ns, sdv2_stream stream) {
+    if (!c) return fail(SDV2_E_ARG, "cache is NULL");
+    if (limit_ns == 0 || limit_ns > kWaitLimitNs) return fail(SDV2_E_ARG, "limit_ns must be in 1..%llu",
+                                                               static_cast<unsigned long long>(kWaitLimitNs));
+    sdv2_status st = check_device(c->device);
+    if (st != SDV2_OK) return st;
+    cudaError_t e = launch_wait_selftest(reinterpret_cast<uint32_t *>(c->base + c->g.status), limit_ns,
+                                         reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "selftest launch");
+    g_launches.fetch_add(1);
+    return SDV2_OK;
+}
+
 // ------------------------------------------------------------------ motion
 
 static sdv2_status check_motion(const sdv2_motion_config *m) {

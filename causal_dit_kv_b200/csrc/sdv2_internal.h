@@ -26,6 +26,7 @@ enum : uint32_t {
     kStatusMmaWait = 1u << 1,
     kStatusSoftmaxWait = 1u << 2,
     kStatusBadArgs = 1u << 3,
+    kStatusSelfTest = 1u << 4,
 };
 
 struct AppendParams {
@@ -123,6 +124,7 @@ inline cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 bl
 cudaError_t launch_append(const AppendParams &p, int sm_count, cudaStream_t s);
 // RoPE(q) -> q_rot for the streams of the launch (lk > 0), then the attention kernel.
 cudaError_t launch_rope_q(const AttnParams &p, int sm_count, cudaStream_t s);
+cudaError_t launch_wait_selftest(uint32_t *status, uint64_t limit_ns, cudaStream_t s);
 // Merge of the KV-split partials into out (a dependent launch after the attention kernel).
 cudaError_t launch_combine(const AttnParams &p, int head_dim, cudaStream_t s);
 cudaError_t launch_attention(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk,

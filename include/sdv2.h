@@ -189,6 +189,15 @@ sdv2_status sdv2_cache_layout_get(const sdv2_cache *cache, sdv2_cache_layout *ou
  * cleared).  Not for the hot path. */
 sdv2_status sdv2_cache_check(sdv2_cache *cache);
 
+/* Failure-detection self-test (no counterpart in the pages): launches one
+ * thread that waits on a device barrier nothing arrives on, bounded by
+ * limit_ns (1 .. 2e9).  The wait gives up, sets a bit in the cache's status
+ * word and the kernel returns normally, so the next sdv2_cache_check()
+ * reports SDV2_E_DEVICE and clears the word; the CUDA context stays usable.
+ * This is the path every real kernel wait takes when it runs out.
+ * Errors: SDV2_E_ARG, SDV2_E_CUDA. */
+sdv2_status sdv2_cache_selftest_wait(sdv2_cache *cache, uint64_t limit_ns, sdv2_stream stream);
+
 /* ------------------------------------------------------------------------
  * Motion-aware noise rate.  [A] method item 2; [Q] "Motion-aware noise
  * scheduler"; [G] Python example (previous_noise_scale carried over).

@@ -169,3 +169,38 @@ def test_full_size_14b_sampled():
     ps = PairedStream(seed=1003, **cfg)
     rows = np.sort(np.random.default_rng(2).choice(1024, 32, replace=False))
     _stream_and_check(ps, 8, check_every=7, attn_rows=rows)
+
+
+@pytest.mark.parametrize("splits", ["split", "unsplit"])
+def test_back_to_back_attention_calls(splits):
+    """Several attention calls on the same appended chunk in a row (and on
+    alternating layers) give the same, correct output: a call's query RoPE pass
+    never overwrites queries an earlier call is still reading."""
+    if splits == "split":
+        cfg = dict(batch=1, layers=2, heads=12, head_dim=128, frame_h=32, frame_w=32, chunk_frames=1,
+                   sink_frames=1, window_frames=6)
+    else:
+        cfg = dict(batch=2, layers=2, heads=40, head_dim=128, frame_h=16, frame_w=16, chunk_frames=1,
+                   sink_frames=1, window_frames=3)
+    ps = PairedStream(seed=1301, **cfg)
+    c = ps.cfg
+    for step in range(c.sink_frames + c.window_frames + 1):
+        ps.step_idx = step
+        f0 = ps.advance()
+        for layer in range(c.layers):
+            _, k, v = ps.inputs(layer)
+            ps.append(layer, f0, k, v)
+    rows = np.arange(0, c.chunk_tokens, 97)
+    qs = [ps.inputs(layer)[0] for layer in range(c.layers)]
+    wants = [O.chunk_attention(ps.ora, layer, synth.bf16_bits(qs[layer]), f0, 1.0 / math.sqrt(c.head_dim), rows=rows)
+             for layer in range(c.layers)]
+    outs = [torch.zeros((c.batch, c.chunk_tokens, c.heads, c.head_dim), dtype=torch.bfloat16, device="cuda")
+            for _ in range(6)]
+    qd = [q.cuda() for q in qs]
+    for i, out in enumerate(outs):                    # no synchronisation between the calls
+        ps.gpu.chunk_attention(i % c.layers, qd[i % c.layers], out, f0)
+    torch.cuda.synchronize()
+    for i, out in enumerate(outs):
+        mx, mean = attn_errors(out, wants[i % c.layers], rows)
+        assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS, (i, mx, mean)
+        assert torch.equal(out, outs[i % c.layers])
