@@ -324,24 +324,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (lane == 0 && n_local > 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kBlockN, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, D, 0, 1);
-            const uint32_t q_base = smem_addr(smem + L::kQ);
-            const uint32_t k_base = smem_addr(smem + L::kK);
-            const uint32_t v_base = smem_addr(smem + L::kV);
+            // Descriptors are built once; each MMA only adds a constant to the start-address
+            // field (bits 0..13, address >> 4; every operand lies below 256 KB, so no carry
+            // leaves the field).  This keeps the issuing thread's instruction count low: it
+            // shares its SM sub-partition with busy softmax warps.
+            const uint64_t dq = smem_desc_sw128(smem_addr(smem + L::kQ), 16, 1024);
+            const uint64_t dk = smem_desc_sw128(smem_addr(smem + L::kK), 16, 1024);
+            const uint64_t dv = smem_desc_sw128(smem_addr(smem + L::kV), L::kSub, 1024);
             auto issue_qk = [&](int t, int st) {
+                const uint64_t a0 = dq + static_cast<uint64_t>(t * (L::kQTile >> 4));
+                const uint64_t b0 = dk + static_cast<uint64_t>(st * (L::kKVTile >> 4));
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * L::kSub + (kk & 3) * 32;
-                    const uint64_t a = smem_desc_sw128(q_base + t * L::kQTile + off, 16, 1024);
-                    const uint64_t b = smem_desc_sw128(k_base + st * L::kKVTile + off, 16, 1024);
-                    umma_ss(tmem + t * 128, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+                    const uint64_t off = static_cast<uint64_t>(((kk >> 2) * L::kSub + (kk & 3) * 32) >> 4);
+                    umma_ss(tmem + t * 128, a0 + off, b0 + off, idesc_qk, kk > 0 ? 1u : 0u);
                 }
             };
             auto issue_pv = [&](int t, int st, bool acc) {
+                const uint64_t b0 = dv + static_cast<uint64_t>(st * (L::kKVTile >> 4));
 #pragma unroll
-                for (int kk = 0; kk < kBlockN / 16; ++kk) {
-                    const uint64_t b = smem_desc_sw128(v_base + st * L::kKVTile + kk * 2048, L::kSub, 1024);
-                    umma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, b, idesc_pv, (acc || kk > 0) ? 1u : 0u);
-                }
+                for (int kk = 0; kk < kBlockN / 16; ++kk)
+                    umma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, b0 + static_cast<uint64_t>((kk * 2048) >> 4),
+                            idesc_pv, (acc || kk > 0) ? 1u : 0u);
             };
             bool ok = mbar_wait(&bars[L::kQFull], 0, abort_flag, p.status, kStatusMmaWait);
             if (ok) {
