@@ -79,12 +79,14 @@ def test_multi_tile_ragged_split_path():
 
 
 def test_many_heads_unsplit_path():
+    # 37 heads x 4 query-tile pairs = 148 CTAs, one full wave: no KV split
     from causal_dit_kv_b200 import binding as B
-    cfg = dict(batch=2, layers=1, heads=40, head_dim=128, frame_h=16, frame_w=16, chunk_frames=1, sink_frames=1,
-               window_frames=3)
+    cfg = dict(batch=1, layers=1, heads=37, head_dim=128, frame_h=32, frame_w=32, chunk_frames=1, sink_frames=1,
+               window_frames=1)
     ps = PairedStream(seed=1004, **cfg)
-    assert B.sdv2_attention_splits(ps.gpu.cfg, [1024, 1024], 148) == 1
-    _stream_and_check(ps, 5)
+    assert B.sdv2_attention_splits(ps.gpu.cfg, [2048], 148) == 1
+    rows = np.sort(np.random.default_rng(4).choice(1024, 48, replace=False))
+    _stream_and_check(ps, 4, attn_rows=rows)
 
 
 def test_window_equals_chunk_and_reset_every_frame():
@@ -180,10 +182,13 @@ def test_back_to_back_attention_calls(splits):
         cfg = dict(batch=1, layers=2, heads=12, head_dim=128, frame_h=32, frame_w=32, chunk_frames=1,
                    sink_frames=1, window_frames=6)
     else:
-        cfg = dict(batch=2, layers=2, heads=40, head_dim=128, frame_h=16, frame_w=16, chunk_frames=1,
-                   sink_frames=1, window_frames=3)
+        cfg = dict(batch=1, layers=2, heads=37, head_dim=128, frame_h=32, frame_w=32, chunk_frames=1,
+                   sink_frames=1, window_frames=1)
     ps = PairedStream(seed=1301, **cfg)
     c = ps.cfg
+    from causal_dit_kv_b200 import binding as B
+    n_split = B.sdv2_attention_splits(ps.gpu.cfg, [(c.sink_frames + c.window_frames) * c.frame_h * c.frame_w], 148)
+    assert (n_split > 1) == (splits == "split")
     for step in range(c.sink_frames + c.window_frames + 1):
         ps.step_idx = step
         f0 = ps.advance()
