@@ -530,6 +530,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                     make_float4(__uint_as_float(r[cb][4 * v]), __uint_as_float(r[cb][4 * v + 1]),
                                                 __uint_as_float(r[cb][4 * v + 2]), __uint_as_float(r[cb][4 * v + 3]));
                     }
+                } else if (valid) {                         // no keys in this split: zero partial
+                    float4 *po = reinterpret_cast<float4 *>(p.part_o) + (split * n_groups + group) * (D / 4) * 256 + srow;
+#pragma unroll
+                    for (int c = 0; c < D / 4; ++c) po[c * 256] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
                 }
                 if (valid)
                     reinterpret_cast<float2 *>(p.part_ml)[((static_cast<int64_t>(split) * p.batch + bg) * p.heads + h) *
@@ -549,20 +553,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 }
 
 // Merge of the KV-split partials: out = sum_s 2^(m_s - m) O_s / sum_s 2^(m_s - m) l_s.
-// Thread = (row, 8 float4 columns) of one (stream, head, query-tile pair) block:
+// Thread = (row, 4 float4 columns) of one (stream, head, query-tile pair) block:
 // consecutive threads take consecutive rows, so every load of a split's column
-// is coalesced, and all splits' loads of a thread are in flight together.
+// is coalesced.  Every split's (max, sum) and columns are loaded unconditionally
+// (a split CTA without keys writes zeros), so all of a thread's loads are in
+// flight at once; the partials are read once (evict-first loads).
 template <int D>
 __global__ void __launch_bounds__(256) attention_combine_kernel(const __grid_constant__ AttnParams p) {
     grid_dependency_wait();                         // the split CTAs' partials
     grid_launch_dependents();
-    constexpr int kC8 = D / 32;                     // 8-column chunks per row
+    constexpr int kC16 = D / 16;                    // 16-column chunks per row
     const int64_t n_groups = static_cast<int64_t>(p.batch) * p.heads * p.n_qpairs;
     const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int srow = static_cast<int>(idx & 255);
     const int64_t rest = idx >> 8;
-    const int c8 = static_cast<int>(rest % kC8);
-    const int64_t gl = rest / kC8;                  // group within this launch's streams
+    const int c16 = static_cast<int>(rest % kC16);
+    const int64_t gl = rest / kC16;                 // group within this launch's streams
     const int64_t per_stream = static_cast<int64_t>(p.heads) * p.n_qpairs;
     const int bl = static_cast<int>(gl / per_stream);
     if (bl >= kMaxBatch || p.lk[bl] <= 0) return;
@@ -573,36 +579,33 @@ __global__ void __launch_bounds__(256) attention_combine_kernel(const __grid_con
     if (token >= p.lq) return;
     const int64_t group = (static_cast<int64_t>(bg) * p.heads + h) * p.n_qpairs + qpair;
     float2 ml[kMaxSplits];
-    float m = -INFINITY;
+    float4 u[kMaxSplits][4];
 #pragma unroll
     for (int s = 0; s < kMaxSplits; ++s) {
         ml[s] = make_float2(-INFINITY, 0.0f);
-        if (s < p.n_split)
-            ml[s] = reinterpret_cast<const float2 *>(p.part_ml)[((static_cast<int64_t>(s) * p.batch + bg) * p.heads + h) *
-                                                                     p.lq_pad + token];
-        m = fmaxf(m, ml[s].x);
-    }
-    float4 u[kMaxSplits][8];
-#pragma unroll
-    for (int s = 0; s < kMaxSplits; ++s) {
-        if (s < p.n_split && ml[s].x != -INFINITY) {
+        if (s < p.n_split) {
+            ml[s] = __ldcs(reinterpret_cast<const float2 *>(p.part_ml) +
+                           ((static_cast<int64_t>(s) * p.batch + bg) * p.heads + h) * p.lq_pad + token);
             const float4 *po = reinterpret_cast<const float4 *>(p.part_o) + (s * n_groups + group) * (D / 4) * 256 +
-                               (c8 * 8) * 256 + srow;
+                               (c16 * 4) * 256 + srow;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) u[s][i] = po[i * 256];
+            for (int i = 0; i < 4; ++i) u[s][i] = __ldcs(po + i * 256);
         }
     }
-    float a[32];
+    float m = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) a[i] = 0.0f;
+    for (int s = 0; s < kMaxSplits; ++s) m = fmaxf(m, ml[s].x);
+    float a[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a[i] = 0.0f;
     float l = 0.0f;
 #pragma unroll
     for (int s = 0; s < kMaxSplits; ++s) {
-        if (s < p.n_split && ml[s].x != -INFINITY) {
-            const float w = exp2f(ml[s].x - m);
+        if (s < p.n_split) {
+            const float w = ml[s].x == -INFINITY ? 0.0f : exp2f(ml[s].x - m);
             l += w * ml[s].y;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int i = 0; i < 4; ++i) {
                 a[4 * i] += w * u[s][i].x;
                 a[4 * i + 1] += w * u[s][i].y;
                 a[4 * i + 2] += w * u[s][i].z;
@@ -611,9 +614,9 @@ __global__ void __launch_bounds__(256) attention_combine_kernel(const __grid_con
         }
     }
     const float inv = 1.0f / l;
-    uint16_t *orow = p.out + ((static_cast<int64_t>(bg) * p.lq + token) * p.heads + h) * D + c8 * 32;
+    uint16_t *orow = p.out + ((static_cast<int64_t>(bg) * p.lq + token) * p.heads + h) * D + c16 * 16;
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
+    for (int v = 0; v < 2; ++v) {
         uint4 w;
         w.x = pack_bf16x2(a[8 * v + 0] * inv, a[8 * v + 1] * inv);
         w.y = pack_bf16x2(a[8 * v + 2] * inv, a[8 * v + 3] * inv);
@@ -674,7 +677,7 @@ cudaError_t launch_combine(const AttnParams &p, int head_dim, cudaStream_t s) {
     for (int i = 0; i < kMaxBatch; ++i)
         if (p.lk[i] > 0) nb = i + 1;
     if (nb == 0 || p.n_split <= 1) return cudaSuccess;
-    const int64_t threads = static_cast<int64_t>(nb) * p.heads * p.n_qpairs * (head_dim / 32) * 256;
+    const int64_t threads = static_cast<int64_t>(nb) * p.heads * p.n_qpairs * (head_dim / 16) * 256;
     const dim3 grid(static_cast<unsigned>((threads + 255) / 256));
     if (head_dim == 64) return launch_dependent(attention_combine_kernel<64>, grid, dim3(256), 0, s, p);
     return launch_dependent(attention_combine_kernel<128>, grid, dim3(256), 0, s, p);
