@@ -59,7 +59,8 @@ __global__ void __launch_bounds__(128) kv_append_kernel(const __grid_constant__ 
     __shared__ double2 s_tab[64];                    // temporal (cos, sin) of this block's frame
     if (!is_v) {
         if (threadIdx.x < p.n_t)
-            s_tab[threadIdx.x] = make_double2(p.tab_t[fi * p.n_t + threadIdx.x][0], p.tab_t[fi * p.n_t + threadIdx.x][1]);
+            s_tab[threadIdx.x] = make_double2(p.tab_t[p.tab_row[fi] * p.n_t + threadIdx.x][0],
+                                              p.tab_t[p.tab_row[fi] * p.n_t + threadIdx.x][1]);
         __syncthreads();
     }
     const int rows = static_cast<int>(p.frame_elems / p.head_dim);     // N * H

@@ -29,6 +29,11 @@
 // (and O is rescaled in TMEM) when a tile's max exceeds it by more than 8,
 // so P stays <= 256.  The exponent arguments and row sums use packed f32x2
 // arithmetic.
+// A CTA whose query-tile pair holds a single tile (chunks of <= 128 queries,
+// or the last pair of a ragged chunk) runs the same pipeline with both
+// accumulator sets on that tile: even KV tiles go to S_0/O_0, odd ones to
+// S_1/O_1, so the softmax of one still overlaps the MMAs of the other; the
+// two partial results are merged in the epilogue.
 // Q: rope_q_kernel rotates the chunk's queries once per call (fp32 RoPE,
 // rounded to bf16) into a scratch buffer; the producer warp TMA-loads the
 // rotated tiles straight into the 128-byte-swizzled K-major layout the MMA
@@ -78,20 +83,6 @@ int attention_smem_bytes(int head_dim) {
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale only when the max grows by > 2^8
 
-// fp32 (cos, sin) of rotation pair j for a query token.
-__device__ __forceinline__ float2 q_cos_sin(const AttnParams &p, int bl, int fi, int row, int col, int j) {
-    if (j < p.n_t) {
-        const int e = (bl * p.chunk_frames + fi) * p.n_t + j;
-        return make_float2(p.tab_t[e][0], p.tab_t[e][1]);
-    }
-    if (j < p.n_t + p.n_h) {
-        const float *t = p.rope_h + 2 * (row * p.n_h + (j - p.n_t));
-        return make_float2(t[0], t[1]);
-    }
-    const float *t = p.rope_w + 2 * (col * p.n_w + (j - p.n_t - p.n_h));
-    return make_float2(t[0], t[1]);
-}
-
 // All 32 lanes wait; the warp proceeds only if every lane saw the phase
 // complete, so the .sync.aligned tcgen05 ops that follow stay warp-uniform.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile uint32_t *abort, uint32_t *status,
@@ -103,7 +94,9 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
 // RoPE of the chunk's queries: q_rot = rotate(q) at (phase(frame), row, col),
 // fp32 arithmetic, bf16 result.  Block = 64 (token, head) rows of one stream,
 // 4 threads per row, every 4th 16-byte vector of the row per thread (loads
-// first).  grid = (row blocks, streams of the launch).
+// first).  grid = (row blocks, streams of the launch).  The temporal angles
+// phase * base^(-j / n_t) of the stream's chunk frames are evaluated in fp64
+// by each block and rounded to fp32, like the row and column tables.
 __global__ void __launch_bounds__(256) rope_q_kernel(const __grid_constant__ AttnParams p, int head_dim) {
     // Launched right behind the KV append, whose own wait already ordered it after
     // the producer of q: q can be read at once.  Completing only after the append
@@ -112,8 +105,13 @@ __global__ void __launch_bounds__(256) rope_q_kernel(const __grid_constant__ Att
     const int bl = blockIdx.y;
     __shared__ float2 s_tab[kAttnTabEntries];        // temporal (cos, sin) of this stream's frames
     for (int e = threadIdx.x; e < p.chunk_frames * p.n_t; e += blockDim.x) {
-        const int src = bl * p.chunk_frames * p.n_t + e;
-        s_tab[e] = make_float2(p.tab_t[src][0], p.tab_t[src][1]);
+        const int fi = e / p.n_t, j = e - fi * p.n_t;
+        const int64_t f = p.f0[bl] + fi;
+        const int64_t ph = p.rope_reset > 0 ? f % p.rope_reset : f;
+        const double a = static_cast<double>(ph) * pow(p.rope_base, -static_cast<double>(j) / static_cast<double>(p.n_t));
+        double sn, cs;
+        sincos(a, &sn, &cs);
+        s_tab[e] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
     }
     __syncthreads();
     const int rows = p.lq * p.heads;
@@ -195,6 +193,25 @@ __device__ __forceinline__ float softmax_exp_store(const uint32_t (&sr)[kBlockN 
     return a0 + a1;
 }
 
+// Single-tile mode: 32 columns of w0 O_0 + w1 O_1 for this thread's row, as
+// fp32 bits in r0 (O_1 is read only if its set received keys).
+__device__ __forceinline__ void merge_sets(uint32_t o0, uint32_t o1, bool has1, float w0, float w1,
+                                           uint32_t (&r0)[32]) {
+    uint32_t r1[32];
+    tmem_ld32(o0, r0);
+    if (has1) {
+        tmem_ld32(o1, r1);
+        tmem_wait_ld_bind(r0);
+        reg_bind(r1);
+    } else {
+        tmem_wait_ld_bind(r0);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) r1[i] = 0u;
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) r0[i] = __float_as_uint(w0 * __uint_as_float(r0[i]) + w1 * __uint_as_float(r1[i]));
+}
+
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     chunk_attention_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
@@ -223,6 +240,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int n_local = kv_end > kv_begin ? kv_end - kv_begin : 0;
     const int q_row0 = qpair * (kBlockM * kQTilesPerCta);
     const int n_qt = (q_row0 + kBlockM < p.lq) ? 2 : 1;
+    const bool dual = n_qt == 1;                // one query tile: the two accumulator sets split the KV tiles
 
     if (threadIdx.x == 0) {
         mbar_init(&bars[L::kQFull], 1);
@@ -332,7 +350,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const uint64_t dk = smem_desc_sw128(smem_addr(smem + L::kK), 16, 1024);
             const uint64_t dv = smem_desc_sw128(smem_addr(smem + L::kV), L::kSub, 1024);
             auto issue_qk = [&](int t, int st) {
-                const uint64_t a0 = dq + static_cast<uint64_t>(t * (L::kQTile >> 4));
+                const uint64_t a0 = dq + static_cast<uint64_t>((dual ? 0 : t) * (L::kQTile >> 4));
                 const uint64_t b0 = dk + static_cast<uint64_t>(st * (L::kKVTile >> 4));
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
@@ -348,6 +366,42 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                             idesc_pv, (acc || kk > 0) ? 1u : 0u);
             };
             bool ok = mbar_wait(&bars[L::kQFull], 0, abort_flag, p.status, kStatusMmaWait);
+            if (dual) {
+                // KV tile i -> accumulator set i & 1.  Prologue: S_0 = Q K_0^T, S_1 = Q K_1^T.
+                for (int i = 0; ok && i < n_local && i < 2; ++i) {
+                    ok = mbar_wait(&bars[L::kKFull + i % L::kKStages], (i / L::kKStages) & 1, abort_flag, p.status,
+                                   kStatusMmaWait);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_qk(i, i % L::kKStages);
+                    umma_commit(&bars[L::kSFull + i]);
+                    umma_commit(&bars[L::kKEmpty + i % L::kKStages]);
+                }
+                for (int i = 0; ok && i < n_local; ++i) {
+                    const int t = i & 1;
+                    const int st = i % L::kVStages;
+                    if (!mbar_wait(&bars[L::kVFull + st], (i / L::kVStages) & 1, abort_flag, p.status, kStatusMmaWait))
+                        break;
+                    if (!mbar_wait(&bars[L::kPFull + t], (i >> 1) & 1, abort_flag, p.status, kStatusMmaWait)) break;
+                    tc_fence_after();
+                    issue_pv(t, st, i >= 2);
+                    umma_commit(&bars[L::kVEmpty + st]);
+                    const int nk = i + 2;
+                    if (nk < n_local) {
+                        const int kst = nk % L::kKStages;
+                        if (!mbar_wait(&bars[L::kKFull + kst], (nk / L::kKStages) & 1, abort_flag, p.status,
+                                       kStatusMmaWait))
+                            break;
+                        tc_fence_after();
+                        issue_qk(t, kst);
+                        umma_commit(&bars[L::kSFull + t]);
+                        umma_commit(&bars[L::kKEmpty + kst]);
+                    } else {
+                        umma_commit(&bars[L::kOFull + t]);
+                    }
+                }
+                ok = false;                              // the two-tile schedule below is skipped
+            }
             if (ok) {
                 tc_fence_after();
                 ok = mbar_wait(&bars[L::kKFull + 0], 0, abort_flag, p.status, kStatusMmaWait);
@@ -410,15 +464,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int t = (warp - 4) >> 2;               // query tile of this warpgroup
         const int row = ((warp & 3) << 5) + lane;    // TMEM lane == query row in the tile
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) << 5) << 16;
-        if (t < n_qt) {
-            const int token = q_row0 + t * kBlockM + row;
+        if (t < n_qt || dual) {
+            // in the single-tile mode, tile 1's warps take the odd KV tiles of tile 0's rows
+            const int token = q_row0 + (dual ? 0 : t) * kBlockM + row;
             const bool valid = token < p.lq;
+            const int n_mine = dual ? (n_local + 1 - t) / 2 : n_local;
             float m_run = -INFINITY;   // running max of scale*log2(e)*s
             float l_run = 0.0f;
             bool ok = true;
             const uint32_t s_tmem = tmem + lane_base + t * 128;
             const uint32_t o_tmem = tmem + lane_base + 256 + t * 128;
-            for (int it = 0; it < n_local; ++it) {
+            for (int it = 0; it < n_mine; ++it) {
                 if (!warp_wait(&bars[L::kSFull + t], it & 1, abort_flag, p.status, kStatusSoftmaxWait)) {
                     ok = false;
                     break;
@@ -430,7 +486,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 tmem_wait_ld_bind(sr[0]);
 #pragma unroll
                 for (int cb = 1; cb < kBlockN / 32; ++cb) reg_bind(sr[cb]);
-                const int valid_cols = lk - (kv_begin + it) * kBlockN;
+                const int valid_cols = lk - (kv_begin + (dual ? 2 * it + t : it)) * kBlockN;
                 if (valid_cols < kBlockN) {
 #pragma unroll
                     for (int cb = 0; cb < kBlockN / 32; ++cb)
@@ -479,66 +535,136 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 mbar_arrive(&bars[L::kPFull + t]);
             }
 
-            // ---- epilogue
-            if (ok && n_local > 0) ok = warp_wait(&bars[L::kOFull + t], 0, abort_flag, p.status, kStatusSoftmaxWait);
-            const int prow_local = q_row0 + t * kBlockM + row;     // row index within the padded query range
-            if (ok) tc_fence_after();
-            if (p.n_split == 1) {
-                if (ok) {
-                    const float inv = 1.0f / l_run;
-                    uint16_t *orow = p.out + ((static_cast<int64_t>(bg) * p.lq + token) * p.heads + h) * D;
+            if (dual) {
+                // ---- single-tile epilogue: merge the two accumulator sets of the row; thread
+                // (t, row) produces output columns [t d/2, (t+1) d/2)
+                const int n0 = (n_local + 1) / 2, n1 = n_local / 2;
+                if (ok && n0 > 0) ok = warp_wait(&bars[L::kOFull + 0], 0, abort_flag, p.status, kStatusSoftmaxWait);
+                if (ok && n1 > 0) ok = warp_wait(&bars[L::kOFull + 1], 0, abort_flag, p.status, kStatusSoftmaxWait);
+                // (max, sum) of both sets through the unused second query-tile slot
+                float2 *xm = reinterpret_cast<float2 *>(smem + L::kQ + L::kQTile);
+                xm[t * kBlockM + row] = make_float2(n_mine > 0 ? m_run : -INFINITY, l_run);
+                ok = named_bar_and(1, 2 * 4 * 32, ok);
+                const float2 a0 = xm[row], a1 = xm[kBlockM + row];
+                const float m = fmaxf(a0.x, a1.x);
+                const float w0 = a0.x == -INFINITY ? 0.0f : ex2_approx(a0.x - m);
+                const float w1 = a1.x == -INFINITY ? 0.0f : ex2_approx(a1.x - m);
+                const float l = w0 * a0.y + w1 * a1.y;
+                if (ok) tc_fence_after();
+                const uint32_t o0 = tmem + lane_base + 256 + t * (D / 2);
+                const uint32_t o1 = o0 + 128;
+                if (p.n_split == 1) {
+                    if (ok) {
+                        const float inv = 1.0f / l;
+                        uint16_t *orow =
+                            p.out + ((static_cast<int64_t>(bg) * p.lq + token) * p.heads + h) * D + t * (D / 2);
+#pragma unroll 1
+                        for (int cb = 0; cb < D / 64; ++cb) {
+                            uint32_t v[32];
+                            merge_sets(o0 + cb * 32, o1 + cb * 32, n1 > 0, w0, w1, v);
+                            if (valid) {
 #pragma unroll
-                    for (int cb = 0; cb < D / 32; ++cb) {
-                        uint32_t r[32];
-                        tmem_ld32(o_tmem + cb * 32, r);
-                        tmem_wait_ld_bind(r);
-                        if (valid) {
-#pragma unroll
-                            for (int v = 0; v < 4; ++v) {
-                                uint4 w;
-                                w.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]) * inv, __uint_as_float(r[8 * v + 1]) * inv);
-                                w.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]) * inv, __uint_as_float(r[8 * v + 3]) * inv);
-                                w.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]) * inv, __uint_as_float(r[8 * v + 5]) * inv);
-                                w.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]) * inv, __uint_as_float(r[8 * v + 7]) * inv);
-                                *reinterpret_cast<uint4 *>(orow + cb * 32 + v * 8) = w;
+                                for (int q = 0; q < 4; ++q) {
+                                    uint4 w;
+                                    w.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]) * inv, __uint_as_float(v[8 * q + 1]) * inv);
+                                    w.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]) * inv, __uint_as_float(v[8 * q + 3]) * inv);
+                                    w.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]) * inv, __uint_as_float(v[8 * q + 5]) * inv);
+                                    w.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]) * inv, __uint_as_float(v[8 * q + 7]) * inv);
+                                    *reinterpret_cast<uint4 *>(orow + cb * 32 + q * 8) = w;
+                                }
                             }
                         }
                     }
-                }
-            } else if (ok) {
-                // ---- KV split: write this split's unnormalised partial for attention_combine_kernel.
-                // part_o: one block per (split, stream, head, query-tile pair) of [D/4 float4
-                // columns][256 rows] (rows t*128 + lane; a warp's 32 rows are 512 contiguous
-                // bytes); part_ml[(split*B + b)*H + h][lq_pad] float2 = (row max in log2 units, sum).
-                const int64_t group = (static_cast<int64_t>(bg) * p.heads + h) * p.n_qpairs + qpair;
-                const int64_t n_groups = static_cast<int64_t>(p.batch) * p.heads * p.n_qpairs;
-                const int srow = t * kBlockM + row;
-                if (n_local > 0) {                         // warp-uniform: every lane takes part in tcgen05.ld
-                    float4 *po = reinterpret_cast<float4 *>(p.part_o) + (split * n_groups + group) * (D / 4) * 256 + srow;
-                    uint32_t r[D / 32][32];
+                } else if (ok) {
+                    // KV split: this split's merged, unnormalised partial (layout as below)
+                    const int64_t group = (static_cast<int64_t>(bg) * p.heads + h) * p.n_qpairs + qpair;
+                    const int64_t n_groups = static_cast<int64_t>(p.batch) * p.heads * p.n_qpairs;
+                    float4 *po = reinterpret_cast<float4 *>(p.part_o) + (split * n_groups + group) * (D / 4) * 256 +
+                                 t * (D / 8) * 256 + row;
+                    if (n_local > 0) {
+#pragma unroll 1
+                        for (int cb = 0; cb < D / 64; ++cb) {
+                            uint32_t v[32];
+                            merge_sets(o0 + cb * 32, o1 + cb * 32, n1 > 0, w0, w1, v);
+                            if (valid) {
 #pragma unroll
-                    for (int cb = 0; cb < D / 32; ++cb) tmem_ld32(o_tmem + cb * 32, r[cb]);
-                    tmem_wait_ld_bind(r[0]);
+                                for (int q = 0; q < 8; ++q)
+                                    po[(cb * 8 + q) * 256] =
+                                        make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                                    __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+                            }
+                        }
+                    } else if (valid) {
 #pragma unroll
-                    for (int cb = 1; cb < D / 32; ++cb) reg_bind(r[cb]);
-                    if (valid) {
-#pragma unroll
-                        for (int cb = 0; cb < D / 32; ++cb)
-#pragma unroll
-                            for (int v = 0; v < 8; ++v)
-                                po[(cb * 8 + v) * 256] =
-                                    make_float4(__uint_as_float(r[cb][4 * v]), __uint_as_float(r[cb][4 * v + 1]),
-                                                __uint_as_float(r[cb][4 * v + 2]), __uint_as_float(r[cb][4 * v + 3]));
+                        for (int c = 0; c < D / 8; ++c) po[c * 256] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
                     }
-                } else if (valid) {                         // no keys in this split: zero partial
-                    float4 *po = reinterpret_cast<float4 *>(p.part_o) + (split * n_groups + group) * (D / 4) * 256 + srow;
-#pragma unroll
-                    for (int c = 0; c < D / 4; ++c) po[c * 256] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                    if (valid && t == 0)
+                        reinterpret_cast<float2 *>(p.part_ml)[((static_cast<int64_t>(split) * p.batch + bg) * p.heads + h) *
+                                                                  p.lq_pad + q_row0 + row] =
+                            make_float2(n_local > 0 ? m : -INFINITY, l);
                 }
-                if (valid)
-                    reinterpret_cast<float2 *>(p.part_ml)[((static_cast<int64_t>(split) * p.batch + bg) * p.heads + h) *
-                                                              p.lq_pad + prow_local] =
-                        make_float2(n_local > 0 ? m_run : -INFINITY, l_run);
+            } else {
+                // ---- epilogue
+                if (ok && n_local > 0) ok = warp_wait(&bars[L::kOFull + t], 0, abort_flag, p.status, kStatusSoftmaxWait);
+                const int prow_local = q_row0 + t * kBlockM + row;     // row index within the padded query range
+                if (ok) tc_fence_after();
+                if (p.n_split == 1) {
+                    if (ok) {
+                        const float inv = 1.0f / l_run;
+                        uint16_t *orow = p.out + ((static_cast<int64_t>(bg) * p.lq + token) * p.heads + h) * D;
+#pragma unroll
+                        for (int cb = 0; cb < D / 32; ++cb) {
+                            uint32_t r[32];
+                            tmem_ld32(o_tmem + cb * 32, r);
+                            tmem_wait_ld_bind(r);
+                            if (valid) {
+#pragma unroll
+                                for (int v = 0; v < 4; ++v) {
+                                    uint4 w;
+                                    w.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]) * inv, __uint_as_float(r[8 * v + 1]) * inv);
+                                    w.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]) * inv, __uint_as_float(r[8 * v + 3]) * inv);
+                                    w.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]) * inv, __uint_as_float(r[8 * v + 5]) * inv);
+                                    w.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]) * inv, __uint_as_float(r[8 * v + 7]) * inv);
+                                    *reinterpret_cast<uint4 *>(orow + cb * 32 + v * 8) = w;
+                                }
+                            }
+                        }
+                    }
+                } else if (ok) {
+                    // ---- KV split: write this split's unnormalised partial for attention_combine_kernel.
+                    // part_o: one block per (split, stream, head, query-tile pair) of [D/4 float4
+                    // columns][256 rows] (rows t*128 + lane; a warp's 32 rows are 512 contiguous
+                    // bytes); part_ml[(split*B + b)*H + h][lq_pad] float2 = (row max in log2 units, sum).
+                    const int64_t group = (static_cast<int64_t>(bg) * p.heads + h) * p.n_qpairs + qpair;
+                    const int64_t n_groups = static_cast<int64_t>(p.batch) * p.heads * p.n_qpairs;
+                    const int srow = t * kBlockM + row;
+                    if (n_local > 0) {                         // warp-uniform: every lane takes part in tcgen05.ld
+                        float4 *po = reinterpret_cast<float4 *>(p.part_o) + (split * n_groups + group) * (D / 4) * 256 + srow;
+                        uint32_t r[D / 32][32];
+#pragma unroll
+                        for (int cb = 0; cb < D / 32; ++cb) tmem_ld32(o_tmem + cb * 32, r[cb]);
+                        tmem_wait_ld_bind(r[0]);
+#pragma unroll
+                        for (int cb = 1; cb < D / 32; ++cb) reg_bind(r[cb]);
+                        if (valid) {
+#pragma unroll
+                            for (int cb = 0; cb < D / 32; ++cb)
+#pragma unroll
+                                for (int v = 0; v < 8; ++v)
+                                    po[(cb * 8 + v) * 256] =
+                                        make_float4(__uint_as_float(r[cb][4 * v]), __uint_as_float(r[cb][4 * v + 1]),
+                                                    __uint_as_float(r[cb][4 * v + 2]), __uint_as_float(r[cb][4 * v + 3]));
+                        }
+                    } else if (valid) {                         // no keys in this split: zero partial
+                        float4 *po = reinterpret_cast<float4 *>(p.part_o) + (split * n_groups + group) * (D / 4) * 256 + srow;
+#pragma unroll
+                        for (int c = 0; c < D / 4; ++c) po[c * 256] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                    }
+                    if (valid)
+                        reinterpret_cast<float2 *>(p.part_ml)[((static_cast<int64_t>(split) * p.batch + bg) * p.heads + h) *
+                                                                  p.lq_pad + prow_local] =
+                            make_float2(n_local > 0 ? m_run : -INFINITY, l_run);
+                }
             }
         }
     }

@@ -73,6 +73,7 @@ double rope_angle(double base, int j, int n, int64_t pos) {
 struct Geometry {
     int64_t N, slots, lq, frame_elems, layer_elems;
     int n_qpairs, lq_pad;
+    int refresh_chunks;  // token chunks of the refresh reduction
     int64_t part_rows;  // capacity of the split-KV partial buffer, rows of d floats
     // region offsets
     uint64_t rope_h64, rope_w64, rope_h32, rope_w32;
@@ -153,10 +154,16 @@ Geometry geometry(const sdv2_cache_config &c) {
     g.status = off;
     off = align_up(off + 4, 256);
     g.scratch = off;
+    // token chunks of the chunk-mean reduction: about two blocks per SM of a 148-SM GPU
+    {
+        const int col_blocks = std::max(1, (c.embed_dim + 255) / 256);
+        const int want = (296 + col_blocks * c.batch - 1) / (col_blocks * c.batch);
+        g.refresh_chunks = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>({kRefreshMaxChunks, want, g.lq})));
+    }
     g.refresh_mean = off;
-    off = align_up(off + 8ull * c.batch * kRefreshRowChunks * (c.embed_dim > 0 ? c.embed_dim : 1), 256);
+    off = align_up(off + 8ull * c.batch * g.refresh_chunks * (c.embed_dim > 0 ? c.embed_dim : 1), 256);
     g.refresh_counter = off;
-    off = align_up(off + 4ull * c.batch, 256);
+    off = align_up(off + 4ull * (kMaxBatch + static_cast<uint64_t>(c.batch) * kRefreshMaxColBlocks), 256);
     // two buffers of rotated queries, used by alternate attention calls: a call's RoPE
     // pass may then start before the previous call's attention kernel has finished
     g.q_rot = off;
@@ -424,7 +431,9 @@ sdv2_status sdv2_kv_append(sdv2_cache *c, int32_t layer, const void *k, const vo
     if ((st = check_device(c->device)) != SDV2_OK) return st;
     const sdv2_cache_config &n = c->cfg;
     const int n_t = n.rope_pairs[0];
-    const int per_launch = std::min(kAppendMaxFrames, kAppendTabEntries / n_t);
+    const int max_rows = kAppendTabEntries / n_t;     // distinct phases per launch
+    int64_t row_phase[kAppendTabEntries];
+    int n_rows = 0;
     AppendParams p;
     std::memset(&p, 0, sizeof(p));
     p.k_in = static_cast<const uint16_t *>(k);
@@ -448,6 +457,7 @@ sdv2_status sdv2_kv_append(sdv2_cache *c, int32_t layer, const void *k, const vo
         if (e != cudaSuccess) return cuda_fail(e, "kv_append launch");
         g_launches.fetch_add(1);
         p.n_frames = 0;
+        n_rows = 0;
         return SDV2_OK;
     };
     for (int b = 0; b < n.batch; ++b) {
@@ -455,18 +465,30 @@ sdv2_status sdv2_kv_append(sdv2_cache *c, int32_t layer, const void *k, const vo
         if (f0 < 0) continue;
         for (int i = 0; i < n.chunk_frames; ++i) {
             const int64_t f = f0 + i;
+            const int64_t ph = phase_of(f, n.rope_reset_period);
+            // streams at the same phase share one row of the temporal table
+            int row = 0;
+            while (row < n_rows && row_phase[row] != ph) ++row;
+            if (row == n_rows) {
+                if (n_rows == max_rows) {
+                    if ((st = flush()) != SDV2_OK) return st;
+                    row = 0;
+                }
+                row_phase[row] = ph;
+                for (int j = 0; j < n_t; ++j) {
+                    const double a = rope_angle(n.rope_base, j, n_t, ph);
+                    p.tab_t[row * n_t + j][0] = std::cos(a);
+                    p.tab_t[row * n_t + j][1] = std::sin(a);
+                }
+                n_rows = row + 1;
+            }
             const int fi = p.n_frames;
             p.src_b[fi] = b;
             p.src_i[fi] = i;
             p.dst_slot[fi] = slot_of(f, n.sink_frames, n.window_frames);
-            const int64_t ph = phase_of(f, n.rope_reset_period);
-            for (int j = 0; j < n_t; ++j) {
-                const double a = rope_angle(n.rope_base, j, n_t, ph);
-                p.tab_t[fi * n_t + j][0] = std::cos(a);
-                p.tab_t[fi * n_t + j][1] = std::sin(a);
-            }
+            p.tab_row[fi] = static_cast<uint8_t>(row);
             ++p.n_frames;
-            if (p.n_frames == per_launch && (st = flush()) != SDV2_OK) return st;
+            if (p.n_frames == kAppendMaxFrames && (st = flush()) != SDV2_OK) return st;
         }
     }
     if ((st = flush()) != SDV2_OK) return st;
@@ -497,7 +519,7 @@ sdv2_status sdv2_chunk_attention(sdv2_cache *c, int32_t layer, const void *q, vo
     }
     const int n_split = plan_splits(n, g, keys.data(), c->sm_count);
     const int n_t = n.rope_pairs[0];
-    const int streams_per_launch = std::min(kMaxBatch, kAttnTabEntries / (n_t * n.chunk_frames));
+    const int streams_per_launch = kMaxBatch;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     AttnParams p;
     std::memset(&p, 0, sizeof(p));
@@ -523,6 +545,8 @@ sdv2_status sdv2_chunk_attention(sdv2_cache *c, int32_t layer, const void *q, vo
     p.n_qpairs = g.n_qpairs;
     p.n_split = n_split;
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.rope_base = n.rope_base;
+    p.rope_reset = n.rope_reset_period;
     for (int b0 = 0; b0 < n.batch; b0 += streams_per_launch) {
         const int nb = std::min(streams_per_launch, n.batch - b0);
         p.b_offset = b0;
@@ -531,17 +555,8 @@ sdv2_status sdv2_chunk_attention(sdv2_cache *c, int32_t layer, const void *q, vo
         for (int bl = 0; bl < nb; ++bl) {
             const int b = b0 + bl;
             p.lk[bl] = static_cast<int32_t>(keys[b]);
-            if (keys[b] <= 0) continue;
-            any = true;
-            const int64_t f0 = chunk_first_frame[b];
-            for (int fi = 0; fi < n.chunk_frames; ++fi) {
-                const int64_t ph = phase_of(f0 + fi, n.rope_reset_period);
-                for (int j = 0; j < n_t; ++j) {
-                    const double a = rope_angle(n.rope_base, j, n_t, ph);
-                    p.tab_t[(bl * n.chunk_frames + fi) * n_t + j][0] = static_cast<float>(std::cos(a));
-                    p.tab_t[(bl * n.chunk_frames + fi) * n_t + j][1] = static_cast<float>(std::sin(a));
-                }
-            }
+            p.f0[bl] = chunk_first_frame[b];
+            if (keys[b] > 0) any = true;
         }
         if (!any) continue;
         cudaError_t e = launch_rope_q(p, c->sm_count, s);
@@ -594,6 +609,7 @@ sdv2_status sdv2_sink_refresh(sdv2_cache *c, const void *hidden, float tau, cons
     p.sinks = n.sink_frames;
     p.slots = static_cast<int32_t>(g.slots);
     p.layers = n.layers;
+    p.row_chunks = g.refresh_chunks;
     p.tau = static_cast<double>(tau);
     for (int b = 0; b < n.batch; ++b) {
         const int64_t f0 = chunk_first_frame[b];
@@ -658,7 +674,8 @@ sdv2_status sdv2_cache_check(sdv2_cache *c) {
     if (word != 0) {
         // A block that gave up may have left the refresh ticket half counted: re-arm it.
         cudaMemset(c->base + c->g.status, 0, 4);
-        cudaMemset(c->base + c->g.refresh_counter, 0, 4ull * c->cfg.batch);
+        cudaMemset(c->base + c->g.refresh_counter, 0,
+                   4ull * (kMaxBatch + static_cast<uint64_t>(c->cfg.batch) * kRefreshMaxColBlocks));
         cudaDeviceSynchronize();
         return fail(SDV2_E_DEVICE, "device status 0x%x (a kernel gave up on a bounded wait)", word);
     }

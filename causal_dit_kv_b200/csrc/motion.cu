@@ -7,8 +7,10 @@
 // 0 < lambda < 1 between s_min and s_max).
 //
 // One launch per call.  Block (x, b) owns a contiguous slice of the latent
-// frame of stream b: it sums squared differences of that slice for every
-// frame of the chunk in fp64, writes one partial per frame, then overwrites
+// frame of stream b (2048 elements, read as 16-byte vectors when the frame
+// size and the latents allow it): it sums squared differences of that slice
+// for every frame of the chunk in fp64 (warp-shuffle, then fixed-order
+// reduction across warps), writes one partial per frame, then overwrites
 // the slice of the stored previous frame with the chunk's last frame (only
 // this block touches that slice, so no ordering across blocks is needed).
 // The last block of a stream to finish (counted with an atomic ticket) sums
@@ -32,15 +34,32 @@ __global__ void __launch_bounds__(kMotionThreads) motion_kernel(const __grid_con
 
     __shared__ double red[kMotionThreads / 32];
     __shared__ int is_last;
+    // 16-byte vectors when every frame starts on a 16-byte boundary (block slices are
+    // multiples of 2048 elements, so they do too)
+    const bool vec = (n & 3) == 0 && (reinterpret_cast<uintptr_t>(p.latents) & 15u) == 0;
 
     for (int t = 0; t < p.chunk_frames; ++t) {
         double acc = 0.0;
         if (t > 0 || had_prev) {
             const float *cur = x + static_cast<int64_t>(t) * n;
             const float *before = t == 0 ? prev : x + static_cast<int64_t>(t - 1) * n;
-            for (int64_t e = begin + tid; e < end; e += kMotionThreads) {
-                const double dlt = static_cast<double>(cur[e]) - static_cast<double>(before[e]);
-                acc += dlt * dlt;
+            if (vec) {
+                const float4 *c4 = reinterpret_cast<const float4 *>(cur);
+                const float4 *b4 = reinterpret_cast<const float4 *>(before);
+#pragma unroll 2
+                for (int64_t e = begin / 4 + tid; e < end / 4; e += kMotionThreads) {
+                    const float4 u = __ldcs(c4 + e), v = __ldcg(b4 + e);
+                    const double d0 = static_cast<double>(u.x) - static_cast<double>(v.x);
+                    const double d1 = static_cast<double>(u.y) - static_cast<double>(v.y);
+                    const double d2 = static_cast<double>(u.z) - static_cast<double>(v.z);
+                    const double d3 = static_cast<double>(u.w) - static_cast<double>(v.w);
+                    acc += d0 * d0 + d1 * d1 + d2 * d2 + d3 * d3;
+                }
+            } else {
+                for (int64_t e = begin + tid; e < end; e += kMotionThreads) {
+                    const double dlt = static_cast<double>(cur[e]) - static_cast<double>(before[e]);
+                    acc += dlt * dlt;
+                }
             }
         }
         for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
@@ -55,7 +74,13 @@ __global__ void __launch_bounds__(kMotionThreads) motion_kernel(const __grid_con
     }
     // This block's slice of the previous frame is no longer needed: replace it.
     const float *last = x + static_cast<int64_t>(p.chunk_frames - 1) * n;
-    for (int64_t e = begin + tid; e < end; e += kMotionThreads) prev[e] = last[e];
+    if (vec) {
+        const float4 *l4 = reinterpret_cast<const float4 *>(last);
+        float4 *p4 = reinterpret_cast<float4 *>(prev);
+        for (int64_t e = begin / 4 + tid; e < end / 4; e += kMotionThreads) p4[e] = __ldcg(l4 + e);
+    } else {
+        for (int64_t e = begin + tid; e < end; e += kMotionThreads) prev[e] = last[e];
+    }
 
     __threadfence();
     __syncthreads();

@@ -6,10 +6,11 @@
 // similarity; replace the least similar sink when the similarity falls
 // below the threshold tau).
 //
-// Kernel 1, grid (column blocks, token chunks, B): block (x, r, b) sums 64
+// Kernel 1, grid (column blocks, token chunks, B): block (x, r, b) sums 256
 // columns of the hidden states over token chunk r in fp64 (warp w takes
-// tokens w, w+8, ...; lane l takes columns 2l, 2l+1; fixed-order reduction
-// across warps).  The last block of stream b (atomic ticket) adds the chunk
+// tokens w, w+8, ...; lane l takes columns 8l..8l+7 with one 16-byte load per
+// token; fixed-order reduction across warps).  The number of token chunks is
+// chosen per cache so the grid covers the GPU about twice.  The last block of stream b (atomic ticket) adds the chunk
 // sums in chunk order, divides by the token count, computes the dot products
 // and norms in fp64, takes the decision, updates the sink embedding and the
 // sink-frame record, and writes out_slot[b].
@@ -23,7 +24,15 @@
 namespace sdv2 {
 
 constexpr int kRefreshThreads = 256;
-constexpr int kRefreshCols = 64;
+constexpr int kRefreshCols = 256;                 // 8 per lane
+
+__device__ __forceinline__ uint4 ld_stream_v4(const uint16_t *p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
 
 __device__ __forceinline__ double block_sum_fixed(double v, double *red) {
     for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
@@ -46,45 +55,78 @@ __global__ void __launch_bounds__(kRefreshThreads) refresh_decide_kernel(const _
     __shared__ double red[kRefreshThreads / 32];
     __shared__ int is_last;
 
-    // column sums of this block's 64 columns over its chunk of tokens
-    const int col0 = blockIdx.x * kRefreshCols + 2 * lane;
-    const int t_begin = static_cast<int>((static_cast<int64_t>(p.lq) * blockIdx.y) / kRefreshRowChunks);
-    const int t_end = static_cast<int>((static_cast<int64_t>(p.lq) * (blockIdx.y + 1)) / kRefreshRowChunks);
+    // column sums of this block's 256 columns over its chunk of tokens
+    const int col0 = blockIdx.x * kRefreshCols + 8 * lane;
+    const int t_begin = static_cast<int>((static_cast<int64_t>(p.lq) * blockIdx.y) / p.row_chunks);
+    const int t_end = static_cast<int>((static_cast<int64_t>(p.lq) * (blockIdx.y + 1)) / p.row_chunks);
     const uint16_t *hb = p.hidden + static_cast<int64_t>(b) * p.lq * p.dim;
-    double a0 = 0.0, a1 = 0.0;
+    double a[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) a[j] = 0.0;
     if (col0 < p.dim) {
+        if ((p.dim & 7) == 0) {                      // rows are 16-byte aligned: one vector per token
 #pragma unroll 4
-        for (int t = t_begin + warp; t < t_end; t += kRefreshThreads / 32) {
-            const uint32_t w = *reinterpret_cast<const uint32_t *>(hb + static_cast<int64_t>(t) * p.dim + col0);
-            a0 += static_cast<double>(bf16_lo(w));
-            a1 += static_cast<double>(bf16_hi(w));
+            for (int t = t_begin + warp; t < t_end; t += kRefreshThreads / 32) {
+                const uint4 w = ld_stream_v4(hb + static_cast<int64_t>(t) * p.dim + col0);
+                const uint32_t v[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    a[2 * q] += static_cast<double>(bf16_lo(v[q]));
+                    a[2 * q + 1] += static_cast<double>(bf16_hi(v[q]));
+                }
+            }
+        } else {
+            for (int t = t_begin + warp; t < t_end; t += kRefreshThreads / 32)
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    if (col0 + j < p.dim)
+                        a[j] += static_cast<double>(
+                            __uint_as_float(static_cast<uint32_t>(hb[static_cast<int64_t>(t) * p.dim + col0 + j]) << 16));
         }
     }
-    part[warp][2 * lane] = a0;
-    part[warp][2 * lane + 1] = a1;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) part[warp][8 * lane + j] = a[j];
     __syncthreads();
-    if (tid < kRefreshCols) {
+    {
         const int c = blockIdx.x * kRefreshCols + tid;
         if (c < p.dim) {
-            double s = 0.0;
-            for (int w = 0; w < kRefreshThreads / 32; ++w) s += part[w][tid];
-            p.partial[(static_cast<int64_t>(b) * kRefreshRowChunks + blockIdx.y) * p.dim + c] = s;
+            double sum = 0.0;
+            for (int w = 0; w < kRefreshThreads / 32; ++w) sum += part[w][tid];
+            p.partial[(static_cast<int64_t>(b) * p.row_chunks + blockIdx.y) * p.dim + c] = sum;
+        }
+    }
+    // Two-level merge.  The last block of each column block adds that block's 256
+    // column sums over the token chunks (in chunk order) and leaves the chunk mean
+    // in place of token chunk 0's sums; the last column block of the stream then
+    // takes the decision.
+    uint32_t *col_counter = p.counter + kMaxBatch + static_cast<int64_t>(b) * kRefreshMaxColBlocks + blockIdx.x;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) is_last = atomicAdd(col_counter, 1u) == gridDim.y - 1;
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    double *pb = p.partial + static_cast<int64_t>(b) * p.row_chunks * p.dim;
+    {
+        const int c = blockIdx.x * kRefreshCols + tid;
+        if (c < p.dim) {
+            double sum = 0.0;
+            for (int r = 0; r < p.row_chunks; ++r) sum += __ldcg(pb + static_cast<int64_t>(r) * p.dim + c);
+            pb[c] = sum / static_cast<double>(p.lq);
         }
     }
     __threadfence();
     __syncthreads();
-    if (tid == 0) is_last = atomicAdd(p.counter + b, 1u) == gridDim.x * gridDim.y - 1;
+    if (tid == 0) {
+        *col_counter = 0u;
+        is_last = atomicAdd(p.counter + b, 1u) == gridDim.x - 1;
+    }
     __syncthreads();
     if (!is_last) return;
     __threadfence();
 
-    // last block of stream b: chunk mean h (row chunks summed in order), then the decision
-    const double *pb = p.partial + static_cast<int64_t>(b) * kRefreshRowChunks * p.dim;
-    auto mean_at = [&](int c) {
-        double s = 0.0;
-        for (int r = 0; r < kRefreshRowChunks; ++r) s += __ldcg(pb + static_cast<int64_t>(r) * p.dim + c);
-        return s / static_cast<double>(p.lq);
-    };
+    // last column block of stream b: the chunk mean h is in pb[0 .. D), then the decision
+    auto mean_at = [&](int c) { return __ldcg(pb + c); };
     double *emb = p.sink_embed + static_cast<int64_t>(b) * p.sinks * p.dim;
     if (p.fill_count[b] > 0) {
         // The chunk fills sink slots itself: record their embedding only.
@@ -165,7 +207,7 @@ __global__ void __launch_bounds__(256) refresh_copy_kernel(const __grid_constant
 }
 
 cudaError_t launch_refresh(const RefreshParams &p, int sm_count, cudaStream_t s, int *launches) {
-    dim3 g1(static_cast<unsigned>((p.dim + kRefreshCols - 1) / kRefreshCols), kRefreshRowChunks,
+    dim3 g1(static_cast<unsigned>((p.dim + kRefreshCols - 1) / kRefreshCols), static_cast<unsigned>(p.row_chunks),
             static_cast<unsigned>(p.batch));
     refresh_decide_kernel<<<g1, kRefreshThreads, 0, s>>>(p);
     cudaError_t e = cudaGetLastError();

@@ -13,10 +13,10 @@ namespace sdv2 {
 
 constexpr int kMaxBatch = 64;
 // fp64 (cos, sin) entries of the temporal axis carried in one append launch.
-constexpr int kAppendTabEntries = 256;    // 4 KB of kernel parameters
-constexpr int kAppendMaxFrames = 16;
+constexpr int kAppendTabEntries = 256;    // 4 KB of kernel parameters (rows of distinct phases)
+constexpr int kAppendMaxFrames = 64;
 // fp32 (cos, sin) entries of the temporal axis carried in one attention launch.
-constexpr int kAttnTabEntries = 256;      // 2 KB of kernel parameters
+constexpr int kAttnTabEntries = 256;      // temporal (cos, sin) of one stream's chunk, in shared memory
 constexpr int kMaxSplits = 4;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits give up after 2 s
 
@@ -43,7 +43,8 @@ struct AppendParams {
     int32_t src_b[kAppendMaxFrames];     // stream of each frame
     int32_t src_i[kAppendMaxFrames];     // index of the frame in the chunk
     int32_t dst_slot[kAppendMaxFrames];  // ring slot it goes to
-    double tab_t[kAppendTabEntries][2];  // [frame][n_t] temporal cos, sin
+    uint8_t tab_row[kAppendMaxFrames];   // row of tab_t with the frame's phase
+    double tab_t[kAppendTabEntries][2];  // [distinct phase][n_t] temporal cos, sin
 };
 
 struct AttnParams {
@@ -60,13 +61,15 @@ struct AttnParams {
     int32_t n_qpairs, n_split, b_offset;
     float scale_log2;           // softmax_scale * log2(e)
     int32_t lk[kMaxBatch];      // valid keys per stream of this launch (0 = skip)
-    float tab_t[kAttnTabEntries][2];     // [b][frame in chunk][n_t] temporal cos, sin
+    double rope_base;           // RoPE frequency base
+    int32_t rope_reset;         // temporal phase period (0: none)
+    int64_t f0[kMaxBatch];      // first frame of each stream's chunk
 };
 
 struct RefreshParams {
     const uint16_t *hidden;     // [B][Lq][D]
-    double *partial;            // scratch [B][kRefreshRowChunks][D]: column sums of each row chunk
-    uint32_t *counter;          // scratch [B]
+    double *partial;            // scratch [B][row_chunks][D]: column sums of each token chunk
+    uint32_t *counter;          // scratch: [kMaxBatch] per-stream tickets, then [B][kRefreshMaxColBlocks] per column block
     double *sink_embed;         // [B][S][D]
     int64_t *sink_frame;        // [B][S]
     int32_t *out_slot;          // [B] (caller's)
@@ -74,7 +77,7 @@ struct RefreshParams {
     uint16_t *v_cache;
     int64_t layer_stride_elems; // elements between layers
     int64_t frame_elems;        // N*H*d
-    int32_t batch, lq, dim, sinks, slots, layers;
+    int32_t batch, lq, dim, sinks, slots, layers, row_chunks;
     double tau;
     int32_t active[kMaxBatch];  // 1 if stream takes part in this call
     int32_t fill_first[kMaxBatch];  // first sink slot this chunk fills itself (-1 none)
@@ -92,7 +95,7 @@ struct MotionParams {
     int32_t *hist_pos;          // [B]
     double *rate;               // [B]
     double *partial;            // scratch [B][T'][n_blocks]
-    uint32_t *counter;          // scratch [B]
+    uint32_t *counter;          // scratch: [kMaxBatch] per-stream tickets, then [B][kRefreshMaxColBlocks] per column block
     float *out_rate;            // [B]
     float *out_d;               // [B][T'] or null
     int64_t frame_elems;        // CHW
@@ -142,7 +145,8 @@ constexpr int kQTilesPerCta = 2;  // two query tiles ping-pong over the tensor c
 constexpr int kAttnThreads = 384;
 int attention_smem_bytes(int head_dim);
 
-constexpr int kRefreshRowChunks = 8;      // token chunks the chunk-mean reduction is split into
+constexpr int kRefreshMaxChunks = 32;     // token chunks the chunk-mean reduction is split into, at most
+constexpr int kRefreshMaxColBlocks = 64;  // 256-column blocks of the refresh reduction (embed_dim <= 16384)
 constexpr int kMotionBlockElems = 2048;   // latent elements per motion block
 constexpr int kMotionThreads = 256;
 

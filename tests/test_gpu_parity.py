@@ -78,6 +78,28 @@ def test_multi_tile_ragged_split_path():
     _stream_and_check(ps, 6, active_fn=lambda s: {0, 1} if s < 2 else {0, 1, 2})
 
 
+@pytest.mark.parametrize("head_dim", [128, 64])
+def test_single_tile_chunks_split_and_ragged(head_dim):
+    # 80 queries (one query tile: the two accumulator sets take alternate KV tiles and
+    # are merged in the CTA), 480 keys in 4 tiles with a ragged last one, split over the
+    # KV range so that some splits hold a single tile (one accumulator set unused).
+    from causal_dit_kv_b200 import binding as B
+    cfg = dict(batch=2, layers=1, heads=3, head_dim=head_dim, frame_h=8, frame_w=10, chunk_frames=1, sink_frames=1,
+               window_frames=5)
+    ps = PairedStream(seed=1010 + head_dim, **cfg)
+    assert B.sdv2_attention_splits(ps.gpu.cfg, [480, 480], 148) > 1
+    _stream_and_check(ps, 8)
+
+
+def test_small_chunk_many_streams():
+    """The 128x128 small-chunk shape: 64 tokens per frame, 12 heads x 128, 1 sink + 6
+    window frames, 16 independent streams, one of them starting late."""
+    cfg = dict(batch=16, layers=1, heads=12, head_dim=128, frame_h=8, frame_w=8, chunk_frames=1, sink_frames=1,
+               window_frames=6)
+    ps = PairedStream(seed=1012, **cfg)
+    _stream_and_check(ps, 9, check_every=4, active_fn=lambda s: set(range(15)) if s < 3 else set(range(16)))
+
+
 def test_many_heads_unsplit_path():
     # 37 heads x 4 query-tile pairs = 148 CTAs, one full wave: no KV split
     from causal_dit_kv_b200 import binding as B
