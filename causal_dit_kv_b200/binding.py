@@ -59,6 +59,7 @@ _SIGNATURES = [
     ("sdv2_cache_layout_get", c_int32, [c_void_p, POINTER(sdv2_cache_layout)]),
     ("sdv2_cache_check", c_int32, [c_void_p]),
     ("sdv2_cache_selftest_wait", c_int32, [c_void_p, c_uint64, c_void_p]),
+    ("sdv2_cache_time_attention", c_int32, [c_void_p, c_void_p, c_void_p]),
     ("sdv2_motion_bytes", c_size_t, [POINTER(sdv2_motion_config)]),
     ("sdv2_motion_create", c_int32, [POINTER(sdv2_motion_config), c_void_p, c_size_t, POINTER(c_void_p)]),
     ("sdv2_motion_destroy", c_int32, [c_void_p]),
@@ -204,6 +205,14 @@ def sdv2_cache_check(cache: int) -> int:
 
 def sdv2_cache_selftest_wait(cache: int, limit_ns: int, stream=None) -> None:
     _check(lib().sdv2_cache_selftest_wait(cache, int(limit_ns), _stream(stream)), "sdv2_cache_selftest_wait")
+
+
+def sdv2_cache_time_attention(cache: int, start=None, stop=None) -> None:
+    """Record torch.cuda.Event `start`/`stop` around the attention kernel of every
+    following sdv2_chunk_attention call (None, None switches it off)."""
+    s = ctypes.c_void_p(start.cuda_event) if start is not None else None
+    t = ctypes.c_void_p(stop.cuda_event) if stop is not None else None
+    _check(lib().sdv2_cache_time_attention(cache, s, t), "sdv2_cache_time_attention")
 
 
 def sdv2_motion_bytes(cfg: sdv2_motion_config) -> int:

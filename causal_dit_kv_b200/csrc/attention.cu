@@ -270,6 +270,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
+    __syncwarp();                               // thread 0 took the set-up branches alone
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -669,6 +670,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
     }
 
+    // Lane 0 of the producer and MMA warps arrives here long after the other lanes:
+    // reconverge each warp first, so that the block barrier counts every warp only
+    // once all its threads are done (TMEM is released right after it).
+    __syncwarp();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

@@ -239,6 +239,8 @@ struct sdv2_cache {
     std::vector<CUtensorMap> tk, tv;  // [L]
     CUtensorMap tq[2];                // the two rotated-query buffers in scratch: (d, H, Lq, B)
     uint64_t attention_calls = 0;     // selects the rotated-query buffer
+    cudaEvent_t time_start = nullptr;  // measurement hook: events around the attention kernel
+    cudaEvent_t time_stop = nullptr;
 };
 
 struct sdv2_motion {
@@ -561,8 +563,16 @@ sdv2_status sdv2_chunk_attention(sdv2_cache *c, int32_t layer, const void *q, vo
         if (!any) continue;
         cudaError_t e = launch_rope_q(p, c->sm_count, s);
         if (e != cudaSuccess) return cuda_fail(e, "rope_q launch");
+        if (c->time_start && b0 == 0) {
+            e = cudaEventRecord(c->time_start, s);
+            if (e != cudaSuccess) return cuda_fail(e, "chunk_attention start event");
+        }
         e = launch_attention(p, c->tq[qbuf], c->tk[layer], c->tv[layer], n.head_dim, s);
         if (e != cudaSuccess) return cuda_fail(e, "chunk_attention launch");
+        if (c->time_stop && b0 + streams_per_launch >= n.batch) {
+            e = cudaEventRecord(c->time_stop, s);
+            if (e != cudaSuccess) return cuda_fail(e, "chunk_attention stop event");
+        }
         g_launches.fetch_add(2);
         if (n_split > 1) {
             e = launch_combine(p, n.head_dim, s);
@@ -628,6 +638,14 @@ sdv2_status sdv2_sink_refresh(sdv2_cache *c, const void *hidden, float tau, cons
     cudaError_t e = launch_refresh(p, c->sm_count, reinterpret_cast<cudaStream_t>(stream), &launches);
     g_launches.fetch_add(static_cast<uint64_t>(launches));
     if (e != cudaSuccess) return cuda_fail(e, "sink_refresh launch");
+    return SDV2_OK;
+}
+
+sdv2_status sdv2_cache_time_attention(sdv2_cache *c, sdv2_event start, sdv2_event stop) {
+    if (!c) return fail(SDV2_E_ARG, "cache is NULL");
+    if ((start == nullptr) != (stop == nullptr)) return fail(SDV2_E_ARG, "give both events or neither");
+    c->time_start = reinterpret_cast<cudaEvent_t>(start);
+    c->time_stop = reinterpret_cast<cudaEvent_t>(stop);
     return SDV2_OK;
 }
 

@@ -48,6 +48,12 @@ class KVCache:
         scale = 1.0 / math.sqrt(self.head_dim) if softmax_scale is None else softmax_scale
         B.sdv2_chunk_attention(self.handle, layer, q, out, chunk_first_frame, scale, self.batch, stream)
 
+    def time_attention(self, start=None, stop=None):
+        """Record torch.cuda.Event start/stop (enable_timing=True, already recorded once so
+        that they exist) around the attention kernel of the following chunk_attention
+        calls; time_attention() switches it off."""
+        B.sdv2_cache_time_attention(self.handle, start, stop)
+
     def sink_refresh(self, hidden, tau, chunk_first_frame, out_slot, stream=None):
         B.sdv2_sink_refresh(self.handle, hidden, tau, chunk_first_frame, out_slot, self.batch, stream)
 

@@ -49,6 +49,8 @@ extern "C" {
 
 /* A CUDA stream (same type as cudaStream_t / CUstream). */
 typedef struct CUstream_st *sdv2_stream;
+/* A CUDA event (same type as cudaEvent_t / CUevent). */
+typedef struct CUevent_st *sdv2_event;
 
 typedef enum {
     SDV2_OK = 0,
@@ -197,6 +199,16 @@ sdv2_status sdv2_cache_check(sdv2_cache *cache);
  * This is the path every real kernel wait takes when it runs out.
  * Errors: SDV2_E_ARG, SDV2_E_CUDA. */
 sdv2_status sdv2_cache_selftest_wait(sdv2_cache *cache, uint64_t limit_ns, sdv2_stream stream);
+
+/* Measurement hook (no counterpart in the pages): while set, every
+ * sdv2_chunk_attention call on this cache records `start` on its stream
+ * right before the attention kernel's launch and `stop` right after it, so
+ * the time between them is that kernel alone (the query RoPE pass before it
+ * and the split merge after it are outside).  Recording events between the
+ * call's launches serialises them; use it in a separate timing pass.  Pass
+ * NULL for both to switch it off.  The events are the caller's.
+ * Errors: SDV2_E_ARG (only one of the two given). */
+sdv2_status sdv2_cache_time_attention(sdv2_cache *cache, sdv2_event start, sdv2_event stop);
 
 /* ------------------------------------------------------------------------
  * Motion-aware noise rate.  [A] method item 2; [Q] "Motion-aware noise
