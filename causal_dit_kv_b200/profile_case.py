@@ -12,13 +12,13 @@ import argparse
 import math
 
 SHAPES = {
-    "wan1.3b-512x512": dict(batch=1, heads=12, head_dim=128, frame_h=32, frame_w=32, chunk_frames=1,
+    "wan1.3b-512x512": dict(batch=1, layers=30, heads=12, head_dim=128, frame_h=32, frame_w=32, chunk_frames=1,
                             sink_frames=1, window_frames=6, embed_dim=1536, motion=(16, 64, 64)),
-    "wan1.3b-480x832-b4": dict(batch=4, heads=12, head_dim=128, frame_h=30, frame_w=52, chunk_frames=2,
+    "wan1.3b-480x832-b4": dict(batch=4, layers=30, heads=12, head_dim=128, frame_h=30, frame_w=52, chunk_frames=2,
                                sink_frames=1, window_frames=8, embed_dim=1536, motion=(16, 60, 104)),
-    "wan1.3b-128x128-b16": dict(batch=16, heads=12, head_dim=128, frame_h=8, frame_w=8, chunk_frames=1,
+    "wan1.3b-128x128-b16": dict(batch=16, layers=30, heads=12, head_dim=128, frame_h=8, frame_w=8, chunk_frames=1,
                                 sink_frames=1, window_frames=6, embed_dim=1536, motion=(16, 16, 16)),
-    "wan14b-512x512-b1": dict(batch=1, heads=40, head_dim=128, frame_h=32, frame_w=32, chunk_frames=1,
+    "wan14b-512x512-b1": dict(batch=1, layers=40, heads=40, head_dim=128, frame_h=32, frame_w=32, chunk_frames=1,
                               sink_frames=1, window_frames=6, embed_dim=5120, motion=(16, 64, 64)),
 }
 
