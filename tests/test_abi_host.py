@@ -89,3 +89,13 @@ def test_split_plan(B):
     tiny = B.make_cache_config(1, 1, 2, 64, 4, 4, 1, 1, 2)
     assert B.sdv2_attention_splits(tiny, [48], 148) == 1
     assert B.sdv2_attention_splits(c2, [0], 148) == 1
+
+
+def test_null_handles_are_rejected_without_a_device(B):
+    import ctypes
+    lib = B.lib()
+    assert lib.sdv2_cache_time_attention(None, None, None) == B.SDV2_E_ARG
+    assert lib.sdv2_cache_check(None) == B.SDV2_E_ARG
+    assert lib.sdv2_cache_selftest_wait(None, ctypes.c_uint64(1000), None) == B.SDV2_E_ARG
+    assert lib.sdv2_kv_append(None, 0, None, None, None, None) == B.SDV2_E_ARG
+    assert "NULL" in lib.sdv2_last_error().decode() or "null" in lib.sdv2_last_error().decode()
