@@ -70,6 +70,8 @@ _SIGNATURES = [
     ("sdv2_rope_phase", c_int64, [c_int64, c_int32]),
     ("sdv2_valid_slots", None, [c_int64, c_int32, c_int32, POINTER(c_int32), POINTER(c_int32)]),
     ("sdv2_attention_splits", c_int32, [POINTER(sdv2_cache_config), POINTER(c_int64), c_int32]),
+    ("sdv2_attention_plan", c_int32, [POINTER(sdv2_cache_config), POINTER(c_int64), c_int32, POINTER(c_int32),
+                                      POINTER(c_int32)]),
     ("sdv2_launch_count", c_uint64, []),
     ("sdv2_last_error", c_char_p, []),
     ("sdv2_version", c_char_p, []),
@@ -264,6 +266,15 @@ def sdv2_valid_slots(frame_end: int, sink_frames: int, window_frames: int):
 def sdv2_attention_splits(cfg: sdv2_cache_config, keys, sm_count: int) -> int:
     arr = (c_int64 * cfg.batch)(*[int(k) for k in keys])
     return int(lib().sdv2_attention_splits(ctypes.byref(cfg), arr, sm_count))
+
+
+def sdv2_attention_plan(cfg: sdv2_cache_config, keys, sm_count: int):
+    """(whole_units, pieces): units [0, whole_units) run whole, the rest in `pieces` KV pieces."""
+    arr = (c_int64 * cfg.batch)(*[int(k) for k in keys])
+    whole, pieces = c_int32(0), c_int32(0)
+    _check(lib().sdv2_attention_plan(ctypes.byref(cfg), arr, sm_count, ctypes.byref(whole), ctypes.byref(pieces)),
+           "sdv2_attention_plan")
+    return int(whole.value), int(pieces.value)
 
 
 def sdv2_launch_count() -> int:

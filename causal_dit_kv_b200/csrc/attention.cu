@@ -13,7 +13,11 @@
 // keys, so the kernel reads keys 0..lk-1 of the slot-major cache directly,
 // without unrolling the ring.
 //
-// One CTA = one (stream, head, pair of 128-row query tiles, KV split):
+// One CTA = one work unit (stream, head, pair of 128-row query tiles) or one
+// KV-range piece of a unit: the host runs as many units whole as fill complete
+// waves of the GPU and splits the remaining ones (or all of them, when there
+// are fewer units than SMs) over the KV range, so the last wave is not left
+// mostly empty.
 //   warp 0      TMA producer: K tiles (128 keys x d) into a 2-slot ring, V tiles
 //               into a 3-slot ring
 //   warp 1      MMA issuer (one thread): S_t = Q_t K^T and O_t += P_t V
@@ -225,16 +229,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int qpair = blockIdx.x / p.n_split;
-    const int split = blockIdx.x - qpair * p.n_split;
-    const int h = blockIdx.y;
-    const int bl = blockIdx.z;                  // stream within this launch
+    // work unit of this CTA: whole units first, then the pieces of the split ones
+    int unit, split, n_split;
+    if (static_cast<int>(blockIdx.x) < p.n_whole) {
+        unit = blockIdx.x;
+        split = 0;
+        n_split = 1;
+    } else {
+        const int j = blockIdx.x - p.n_whole;
+        unit = p.n_whole + j / p.n_pieces;
+        split = j - (j / p.n_pieces) * p.n_pieces;
+        n_split = p.n_pieces;
+    }
+    const int su = unit - p.n_whole;            // index among the split units (split CTAs only)
+    const int n_su = p.n_units - p.n_whole;
+    const int qpair = unit % p.n_qpairs;
+    const int h = (unit / p.n_qpairs) % p.heads;
+    const int bl = p.unit_stream[unit / (p.n_qpairs * p.heads)];   // stream within this launch
     const int bg = p.b_offset + bl;             // stream index in the cache
     const int lk = p.lk[bl];
-    if (lk <= 0) return;                        // stream not part of this call (uniform per CTA)
+    if (lk <= 0) return;                        // (active streams only; uniform per CTA)
 
     const int n_kv = (lk + kBlockN - 1) / kBlockN;
-    const int per = (n_kv + p.n_split - 1) / p.n_split;
+    const int per = (n_kv + n_split - 1) / n_split;
     const int kv_begin = split * per;
     const int kv_end = min(n_kv, kv_begin + per);
     const int n_local = kv_end > kv_begin ? kv_end - kv_begin : 0;
@@ -554,7 +571,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 if (ok) tc_fence_after();
                 const uint32_t o0 = tmem + lane_base + 256 + t * (D / 2);
                 const uint32_t o1 = o0 + 128;
-                if (p.n_split == 1) {
+                if (n_split == 1) {
                     if (ok) {
                         const float inv = 1.0f / l;
                         uint16_t *orow =
@@ -578,10 +595,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     }
                 } else if (ok) {
                     // KV split: this split's merged, unnormalised partial (layout as below)
-                    const int64_t group = (static_cast<int64_t>(bg) * p.heads + h) * p.n_qpairs + qpair;
-                    const int64_t n_groups = static_cast<int64_t>(p.batch) * p.heads * p.n_qpairs;
-                    float4 *po = reinterpret_cast<float4 *>(p.part_o) + (split * n_groups + group) * (D / 4) * 256 +
-                                 t * (D / 8) * 256 + row;
+                    float4 *po = reinterpret_cast<float4 *>(p.part_o) +
+                                 (static_cast<int64_t>(split) * n_su + su) * (D / 4) * 256 + t * (D / 8) * 256 + row;
                     if (n_local > 0) {
 #pragma unroll 1
                         for (int cb = 0; cb < D / 64; ++cb) {
@@ -600,16 +615,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         for (int c = 0; c < D / 8; ++c) po[c * 256] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
                     }
                     if (valid && t == 0)
-                        reinterpret_cast<float2 *>(p.part_ml)[((static_cast<int64_t>(split) * p.batch + bg) * p.heads + h) *
-                                                                  p.lq_pad + q_row0 + row] =
+                        reinterpret_cast<float2 *>(p.part_ml)[(static_cast<int64_t>(split) * n_su + su) * 256 + row] =
                             make_float2(n_local > 0 ? m : -INFINITY, l);
                 }
             } else {
                 // ---- epilogue
                 if (ok && n_local > 0) ok = warp_wait(&bars[L::kOFull + t], 0, abort_flag, p.status, kStatusSoftmaxWait);
-                const int prow_local = q_row0 + t * kBlockM + row;     // row index within the padded query range
                 if (ok) tc_fence_after();
-                if (p.n_split == 1) {
+                if (n_split == 1) {
                     if (ok) {
                         const float inv = 1.0f / l_run;
                         uint16_t *orow = p.out + ((static_cast<int64_t>(bg) * p.lq + token) * p.heads + h) * D;
@@ -633,14 +646,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     }
                 } else if (ok) {
                     // ---- KV split: write this split's unnormalised partial for attention_combine_kernel.
-                    // part_o: one block per (split, stream, head, query-tile pair) of [D/4 float4
-                    // columns][256 rows] (rows t*128 + lane; a warp's 32 rows are 512 contiguous
-                    // bytes); part_ml[(split*B + b)*H + h][lq_pad] float2 = (row max in log2 units, sum).
-                    const int64_t group = (static_cast<int64_t>(bg) * p.heads + h) * p.n_qpairs + qpair;
-                    const int64_t n_groups = static_cast<int64_t>(p.batch) * p.heads * p.n_qpairs;
+                    // part_o: one block per (piece, split unit) of [D/4 float4 columns][256 rows]
+                    // (rows t*128 + lane; a warp's 32 rows are 512 contiguous bytes);
+                    // part_ml[piece][split unit][256] float2 = (row max in log2 units, sum).
+                    const int64_t blk = static_cast<int64_t>(split) * n_su + su;
                     const int srow = t * kBlockM + row;
                     if (n_local > 0) {                         // warp-uniform: every lane takes part in tcgen05.ld
-                        float4 *po = reinterpret_cast<float4 *>(p.part_o) + (split * n_groups + group) * (D / 4) * 256 + srow;
+                        float4 *po = reinterpret_cast<float4 *>(p.part_o) + blk * (D / 4) * 256 + srow;
                         uint32_t r[D / 32][32];
 #pragma unroll
                         for (int cb = 0; cb < D / 32; ++cb) tmem_ld32(o_tmem + cb * 32, r[cb]);
@@ -657,13 +669,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                                     __uint_as_float(r[cb][4 * v + 2]), __uint_as_float(r[cb][4 * v + 3]));
                         }
                     } else if (valid) {                         // no keys in this split: zero partial
-                        float4 *po = reinterpret_cast<float4 *>(p.part_o) + (split * n_groups + group) * (D / 4) * 256 + srow;
+                        float4 *po = reinterpret_cast<float4 *>(p.part_o) + blk * (D / 4) * 256 + srow;
 #pragma unroll
                         for (int c = 0; c < D / 4; ++c) po[c * 256] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
                     }
                     if (valid)
-                        reinterpret_cast<float2 *>(p.part_ml)[((static_cast<int64_t>(split) * p.batch + bg) * p.heads + h) *
-                                                                  p.lq_pad + prow_local] =
+                        reinterpret_cast<float2 *>(p.part_ml)[blk * 256 + srow] =
                             make_float2(n_local > 0 ? m_run : -INFINITY, l_run);
                 }
             }
@@ -694,31 +705,28 @@ __global__ void __launch_bounds__(256) attention_combine_kernel(const __grid_con
     grid_dependency_wait();                         // the split CTAs' partials
     grid_launch_dependents();
     constexpr int kC16 = D / 16;                    // 16-column chunks per row
-    const int64_t n_groups = static_cast<int64_t>(p.batch) * p.heads * p.n_qpairs;
+    const int n_su = p.n_units - p.n_whole;         // split units
     const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int srow = static_cast<int>(idx & 255);
     const int64_t rest = idx >> 8;
     const int c16 = static_cast<int>(rest % kC16);
-    const int64_t gl = rest / kC16;                 // group within this launch's streams
-    const int64_t per_stream = static_cast<int64_t>(p.heads) * p.n_qpairs;
-    const int bl = static_cast<int>(gl / per_stream);
-    if (bl >= kMaxBatch || p.lk[bl] <= 0) return;
-    const int bg = p.b_offset + bl;
-    const int h = static_cast<int>((gl % per_stream) / p.n_qpairs);
-    const int qpair = static_cast<int>(gl % p.n_qpairs);
+    const int su = static_cast<int>(rest / kC16);
+    if (su >= n_su) return;
+    const int unit = p.n_whole + su;
+    const int qpair = unit % p.n_qpairs;
+    const int h = (unit / p.n_qpairs) % p.heads;
+    const int bg = p.b_offset + p.unit_stream[unit / (p.n_qpairs * p.heads)];
     const int token = qpair * 256 + srow;
     if (token >= p.lq) return;
-    const int64_t group = (static_cast<int64_t>(bg) * p.heads + h) * p.n_qpairs + qpair;
     float2 ml[kMaxSplits];
     float4 u[kMaxSplits][4];
 #pragma unroll
     for (int s = 0; s < kMaxSplits; ++s) {
         ml[s] = make_float2(-INFINITY, 0.0f);
-        if (s < p.n_split) {
-            ml[s] = __ldcs(reinterpret_cast<const float2 *>(p.part_ml) +
-                           ((static_cast<int64_t>(s) * p.batch + bg) * p.heads + h) * p.lq_pad + token);
-            const float4 *po = reinterpret_cast<const float4 *>(p.part_o) + (s * n_groups + group) * (D / 4) * 256 +
-                               (c16 * 4) * 256 + srow;
+        if (s < p.n_pieces) {
+            const int64_t blk = static_cast<int64_t>(s) * n_su + su;
+            ml[s] = __ldcs(reinterpret_cast<const float2 *>(p.part_ml) + blk * 256 + srow);
+            const float4 *po = reinterpret_cast<const float4 *>(p.part_o) + blk * (D / 4) * 256 + (c16 * 4) * 256 + srow;
 #pragma unroll
             for (int i = 0; i < 4; ++i) u[s][i] = __ldcs(po + i * 256);
         }
@@ -732,7 +740,7 @@ __global__ void __launch_bounds__(256) attention_combine_kernel(const __grid_con
     float l = 0.0f;
 #pragma unroll
     for (int s = 0; s < kMaxSplits; ++s) {
-        if (s < p.n_split) {
+        if (s < p.n_pieces) {
             const float w = ml[s].x == -INFINITY ? 0.0f : exp2f(ml[s].x - m);
             l += w * ml[s].y;
 #pragma unroll
@@ -789,11 +797,8 @@ static cudaError_t launch_attention_d(const AttnParams &p, const CUtensorMap &tq
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    int nb = 0;
-    for (int i = 0; i < kMaxBatch; ++i)
-        if (p.lk[i] > 0) nb = i + 1;
-    if (nb == 0) return cudaSuccess;
-    dim3 grid(static_cast<unsigned>(p.n_qpairs * p.n_split), static_cast<unsigned>(p.heads), static_cast<unsigned>(nb));
+    if (p.n_units == 0) return cudaSuccess;
+    dim3 grid(static_cast<unsigned>(p.n_whole + (p.n_units - p.n_whole) * p.n_pieces));
     return launch_dependent(chunk_attention_kernel<D>, grid, dim3(kAttnThreads), static_cast<size_t>(smem), s, p, tq, tk, tv);
 }
 
@@ -804,11 +809,8 @@ cudaError_t launch_attention(const AttnParams &p, const CUtensorMap &tq, const C
 }
 
 cudaError_t launch_combine(const AttnParams &p, int head_dim, cudaStream_t s) {
-    int nb = 0;
-    for (int i = 0; i < kMaxBatch; ++i)
-        if (p.lk[i] > 0) nb = i + 1;
-    if (nb == 0 || p.n_split <= 1) return cudaSuccess;
-    const int64_t threads = static_cast<int64_t>(nb) * p.heads * p.n_qpairs * (head_dim / 16) * 256;
+    if (p.n_units == p.n_whole) return cudaSuccess;
+    const int64_t threads = static_cast<int64_t>(p.n_units - p.n_whole) * (head_dim / 16) * 256;
     const dim3 grid(static_cast<unsigned>((threads + 255) / 256));
     if (head_dim == 64) return launch_dependent(attention_combine_kernel<64>, grid, dim3(256), 0, s, p);
     return launch_dependent(attention_combine_kernel<128>, grid, dim3(256), 0, s, p);

@@ -130,9 +130,9 @@ Geometry geometry(const sdv2_cache_config &c) {
     g.layer_elems = static_cast<int64_t>(c.batch) * g.slots * g.frame_elems;
     g.n_qpairs = static_cast<int>((g.lq + kBlockM * kQTilesPerCta - 1) / (kBlockM * kQTilesPerCta));
     g.lq_pad = g.n_qpairs * kBlockM * kQTilesPerCta;
-    const int64_t rows_one = static_cast<int64_t>(c.batch) * c.heads * g.lq_pad;
-    g.part_rows = rows_one * kMaxSplits;
-    if (g.part_rows > kPartRowsCap) g.part_rows = (kPartRowsCap / rows_one) * rows_one;
+    // partial blocks (256 rows each) for the split units of one launch
+    g.part_rows = std::min<int64_t>(static_cast<int64_t>(std::min(c.batch, kMaxBatch)) * c.heads * g.n_qpairs *
+                                        kMaxSplits, kPartRowsCap / 256) * 256;
     uint64_t off = 0;
     g.k = off;
     g.layer_stride = static_cast<uint64_t>(g.layer_elems) * 2;
@@ -178,41 +178,56 @@ Geometry geometry(const sdv2_cache_config &c) {
     return g;
 }
 
-// Split-KV partition count for one attention call: minimises an estimate of
-// the makespan (waves x KV tiles per CTA) plus the cost of writing and
-// merging partials, within the partial buffer's capacity.
-int plan_splits(const sdv2_cache_config &c, const Geometry &g, const int64_t *keys, int sm_count) {
-    int64_t max_tiles = 0;
-    int active = 0;
-    for (int b = 0; b < c.batch; ++b) {
-        if (keys[b] <= 0) continue;
-        ++active;
-        const int64_t t = (keys[b] + kBlockN - 1) / kBlockN;
-        if (t > max_tiles) max_tiles = t;
-    }
-    if (active == 0 || max_tiles <= 1 || sm_count <= 0) return 1;
-    const int64_t ctas1 = static_cast<int64_t>(c.batch) * c.heads * g.n_qpairs;
-    const int64_t rows_one = static_cast<int64_t>(c.batch) * c.heads * g.lq_pad;
+// Work decomposition of one attention launch over `units` (stream, head,
+// query-tile pair) units of at most max_tiles KV tiles each.  Either every
+// unit runs whole (one CTA each), or the units beyond the last complete wave
+// (all of them, when there are fewer units than SMs) are split over the KV
+// range into `pieces` CTAs each and merged afterwards.  Chosen by an estimate
+// of the makespan: whole waves x tiles per unit + waves of pieces x tiles per
+// piece + the merge (a fixed cost plus the partials written and read back),
+// within the partial buffer's capacity.
+struct AttnPlan {
+    int64_t whole;
+    int pieces;
+};
+
+AttnPlan plan_attention(const sdv2_cache_config &c, const Geometry &g, int64_t units, int64_t max_tiles,
+                        int sm_count) {
+    AttnPlan best{units, 1};
+    if (units <= 0 || max_tiles <= 1 || sm_count <= 0) return best;
     // Cost units: one KV tile of one CTA (~2.5 us on a B200 SM at these sizes).
-    // Partial traffic per split: rows * (d + 2) floats written and read back.
     const double tile_us = 2.5;
+    const double merge_us = 3.0;
     const double bytes_per_us = 6.0e6;   // ~6 TB/s
-    double best_cost = 1e300;
-    int best = 1;
-    for (int s = 1; s <= kMaxSplits; ++s) {
-        if (s > 1 && rows_one * s > g.part_rows) break;
+    const int64_t cap = g.part_rows / 256;  // partial blocks of 256 rows
+    auto waves = [&](int64_t ctas) { return (ctas + sm_count - 1) / sm_count; };
+    double best_cost = static_cast<double>(waves(units) * max_tiles) * tile_us;
+    const int64_t full = (units / sm_count) * sm_count;   // units that fill whole waves
+    for (int s = 2; s <= kMaxSplits; ++s) {
         const int64_t per = (max_tiles + s - 1) / s;
-        const int64_t ctas = ctas1 * s;
-        const int64_t waves = (ctas + sm_count - 1) / sm_count;
-        double cost = static_cast<double>(waves * per) * tile_us;
-        if (s > 1) cost += 3.0 + static_cast<double>(s) * rows_one * (c.head_dim + 2) * 8.0 / bytes_per_us;
-        if (cost < best_cost - 1e-9) {
-            best_cost = cost;
-            best = s;
+        for (int tail = 0; tail < 2; ++tail) {
+            const int64_t whole = tail ? full : 0;
+            if (tail && (full == 0 || full == units)) continue;
+            const int64_t rest = units - whole;
+            if (rest * s > cap) continue;
+            const double cost = static_cast<double>(whole / sm_count * max_tiles) * tile_us +
+                                static_cast<double>(waves(rest * s) * per) * tile_us + merge_us +
+                                static_cast<double>(rest * s) * 256.0 * (c.head_dim + 2) * 8.0 / bytes_per_us;
+            if (cost < best_cost - 1e-9) {
+                best_cost = cost;
+                best = {whole, s};
+            }
         }
         if (per <= 1) break;
     }
     return best;
+}
+
+int64_t max_kv_tiles(const int64_t *keys, int n) {
+    int64_t m = 0;
+    for (int b = 0; b < n; ++b)
+        if (keys[b] > 0) m = std::max<int64_t>(m, (keys[b] + kBlockN - 1) / kBlockN);
+    return m;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
@@ -519,7 +534,6 @@ sdv2_status sdv2_chunk_attention(sdv2_cache *c, int32_t layer, const void *q, vo
         valid_counts(chunk_first_frame[b] + n.chunk_frames, n.sink_frames, n.window_frames, &sv, &wv);
         keys[b] = static_cast<int64_t>(sv + wv) * g.N;
     }
-    const int n_split = plan_splits(n, g, keys.data(), c->sm_count);
     const int n_t = n.rope_pairs[0];
     const int streams_per_launch = kMaxBatch;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -537,7 +551,6 @@ sdv2_status sdv2_chunk_attention(sdv2_cache *c, int32_t layer, const void *q, vo
     p.batch = n.batch;
     p.heads = n.heads;
     p.lq = static_cast<int32_t>(g.lq);
-    p.lq_pad = g.lq_pad;
     p.tokens_per_frame = static_cast<int32_t>(g.N);
     p.frame_w = n.frame_w;
     p.chunk_frames = n.chunk_frames;
@@ -545,7 +558,6 @@ sdv2_status sdv2_chunk_attention(sdv2_cache *c, int32_t layer, const void *q, vo
     p.n_h = n.rope_pairs[1];
     p.n_w = n.rope_pairs[2];
     p.n_qpairs = g.n_qpairs;
-    p.n_split = n_split;
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
     p.rope_base = n.rope_base;
     p.rope_reset = n.rope_reset_period;
@@ -553,14 +565,22 @@ sdv2_status sdv2_chunk_attention(sdv2_cache *c, int32_t layer, const void *q, vo
         const int nb = std::min(streams_per_launch, n.batch - b0);
         p.b_offset = b0;
         bool any = false;
+        int n_active = 0;
         for (int bl = 0; bl < kMaxBatch; ++bl) p.lk[bl] = 0;
         for (int bl = 0; bl < nb; ++bl) {
             const int b = b0 + bl;
             p.lk[bl] = static_cast<int32_t>(keys[b]);
             p.f0[bl] = chunk_first_frame[b];
-            if (keys[b] > 0) any = true;
+            if (keys[b] > 0) {
+                any = true;
+                p.unit_stream[n_active++] = static_cast<uint8_t>(bl);
+            }
         }
         if (!any) continue;
+        p.n_units = n_active * n.heads * g.n_qpairs;
+        const AttnPlan plan = plan_attention(n, g, p.n_units, max_kv_tiles(keys.data() + b0, nb), c->sm_count);
+        p.n_whole = static_cast<int32_t>(plan.whole);
+        p.n_pieces = plan.pieces;
         cudaError_t e = launch_rope_q(p, c->sm_count, s);
         if (e != cudaSuccess) return cuda_fail(e, "rope_q launch");
         if (c->time_start && b0 == 0) {
@@ -574,7 +594,7 @@ sdv2_status sdv2_chunk_attention(sdv2_cache *c, int32_t layer, const void *q, vo
             if (e != cudaSuccess) return cuda_fail(e, "chunk_attention stop event");
         }
         g_launches.fetch_add(2);
-        if (n_split > 1) {
+        if (p.n_whole < p.n_units) {
             e = launch_combine(p, n.head_dim, s);
             if (e != cudaSuccess) return cuda_fail(e, "attention combine launch");
             g_launches.fetch_add(1);
@@ -898,9 +918,26 @@ void sdv2_valid_slots(int64_t frame_end, int32_t sink_frames, int32_t window_fra
 }
 
 int32_t sdv2_attention_splits(const sdv2_cache_config *cfg, const int64_t *keys, int32_t sm_count) {
+    int32_t whole = 0, pieces = 0;
+    if (sdv2_attention_plan(cfg, keys, sm_count, &whole, &pieces) != SDV2_OK) return -1;
+    return pieces;
+}
+
+sdv2_status sdv2_attention_plan(const sdv2_cache_config *cfg, const int64_t *keys, int32_t sm_count,
+                                int32_t *whole_units, int32_t *pieces) {
     sdv2_cache_config n;
-    if (!keys || check_config(cfg, &n) != SDV2_OK) return -1;
-    return plan_splits(n, geometry(n), keys, sm_count);
+    if (!keys || !whole_units || !pieces) return fail(SDV2_E_ARG, "NULL argument");
+    sdv2_status st = check_config(cfg, &n);
+    if (st != SDV2_OK) return st;
+    const Geometry g = geometry(n);
+    int active = 0;
+    for (int b = 0; b < std::min(n.batch, kMaxBatch); ++b)
+        if (keys[b] > 0) ++active;
+    const AttnPlan plan = plan_attention(n, g, static_cast<int64_t>(active) * n.heads * g.n_qpairs,
+                                         max_kv_tiles(keys, std::min(n.batch, kMaxBatch)), sm_count);
+    *whole_units = static_cast<int32_t>(plan.whole);
+    *pieces = plan.pieces;
+    return SDV2_OK;
 }
 
 uint64_t sdv2_launch_count(void) { return g_launches.load(); }

@@ -51,14 +51,20 @@ struct AttnParams {
     const uint16_t *q;          // [B][Lq][H][d] as given (not rotated)
     uint16_t *q_rot;            // [B][Lq][H][d] RoPE(q) in bf16, scratch (read by TMA)
     uint16_t *out;              // [B][Lq][H][d]
-    float *part_o;              // [split][B][H][d/4][Lq_pad] float4 (split > 1)
-    float *part_ml;             // [split][B][H][Lq_pad] float2 (row max in log2 units, row sum)
+    float *part_o;              // [piece][split unit][d/4][256] float4 (split units only)
+    float *part_ml;             // [piece][split unit][256] float2 (row max in log2 units, row sum)
     const float *rope_h;        // [frame_h][n_h][2] fp32
     const float *rope_w;        // [frame_w][n_w][2]
     uint32_t *status;
-    int32_t batch, heads, lq, lq_pad, tokens_per_frame, frame_w, chunk_frames;
+    int32_t batch, heads, lq, tokens_per_frame, frame_w, chunk_frames;
     int32_t n_t, n_h, n_w;
-    int32_t n_qpairs, n_split, b_offset;
+    int32_t n_qpairs, b_offset;
+    // Work units u = (i * heads + h) * n_qpairs + qpair over the launch's active streams
+    // unit_stream[i]: units [0, n_whole) run whole, one CTA each; units [n_whole,
+    // n_units) are split over the KV range into n_pieces CTAs each and merged by
+    // attention_combine_kernel.
+    int32_t n_units, n_whole, n_pieces;
+    uint8_t unit_stream[kMaxBatch];
     float scale_log2;           // softmax_scale * log2(e)
     int32_t lk[kMaxBatch];      // valid keys per stream of this launch (0 = skip)
     double rope_base;           // RoPE frequency base

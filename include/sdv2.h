@@ -288,8 +288,16 @@ int64_t sdv2_rope_phase(int64_t f, int32_t rope_reset_period);
 /* Valid sink and window slot counts once frames 0..frame_end-1 exist. */
 void sdv2_valid_slots(int64_t frame_end, int32_t sink_frames, int32_t window_frames,
                       int32_t *sink_valid, int32_t *window_valid);
-/* Number of split-KV partitions sdv2_chunk_attention would use for streams
- * whose valid key counts are keys[0..batch-1] (host-side plan). */
+/* Work plan sdv2_chunk_attention would use on a GPU with sm_count SMs for
+ * streams whose valid key counts are keys[0..batch-1] (0: stream skipped),
+ * for the first launch (up to 64 streams).  Units are (stream, head, pair of
+ * 128-query tiles); units [0, *whole_units) run whole and the rest are split
+ * over the KV range into *pieces CTAs each (*pieces == 1: nothing split).
+ * Host-side, no device needed.  Errors: SDV2_E_ARG, SDV2_E_SHAPE. */
+sdv2_status sdv2_attention_plan(const sdv2_cache_config *cfg, const int64_t *keys, int32_t sm_count,
+                                int32_t *whole_units, int32_t *pieces);
+/* *pieces of sdv2_attention_plan (1 if no unit is split), or -1 on a bad
+ * argument. */
 int32_t sdv2_attention_splits(const sdv2_cache_config *cfg, const int64_t *keys, int32_t sm_count);
 
 /* Kernels launched by this library in this process so far. */

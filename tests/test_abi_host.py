@@ -81,14 +81,24 @@ def test_layout_regions_are_disjoint_and_aligned(B):
 
 def test_split_plan(B):
     c2 = B.make_cache_config(1, 30, 12, 128, 32, 32, 1, 1, 6)
-    s = B.sdv2_attention_splits(c2, [7168], 148)
-    # 48 CTAs unsplit on 148 SMs: the plan splits the KV range to fill the GPU
-    assert 2 <= s <= 4 and 48 * s <= 148
+    # 48 units (12 heads x 4 query-tile pairs) on 148 SMs: every unit split over the KV range
+    whole, pieces = B.sdv2_attention_plan(c2, [7168], 148)
+    assert whole == 0 and 2 <= pieces <= 4 and 48 * pieces <= 148
+    assert B.sdv2_attention_splits(c2, [7168], 148) == pieces
+    # 37 heads x 4 pairs = 148 units fill the GPU exactly once: nothing split
+    full = B.make_cache_config(1, 1, 37, 128, 32, 32, 1, 1, 6)
+    assert B.sdv2_attention_plan(full, [7168], 148) == (148, 1)
+    # 624 units are 4 full waves + 32: the 32 of the last wave are split, the rest run whole
     c3 = B.make_cache_config(4, 30, 12, 128, 30, 52, 2, 1, 8)
-    assert B.sdv2_attention_splits(c3, [14040] * 4, 148) == 1
+    whole, pieces = B.sdv2_attention_plan(c3, [14040] * 4, 148)
+    assert whole == 4 * 148 and pieces > 1 and (624 - whole) * pieces <= 148
+    # 160 units: one full wave whole, the 12 left split
+    c4 = B.make_cache_config(1, 40, 40, 128, 32, 32, 1, 1, 6)
+    whole, pieces = B.sdv2_attention_plan(c4, [7168], 148)
+    assert whole == 148 and pieces > 1
     tiny = B.make_cache_config(1, 1, 2, 64, 4, 4, 1, 1, 2)
-    assert B.sdv2_attention_splits(tiny, [48], 148) == 1
-    assert B.sdv2_attention_splits(c2, [0], 148) == 1
+    assert B.sdv2_attention_plan(tiny, [48], 148) == (2, 1)     # 2 heads, a single KV tile: nothing to split
+    assert B.sdv2_attention_plan(c2, [0], 148) == (0, 1)        # no active stream
 
 
 def test_null_handles_are_rejected_without_a_device(B):
