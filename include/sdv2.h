@@ -140,9 +140,9 @@ sdv2_status sdv2_kv_append(sdv2_cache *cache, int32_t layer, const void *k, cons
 /* Attention of the chunk's queries over the valid sink + window keys of
  * layer `layer`: out = softmax(softmax_scale * RoPE(q) K^T) V.
  * [A] "深入分析" (KV-cache load per chunk), [Q] "Adaptive sink and RoPE refresh".
- * q:   device bf16 [B][T'*N][H][d], NOT rotated: RoPE is applied on load (fp32,
- *      then rounded to bf16 for the tensor cores) at the same (phase, row, col)
- *      as the chunk's keys.
+ * q:   device bf16 [B][T'*N][H][d], NOT rotated: the call rotates it (fp32,
+ *      rounded to bf16 for the tensor cores, into the cache's scratch) at the
+ *      same (phase, row, col) as the chunk's keys.
  * out: device bf16 [B][T'*N][H][d].
  * chunk_first_frame: HOST int64 [B], the frames of this chunk; the chunk must
  *      already be appended to this layer (f0 + T' == frames appended).
