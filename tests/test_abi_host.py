@@ -109,3 +109,25 @@ def test_null_handles_are_rejected_without_a_device(B):
     assert lib.sdv2_cache_selftest_wait(None, ctypes.c_uint64(1000), None) == B.SDV2_E_ARG
     assert lib.sdv2_kv_append(None, 0, None, None, None, None) == B.SDV2_E_ARG
     assert "NULL" in lib.sdv2_last_error().decode() or "null" in lib.sdv2_last_error().decode()
+
+
+def test_plan_properties_over_random_shapes(B):
+    import random
+    rng = random.Random(11)
+    for _ in range(300):
+        b, h = rng.randint(1, 16), rng.choice([1, 2, 8, 12, 24, 40])
+        fh, fw, tp = rng.randint(1, 40), rng.randint(1, 60), rng.randint(1, 3)
+        s_, w = rng.randint(1, 3), rng.randint(3, 10)
+        cfg = B.make_cache_config(b, 1, h, 128, fh, fw, tp, s_, max(w, tp))
+        n = fh * fw
+        keys = [rng.choice([0, (s_ + max(w, tp)) * n, rng.randint(1, (s_ + max(w, tp)) * n)]) for _ in range(b)]
+        sms = rng.choice([132, 148, 160])
+        whole, pieces = B.sdv2_attention_plan(cfg, keys, sms)
+        units = sum(1 for k in keys if k > 0) * h * ((tp * n + 255) // 256)
+        assert 1 <= pieces <= 4
+        assert 0 <= whole <= units
+        if pieces == 1:
+            assert whole == units                     # nothing split
+        else:
+            assert whole == 0 or whole % sms == 0    # whole units fill complete waves
+            assert whole < units
