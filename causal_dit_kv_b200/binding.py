@@ -10,7 +10,7 @@ from __future__ import annotations
 
 import ctypes
 import os
-from ctypes import POINTER, c_char_p, c_double, c_float, c_int32, c_int64, c_size_t, c_uint64, c_void_p
+from ctypes import POINTER, c_char_p, c_double, c_float, c_int32, c_int64, c_size_t, c_uint32, c_uint64, c_void_p
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsdv2.so")
 
@@ -23,13 +23,19 @@ class sdv2_cache_config(ctypes.Structure):
     _fields_ = [("batch", c_int32), ("layers", c_int32), ("heads", c_int32), ("head_dim", c_int32),
                 ("frame_h", c_int32), ("frame_w", c_int32), ("chunk_frames", c_int32), ("sink_frames", c_int32),
                 ("window_frames", c_int32), ("rope_pairs", c_int32 * 3), ("rope_reset_period", c_int32),
-                ("embed_dim", c_int32), ("rope_base", c_double)]
+                ("embed_dim", c_int32), ("rope_base", c_double), ("kv_format", c_int32)]
+
+
+KV_BF16, KV_FP8_E4M3 = 0, 1
+KV_FORMATS = {"bf16": KV_BF16, "fp8": KV_FP8_E4M3}
 
 
 class sdv2_cache_layout(ctypes.Structure):
     _fields_ = [("k_offset", c_uint64), ("v_offset", c_uint64), ("layer_stride", c_uint64),
                 ("sink_embed_offset", c_uint64), ("sink_frame_offset", c_uint64), ("status_offset", c_uint64),
-                ("scratch_offset", c_uint64), ("scratch_bytes", c_uint64), ("total_bytes", c_uint64)]
+                ("scratch_offset", c_uint64), ("scratch_bytes", c_uint64), ("total_bytes", c_uint64),
+                ("k_scale_offset", c_uint64), ("v_scale_offset", c_uint64), ("scale_layer_stride", c_uint64),
+                ("scale_slot_stride", c_uint32), ("tokens_padded", c_uint32)]
 
 
 class sdv2_motion_config(ctypes.Structure):
@@ -128,13 +134,15 @@ def _frames(chunk_first_frame, batch: int):
 
 
 def make_cache_config(batch, layers, heads, head_dim, frame_h, frame_w, chunk_frames, sink_frames, window_frames,
-                      rope_pairs=(0, 0, 0), rope_reset_period=0, embed_dim=0, rope_base=10000.0) -> sdv2_cache_config:
+                      rope_pairs=(0, 0, 0), rope_reset_period=0, embed_dim=0, rope_base=10000.0,
+                      kv_format="bf16") -> sdv2_cache_config:
     cfg = sdv2_cache_config()
     cfg.batch, cfg.layers, cfg.heads, cfg.head_dim = batch, layers, heads, head_dim
     cfg.frame_h, cfg.frame_w, cfg.chunk_frames = frame_h, frame_w, chunk_frames
     cfg.sink_frames, cfg.window_frames = sink_frames, window_frames
     cfg.rope_pairs = (c_int32 * 3)(*rope_pairs)
     cfg.rope_reset_period, cfg.embed_dim, cfg.rope_base = rope_reset_period, embed_dim, rope_base
+    cfg.kv_format = KV_FORMATS[kv_format] if isinstance(kv_format, str) else int(kv_format)
     return cfg
 
 

@@ -53,10 +53,11 @@
 
 namespace sdv2 {
 
-template <int D>
+template <int D, bool F8 = false>
 struct AttnLayout {
-    static constexpr int kQTile = kBlockM * D * 2;    // bytes of one Q tile
-    static constexpr int kKVTile = kBlockN * D * 2;   // bytes of one K (or V) tile
+    static constexpr int kElem = F8 ? 1 : 2;          // bytes per element of Q, K, V
+    static constexpr int kQTile = kBlockM * D * kElem;    // bytes of one Q tile
+    static constexpr int kKVTile = kBlockN * D * kElem;   // bytes of one K (or V) tile
     static constexpr int kSub = kBlockM * 128;        // one 64-column (128-byte) sub-tile
     static constexpr int kKStages = 2;                // K tile i is needed one half-iteration before V tile i,
     static constexpr int kVStages = 3;                // so V gets the deeper ring to hide its load latency
@@ -150,17 +151,51 @@ __global__ void __launch_bounds__(256) rope_q_kernel(const __grid_constant__ Att
             cs[i][q] = *(j < p.n_t ? tab_t + j : (j < p.n_t + p.n_h ? tab_h + j : tab_w + j));
         }
     }
+    if (p.q_scale == nullptr) {
 #pragma unroll
-    for (int i = 0; i < kMaxVec; ++i) {
-        if (i >= nvec) break;
-        const uint32_t in[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
-        uint32_t o[4];
+        for (int i = 0; i < kMaxVec; ++i) {
+            if (i >= nvec) break;
+            const uint32_t in[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
+            uint32_t o[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float x0 = bf16_lo(in[q]), x1 = bf16_hi(in[q]);
-            o[q] = pack_bf16x2(x0 * cs[i][q].x - x1 * cs[i][q].y, x0 * cs[i][q].y + x1 * cs[i][q].x);
+            for (int q = 0; q < 4; ++q) {
+                const float x0 = bf16_lo(in[q]), x1 = bf16_hi(in[q]);
+                o[q] = pack_bf16x2(x0 * cs[i][q].x - x1 * cs[i][q].y, x0 * cs[i][q].y + x1 * cs[i][q].x);
+            }
+            *reinterpret_cast<uint4 *>(p.q_rot + off + (sub + 4 * i) * 8) = make_uint4(o[0], o[1], o[2], o[3]);
         }
-        *reinterpret_cast<uint4 *>(p.q_rot + off + (sub + 4 * i) * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+    } else {
+        // fp8 cache (head_dim 128): the rotated row is coded as E4M3 with its own scale
+        // amax / 448, amax over the row's 128 channels (the row's 4 threads combine theirs).
+        float r[kMaxVec][8];
+        float am = 0.0f;
+#pragma unroll
+        for (int i = 0; i < kMaxVec; ++i) {
+            const uint32_t in[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float x0 = bf16_lo(in[q]), x1 = bf16_hi(in[q]);
+                r[i][2 * q] = x0 * cs[i][q].x - x1 * cs[i][q].y;
+                r[i][2 * q + 1] = x0 * cs[i][q].y + x1 * cs[i][q].x;
+                am = fmaxf(am, fmaxf(fabsf(r[i][2 * q]), fabsf(r[i][2 * q + 1])));
+            }
+        }
+        const unsigned group = 0xFu << (threadIdx.x & 28u);
+        am = fmaxf(am, __shfl_xor_sync(group, am, 1));
+        am = fmaxf(am, __shfl_xor_sync(group, am, 2));
+        float scale, inv;
+        e4m3_scale_inv(am, scale, inv);
+        uint8_t *q8 = reinterpret_cast<uint8_t *>(p.q_rot);
+#pragma unroll
+        for (int i = 0; i < kMaxVec; ++i) {
+            uint32_t c[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k)
+                c[k] = pack_e4m3x2(r[i][4 * k] * inv, r[i][4 * k + 1] * inv) |
+                       (pack_e4m3x2(r[i][4 * k + 2] * inv, r[i][4 * k + 3] * inv) << 16);
+            *reinterpret_cast<uint2 *>(q8 + off + (sub + 4 * i) * 8) = make_uint2(c[0], c[1]);
+        }
+        if (sub == 0) p.q_scale[static_cast<int64_t>(p.b_offset + bl) * rows + row] = scale;
     }
     grid_dependency_wait();
 }
@@ -197,6 +232,46 @@ __device__ __forceinline__ float softmax_exp_store(const uint32_t (&sr)[kBlockN 
     return a0 + a1;
 }
 
+// fp8 cache: P = 2^(s*c - m) as above, the row sum from P, and P * r coded as
+// E4M3 (four keys per 32-bit TMEM column, key order in the bytes) into columns
+// [0, 32) of the row's S region; r = (this tile's V scale) / (the CTA's
+// largest V scale) folds the tile's V scale into P, so one O accumulates
+// tiles of different scales.
+__device__ __forceinline__ float softmax_exp_store_f8(const uint32_t (&sr)[kBlockN / 32][32], float c, float neg_m,
+                                                      float r, uint32_t s_tmem) {
+    const uint64_t scale2 = f2_pack(c, c);
+    const uint64_t negm2 = f2_pack(neg_m, neg_m);
+    const uint64_t r2 = f2_pack(r, r);
+    const uint64_t zero2 = f2_pack(0.0f, 0.0f);
+    uint64_t acc[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i] = 0ull;
+#pragma unroll
+    for (int cb = 0; cb < kBlockN / 32; ++cb) {
+        uint32_t pk[8];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const uint64_t x = f2_fma(f2_pack(__uint_as_float(sr[cb][2 * i]), __uint_as_float(sr[cb][2 * i + 1])),
+                                      scale2, negm2);
+            float x0, x1;
+            f2_unpack(x, x0, x1);
+            const uint64_t pp = f2_pack(ex2_approx(x0), ex2_approx(x1));
+            acc[i & 3] = f2_add(acc[i & 3], pp);
+            float q0, q1;
+            f2_unpack(f2_fma(pp, r2, zero2), q0, q1);
+            const uint32_t h16 = pack_e4m3x2(q0, q1);
+            if (i & 1)
+                pk[i >> 1] |= h16 << 16;
+            else
+                pk[i >> 1] = h16;
+        }
+        tmem_st8(s_tmem + cb * 8, pk);
+    }
+    float a0, a1;
+    f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
+    return a0 + a1;
+}
+
 // Single-tile mode: 32 columns of w0 O_0 + w1 O_1 for this thread's row, as
 // fp32 bits in r0 (O_1 is read only if its set received keys).
 __device__ __forceinline__ void merge_sets(uint32_t o0, uint32_t o1, bool has1, float w0, float w1,
@@ -216,11 +291,12 @@ __device__ __forceinline__ void merge_sets(uint32_t o0, uint32_t o1, bool has1, 
     for (int i = 0; i < 32; ++i) r0[i] = __float_as_uint(w0 * __uint_as_float(r0[i]) + w1 * __uint_as_float(r1[i]));
 }
 
-template <int D>
+template <int D, bool F8>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     chunk_attention_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
                            const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v) {
-    using L = AttnLayout<D>;
+    using L = AttnLayout<D, F8>;
+    static_assert(!F8 || D == 128, "the fp8 cache is built for head_dim 128");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBar);
@@ -250,7 +326,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int lk = p.lk[bl];
     if (lk <= 0) return;                        // (active streams only; uniform per CTA)
 
-    const int n_kv = (lk + kBlockN - 1) / kBlockN;
+    // KV tiles: 128-key runs of the valid prefix (bf16), or the 128-token blocks of each
+    // valid slot (fp8: tile g is block g % n_blk of slot g / n_blk)
+    const int n_kv = F8 ? (lk / p.tokens_per_frame) * p.n_blk : (lk + kBlockN - 1) / kBlockN;
     const int per = (n_kv + n_split - 1) / n_split;
     const int kv_begin = split * per;
     const int kv_end = min(n_kv, kv_begin + per);
@@ -304,11 +382,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (lane == 0 && n_local > 0) {
             // rotated query tiles of this CTA (rows past lq are filled with zeros)
             mbar_arrive_expect_tx(&bars[L::kQFull], n_qt * L::kQTile);
-            for (int t = 0; t < n_qt; ++t)
+            for (int t = 0; t < n_qt; ++t) {
+                if constexpr (F8) {
+                    tma_load_4d(smem + L::kQ + t * L::kQTile, &tmap_q, &bars[L::kQFull], 0, h, q_row0 + t * kBlockM, bg);
+                } else {
 #pragma unroll
-                for (int kb = 0; kb < D / 64; ++kb)
-                    tma_load_4d(smem + L::kQ + t * L::kQTile + kb * L::kSub, &tmap_q, &bars[L::kQFull], kb * 64, h,
-                                q_row0 + t * kBlockM, bg);
+                    for (int kb = 0; kb < D / 64; ++kb)
+                        tma_load_4d(smem + L::kQ + t * L::kQTile + kb * L::kSub, &tmap_q, &bars[L::kQFull], kb * 64,
+                                    h, q_row0 + t * kBlockM, bg);
+                }
+            }
             // K tile `it` and V tile `it` are issued as soon as their own ring slot is free.
             int k_issued = 0, v_issued = 0;
             bool ok = true;
@@ -321,10 +404,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         break;
                     }
                     mbar_arrive_expect_tx(&bars[L::kKFull + st], L::kKVTile);
+                    if constexpr (F8) {
+                        const int g = kv_begin + k_issued, sl = g / p.n_blk;
+                        tma_load_4d(smem + L::kK + st * L::kKVTile, &tmap_k, &bars[L::kKFull + st], 0, h,
+                                    sl * p.np_tokens + (g - sl * p.n_blk) * kBlockN, bg);
+                    } else {
 #pragma unroll
-                    for (int kb = 0; kb < D / 64; ++kb)
-                        tma_load_4d(smem + L::kK + st * L::kKVTile + kb * L::kSub, &tmap_k, &bars[L::kKFull + st],
-                                    kb * 64, h, (kv_begin + k_issued) * kBlockN, bg);
+                        for (int kb = 0; kb < D / 64; ++kb)
+                            tma_load_4d(smem + L::kK + st * L::kKVTile + kb * L::kSub, &tmap_k, &bars[L::kKFull + st],
+                                        kb * 64, h, (kv_begin + k_issued) * kBlockN, bg);
+                    }
                     ++k_issued;
                 }
                 const int st = v_issued % L::kVStages;
@@ -334,10 +423,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     break;
                 }
                 mbar_arrive_expect_tx(&bars[L::kVFull + st], L::kKVTile);
+                if constexpr (F8) {
+                    const int g = kv_begin + v_issued, sl = g / p.n_blk;
+                    tma_load_5d(smem + L::kV + st * L::kKVTile, &tmap_v, &bars[L::kVFull + st],
+                                (g - sl * p.n_blk) * kBlockN, 0, h, sl, bg);
+                } else {
 #pragma unroll
-                for (int kb = 0; kb < D / 64; ++kb)
-                    tma_load_4d(smem + L::kV + st * L::kKVTile + kb * L::kSub, &tmap_v, &bars[L::kVFull + st],
-                                kb * 64, h, (kv_begin + v_issued) * kBlockN, bg);
+                    for (int kb = 0; kb < D / 64; ++kb)
+                        tma_load_4d(smem + L::kV + st * L::kKVTile + kb * L::kSub, &tmap_v, &bars[L::kVFull + st],
+                                    kb * 64, h, (kv_begin + v_issued) * kBlockN, bg);
+                }
                 ++v_issued;
             }
             if (!ok) {
@@ -358,30 +453,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0 && n_local > 0) {
-            constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kBlockN, 0, 0);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, D, 0, 1);
+            // fp8: E4M3 operands, K = 32 per MMA; V is stored transposed, so both B operands
+            // are K-major 128-byte rows
+            constexpr uint32_t idesc_qk = F8 ? idesc_e4m3_f32(kBlockM, kBlockN, 0, 0) : idesc_bf16_f32(kBlockM, kBlockN, 0, 0);
+            constexpr uint32_t idesc_pv = F8 ? idesc_e4m3_f32(kBlockM, D, 0, 0) : idesc_bf16_f32(kBlockM, D, 0, 1);
             // Descriptors are built once; each MMA only adds a constant to the start-address
             // field (bits 0..13, address >> 4; every operand lies below 256 KB, so no carry
             // leaves the field).  This keeps the issuing thread's instruction count low: it
             // shares its SM sub-partition with busy softmax warps.
             const uint64_t dq = smem_desc_sw128(smem_addr(smem + L::kQ), 16, 1024);
             const uint64_t dk = smem_desc_sw128(smem_addr(smem + L::kK), 16, 1024);
-            const uint64_t dv = smem_desc_sw128(smem_addr(smem + L::kV), L::kSub, 1024);
+            const uint64_t dv = smem_desc_sw128(smem_addr(smem + L::kV), F8 ? 16 : L::kSub, 1024);
             auto issue_qk = [&](int t, int st) {
                 const uint64_t a0 = dq + static_cast<uint64_t>((dual ? 0 : t) * (L::kQTile >> 4));
                 const uint64_t b0 = dk + static_cast<uint64_t>(st * (L::kKVTile >> 4));
+                if constexpr (F8) {
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t off = static_cast<uint64_t>(((kk >> 2) * L::kSub + (kk & 3) * 32) >> 4);
-                    umma_ss(tmem + t * 128, a0 + off, b0 + off, idesc_qk, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < D / 32; ++kk)
+                        umma_ss_f8(tmem + t * 128, a0 + kk * 2, b0 + kk * 2, idesc_qk, kk > 0 ? 1u : 0u);
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint64_t off = static_cast<uint64_t>(((kk >> 2) * L::kSub + (kk & 3) * 32) >> 4);
+                        umma_ss(tmem + t * 128, a0 + off, b0 + off, idesc_qk, kk > 0 ? 1u : 0u);
+                    }
                 }
             };
             auto issue_pv = [&](int t, int st, bool acc) {
                 const uint64_t b0 = dv + static_cast<uint64_t>(st * (L::kKVTile >> 4));
+                if constexpr (F8) {
 #pragma unroll
-                for (int kk = 0; kk < kBlockN / 16; ++kk)
-                    umma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, b0 + static_cast<uint64_t>((kk * 2048) >> 4),
-                            idesc_pv, (acc || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < kBlockN / 32; ++kk)
+                        umma_ts_f8(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, b0 + kk * 2, idesc_pv,
+                                   (acc || kk > 0) ? 1u : 0u);
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < kBlockN / 16; ++kk)
+                        umma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
+                                b0 + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv, (acc || kk > 0) ? 1u : 0u);
+                }
             };
             bool ok = mbar_wait(&bars[L::kQFull], 0, abort_flag, p.status, kStatusMmaWait);
             if (dual) {
@@ -492,7 +602,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             bool ok = true;
             const uint32_t s_tmem = tmem + lane_base + t * 128;
             const uint32_t o_tmem = tmem + lane_base + 256 + t * 128;
+            // fp8: this row's query scale, and the largest V scale of the CTA's tiles (every
+            // tile's P is multiplied by its V scale over this one; the epilogue multiplies back)
+            float sq = 1.0f, sv_ref = 1.0f;
+            int64_t scale_base = 0;
+            if constexpr (F8) {
+                sq = valid ? p.q_scale[(static_cast<int64_t>(bg) * p.lq + token) * p.heads + h] : 0.0f;
+                scale_base = static_cast<int64_t>(bg) * p.slots * p.scale_slot_stride + h * p.n_blk;
+                sv_ref = 0.0f;
+                for (int i = 0; i < n_local; ++i) {
+                    const int g = kv_begin + i, sl = g / p.n_blk;
+                    sv_ref = fmaxf(sv_ref, p.v_scale[scale_base + sl * (p.scale_slot_stride - p.n_blk) + g]);
+                }
+                sv_ref = fmaxf(sv_ref, 1e-30f);
+            }
             for (int it = 0; it < n_mine; ++it) {
+                const int g = kv_begin + (dual ? 2 * it + t : it);   // KV tile of this iteration
+                float c_t = p.scale_log2, r_t = 1.0f;
+                int valid_cols;
+                if constexpr (F8) {
+                    const int sl = g / p.n_blk;
+                    const int64_t si = scale_base + sl * (p.scale_slot_stride - p.n_blk) + g;
+                    c_t = fmaxf(p.scale_log2 * sq * p.k_scale[si], 1e-30f);
+                    r_t = p.v_scale[si] / sv_ref;
+                    valid_cols = p.tokens_per_frame - (g - sl * p.n_blk) * kBlockN;
+                } else {
+                    valid_cols = lk - g * kBlockN;
+                }
                 if (!warp_wait(&bars[L::kSFull + t], it & 1, abort_flag, p.status, kStatusSoftmaxWait)) {
                     ok = false;
                     break;
@@ -504,7 +640,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 tmem_wait_ld_bind(sr[0]);
 #pragma unroll
                 for (int cb = 1; cb < kBlockN / 32; ++cb) reg_bind(sr[cb]);
-                const int valid_cols = lk - (kv_begin + (dual ? 2 * it + t : it)) * kBlockN;
                 if (valid_cols < kBlockN) {
 #pragma unroll
                     for (int cb = 0; cb < kBlockN / 32; ++cb)
@@ -523,7 +658,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     m4[cb] = fmaxf(m, __uint_as_float(sr[cb][31]));
                 }
                 const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-                const float m_tile = mx * p.scale_log2;
+                const float m_tile = mx * c_t;
                 bool rescale = false;
                 float alpha = 1.0f;
                 if (it == 0) {
@@ -534,7 +669,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     l_run *= alpha;
                     m_run = m_tile;
                 }
-                l_run += softmax_exp_store(sr, p.scale_log2, -m_run, s_tmem);
+                if constexpr (F8)
+                    l_run += softmax_exp_store_f8(sr, c_t, -m_run, r_t, s_tmem);
+                else
+                    l_run += softmax_exp_store(sr, c_t, -m_run, s_tmem);
                 // O_t is idle here (PV(t, it-1) completed before S(t, it) was signalled and
                 // PV(t, it) waits for this thread's arrival below), so it can be rescaled now.
                 if (__any_sync(0xffffffffu, rescale)) {
@@ -568,12 +706,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const float w0 = a0.x == -INFINITY ? 0.0f : ex2_approx(a0.x - m);
                 const float w1 = a1.x == -INFINITY ? 0.0f : ex2_approx(a1.x - m);
                 const float l = w0 * a0.y + w1 * a1.y;
+                const float svr = F8 ? sv_ref : 1.0f;      // fp8: undo the V-scale normalisation of P
                 if (ok) tc_fence_after();
                 const uint32_t o0 = tmem + lane_base + 256 + t * (D / 2);
                 const uint32_t o1 = o0 + 128;
                 if (n_split == 1) {
                     if (ok) {
-                        const float inv = 1.0f / l;
+                        const float inv = svr / l;
                         uint16_t *orow =
                             p.out + ((static_cast<int64_t>(bg) * p.lq + token) * p.heads + h) * D + t * (D / 2);
 #pragma unroll 1
@@ -601,7 +740,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll 1
                         for (int cb = 0; cb < D / 64; ++cb) {
                             uint32_t v[32];
-                            merge_sets(o0 + cb * 32, o1 + cb * 32, n1 > 0, w0, w1, v);
+                            merge_sets(o0 + cb * 32, o1 + cb * 32, n1 > 0, w0 * svr, w1 * svr, v);
                             if (valid) {
 #pragma unroll
                                 for (int q = 0; q < 8; ++q)
@@ -622,9 +761,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 // ---- epilogue
                 if (ok && n_local > 0) ok = warp_wait(&bars[L::kOFull + t], 0, abort_flag, p.status, kStatusSoftmaxWait);
                 if (ok) tc_fence_after();
+                const float svr = F8 ? sv_ref : 1.0f;          // fp8: undo the V-scale normalisation of P
                 if (n_split == 1) {
                     if (ok) {
-                        const float inv = 1.0f / l_run;
+                        const float inv = svr / l_run;
                         uint16_t *orow = p.out + ((static_cast<int64_t>(bg) * p.lq + token) * p.heads + h) * D;
 #pragma unroll
                         for (int cb = 0; cb < D / 32; ++cb) {
@@ -664,9 +804,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                             for (int cb = 0; cb < D / 32; ++cb)
 #pragma unroll
                                 for (int v = 0; v < 8; ++v)
-                                    po[(cb * 8 + v) * 256] =
-                                        make_float4(__uint_as_float(r[cb][4 * v]), __uint_as_float(r[cb][4 * v + 1]),
-                                                    __uint_as_float(r[cb][4 * v + 2]), __uint_as_float(r[cb][4 * v + 3]));
+                                    po[(cb * 8 + v) * 256] = make_float4(
+                                        __uint_as_float(r[cb][4 * v]) * svr, __uint_as_float(r[cb][4 * v + 1]) * svr,
+                                        __uint_as_float(r[cb][4 * v + 2]) * svr, __uint_as_float(r[cb][4 * v + 3]) * svr);
                         }
                     } else if (valid) {                         // no keys in this split: zero partial
                         float4 *po = reinterpret_cast<float4 *>(p.part_o) + blk * (D / 4) * 256 + srow;
@@ -787,25 +927,28 @@ cudaError_t launch_wait_selftest(uint32_t *status, uint64_t limit_ns, cudaStream
     return cudaGetLastError();
 }
 
-template <int D>
+template <int D, bool F8>
 static cudaError_t launch_attention_d(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
                                       const CUtensorMap &tv, cudaStream_t s) {
     static bool configured = false;
-    const int smem = AttnLayout<D>::kAlloc;
+    const int smem = AttnLayout<D, F8>::kAlloc;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(chunk_attention_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        cudaError_t e =
+            cudaFuncSetAttribute(chunk_attention_kernel<D, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         configured = true;
     }
     if (p.n_units == 0) return cudaSuccess;
     dim3 grid(static_cast<unsigned>(p.n_whole + (p.n_units - p.n_whole) * p.n_pieces));
-    return launch_dependent(chunk_attention_kernel<D>, grid, dim3(kAttnThreads), static_cast<size_t>(smem), s, p, tq, tk, tv);
+    return launch_dependent(chunk_attention_kernel<D, F8>, grid, dim3(kAttnThreads), static_cast<size_t>(smem), s, p,
+                            tq, tk, tv);
 }
 
 cudaError_t launch_attention(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
                              const CUtensorMap &tv, int head_dim, cudaStream_t s) {
-    if (head_dim == 64) return launch_attention_d<64>(p, tq, tk, tv, s);
-    return launch_attention_d<128>(p, tq, tk, tv, s);
+    if (p.q_scale != nullptr) return launch_attention_d<128, true>(p, tq, tk, tv, s);
+    if (head_dim == 64) return launch_attention_d<64, false>(p, tq, tk, tv, s);
+    return launch_attention_d<128, false>(p, tq, tk, tv, s);
 }
 
 cudaError_t launch_combine(const AttnParams &p, int head_dim, cudaStream_t s) {

@@ -72,6 +72,10 @@ double rope_angle(double base, int j, int n, int64_t pos) {
 
 struct Geometry {
     int64_t N, slots, lq, frame_elems, layer_elems;
+    bool f8;                 // fp8 (E4M3) block-scaled cache
+    int64_t np_tokens;       // fp8: tokens per slot padded to whole 128-token blocks
+    int n_blk, scale_slot_stride;
+    uint64_t k_scale, v_scale, scale_layer_stride, q_scale, q_scale_bytes;
     int n_qpairs, lq_pad;
     int refresh_chunks;  // token chunks of the refresh reduction
     int64_t part_rows;  // capacity of the split-KV partial buffer, rows of d floats
@@ -98,6 +102,10 @@ sdv2_status check_config(const sdv2_cache_config *c, sdv2_cache_config *norm) {
     if (n.embed_dim < 0 || (n.embed_dim & 1) || n.embed_dim > 16384)
         return fail(SDV2_E_SHAPE, "embed_dim must be even and in 0..16384");
     if (!(n.rope_base > 0.0)) n.rope_base = 10000.0;
+    if (n.kv_format != SDV2_KV_BF16 && n.kv_format != SDV2_KV_FP8_E4M3)
+        return fail(SDV2_E_SHAPE, "kv_format must be SDV2_KV_BF16 or SDV2_KV_FP8_E4M3");
+    if (n.kv_format == SDV2_KV_FP8_E4M3 && n.head_dim != 128)
+        return fail(SDV2_E_SHAPE, "the fp8 cache requires head_dim 128");
     const int c2 = n.head_dim / 2;
     if (n.rope_pairs[0] == 0 && n.rope_pairs[1] == 0 && n.rope_pairs[2] == 0) {
         n.rope_pairs[1] = c2 / 3;
@@ -114,7 +122,8 @@ sdv2_status check_config(const sdv2_cache_config *c, sdv2_cache_config *norm) {
     const int64_t N = static_cast<int64_t>(n.frame_h) * n.frame_w;
     const int64_t slots = n.sink_frames + n.window_frames;
     const int64_t fe = N * n.heads * n.head_dim;
-    if (slots * N >= (1ll << 31) || fe * kAppendMaxFrames * 2 / 8 >= (1ll << 31) ||
+    const int64_t np_tok = (N + 127) / 128 * 128;
+    if (slots * np_tok >= (1ll << 31) || fe * kAppendMaxFrames * 2 / 8 >= (1ll << 31) ||
         N * n.chunk_frames >= (1ll << 30))
         return fail(SDV2_E_SHAPE, "cache dimensions exceed the supported 32-bit index range");
     *norm = n;
@@ -128,6 +137,10 @@ Geometry geometry(const sdv2_cache_config &c) {
     g.lq = g.N * c.chunk_frames;
     g.frame_elems = g.N * c.heads * c.head_dim;
     g.layer_elems = static_cast<int64_t>(c.batch) * g.slots * g.frame_elems;
+    g.f8 = c.kv_format == SDV2_KV_FP8_E4M3;
+    g.np_tokens = (g.N + kBlockN - 1) / kBlockN * kBlockN;
+    g.n_blk = static_cast<int>(g.np_tokens / kBlockN);
+    g.scale_slot_stride = (c.heads * g.n_blk + 3) / 4 * 4;
     g.n_qpairs = static_cast<int>((g.lq + kBlockM * kQTilesPerCta - 1) / (kBlockM * kQTilesPerCta));
     g.lq_pad = g.n_qpairs * kBlockM * kQTilesPerCta;
     // partial blocks (256 rows each) for the split units of one launch
@@ -135,10 +148,18 @@ Geometry geometry(const sdv2_cache_config &c) {
                                         kMaxSplits, kPartRowsCap / 256) * 256;
     uint64_t off = 0;
     g.k = off;
-    g.layer_stride = static_cast<uint64_t>(g.layer_elems) * 2;
+    g.layer_stride = g.f8 ? static_cast<uint64_t>(c.batch) * g.slots * g.np_tokens * c.heads * c.head_dim
+                          : static_cast<uint64_t>(g.layer_elems) * 2;
     off = align_up(off + g.layer_stride * c.layers, 256);
     g.v = off;
     off = align_up(off + g.layer_stride * c.layers, 256);
+    if (g.f8) {
+        g.scale_layer_stride = 4ull * c.batch * g.slots * g.scale_slot_stride;
+        g.k_scale = off;
+        off = align_up(off + g.scale_layer_stride * c.layers, 256);
+        g.v_scale = off;
+        off = align_up(off + g.scale_layer_stride * c.layers, 256);
+    }
     g.rope_h64 = off;
     off = align_up(off + 16ull * c.frame_h * c.rope_pairs[1], 256);
     g.rope_w64 = off;
@@ -169,6 +190,11 @@ Geometry geometry(const sdv2_cache_config &c) {
     g.q_rot = off;
     g.q_rot_bytes = align_up(2ull * c.batch * g.lq * c.heads * c.head_dim, 1024);
     off = align_up(off + 2 * g.q_rot_bytes, 1024);
+    if (g.f8) {                       // per-row scales of the E4M3 queries, one per query buffer
+        g.q_scale = off;
+        g.q_scale_bytes = align_up(4ull * c.batch * g.lq * c.heads, 256);
+        off = align_up(off + 2 * g.q_scale_bytes, 256);
+    }
     g.part_ml = off;
     off = align_up(off + 8ull * g.part_rows, 256);
     g.part_o = off;
@@ -223,10 +249,13 @@ AttnPlan plan_attention(const sdv2_cache_config &c, const Geometry &g, int64_t u
     return best;
 }
 
-int64_t max_kv_tiles(const int64_t *keys, int n) {
+// KV tiles of the longest stream: 128-key runs of its valid prefix, or for the fp8 cache
+// the 128-token blocks of each valid slot.
+int64_t max_kv_tiles(const Geometry &g, const int64_t *keys, int n) {
     int64_t m = 0;
     for (int b = 0; b < n; ++b)
-        if (keys[b] > 0) m = std::max<int64_t>(m, (keys[b] + kBlockN - 1) / kBlockN);
+        if (keys[b] > 0)
+            m = std::max<int64_t>(m, g.f8 ? keys[b] / g.N * g.n_blk : (keys[b] + kBlockN - 1) / kBlockN);
     return m;
 }
 
@@ -319,6 +348,11 @@ static void fill_layout(const sdv2_cache_config &n, const Geometry &g, sdv2_cach
     out->scratch_offset = g.scratch;
     out->scratch_bytes = g.scratch_end - g.scratch;
     out->total_bytes = g.total;
+    out->k_scale_offset = g.f8 ? g.k_scale : 0;
+    out->v_scale_offset = g.f8 ? g.v_scale : 0;
+    out->scale_layer_stride = g.f8 ? g.scale_layer_stride : 0;
+    out->scale_slot_stride = g.f8 ? static_cast<uint32_t>(g.scale_slot_stride) : 0;
+    out->tokens_padded = g.f8 ? static_cast<uint32_t>(g.np_tokens) : 0;
     (void)n;
 }
 
@@ -388,22 +422,49 @@ sdv2_status sdv2_cache_create(const sdv2_cache_config *cfg, void *dev_buf, size_
             return cuda_fail(e, "cache_create upload");
         }
     }
-    // One TMA descriptor per layer for K and for V: dims (d, H, slots*N, B).
+    // One TMA descriptor per layer for K and for V.  bf16: dims (d, H, slots*N, B), boxes of
+    // 64 channels x 128 keys.  fp8: K codes (d, H, slots*Np, B) and transposed V codes
+    // (Np, d, H, slots, B), boxes of 128 bytes x 128 rows.
     c->tk.resize(n.layers);
     c->tv.resize(n.layers);
-    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(n.head_dim), static_cast<cuuint64_t>(n.heads),
-                                static_cast<cuuint64_t>(g.slots * g.N), static_cast<cuuint64_t>(n.batch)};
-    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(n.head_dim) * 2,
-                                   static_cast<cuuint64_t>(n.heads) * n.head_dim * 2,
-                                   static_cast<cuuint64_t>(g.slots * g.frame_elems) * 2};
-    const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kBlockN), 1};
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     for (int l = 0; l < n.layers; ++l) {
         for (int kv = 0; kv < 2; ++kv) {
             void *ptr = c->base + (kv ? g.v : g.k) + g.layer_stride * l;
-            CUresult r = encode(kv ? &c->tv[l] : &c->tk[l], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, ptr, dims, strides,
-                                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+            CUresult r;
+            if (!g.f8) {
+                const cuuint64_t dims[4] = {static_cast<cuuint64_t>(n.head_dim), static_cast<cuuint64_t>(n.heads),
+                                            static_cast<cuuint64_t>(g.slots * g.N), static_cast<cuuint64_t>(n.batch)};
+                const cuuint64_t strides[3] = {static_cast<cuuint64_t>(n.head_dim) * 2,
+                                               static_cast<cuuint64_t>(n.heads) * n.head_dim * 2,
+                                               static_cast<cuuint64_t>(g.slots * g.frame_elems) * 2};
+                const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kBlockN), 1};
+                r = encode(kv ? &c->tv[l] : &c->tk[l], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, ptr, dims, strides, box,
+                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+            } else if (kv == 0) {
+                const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(n.heads),
+                                            static_cast<cuuint64_t>(g.slots * g.np_tokens),
+                                            static_cast<cuuint64_t>(n.batch)};
+                const cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(n.heads) * 128,
+                                               static_cast<cuuint64_t>(g.slots * g.np_tokens * n.heads) * 128};
+                const cuuint32_t box[4] = {128, 1, static_cast<cuuint32_t>(kBlockN), 1};
+                r = encode(&c->tk[l], CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, ptr, dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+            } else {
+                const cuuint64_t dims[5] = {static_cast<cuuint64_t>(g.np_tokens), 128,
+                                            static_cast<cuuint64_t>(n.heads), static_cast<cuuint64_t>(g.slots),
+                                            static_cast<cuuint64_t>(n.batch)};
+                const cuuint64_t strides[4] = {static_cast<cuuint64_t>(g.np_tokens),
+                                               static_cast<cuuint64_t>(g.np_tokens) * 128,
+                                               static_cast<cuuint64_t>(g.np_tokens) * 128 * n.heads,
+                                               static_cast<cuuint64_t>(g.np_tokens) * 128 * n.heads * g.slots};
+                const cuuint32_t box[5] = {static_cast<cuuint32_t>(kBlockN), 128, 1, 1, 1};
+                r = encode(&c->tv[l], CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, ptr, dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+            }
             if (r != CUDA_SUCCESS) {
                 delete c;
                 return fail(SDV2_E_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
@@ -411,15 +472,18 @@ sdv2_status sdv2_cache_create(const sdv2_cache_config *cfg, void *dev_buf, size_
         }
     }
     {
+        // rotated queries: bf16 (d, H, Lq, B) in 64-channel boxes, or E4M3 codes in 128-byte boxes
+        const cuuint64_t esz = g.f8 ? 1 : 2;
         const cuuint64_t qdims[4] = {static_cast<cuuint64_t>(n.head_dim), static_cast<cuuint64_t>(n.heads),
                                      static_cast<cuuint64_t>(g.lq), static_cast<cuuint64_t>(n.batch)};
-        const cuuint64_t qstrides[3] = {static_cast<cuuint64_t>(n.head_dim) * 2,
-                                        static_cast<cuuint64_t>(n.heads) * n.head_dim * 2,
-                                        static_cast<cuuint64_t>(g.lq) * n.heads * n.head_dim * 2};
-        const cuuint32_t qbox[4] = {64, 1, static_cast<cuuint32_t>(kBlockM), 1};
+        const cuuint64_t qstrides[3] = {static_cast<cuuint64_t>(n.head_dim) * esz,
+                                        static_cast<cuuint64_t>(n.heads) * n.head_dim * esz,
+                                        static_cast<cuuint64_t>(g.lq) * n.heads * n.head_dim * esz};
+        const cuuint32_t qbox[4] = {g.f8 ? 128u : 64u, 1, static_cast<cuuint32_t>(kBlockM), 1};
         for (int buf = 0; buf < 2; ++buf) {
-            CUresult r = encode(&c->tq[buf], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, c->base + g.q_rot + buf * g.q_rot_bytes,
-                                qdims, qstrides, qbox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CUresult r = encode(&c->tq[buf], g.f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                                c->base + g.q_rot + buf * g.q_rot_bytes, qdims, qstrides, qbox, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
             if (r != CUDA_SUCCESS) {
                 delete c;
@@ -468,6 +532,17 @@ sdv2_status sdv2_kv_append(sdv2_cache *c, int32_t layer, const void *k, const vo
     p.n_h = n.rope_pairs[1];
     p.n_w = n.rope_pairs[2];
     p.slots = static_cast<int32_t>(c->g.slots);
+    if (c->g.f8) {
+        p.k_layer = p.v_layer = nullptr;
+        p.k8_layer = reinterpret_cast<uint8_t *>(c->base + c->g.k + c->g.layer_stride * layer);
+        p.v8t_layer = reinterpret_cast<uint8_t *>(c->base + c->g.v + c->g.layer_stride * layer);
+        p.k_scale_layer = reinterpret_cast<float *>(c->base + c->g.k_scale + c->g.scale_layer_stride * layer);
+        p.v_scale_layer = reinterpret_cast<float *>(c->base + c->g.v_scale + c->g.scale_layer_stride * layer);
+        p.tokens = static_cast<int32_t>(c->g.N);
+        p.np_tokens = static_cast<int32_t>(c->g.np_tokens);
+        p.n_blk = c->g.n_blk;
+        p.scale_slot_stride = c->g.scale_slot_stride;
+    }
     auto flush = [&]() -> sdv2_status {
         if (p.n_frames == 0) return SDV2_OK;
         cudaError_t e = launch_append(p, c->sm_count, reinterpret_cast<cudaStream_t>(stream));
@@ -561,6 +636,15 @@ sdv2_status sdv2_chunk_attention(sdv2_cache *c, int32_t layer, const void *q, vo
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
     p.rope_base = n.rope_base;
     p.rope_reset = n.rope_reset_period;
+    if (g.f8) {
+        p.k_scale = reinterpret_cast<const float *>(c->base + g.k_scale + g.scale_layer_stride * layer);
+        p.v_scale = reinterpret_cast<const float *>(c->base + g.v_scale + g.scale_layer_stride * layer);
+        p.q_scale = reinterpret_cast<float *>(c->base + g.q_scale + qbuf * g.q_scale_bytes);
+        p.slots = static_cast<int32_t>(g.slots);
+        p.np_tokens = static_cast<int32_t>(g.np_tokens);
+        p.n_blk = g.n_blk;
+        p.scale_slot_stride = g.scale_slot_stride;
+    }
     for (int b0 = 0; b0 < n.batch; b0 += streams_per_launch) {
         const int nb = std::min(streams_per_launch, n.batch - b0);
         p.b_offset = b0;
@@ -578,7 +662,7 @@ sdv2_status sdv2_chunk_attention(sdv2_cache *c, int32_t layer, const void *q, vo
         }
         if (!any) continue;
         p.n_units = n_active * n.heads * g.n_qpairs;
-        const AttnPlan plan = plan_attention(n, g, p.n_units, max_kv_tiles(keys.data() + b0, nb), c->sm_count);
+        const AttnPlan plan = plan_attention(n, g, p.n_units, max_kv_tiles(g, keys.data() + b0, nb), c->sm_count);
         p.n_whole = static_cast<int32_t>(plan.whole);
         p.n_pieces = plan.pieces;
         cudaError_t e = launch_rope_q(p, c->sm_count, s);
@@ -629,10 +713,20 @@ sdv2_status sdv2_sink_refresh(sdv2_cache *c, const void *hidden, float tau, cons
     p.sink_embed = reinterpret_cast<double *>(c->base + g.sink_embed);
     p.sink_frame = reinterpret_cast<int64_t *>(c->base + g.sink_frame);
     p.out_slot = out_slot_dev;
-    p.k_cache = reinterpret_cast<uint16_t *>(c->base + g.k);
-    p.v_cache = reinterpret_cast<uint16_t *>(c->base + g.v);
-    p.layer_stride_elems = static_cast<int64_t>(g.layer_stride / 2);
-    p.frame_elems = g.frame_elems;
+    // slot-to-slot copy regions: K and V (codes, for the fp8 cache, plus their scales)
+    const int64_t kv_slot_bytes = g.layer_stride / (static_cast<int64_t>(n.batch) * g.slots);
+    p.copy_base[0] = c->base + g.k;
+    p.copy_base[1] = c->base + g.v;
+    p.copy_layer_bytes[0] = p.copy_layer_bytes[1] = static_cast<int64_t>(g.layer_stride);
+    p.copy_slot_bytes[0] = p.copy_slot_bytes[1] = kv_slot_bytes;
+    p.n_copy = 2;
+    if (g.f8) {
+        p.copy_base[2] = c->base + g.k_scale;
+        p.copy_base[3] = c->base + g.v_scale;
+        p.copy_layer_bytes[2] = p.copy_layer_bytes[3] = static_cast<int64_t>(g.scale_layer_stride);
+        p.copy_slot_bytes[2] = p.copy_slot_bytes[3] = 4ll * g.scale_slot_stride;
+        p.n_copy = 4;
+    }
     p.batch = n.batch;
     p.lq = static_cast<int32_t>(g.lq);
     p.dim = n.embed_dim;
@@ -934,7 +1028,7 @@ sdv2_status sdv2_attention_plan(const sdv2_cache_config *cfg, const int64_t *key
     for (int b = 0; b < std::min(n.batch, kMaxBatch); ++b)
         if (keys[b] > 0) ++active;
     const AttnPlan plan = plan_attention(n, g, static_cast<int64_t>(active) * n.heads * g.n_qpairs,
-                                         max_kv_tiles(keys, std::min(n.batch, kMaxBatch)), sm_count);
+                                         max_kv_tiles(g, keys, std::min(n.batch, kMaxBatch)), sm_count);
     *whole_units = static_cast<int32_t>(plan.whole);
     *pieces = plan.pieces;
     return SDV2_OK;

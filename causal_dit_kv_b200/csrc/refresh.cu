@@ -15,8 +15,9 @@
 // and norms in fp64, takes the decision, updates the sink embedding and the
 // sink-frame record, and writes out_slot[b].
 // Kernel 2, grid (blocks, B): if out_slot[b] >= 0, copies slot last_slot[b]
-// to slot out_slot[b] in every layer, K and V, as 16-byte vectors; otherwise
-// the blocks return at once.
+// to slot out_slot[b] in every layer, K and V (for the fp8 cache: K and V
+// codes and their block scales), as 16-byte vectors; otherwise the blocks
+// return at once.
 #include <cmath>
 
 #include "ptx.cuh"
@@ -191,18 +192,18 @@ __global__ void __launch_bounds__(256) refresh_copy_kernel(const __grid_constant
     const int dst_slot = *reinterpret_cast<volatile const int32_t *>(p.out_slot + b);
     if (dst_slot < 0) return;
     const int src_slot = p.last_slot[b];
-    const int64_t vec_per_frame = p.frame_elems / 8;
-    const int64_t total = 2ll * p.layers * vec_per_frame;
-    for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < total;
-         g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t per_kv = p.layers * vec_per_frame;
-        uint16_t *base = g < per_kv ? p.k_cache : p.v_cache;
-        const int64_t r = g < per_kv ? g : g - per_kv;
-        const int64_t layer = r / vec_per_frame;
-        const int64_t vec = r - layer * vec_per_frame;
-        uint16_t *lb = base + layer * p.layer_stride_elems + static_cast<int64_t>(b) * p.slots * p.frame_elems;
-        const uint4 x = *reinterpret_cast<const uint4 *>(lb + static_cast<int64_t>(src_slot) * p.frame_elems + vec * 8);
-        *reinterpret_cast<uint4 *>(lb + static_cast<int64_t>(dst_slot) * p.frame_elems + vec * 8) = x;
+    for (int r = 0; r < p.n_copy; ++r) {
+        const int64_t vec_per_slot = p.copy_slot_bytes[r] / 16;
+        const int64_t total = static_cast<int64_t>(p.layers) * vec_per_slot;
+        for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < total;
+             g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+            const int64_t layer = g / vec_per_slot;
+            const int64_t vec = g - layer * vec_per_slot;
+            uint8_t *lb = p.copy_base[r] + layer * p.copy_layer_bytes[r] +
+                          static_cast<int64_t>(b) * p.slots * p.copy_slot_bytes[r];
+            const uint4 x = *reinterpret_cast<const uint4 *>(lb + src_slot * p.copy_slot_bytes[r] + vec * 16);
+            *reinterpret_cast<uint4 *>(lb + dst_slot * p.copy_slot_bytes[r] + vec * 16) = x;
+        }
     }
 }
 

@@ -45,6 +45,12 @@ struct AppendParams {
     int32_t dst_slot[kAppendMaxFrames];  // ring slot it goes to
     uint8_t tab_row[kAppendMaxFrames];   // row of tab_t with the frame's phase
     double tab_t[kAppendTabEntries][2];  // [distinct phase][n_t] temporal cos, sin
+    // fp8 (E4M3) cache only: codes and per-(slot, head, 128-token block) scales of this layer
+    uint8_t *k8_layer;          // [B][slots][Np][H][d]
+    uint8_t *v8t_layer;         // [B][slots][H][d][Np]
+    float *k_scale_layer;       // [B][slots][scale_slot_stride] (head h, block j at h * n_blk + j)
+    float *v_scale_layer;
+    int32_t tokens, np_tokens, n_blk, scale_slot_stride;
 };
 
 struct AttnParams {
@@ -70,6 +76,12 @@ struct AttnParams {
     double rope_base;           // RoPE frequency base
     int32_t rope_reset;         // temporal phase period (0: none)
     int64_t f0[kMaxBatch];      // first frame of each stream's chunk
+    // fp8 (E4M3) cache only: KV tiles are 128-token blocks of one slot (slot s, block j at
+    // tile s * n_blk + j), each with its own K and V scale; queries are rounded to E4M3 per row
+    const float *k_scale;       // this layer: [B][slots][scale_slot_stride]
+    const float *v_scale;
+    float *q_scale;             // scratch [B][Lq][H]: scale of each rotated query row
+    int32_t slots, np_tokens, n_blk, scale_slot_stride;
 };
 
 struct RefreshParams {
@@ -79,10 +91,13 @@ struct RefreshParams {
     double *sink_embed;         // [B][S][D]
     int64_t *sink_frame;        // [B][S]
     int32_t *out_slot;          // [B] (caller's)
-    uint16_t *k_cache;          // all layers [L][B][slots][N][H][d]
-    uint16_t *v_cache;
-    int64_t layer_stride_elems; // elements between layers
-    int64_t frame_elems;        // N*H*d
+    // Regions copied slot to slot on a refresh (bf16 cache: K, V; fp8 cache: K, V codes and
+    // their scales); region r of stream b, slot s, layer l starts at
+    // copy_base[r] + l * copy_layer_bytes[r] + (b * slots + s) * copy_slot_bytes[r].
+    uint8_t *copy_base[4];
+    int64_t copy_layer_bytes[4];
+    int64_t copy_slot_bytes[4]; // multiples of 16
+    int32_t n_copy;
     int32_t batch, lq, dim, sinks, slots, layers, row_chunks;
     double tau;
     int32_t active[kMaxBatch];  // 1 if stream takes part in this call

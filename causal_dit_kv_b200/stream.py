@@ -14,10 +14,12 @@ class KVCache:
     """Sink + rolling-window K/V cache of ``layers`` DiT layers for ``batch`` streams."""
 
     def __init__(self, batch, layers, heads, head_dim, frame_h, frame_w, chunk_frames, sink_frames, window_frames,
-                 rope_pairs=(0, 0, 0), rope_reset_period=0, embed_dim=0, rope_base=10000.0, device="cuda"):
+                 rope_pairs=(0, 0, 0), rope_reset_period=0, embed_dim=0, rope_base=10000.0, device="cuda",
+                 kv_format="bf16"):
         import torch
         self.cfg = B.make_cache_config(batch, layers, heads, head_dim, frame_h, frame_w, chunk_frames, sink_frames,
-                                       window_frames, rope_pairs, rope_reset_period, embed_dim, rope_base)
+                                       window_frames, rope_pairs, rope_reset_period, embed_dim, rope_base, kv_format)
+        self.kv_format = kv_format
         self.nbytes = B.sdv2_cache_bytes(self.cfg)
         self.buffer = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
         self.handle = B.sdv2_cache_create(self.cfg, self.buffer, self.nbytes)
@@ -64,15 +66,48 @@ class KVCache:
 
     def k_cache(self, layer):
         import torch
+        if self.kv_format != "bf16":
+            raise ValueError("an fp8 cache holds codes: use k_codes / v_codes / k_scales / v_scales")
         shape = (self.batch, self.slots, self.tokens_per_frame, self.heads, self.head_dim)
         off = self.layout.k_offset + layer * self.layout.layer_stride
         return self._region(off, self.layout.layer_stride, torch.bfloat16, shape)
 
     def v_cache(self, layer):
         import torch
+        if self.kv_format != "bf16":
+            raise ValueError("an fp8 cache holds codes: use k_codes / v_codes / k_scales / v_scales")
         shape = (self.batch, self.slots, self.tokens_per_frame, self.heads, self.head_dim)
         off = self.layout.v_offset + layer * self.layout.layer_stride
         return self._region(off, self.layout.layer_stride, torch.bfloat16, shape)
+
+    # fp8 cache: E4M3 codes (uint8) and their per-block scales
+    def k_codes(self, layer):
+        """uint8 [B][S+W][Np][H][d]."""
+        import torch
+        shape = (self.batch, self.slots, self.layout.tokens_padded, self.heads, self.head_dim)
+        return self._region(self.layout.k_offset + layer * self.layout.layer_stride, self.layout.layer_stride,
+                            torch.uint8, shape)
+
+    def v_codes(self, layer):
+        """uint8 [B][S+W][H][d][Np] (token index innermost)."""
+        import torch
+        shape = (self.batch, self.slots, self.heads, self.head_dim, self.layout.tokens_padded)
+        return self._region(self.layout.v_offset + layer * self.layout.layer_stride, self.layout.layer_stride,
+                            torch.uint8, shape)
+
+    def _scales(self, offset, layer):
+        import torch
+        nb = self.layout.tokens_padded // 128
+        full = self._region(offset + layer * self.layout.scale_layer_stride, self.layout.scale_layer_stride,
+                            torch.float32, (self.batch, self.slots, self.layout.scale_slot_stride))
+        return full[:, :, :self.heads * nb].reshape(self.batch, self.slots, self.heads, nb)
+
+    def k_scales(self, layer):
+        """fp32 [B][S+W][H][Np/128]."""
+        return self._scales(self.layout.k_scale_offset, layer)
+
+    def v_scales(self, layer):
+        return self._scales(self.layout.v_scale_offset, layer)
 
     def sink_embed(self):
         import torch

@@ -80,7 +80,24 @@ typedef struct {
     int32_t rope_reset_period; /* T_reset: temporal phase = frame mod T_reset; 0 = never reset */
     int32_t embed_dim;      /* D: width of the hidden states used for sink refresh (0 = no refresh) */
     double rope_base;       /* RoPE base (10000 when <= 0) */
+    int32_t kv_format;      /* SDV2_KV_BF16 (0) or SDV2_KV_FP8_E4M3 (1) */
 } sdv2_cache_config;
+
+/* Storage format of the cached K and V.
+ * SDV2_KV_BF16: the rotated keys and the values as bf16.
+ * SDV2_KV_FP8_E4M3: the same values quantised to FP8 E4M3 in blocks, a
+ *   reading of the FP8 item on the roadmap of [G] (the page names the format
+ *   only).  A slot's N tokens are padded to Np = ceil(N/128)*128 and cut into
+ *   blocks of 128 tokens; each (layer, stream, slot, head, block) has one fp32
+ *   scale for K and one for V: scale = amax/448 over the block's tokens and the
+ *   head's d channels, code = E4M3(x * (448/amax)) with round-to-nearest-even
+ *   and saturation (codes 0 for amax = 0); the dequantised value is
+ *   code * scale.  K codes are token-major [B][S+W][Np][H][d]; V codes are
+ *   transposed per slot, [B][S+W][H][d][Np], so both tensor-core operands are
+ *   K-major; padding tokens hold code 0.  The attention rounds each rotated
+ *   query row to E4M3 with its own scale and the probabilities to E4M3 before
+ *   the products (fp32 accumulation).  Requires head_dim 128. */
+enum { SDV2_KV_BF16 = 0, SDV2_KV_FP8_E4M3 = 1 };
 
 typedef struct sdv2_cache sdv2_cache;
 
@@ -95,6 +112,13 @@ typedef struct {
     uint64_t scratch_offset;  /* attention split-KV partials and refresh reductions */
     uint64_t scratch_bytes;
     uint64_t total_bytes;     /* == sdv2_cache_bytes(cfg) */
+    /* fp8 cache only (zero for bf16): k_offset / v_offset then hold the E4M3 codes,
+     * K [L][B][S+W][Np][H][d] and V [L][B][S+W][H][d][Np], layer_stride bytes apart. */
+    uint64_t k_scale_offset;  /* fp32 [L][B][S+W][scale_slot_stride]: head h, block j at h*(Np/128)+j */
+    uint64_t v_scale_offset;
+    uint64_t scale_layer_stride; /* bytes between layers of the scales */
+    uint32_t scale_slot_stride;  /* floats per slot (H*Np/128 rounded up to a multiple of 4) */
+    uint32_t tokens_padded;      /* Np */
 } sdv2_cache_layout;
 
 /* Device bytes the caller must allocate for a cache with this config;

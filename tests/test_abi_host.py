@@ -79,6 +79,30 @@ def test_layout_regions_are_disjoint_and_aligned(B):
     assert lay.scratch_offset + lay.scratch_bytes == lay.total_bytes == B.sdv2_cache_bytes(cfg)
 
 
+def test_fp8_layout_and_validation(B):
+    # 480x832 latent (N = 1560): slots padded to 13 blocks of 128 tokens
+    cfg = B.make_cache_config(4, 30, 12, 128, 30, 52, 2, 1, 8, embed_dim=1536, kv_format="fp8")
+    lay = B.sdv2_cache_layout_of(cfg)
+    assert lay.tokens_padded == 1664
+    assert lay.layer_stride == 4 * 9 * 1664 * 12 * 128                 # one byte per code
+    assert lay.scale_slot_stride == 12 * 13 == 156
+    assert lay.scale_layer_stride == 4 * 9 * 156 * 4
+    offs = [lay.k_offset, lay.v_offset, lay.k_scale_offset, lay.v_scale_offset, lay.sink_embed_offset,
+            lay.scratch_offset]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    assert lay.v_offset >= lay.k_offset + 30 * lay.layer_stride
+    assert lay.v_scale_offset >= lay.k_scale_offset + 30 * lay.scale_layer_stride
+    bf16 = B.sdv2_cache_layout_of(B.make_cache_config(4, 30, 12, 128, 30, 52, 2, 1, 8, embed_dim=1536))
+    assert bf16.k_scale_offset == 0 and bf16.tokens_padded == 0
+    assert lay.total_bytes < bf16.total_bytes                          # half the K/V bytes plus scales
+    odd = B.make_cache_config(1, 1, 3, 128, 4, 4, 1, 1, 2, kv_format="fp8")
+    assert B.sdv2_cache_layout_of(odd).scale_slot_stride == 4        # 3 heads x 1 block, padded to 4 floats
+    for bad in (B.make_cache_config(1, 1, 1, 64, 4, 4, 1, 1, 2, kv_format="fp8"),   # head_dim 64
+                B.make_cache_config(1, 1, 1, 128, 4, 4, 1, 1, 2, kv_format=7)):     # unknown format
+        with pytest.raises(B.SDV2Error):
+            B.sdv2_cache_bytes(bad)
+
+
 def test_split_plan(B):
     c2 = B.make_cache_config(1, 30, 12, 128, 32, 32, 1, 1, 6)
     # 48 units (12 heads x 4 query-tile pairs) on 148 SMs: every unit split over the KV range

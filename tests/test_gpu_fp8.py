@@ -1,0 +1,165 @@
+"""fp8 (E4M3) cache: CUDA path vs the oracle through the C ABI (B200).
+
+Codes and block scales of the cache are compared bit for bit (both sides take
+every rounding in fp32 with nearest-even).  The attention output is compared
+with the oracle's fp64 attention over the dequantised cache.  The CUDA path
+also rounds each rotated query row and the probabilities to E4M3 before its
+tensor-core products, so the tolerance is derived from those two roundings,
+each a relative error of RMS at most rho = 2^-4 / sqrt(3) per element:
+
+  * the logit of key j moves by ds_j, RMS scale * rho * sqrt(sum_k q_k^2 k_jk^2);
+  * so p_j moves by a relative eps_j with eps_j^2 = ds_j^2 + rho^2 (its own rounding);
+  * the output o_c = sum_j p_j v_jc (p normalised) moves by sum_j p_j eps_j (v_jc - o_c),
+    RMS sigma_c = sqrt(sum_j p_j^2 eps_j^2 (v_jc - o_c)^2).
+
+Every element must lie within 6 sigma (+ the bf16 rounding of the output), and
+the mean of |error| / sigma must stay below 1.2 (0.8 for an exact Gaussian
+model; the rho above over-estimates the RMS of E4M3 rounding).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+from harness import f32
+from oracle.sdv2_fp8 import OracleFp8Cache, chunk_attention_fp8, kv_append_fp8, sink_refresh_fp8
+
+pytestmark = pytest.mark.gpu
+
+
+RHO = 2.0 ** -4 / math.sqrt(3.0)
+
+
+def fp8_sigma(qr, k, v, scale):
+    """Per-element RMS of the CUDA path's deviation (model above) and the reference output.
+    qr [rows][d] rotated queries, k, v [Lk][d] dequantised cache of one head."""
+    o, p = O.attention_reference(qr, k, v, scale)
+    ds2 = (scale * RHO) ** 2 * ((qr ** 2) @ (k ** 2).T)
+    w = p ** 2 * (ds2 + RHO ** 2)                                   # [rows][Lk]
+    var = w @ (v ** 2) - 2.0 * o * (w @ v) + o ** 2 * w.sum(axis=1, keepdims=True)
+    return np.sqrt(np.maximum(var, 0.0)), o
+
+
+class Fp8Pair:
+    def __init__(self, seed, **cfg):
+        from causal_dit_kv_b200 import KVCache
+        self.seed = seed
+        self.cfg = O.CacheConfig(**cfg)
+        self.gpu = KVCache(**cfg, kv_format="fp8")
+        self.ora = OracleFp8Cache(self.cfg)
+        self.next = [0] * self.cfg.batch
+
+    def step_frames(self, active=None):
+        f0 = []
+        for b in range(self.cfg.batch):
+            if active is None or b in active:
+                f0.append(self.next[b])
+                self.next[b] += self.cfg.chunk_frames
+            else:
+                f0.append(-1)
+        return f0
+
+    def run_layer(self, step, layer, f0, rows=None):
+        c = self.cfg
+        q, k, v = synth.chunk_qkv(self.seed, c.batch, c.chunk_tokens, c.heads, c.head_dim, step, layer)
+        self.q_bits = synth.bf16_bits(q)
+        self.gpu.kv_append(layer, k.cuda(), v.cuda(), f0)
+        kv_append_fp8(self.ora, layer, synth.bf16_bits(k), synth.bf16_bits(v), f0)
+        out = torch.zeros((c.batch, c.chunk_tokens, c.heads, c.head_dim), dtype=torch.bfloat16, device="cuda")
+        scale = 1.0 / math.sqrt(c.head_dim)
+        self.gpu.chunk_attention(layer, q.cuda(), out, f0, scale)
+        want = chunk_attention_fp8(self.ora, layer, self.q_bits, f0, f32(scale), rows=rows)
+        return out, want
+
+    def cache_equal(self, layer):
+        g = self.gpu
+        return (np.array_equal(g.k_codes(layer).cpu().numpy(), self.ora.k8[layer]),
+                np.array_equal(g.v_codes(layer).cpu().numpy(), self.ora.v8t[layer]),
+                np.array_equal(g.k_scales(layer).cpu().numpy(), self.ora.k_scale[layer]),
+                np.array_equal(g.v_scales(layer).cpu().numpy(), self.ora.v_scale[layer]))
+
+
+def _check_out(pair, out, want, layer, f0, q_bits, rows=None):
+    c = pair.cfg
+    g = out.float().cpu().numpy().astype(np.float64)
+    sel = np.arange(c.chunk_tokens) if rows is None else np.asarray(rows)
+    scale = float(f32(1.0 / math.sqrt(c.head_dim)))
+    ratios = []
+    for b in range(c.batch):
+        if f0[b] < 0:
+            continue
+        sv, wv = O.valid_slot_counts(f0[b] + c.chunk_frames, c.sink_frames, c.window_frames)
+        k, v = pair.ora.dequantized(layer, b, sv + wv)
+        qr = O.chunk_queries_rotated(c, q_bits[b], f0[b])[sel]
+        for h in range(c.heads):
+            sigma, o = fp8_sigma(qr[:, h], k[:, h], v[:, h], scale)
+            assert np.allclose(o, want[b, sel, h], rtol=0, atol=1e-12)
+            err = np.abs(g[b, sel, h] - o)
+            bound = 6.0 * sigma + 2.0 ** -8 * np.abs(o) + 1e-4
+            assert (err <= bound).all(), (b, h, float((err / bound).max()))
+            ratios.append(err / (sigma + 1e-6))
+    assert float(np.concatenate([r.ravel() for r in ratios]).mean()) < 1.2
+
+
+@pytest.mark.parametrize("case", ["ragged_single_tile", "two_tiles", "multi_frame_chunks"])
+def test_fp8_stream_parity(case):
+    cfg = {
+        # N = 150: two blocks per slot, the second of 22 tokens; one query tile (both accumulator sets)
+        "ragged_single_tile": dict(batch=2, layers=1, heads=2, head_dim=128, frame_h=10, frame_w=15, chunk_frames=1,
+                                   sink_frames=1, window_frames=3, rope_reset_period=4),
+        # N = 320: three blocks per slot; query-tile pairs of 2 tiles and of 1 tile
+        "two_tiles": dict(batch=1, layers=2, heads=3, head_dim=128, frame_h=16, frame_w=20, chunk_frames=1,
+                          sink_frames=1, window_frames=2),
+        # T' = 2, N = 128 (whole blocks), streams at different positions
+        "multi_frame_chunks": dict(batch=3, layers=1, heads=2, head_dim=128, frame_h=8, frame_w=16, chunk_frames=2,
+                                   sink_frames=2, window_frames=4),
+    }[case]
+    pair = Fp8Pair(seed=3001, **cfg)
+    for step in range(7):
+        active = None if case != "multi_frame_chunks" else [b for b in range(3) if step >= b]
+        f0 = pair.step_frames(active)
+        for layer in range(pair.cfg.layers):
+            out, want = pair.run_layer(step, layer, f0)
+            assert all(pair.cache_equal(layer)), (step, layer, pair.cache_equal(layer))
+            _check_out(pair, out, want, layer, f0, pair.q_bits)
+    assert pair.gpu.check() == 0
+
+
+def test_fp8_refresh_copies_codes_and_scales():
+    cfg = dict(batch=2, layers=2, heads=2, head_dim=128, frame_h=8, frame_w=20, chunk_frames=1, sink_frames=2,
+               window_frames=2, embed_dim=64)
+    pair = Fp8Pair(seed=3002, **cfg)
+    D = cfg["embed_dim"]
+    slot = torch.empty(2, dtype=torch.int32, device="cuda")
+    for step in range(6):
+        f0 = pair.step_frames()
+        for layer in range(2):
+            pair.run_layer(step, layer, f0)
+        # alternate the chunk embedding between two orthogonal directions: refreshes fire
+        hid = torch.zeros((2, pair.cfg.chunk_tokens, D), dtype=torch.bfloat16)
+        hid[:, :, step % 2] = 1.0
+        pair.gpu.sink_refresh(hid.cuda(), 0.9, f0, slot)
+        want = sink_refresh_fp8(pair.ora, synth.bf16_bits(hid), 0.9, f0)
+        assert slot.cpu().tolist() == [int(x) for x in want]
+        for layer in range(2):
+            assert all(pair.cache_equal(layer)), (step, layer)
+    assert pair.gpu.check() == 0
+
+
+def test_fp8_full_size_1p3b_sampled():
+    """Wan-1.3B 512x512 layer shape (12 heads, 1024 tokens per frame, 7 slots) in the
+    fp8 format, after the ring has wrapped; attention checked on sampled rows."""
+    cfg = dict(batch=1, layers=1, heads=12, head_dim=128, frame_h=32, frame_w=32, chunk_frames=1, sink_frames=1,
+               window_frames=6)
+    pair = Fp8Pair(seed=3003, **cfg)
+    rows = np.concatenate([np.arange(0, 8), np.arange(250, 262), np.arange(1016, 1024)])
+    for step in range(9):
+        f0 = pair.step_frames()
+        out, want = pair.run_layer(step, 0, f0, rows=rows if step >= 7 else np.arange(1))
+        if step >= 7:
+            assert all(pair.cache_equal(0))
+            _check_out(pair, out, want, 0, f0, pair.q_bits, rows)
+    assert pair.gpu.check() == 0
