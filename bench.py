@@ -47,6 +47,14 @@ WORKLOADS = {
 WORKLOADS["wan1.3b-128x128-b16"] = dict(batch=16, layers=30, heads=12, head_dim=128, frame_h=8, frame_w=8,
                                         chunk_frames=1, sink_frames=1, window_frames=6, embed_dim=1536,
                                         motion=(16, 16, 16))
+# the same shapes with the fp8 (E4M3) block-scaled cache; 128x256 video (8x16 = 128 latent
+# tokens per frame, whole 128-token blocks) for the memory-bound regime in both formats
+WORKLOADS["wan1.3b-512x512-fp8"] = dict(WORKLOADS["wan1.3b-512x512"], kv_format="fp8")
+WORKLOADS["wan14b-512x512-b8-fp8"] = dict(WORKLOADS["wan14b-512x512-b8"], kv_format="fp8")
+WORKLOADS["wan1.3b-128x256-b16"] = dict(batch=16, layers=30, heads=12, head_dim=128, frame_h=8, frame_w=16,
+                                        chunk_frames=1, sink_frames=1, window_frames=6, embed_dim=1536,
+                                        motion=(16, 16, 32))
+WORKLOADS["wan1.3b-128x256-b16-fp8"] = dict(WORKLOADS["wan1.3b-128x256-b16"], kv_format="fp8")
 WORKLOADS["tiny-stream"] = dict(batch=1, layers=1, heads=2, head_dim=64, frame_h=4, frame_w=4, chunk_frames=1,
                                 sink_frames=1, window_frames=2, embed_dim=64, motion=(16, 4, 4))
 DEFAULT_WORKLOAD = "wan1.3b-512x512"
@@ -88,14 +96,19 @@ def workload_config(name, w, world):
     """The JSON config block of a workload (shared by both arms)."""
     n = w["frame_h"] * w["frame_w"]
     slots = w["sink_frames"] + w["window_frames"]
-    cache_mb = 2.0 * w["layers"] * w["batch"] * slots * n * w["heads"] * w["head_dim"] * 2 / 1e6
+    cache_mb = 2.0 * w["layers"] * w["batch"] * slots * n * w["heads"] * w["head_dim"] * kv_elem(w) / 1e6
     return {"workload": name, "batch": w["batch"], "layers": w["layers"], "heads": w["heads"],
             "head_dim": w["head_dim"], "tokens_per_frame": n, "chunk_frames": w["chunk_frames"],
             "sink_frames": w["sink_frames"], "window_frames": w["window_frames"], "keys_per_stream": slots * n,
             "queries_per_stream": w["chunk_frames"] * n, "refresh_embed_dim": w["embed_dim"],
             "motion_latent": list(w["motion"]),
             "l2": "inputs larger than L2 (per-step caches %.0f MB over %d layers)" % (cache_mb, w["layers"]),
-            "parallelism": f"replicas x{world}"}
+            "kv_format": w.get("kv_format", "bf16"), "parallelism": f"replicas x{world}"}
+
+
+def kv_elem(w):
+    """Bytes per cached K or V element."""
+    return 1 if w.get("kv_format", "bf16") == "fp8" else 2
 
 
 def attn_flops(w, keys):
@@ -104,9 +117,18 @@ def attn_flops(w, keys):
 
 
 def attn_bytes(w, keys):
+    """Bytes one attention kernel launch must move: K and V read once, the rotated queries
+    read, O (bf16) written.  The fp8 cache stores 1-byte codes, reads E4M3 queries, and adds
+    one K and one V scale per 128-token block and head and one scale per query row."""
     lq = w["chunk_frames"] * w["frame_h"] * w["frame_w"]
     hd = w["heads"] * w["head_dim"]
-    return sum(2.0 * 2 * k * hd + 2.0 * 2 * lq * hd for k in keys)   # K+V read once, Q read, O written
+    e = kv_elem(w)
+    total = 0.0
+    for k in keys:
+        total += 2.0 * e * k * hd + e * lq * hd + 2.0 * lq * hd
+        if e == 1:
+            total += 2 * 4.0 * w["heads"] * k / 128 + 4.0 * w["heads"] * lq
+    return total
 
 
 def steady_keys(w):
@@ -207,7 +229,9 @@ def run_ours(args, w, name):
     Lq = Tp * N
     E = w["embed_dim"]
     C, MH, MW = w["motion"]
-    cache = KVCache(B, L, H, D, w["frame_h"], w["frame_w"], Tp, w["sink_frames"], w["window_frames"], embed_dim=E)
+    fp8 = w.get("kv_format", "bf16") == "fp8"
+    cache = KVCache(B, L, H, D, w["frame_h"], w["frame_w"], Tp, w["sink_frames"], w["window_frames"], embed_dim=E,
+                    kv_format=w.get("kv_format", "bf16"))
     mot = MotionState(B, Tp, C, MH, MW, window=4, sigma=2.0, lam=0.9)
     scale = 1.0 / math.sqrt(D)
     dev = torch.device("cuda", local)
@@ -411,6 +435,10 @@ def run_ours(args, w, name):
     kern_avg_s = call_us["attn_kernel"] / 1e6                # chunk_attention_kernel alone
     peaks, peak_src = load_peaks()
     peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    peak_name = "bf16_tflops_sustained"
+    if fp8:
+        # E4M3 products: the measured bf16 peak times the nominal fp8 / bf16 ratio (4.5 / 2.25)
+        peak, peak_name = 2.0 * peak, "bf16_tflops_sustained x 2 (nominal fp8/bf16 ratio)"
     hbm = peaks["hbm_gbs"]
     achieved = flops / attn_avg_s / 1e12
     k_achieved = flops / kern_avg_s / 1e12
@@ -420,20 +448,20 @@ def run_ours(args, w, name):
     kv_gbs = abytes / attn_avg_s / 1e9
     k_kv_gbs = abytes / kern_avg_s / 1e9
     kv_chunk = 2.0 * B * Lq * H * D * 2                      # K + V of the chunk, bf16
-    append_bytes = 2 * kv_chunk                               # read + written
+    append_bytes = kv_chunk + kv_chunk * kv_elem(w) / 2       # read (bf16) + written (bf16 or E4M3 codes)
     refresh_bytes = B * Lq * E * 2 + B * E * 8 * (w["sink_frames"] + 1)
     motion_bytes = B * (Tp + 2) * C * MH * MW * 4             # chunk + previous frame read, last frame written
     traffic = profiled_traffic(name)
     result = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3" if fp8 else "bf16", "data": "synthetic",
         "config": workload_config(name, w, world),
         "roofline": {"kernel": "chunk_attention_kernel", "bound": "hbm" if hbm_bound else "tensor",
                      "achieved": round(k_kv_gbs if hbm_bound else k_achieved, 2), "peak": hbm if hbm_bound else peak,
                      "unit": "GB/s" if hbm_bound else "TFLOP/s",
                      "frac": round(k_kv_gbs / hbm if hbm_bound else k_achieved / peak, 4), "traffic": traffic,
-                     "peak_source": f"{peak_src} " + ("hbm_gbs" if hbm_bound else "bf16_tflops_sustained"),
+                     "peak_source": f"{peak_src} " + ("hbm_gbs" if hbm_bound else peak_name),
                      "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": abytes,
                      "avg_launch_us": round(kern_avg_s * 1e6, 3),
                      "timing": "CUDA events recorded by the library right before and after the kernel's launch "
@@ -488,12 +516,18 @@ def oracle_sample(w, threads=None):
     cfg = O.CacheConfig(batch=B, layers=1, heads=H, head_dim=D, frame_h=w["frame_h"], frame_w=w["frame_w"],
                         chunk_frames=Tp, sink_frames=w["sink_frames"], window_frames=w["window_frames"],
                         embed_dim=w["embed_dim"])
-    cache = O.OracleCache(cfg)
+    if w.get("kv_format", "bf16") == "fp8":
+        from oracle import sdv2_fp8 as F
+        cache = F.OracleFp8Cache(cfg)
+        append, attention, refresh = F.kv_append_fp8, F.chunk_attention_fp8, F.sink_refresh_fp8
+    else:
+        cache = O.OracleCache(cfg)
+        append, attention, refresh = O.kv_append, O.chunk_attention, O.sink_refresh
     # fill to steady state (not timed)
     pre = (w["sink_frames"] + w["window_frames"] + Tp - 1) // Tp + 1
     for s in range(pre):
         _, k, v = synth.chunk_qkv(5, B, Lq, H, D, s, 0)
-        O.kv_append(cache, 0, synth.bf16_bits(k), synth.bf16_bits(v), [s * Tp] * B)
+        append(cache, 0, synth.bf16_bits(k), synth.bf16_bits(v), [s * Tp] * B)
     mcfg = O.MotionConfig(batch=B, channels=w["motion"][0], height=w["motion"][1], width=w["motion"][2])
     mstate = O.MotionState(mcfg)
     lat = synth.motion_latents(5, B, Tp, *w["motion"], n_chunks=2)
@@ -503,10 +537,10 @@ def oracle_sample(w, threads=None):
     f0 = [pre * Tp] * B
     x = next(lat).numpy()
     t0 = time.perf_counter()
-    O.kv_append(cache, 0, synth.bf16_bits(k), synth.bf16_bits(v), f0)
-    O.chunk_attention(cache, 0, synth.bf16_bits(q), f0, 1.0 / math.sqrt(D))
+    append(cache, 0, synth.bf16_bits(k), synth.bf16_bits(v), f0)
+    attention(cache, 0, synth.bf16_bits(q), f0, 1.0 / math.sqrt(D))
     t1 = time.perf_counter()
-    O.sink_refresh(cache, synth.bf16_bits(hid), TAU, f0)
+    refresh(cache, synth.bf16_bits(hid), TAU, f0)
     O.motion_noise_rate(mstate, x)
     t2 = time.perf_counter()
     layer_s = t1 - t0

@@ -115,16 +115,16 @@ __global__ void __launch_bounds__(128) kv_append_kernel(const __grid_constant__ 
 }
 
 // fp8 (E4M3) cache.  Block = one 128-token block of one frame and one head, K
-// (blockIdx.z == 0) or V; thread t takes token t/2 of the block and channels
-// [64 (t & 1), 64 (t & 1) + 64).  Keys are rotated exactly as above (so the
+// (blockIdx.z == 0) or V; thread t takes token t/4 of the block and channels
+// [32 (t & 3), 32 (t & 3) + 32).  Keys are rotated exactly as above (so the
 // quantised values are the bf16 cache's values), the block's largest magnitude
 // is reduced over the block, and every value is coded as E4M3(x * 448/amax)
 // (fp32 product, nearest even, saturating).  K codes go out token-major; V
 // codes are transposed through shared memory into the slot's [H][d][Np] rows.
 // Tokens past N in the last block get code 0 and take no part in the maximum.
-constexpr int kF8AppendThreads = 256;
+constexpr int kF8AppendThreads = 512;
 
-__global__ void __launch_bounds__(kF8AppendThreads) kv_append_fp8_kernel(const __grid_constant__ AppendParams p) {
+__global__ void __launch_bounds__(kF8AppendThreads, 2) kv_append_fp8_kernel(const __grid_constant__ AppendParams p) {
     grid_dependency_wait();
     grid_launch_dependents();
     const int fi = blockIdx.y;
@@ -132,7 +132,7 @@ __global__ void __launch_bounds__(kF8AppendThreads) kv_append_fp8_kernel(const _
     const int h = static_cast<int>(blockIdx.x) % p.heads;
     const int blk = static_cast<int>(blockIdx.x) / p.heads;
     const int tid = threadIdx.x;
-    const int tok = tid >> 1, half = tid & 1;
+    const int tok = tid >> 2, sub = tid & 3;
     const int n = blk * kBlockN + tok;                // token in the frame
     const bool real = n < p.tokens;
     __shared__ double2 s_tab[64];                     // temporal (cos, sin) of this block's frame
@@ -143,13 +143,13 @@ __global__ void __launch_bounds__(kF8AppendThreads) kv_append_fp8_kernel(const _
     __syncthreads();
     const int b = p.src_b[fi];
     const int slot = p.dst_slot[fi];
-    uint32_t w[32];                                   // 64 bf16 values, packed pairs (dims 2j, 2j+1)
+    uint32_t w[16];                                   // 32 bf16 values, packed pairs (dims 2j, 2j+1)
     if (real) {
         const uint16_t *in = (is_v ? p.v_in : p.k_in) + static_cast<int64_t>(b) * p.chunk_tokens * p.heads * 128 +
                              static_cast<int64_t>(p.src_i[fi]) * p.frame_elems +
-                             (static_cast<int64_t>(n) * p.heads + h) * 128 + half * 64;
+                             (static_cast<int64_t>(n) * p.heads + h) * 128 + sub * 32;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 4; ++i) {
             const uint4 x = ld_nc_v4(in + i * 8);
             w[4 * i] = x.x;
             w[4 * i + 1] = x.y;
@@ -163,19 +163,24 @@ __global__ void __launch_bounds__(kF8AppendThreads) kv_append_fp8_kernel(const _
             const double2 *tab_w =
                 reinterpret_cast<const double2 *>(p.rope_w) + static_cast<int64_t>(pcol) * p.n_w - p.n_t - p.n_h;
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
-                const int j = half * 32 + q;
-                const double2 cs = j < p.n_t ? s_tab[j] : (j < p.n_t + p.n_h ? tab_h[j] : tab_w[j]);
-                w[q] = rotate_pair(w[q], cs.x, cs.y);
+            for (int q0 = 0; q0 < 16; q0 += 4) {             // table loads of 4 pairs in flight at a time
+                double2 cs[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int j = sub * 16 + q0 + q;
+                    cs[q] = j < p.n_t ? s_tab[j] : (j < p.n_t + p.n_h ? tab_h[j] : tab_w[j]);
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) w[q0 + q] = rotate_pair(w[q0 + q], cs[q].x, cs[q].y);
             }
         }
     } else {
 #pragma unroll
-        for (int q = 0; q < 32; ++q) w[q] = 0u;
+        for (int q = 0; q < 16; ++q) w[q] = 0u;
     }
     float am = 0.0f;
 #pragma unroll
-    for (int q = 0; q < 32; ++q) am = fmaxf(am, fmaxf(fabsf(bf16_lo(w[q])), fabsf(bf16_hi(w[q]))));
+    for (int q = 0; q < 16; ++q) am = fmaxf(am, fmaxf(fabsf(bf16_lo(w[q])), fabsf(bf16_hi(w[q]))));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
     if ((tid & 31) == 0) s_max[tid >> 5] = am;
@@ -185,9 +190,9 @@ __global__ void __launch_bounds__(kF8AppendThreads) kv_append_fp8_kernel(const _
     for (int i = 1; i < kF8AppendThreads / 32; ++i) amax = fmaxf(amax, s_max[i]);
     float scale, inv;
     e4m3_scale_inv(amax, scale, inv);
-    uint32_t c4[16];                                  // 64 codes, 4 per word, channel order
+    uint32_t c4[8];                                   // 32 codes, 4 per word, channel order
 #pragma unroll
-    for (int q = 0; q < 16; ++q) {
+    for (int q = 0; q < 8; ++q) {
         const uint32_t lo = pack_e4m3x2(__fmul_rn(bf16_lo(w[2 * q]), inv), __fmul_rn(bf16_hi(w[2 * q]), inv));
         const uint32_t hi =
             pack_e4m3x2(__fmul_rn(bf16_lo(w[2 * q + 1]), inv), __fmul_rn(bf16_hi(w[2 * q + 1]), inv));
@@ -197,14 +202,17 @@ __global__ void __launch_bounds__(kF8AppendThreads) kv_append_fp8_kernel(const _
     if (tid == 0)
         (is_v ? p.v_scale_layer : p.k_scale_layer)[bs * p.scale_slot_stride + h * p.n_blk + blk] = scale;
     if (!is_v) {
-        uint8_t *dst = p.k8_layer + ((bs * p.np_tokens + n) * p.heads + h) * 128 + half * 64;
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            *reinterpret_cast<uint4 *>(dst + 16 * i) = make_uint4(c4[4 * i], c4[4 * i + 1], c4[4 * i + 2], c4[4 * i + 3]);
+        uint8_t *dst = p.k8_layer + ((bs * p.np_tokens + n) * p.heads + h) * 128 + sub * 32;
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(c4[0], c4[1], c4[2], c4[3]);
+        *reinterpret_cast<uint4 *>(dst + 16) = make_uint4(c4[4], c4[5], c4[6], c4[7]);
         return;
     }
+    // channel order rotated by sub, so the four channel groups of a warp hit different banks
 #pragma unroll
-    for (int q = 0; q < 64; ++q) s_vt[half * 64 + q][tok] = static_cast<uint8_t>(c4[q >> 2] >> (8 * (q & 3)));
+    for (int i = 0; i < 32; ++i) {
+        const int q = (i + sub) & 31;
+        s_vt[sub * 32 + q][tok] = static_cast<uint8_t>(c4[q >> 2] >> (8 * (q & 3)));
+    }
     __syncthreads();
     uint8_t *dst = p.v8t_layer + (bs * p.heads + h) * 128 * p.np_tokens + blk * kBlockN;
     for (int i = tid; i < 128 * 8; i += kF8AppendThreads) {

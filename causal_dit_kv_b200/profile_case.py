@@ -18,6 +18,13 @@ SHAPES = {
                                sink_frames=1, window_frames=8, embed_dim=1536, motion=(16, 60, 104)),
     "wan1.3b-128x128-b16": dict(batch=16, layers=30, heads=12, head_dim=128, frame_h=8, frame_w=8, chunk_frames=1,
                                 sink_frames=1, window_frames=6, embed_dim=1536, motion=(16, 16, 16)),
+    "wan1.3b-512x512-fp8": dict(batch=1, layers=30, heads=12, head_dim=128, frame_h=32, frame_w=32, chunk_frames=1,
+                                sink_frames=1, window_frames=6, embed_dim=1536, motion=(16, 64, 64), kv_format="fp8"),
+    "wan1.3b-128x256-b16": dict(batch=16, layers=30, heads=12, head_dim=128, frame_h=8, frame_w=16, chunk_frames=1,
+                                sink_frames=1, window_frames=6, embed_dim=1536, motion=(16, 16, 32)),
+    "wan1.3b-128x256-b16-fp8": dict(batch=16, layers=30, heads=12, head_dim=128, frame_h=8, frame_w=16,
+                                    chunk_frames=1, sink_frames=1, window_frames=6, embed_dim=1536,
+                                    motion=(16, 16, 32), kv_format="fp8"),
     "wan14b-512x512-b1": dict(batch=1, layers=40, heads=40, head_dim=128, frame_h=32, frame_w=32, chunk_frames=1,
                               sink_frames=1, window_frames=6, embed_dim=5120, motion=(16, 64, 64)),
 }
@@ -38,7 +45,7 @@ def main():
     N = w["frame_h"] * w["frame_w"]
     Lq = Tp * N
     cache = KVCache(B, 1, H, D, w["frame_h"], w["frame_w"], Tp, w["sink_frames"], w["window_frames"],
-                    embed_dim=w["embed_dim"])
+                    embed_dim=w["embed_dim"], kv_format=w.get("kv_format", "bf16"))
     g = torch.Generator(device="cuda").manual_seed(3)
     k = torch.randn((B, Lq, H, D), generator=g, device="cuda").to(torch.bfloat16)
     v = torch.randn((B, Lq, H, D), generator=g, device="cuda").to(torch.bfloat16)
