@@ -28,7 +28,8 @@ def measure_step_latency(shape: dict, batch: int, steps: int = 3, warmup: int = 
     N = shape["frame_h"] * shape["frame_w"]
     Lq, E = Tp * N, shape["embed_dim"]
     C, MH, MW = shape["motion"]
-    cache = KVCache(batch, L, H, D, shape["frame_h"], shape["frame_w"], Tp, S, W, embed_dim=E)
+    cache = KVCache(batch, L, H, D, shape["frame_h"], shape["frame_w"], Tp, S, W, embed_dim=E,
+                    kv_format=shape.get("kv_format", "bf16"))
     mot = MotionState(batch, Tp, C, MH, MW)
     g = torch.Generator(device="cuda").manual_seed(seed)
     mk = lambda *s: torch.randn(s, generator=g, device="cuda").to(torch.bfloat16)

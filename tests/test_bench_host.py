@@ -71,3 +71,19 @@ def test_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
     assert bench.profiled_traffic("w") == 123
     (csrc / "attention.cu").write_bytes(b"kernel v2")
     assert bench.profiled_traffic("w") is None
+
+
+def test_fp8_workloads_byte_accounting():
+    import bench
+    w16, w8 = bench.WORKLOADS["wan1.3b-512x512"], bench.WORKLOADS["wan1.3b-512x512-fp8"]
+    keys = bench.steady_keys(w16)
+    assert bench.steady_keys(w8) == keys == [7168]
+    b16, b8 = bench.attn_bytes(w16, keys), bench.attn_bytes(w8, keys)
+    hd, lq = 12 * 128, 1024
+    assert b16 == 4 * 7168 * hd + 4 * lq * hd                               # K+V, Q, O in bf16
+    # codes for K, V and Q, bf16 O, one K and one V scale per block and head, one scale per query row
+    assert b8 == 2 * 7168 * hd + lq * hd + 2 * lq * hd + 2 * 4 * 12 * 56 + 4 * 12 * lq
+    assert bench.attn_flops(w8, keys) == bench.attn_flops(w16, keys)
+    assert bench.workload_config("x", w8, 1)["kv_format"] == "fp8"
+    assert bench.workload_config("x", w16, 1)["kv_format"] == "bf16"
+    assert bench.kv_elem(w8) == 1 and bench.kv_elem(w16) == 2
