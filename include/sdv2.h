@@ -156,7 +156,9 @@ sdv2_status sdv2_cache_destroy(sdv2_cache *cache);
  * first, then h, then w; frequency of pair j on an axis with n pairs is
  * base^(-j/n).  Each rotation is r0 = x0*c - x1*s, r1 = x0*s + x1*c in fp64
  * without fused multiply-add, rounded once to bf16 (nearest, ties to even).
- * V is copied unchanged.
+ * V is copied unchanged.  With SDV2_KV_FP8_E4M3 the same rotated keys and
+ * the values are then quantised per 128-token block and head (see
+ * sdv2_cache_config.kv_format) and only the codes and scales are stored.
  * Errors: SDV2_E_ARG, SDV2_E_ALIGN, SDV2_E_STATE (wrong f0), SDV2_E_CUDA. */
 sdv2_status sdv2_kv_append(sdv2_cache *cache, int32_t layer, const void *k, const void *v,
                            const int64_t *chunk_first_frame, sdv2_stream stream);
@@ -166,7 +168,9 @@ sdv2_status sdv2_kv_append(sdv2_cache *cache, int32_t layer, const void *k, cons
  * [A] "深入分析" (KV-cache load per chunk), [Q] "Adaptive sink and RoPE refresh".
  * q:   device bf16 [B][T'*N][H][d], NOT rotated: the call rotates it (fp32,
  *      rounded to bf16 for the tensor cores, into the cache's scratch) at the
- *      same (phase, row, col) as the chunk's keys.
+ *      same (phase, row, col) as the chunk's keys.  With the fp8 cache each
+ *      rotated row is coded as E4M3 with its own scale instead, the products
+ *      run on E4M3 operands and the probabilities are coded as E4M3 too.
  * out: device bf16 [B][T'*N][H][d].
  * chunk_first_frame: HOST int64 [B], the frames of this chunk; the chunk must
  *      already be appended to this layer (f0 + T' == frames appended).
