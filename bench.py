@@ -70,15 +70,27 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+def source_digest(path):
+    """sha256 prefix of a CUDA/C++ source with its // comments and blank lines removed:
+    the same for two versions of the file that differ only in comments."""
+    import hashlib
+    lines = []
+    for line in open(path, encoding="utf-8").read().splitlines():
+        i = line.find("//")
+        line = (line[:i] if i >= 0 else line).rstrip()
+        if line:
+            lines.append(line)
+    return hashlib.sha256("\n".join(lines).encode()).hexdigest()[:16]
+
+
 def profiled_traffic(workload):
     """DRAM bytes per attention launch from the committed ncu summary, if it was
-    taken on the current kernel source (else None)."""
-    import hashlib
+    taken on the current kernel code (else None)."""
     path = os.path.join(ROOT, "profiles", f"chunk_attention_{workload}.md")
     src = os.path.join(ROOT, "causal_dit_kv_b200", "csrc", "attention.cu")
     if not os.path.exists(path):
         return None
-    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    digest = source_digest(src)
     fields = {}
     for line in open(path):
         if ":" in line and line.split(":")[0].strip() in ("traffic_bytes_per_launch", "source_sha256_prefix"):

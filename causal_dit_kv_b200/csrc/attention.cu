@@ -42,6 +42,14 @@
 // rounded to bf16) into a scratch buffer; the producer warp TMA-loads the
 // rotated tiles straight into the 128-byte-swizzled K-major layout the MMA
 // reads.
+// fp8 (E4M3) cache (the F8 instantiation, head_dim 128): KV tiles are the
+// 128-token blocks of each valid slot (tile g = block g % n_blk of slot
+// g / n_blk, padding tokens masked), V tiles come from the slot's transposed
+// codes, and Q, K, P and V enter kind::f8f6f4 MMAs (K = 32 per instruction).
+// Each tile's K scale and the query row's scale fold into the softmax scale of
+// that tile; each tile's V scale divided by the CTA's largest V scale
+// multiplies P before its E4M3 coding, and the epilogue multiplies O back by
+// that largest scale.  P takes columns [0, 32) of S_t.
 // KV splits: each split CTA writes its unnormalised O, row max and row sum;
 // attention_combine_kernel (a dependent launch) merges them over the whole
 // GPU.

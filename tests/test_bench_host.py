@@ -63,11 +63,13 @@ def test_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
     (tmp_path / "profiles").mkdir()
     csrc = tmp_path / "causal_dit_kv_b200" / "csrc"
     csrc.mkdir(parents=True)
-    (csrc / "attention.cu").write_bytes(b"kernel v1")
+    (csrc / "attention.cu").write_bytes(b"kernel v1 // first\n")
     import hashlib
     h = hashlib.sha256(b"kernel v1").hexdigest()[:16]
     (tmp_path / "profiles" / "chunk_attention_w.md").write_text(
         f"traffic_bytes_per_launch: 123\nsource_sha256_prefix: {h}\n")
+    assert bench.profiled_traffic("w") == 123
+    (csrc / "attention.cu").write_bytes(b"// a comment-only edit\nkernel v1 // reworded\n\n")
     assert bench.profiled_traffic("w") == 123
     (csrc / "attention.cu").write_bytes(b"kernel v2")
     assert bench.profiled_traffic("w") is None
