@@ -411,7 +411,7 @@ def run_ours(args, w, name):
     # work (ring bookkeeping, plans, launch set-up) leaves the timed region.  Every replay
     # repeats the captured step's slots and positions, so this is a timing of the
     # kernels as launched, reported beside the streamed value, not instead of it.
-    graph_ms, graph_err = 0.0, ""
+    graph_ms, graph_err, graph = 0.0, "", None
     try:
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
@@ -419,19 +419,23 @@ def run_ours(args, w, name):
         for _ in range(3):
             graph.replay()
         torch.cuda.synchronize()
-        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if pg:
-            pg.barrier()
-        g0.record(stream)
-        for _ in range(args.steps):
-            graph.replay()
-        g1.record(stream)
-        torch.cuda.synchronize()
-        graph_ms = g0.elapsed_time(g1)
-        assert cache.check() == 0 and mot.check() == 0, "device status word set"
-        del graph
     except Exception as exc:                                   # reported, the streamed numbers stand
         graph_err = f"{type(exc).__name__}: {exc}"[:200]
+    if pg:
+        pg.barrier()                                           # every rank, whatever its capture did
+    if not graph_err:
+        try:
+            g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            g0.record(stream)
+            for _ in range(args.steps):
+                graph.replay()
+            g1.record(stream)
+            torch.cuda.synchronize()
+            graph_ms = g0.elapsed_time(g1)
+            assert cache.check() == 0 and mot.check() == 0, "device status word set"
+        except Exception as exc:
+            graph_err = f"{type(exc).__name__}: {exc}"[:200]
+    del graph
     graph_fail = 1.0 if graph_err else 0.0
 
     if pg:
