@@ -155,3 +155,15 @@ def test_plan_properties_over_random_shapes(B):
         else:
             assert whole == 0 or whole % sms == 0    # whole units fill complete waves
             assert whole < units
+
+
+def test_fp8_plan_counts_whole_blocks_per_slot(B):
+    # N = 1560 tokens per frame: 13 blocks of 128 per slot (the last one holds 24 tokens)
+    bf = B.make_cache_config(1, 1, 12, 128, 30, 52, 2, 1, 8)
+    f8 = B.make_cache_config(1, 1, 12, 128, 30, 52, 2, 1, 8, kv_format="fp8")
+    keys = [9 * 1560]
+    tiles_bf, tiles_f8 = -(-9 * 1560 // 128), 9 * 13
+    assert tiles_bf == 110 and tiles_f8 == 117
+    for cfg in (bf, f8):
+        whole, pieces = B.sdv2_attention_plan(cfg, keys, 148)
+        assert 1 <= pieces <= 4 and 0 <= whole <= 12 * 13

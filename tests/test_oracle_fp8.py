@@ -111,3 +111,17 @@ def test_fp8_attention_close_to_bf16_attention_and_refresh_copies_codes():
     s_last = O.slot_of_frame(3, cfg.sink_frames, cfg.window_frames)
     for arr in (c8.k8, c8.v8t, c8.k_scale, c8.v_scale):
         assert np.array_equal(arr[:, 0, 0], arr[:, 0, s_last])
+
+
+def test_block_quantiser_tiny_block_clamps_the_inverse():
+    # amax below 448 / FLT_MAX: 448 / amax overflows fp32 and the inverse is clamped to the
+    # largest finite fp32 (not infinity), so zeros stay zero (no 0 * inf) and every code is
+    # finite; the largest element then maps to amax * FLT_MAX (about 3.4 here), not to 448
+    x = np.array([0.0, 1e-38, -5e-39, 2.0 ** -130], dtype=np.float32).astype(np.float64)
+    codes, scale = quantize_block(x)
+    assert scale == np.float32(np.float32(1e-38) / np.float32(448.0))
+    assert codes[0] == 0x00 and codes[1] == 0x46 and codes[2] & 0x80          # 0x46 = 3.5
+    with np.errstate(over="ignore"):
+        inv = np.float32(np.finfo(np.float32).max)
+        want = e4m3_encode((x.astype(np.float32) * inv).astype(np.float64))
+    assert np.array_equal(codes, want)
