@@ -13,10 +13,9 @@ readings taken here:
     finite magnitude 448 (1.75 * 2^8); subnormals are m * 2^-9, m = 1..7.
   * What is stored: the same values the bf16 cache holds (keys rotated by
     3D RoPE and rounded to bf16 once, values as given), quantised in blocks.
-    A slot's N tokens are padded to Np = ceil(N / 128) * 128 and cut into
-    Np / 128 blocks of 128 tokens; every (layer, stream, slot, head, block)
-    has one fp32 scale for K and one for V.  Padding tokens hold code 0 and
-    take no part in the block's maximum.
+    A slot's N tokens are cut into blocks of 128 consecutive tokens (the
+    last block may be shorter); every (layer, stream, slot, head, block) has
+    one fp32 scale for K and one for V.
   * Quantisation of a block, all in fp32 with round-to-nearest-even:
         amax  = max |x| over the block's tokens and the head's d channels
         scale = amax / 448                    (the stored scale)
@@ -24,9 +23,13 @@ readings taken here:
                 largest finite fp32 value (amax below 448 / FLT_MAX)
         code  = E4M3_RNE(x * inv), saturating to +-448
     The dequantised value is decode(code) * scale.
-  * Layouts: K8 [L][B][S+W][Np][H][d] (token-major, like the bf16 cache);
-    V8 transposed per slot, [L][B][S+W][H][d][Np] (token index innermost);
-    scales [L][B][S+W][H][Np / 128].
+  * What the format is, independent of any storage order: for every
+    (layer, stream, slot, token, head) the d codes of K and the d codes of V,
+    and for every (layer, stream, slot, head, block of 128 tokens) one K
+    scale and one V scale.  The arrays below index exactly that:
+    K8, V8 [L][B][S+W][N][H][d], scales [L][B][S+W][H][ceil(N / 128)].
+    The last block of a slot whose N is not a multiple of 128 holds fewer
+    tokens; its scale is taken over those tokens only.
   * Attention: softmax(scale * RoPE(q) K^T) V evaluated in fp64 on the
     dequantised K and V of the valid slots, with q unquantised.  The CUDA
     path also rounds q (per row) and the probabilities to E4M3 before its
@@ -124,8 +127,9 @@ def quantize_block(x: np.ndarray):
 # Cache
 # --------------------------------------------------------------------------
 
-def padded_tokens(tokens_per_frame: int) -> int:
-    return -(-tokens_per_frame // BLOCK_TOKENS) * BLOCK_TOKENS
+def blocks_per_slot(tokens_per_frame: int) -> int:
+    """Blocks of 128 tokens (the last one possibly shorter) that cover one slot."""
+    return -(-tokens_per_frame // BLOCK_TOKENS)
 
 
 class OracleFp8Cache:
@@ -137,12 +141,12 @@ class OracleFp8Cache:
         self.cfg = cfg
         self.base = OracleCache(cfg)
         c = cfg
-        self.np_tokens = padded_tokens(c.tokens_per_frame)
-        nb = self.np_tokens // BLOCK_TOKENS
-        self.k8 = np.zeros((c.layers, c.batch, c.slots, self.np_tokens, c.heads, c.head_dim), np.uint8)
-        self.v8t = np.zeros((c.layers, c.batch, c.slots, c.heads, c.head_dim, self.np_tokens), np.uint8)
-        self.k_scale = np.zeros((c.layers, c.batch, c.slots, c.heads, nb), np.float32)
-        self.v_scale = np.zeros((c.layers, c.batch, c.slots, c.heads, nb), np.float32)
+        self.n_blk = blocks_per_slot(c.tokens_per_frame)
+        shape = (c.layers, c.batch, c.slots, c.tokens_per_frame, c.heads, c.head_dim)
+        self.k8 = np.zeros(shape, np.uint8)
+        self.v8 = np.zeros(shape, np.uint8)
+        self.k_scale = np.zeros((c.layers, c.batch, c.slots, c.heads, self.n_blk), np.float32)
+        self.v_scale = np.zeros((c.layers, c.batch, c.slots, c.heads, self.n_blk), np.float32)
 
     def quantize_slot(self, layer: int, b: int, s: int) -> None:
         """Re-derive slot s's E4M3 codes and scales from the bf16 values it holds."""
@@ -150,28 +154,27 @@ class OracleFp8Cache:
         N = c.tokens_per_frame
         k = bf16_decode(self.base.k[layer, b, s])             # [N][H][d]
         v = bf16_decode(self.base.v[layer, b, s])
-        for blk in range(self.np_tokens // BLOCK_TOKENS):
+        for blk in range(self.n_blk):
             t0, t1 = blk * BLOCK_TOKENS, min(N, (blk + 1) * BLOCK_TOKENS)
             for h in range(c.heads):
                 kc, ks = quantize_block(k[t0:t1, h])
                 vc, vs = quantize_block(v[t0:t1, h])
                 self.k8[layer, b, s, t0:t1, h] = kc
-                self.k8[layer, b, s, t1:(blk + 1) * BLOCK_TOKENS, h] = 0
-                self.v8t[layer, b, s, h, :, t0:t1] = vc.T
-                self.v8t[layer, b, s, h, :, t1:(blk + 1) * BLOCK_TOKENS] = 0
+                self.v8[layer, b, s, t0:t1, h] = vc
                 self.k_scale[layer, b, s, h, blk] = ks
                 self.v_scale[layer, b, s, h, blk] = vs
 
     def dequantized(self, layer: int, b: int, n_slots: int):
-        """K, V of the first n_slots slots, fp64 [n_slots * N][H][d] (padding dropped)."""
+        """K, V of the first n_slots slots, fp64 [n_slots * N][H][d]: token n of a slot
+        takes the scale of its head and of block n // 128."""
         c = self.cfg
-        N, H, d, nb = c.tokens_per_frame, c.heads, c.head_dim, self.np_tokens // BLOCK_TOKENS
-        ks = np.repeat(self.k_scale[layer, b, :n_slots].astype(np.float64), BLOCK_TOKENS, axis=-1)  # [s][H][Np]
-        vs = np.repeat(self.v_scale[layer, b, :n_slots].astype(np.float64), BLOCK_TOKENS, axis=-1)
-        k = e4m3_decode(self.k8[layer, b, :n_slots]) * ks.transpose(0, 2, 1)[..., None]  # [s][Np][H][d]
-        v = e4m3_decode(self.v8t[layer, b, :n_slots]).transpose(0, 3, 1, 2) * vs.transpose(0, 2, 1)[..., None]
-        assert nb * BLOCK_TOKENS == self.np_tokens
-        return (k[:, :N].reshape(n_slots * N, H, d), v[:, :N].reshape(n_slots * N, H, d))
+        N, H, d = c.tokens_per_frame, c.heads, c.head_dim
+        blk = np.arange(N) // BLOCK_TOKENS
+        ks = self.k_scale[layer, b, :n_slots][:, :, blk].astype(np.float64)   # [s][H][N]
+        vs = self.v_scale[layer, b, :n_slots][:, :, blk].astype(np.float64)
+        k = e4m3_decode(self.k8[layer, b, :n_slots]) * ks.transpose(0, 2, 1)[..., None]   # [s][N][H][d]
+        v = e4m3_decode(self.v8[layer, b, :n_slots]) * vs.transpose(0, 2, 1)[..., None]
+        return k.reshape(n_slots * N, H, d), v.reshape(n_slots * N, H, d)
 
 
 def kv_append_fp8(cache: OracleFp8Cache, layer: int, k_bits: np.ndarray, v_bits: np.ndarray,
@@ -219,6 +222,6 @@ def sink_refresh_fp8(cache: OracleFp8Cache, hidden_bits: np.ndarray, tau: float,
             continue
         f_last = int(chunk_first_frame[b]) + c.chunk_frames - 1
         s_last = slot_of_frame(f_last, c.sink_frames, c.window_frames)
-        for arr in (cache.k8, cache.v8t, cache.k_scale, cache.v_scale):
+        for arr in (cache.k8, cache.v8, cache.k_scale, cache.v_scale):
             arr[:, b, j] = arr[:, b, s_last]
     return out

@@ -75,9 +75,17 @@ class Fp8Pair:
         return out, want
 
     def cache_equal(self, layer):
-        g = self.gpu
-        return (np.array_equal(g.k_codes(layer).cpu().numpy(), self.ora.k8[layer]),
-                np.array_equal(g.v_codes(layer).cpu().numpy(), self.ora.v8t[layer]),
+        """Codes and scales of the GPU cache against the oracle's, element by element.  The
+        CUDA cache stores each slot's tokens padded to whole 128-token blocks and V
+        transposed per slot; this converts it to the oracle's (slot, token, head) order and
+        checks that the padding holds code 0."""
+        g, N = self.gpu, self.cfg.tokens_per_frame
+        k = g.k_codes(layer).cpu().numpy()                          # [B][slots][Np][H][d]
+        vt = g.v_codes(layer).cpu().numpy()                         # [B][slots][H][d][Np]
+        v = vt.transpose(0, 1, 4, 2, 3)                             # [B][slots][Np][H][d]
+        pad_zero = not k[:, :, N:].any() and not v[:, :, N:].any()
+        return (np.array_equal(k[:, :, :N], self.ora.k8[layer]) and pad_zero,
+                np.array_equal(v[:, :, :N], self.ora.v8[layer]),
                 np.array_equal(g.k_scales(layer).cpu().numpy(), self.ora.k_scale[layer]),
                 np.array_equal(g.v_scales(layer).cpu().numpy(), self.ora.v_scale[layer]))
 

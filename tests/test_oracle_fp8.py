@@ -69,11 +69,25 @@ def _cfg(**kw):
     return O.CacheConfig(**base)
 
 
-def test_fp8_cache_layouts_track_the_bf16_cache():
+def _quant_err(x, scales_per_elem):
+    """Largest error the block quantiser may make on x (see the quantiser bound test):
+    half a quantum of x's binade, 2^-4 |x| in the normal range, 2^-10 * scale below it,
+    with room for the fp32 roundings of the scale and the product."""
+    return np.maximum(2.0 ** -4 * np.abs(x), 2.0 ** -10 * scales_per_elem) * (1 + 1e-6) + 1e-12
+
+
+def _block_scales(sc, n_tokens):
+    """Per-token scales [slots * N][H] from per-(slot, head, block) scales [slots][H][n_blk]."""
+    blk = np.arange(n_tokens) // BLOCK_TOKENS
+    per_tok = sc[:, :, blk].astype(np.float64)                     # [slots][H][N]
+    return per_tok.transpose(0, 2, 1).reshape(-1, sc.shape[1])
+
+
+def test_fp8_cache_tracks_the_bf16_cache():
     cfg = _cfg()
     c8 = OracleFp8Cache(cfg)
-    N = cfg.tokens_per_frame                                  # 150 tokens: one full block and one ragged block
-    assert c8.np_tokens == 256
+    N = cfg.tokens_per_frame                                  # 150 tokens: one full block and one of 22 tokens
+    assert c8.n_blk == 2
     for step in range(6):                                     # wraps the window
         q, k, v = synth.chunk_qkv(31, cfg.batch, cfg.chunk_tokens, cfg.heads, cfg.head_dim, step, 0)
         kv_append_fp8(c8, 0, k.view(torch.int16).numpy().view(np.uint16), v.view(torch.int16).numpy().view(np.uint16),
@@ -82,35 +96,97 @@ def test_fp8_cache_layouts_track_the_bf16_cache():
         kq, vq = c8.dequantized(0, b, cfg.slots)
         kb = O.bf16_decode(c8.base.k[0, b]).reshape(cfg.slots * N, cfg.heads, cfg.head_dim)
         vb = O.bf16_decode(c8.base.v[0, b]).reshape(cfg.slots * N, cfg.heads, cfg.head_dim)
-        for got, want, sc in ((kq, kb, c8.k_scale), (vq, vb, c8.v_scale)):
-            bound = np.maximum(2.0 ** -4 * np.abs(want), 2.0 ** -10 * float(sc[0, b].max())) * (1 + 1e-6) + 1e-12
-            assert (np.abs(got - want) <= bound).all()
-    assert not c8.k8[:, :, :, N:].any() and not c8.v8t[..., N:].any()   # padding tokens hold code 0
-    assert c8.k_scale.shape[-1] == 256 // BLOCK_TOKENS
+        for got, want, sc in ((kq, kb, c8.k_scale[0, b]), (vq, vb, c8.v_scale[0, b])):
+            # element by element, each against the scale of its own (slot, head, block): a
+            # transposed or misplaced block, or a scale taken over the wrong tokens, fails here
+            assert (np.abs(got - want) <= _quant_err(want, _block_scales(sc, N)[..., None])).all()
+            # every block's largest element is coded as +-448 exactly
+            for s in range(cfg.slots):
+                for h in range(cfg.heads):
+                    for j in range(c8.n_blk):
+                        t0, t1 = s * N + j * BLOCK_TOKENS, s * N + min(N, (j + 1) * BLOCK_TOKENS)
+                        amax = np.abs(want[t0:t1, h]).max()
+                        assert sc[s, h, j] == np.float32(np.float32(amax) / np.float32(448.0))
 
 
-def test_fp8_attention_close_to_bf16_attention_and_refresh_copies_codes():
+def _fp8_attention_sigma(qr, kb, vb, ks, vs, scale):
+    """Per-element RMS of |fp8 attention - bf16 attention| implied by the quantiser's
+    per-element error bound e (uniform rounding error in [-e, e], RMS e / sqrt(3),
+    independent between elements).  qr [rows][d]; kb, vb [Lk][d] the bf16 values; ks, vs
+    [Lk] the scale of each key's block.  To first order, with p the bf16 probabilities
+    and o the bf16 output,
+        do_c = sum_j p_j dv_jc + sum_j p_j (ds_j - mean_p ds)(v_jc - o_c),
+        ds_j = scale * sum_c q_c dk_jc,
+    so sigma_c^2 = sum_j p_j^2 (ev_jc^2 / 3 + var(ds_j) (v_jc - o_c)^2) with
+    var(ds_j) = scale^2 sum_c q_c^2 ek_jc^2 / 3 (the mean term is dropped: p is spread
+    over thousands of keys)."""
+    o, p = O.attention_reference(qr, kb, vb, scale)
+    ek = _quant_err(kb, ks[:, None])
+    ev = _quant_err(vb, vs[:, None])
+    var_s = scale ** 2 * ((qr ** 2) @ (ek ** 2).T) / 3.0                     # [rows][Lk]
+    p2 = p ** 2
+    dv = vb[None, :, :] - o[:, None, :]                                       # [rows][Lk][d]
+    var = p2 @ (ev ** 2 / 3.0) + np.einsum("rj,rjc->rc", p2 * var_s, dv ** 2)
+    return np.sqrt(var), o
+
+
+def test_fp8_attention_within_the_quantisation_bound_and_refresh_copies_codes():
     cfg = _cfg(batch=1, window_frames=2)
     c8 = OracleFp8Cache(cfg)
+    N = cfg.tokens_per_frame
     scale = 1.0 / np.sqrt(cfg.head_dim)
+    as16 = lambda t: t.view(torch.int16).numpy().view(np.uint16)
     for step in range(4):
         q, k, v = synth.chunk_qkv(41, 1, cfg.chunk_tokens, cfg.heads, cfg.head_dim, step, 0)
-        as16 = lambda t: t.view(torch.int16).numpy().view(np.uint16)
         for layer in range(cfg.layers):
             kv_append_fp8(c8, layer, as16(k), as16(v), [step])
         got = chunk_attention_fp8(c8, 0, as16(q), [step], scale)
         want = O.chunk_attention(c8.base, 0, as16(q), [step], scale)
-        err = np.abs(got - want)
-        # K, V each within 2^-4 relative: logits move by < 0.1 here, outputs by a few 1e-2 at most
-        assert err.max() < 6e-2 and err.mean() < 1e-2
+        sv, wv = O.valid_slot_counts(step + 1, cfg.sink_frames, cfg.window_frames)
+        kb, vb = O.valid_keys(c8.base, 0, 0)
+        qr = O.chunk_queries_rotated(cfg, as16(q)[0], step)
+        ks = _block_scales(c8.k_scale[0, 0, :sv + wv], N)
+        vs = _block_scales(c8.v_scale[0, 0, :sv + wv], N)
+        ratios = []
+        for h in range(cfg.heads):
+            sigma, o = _fp8_attention_sigma(qr[:, h], kb[:, h], vb[:, h], ks[:, h], vs[:, h], scale)
+            assert np.allclose(o, want[0, :, h], rtol=0, atol=1e-12)
+            err = np.abs(got[0, :, h] - want[0, :, h])
+            assert (err <= 6.0 * sigma).all(), (step, h, float((err / sigma).max()))
+            ratios.append(err / sigma)
+        # |N(0, 1)| has mean 0.80; the uniform-error RMS over-estimates E4M3's rounding error
+        assert float(np.concatenate(ratios).mean()) < 1.0
     hid = np.zeros((1, cfg.chunk_tokens, cfg.embed_dim), np.uint16)
     hid[..., 0] = 0x3F80                                   # the chunk embedding e_0 = (1, 0, ...)
     c8.base.sink_embed[0, 0, 1] = 1.0                       # a sink embedding orthogonal to it
     slot = sink_refresh_fp8(c8, hid, 0.9, [3])
     assert slot[0] == 0
     s_last = O.slot_of_frame(3, cfg.sink_frames, cfg.window_frames)
-    for arr in (c8.k8, c8.v8t, c8.k_scale, c8.v_scale):
+    for arr in (c8.k8, c8.v8, c8.k_scale, c8.v_scale):
         assert np.array_equal(arr[:, 0, 0], arr[:, 0, s_last])
+
+
+def test_fp8_attention_bound_catches_a_planted_scale_error():
+    """The tolerance of the test above has power: with one block's V scale doubled in the
+    oracle's copy (a plausible indexing slip), the fp8 attention leaves it."""
+    cfg = _cfg(batch=1, window_frames=2, heads=1)
+    c8 = OracleFp8Cache(cfg)
+    N = cfg.tokens_per_frame
+    scale = 1.0 / np.sqrt(cfg.head_dim)
+    as16 = lambda t: t.view(torch.int16).numpy().view(np.uint16)
+    for step in range(3):
+        q, k, v = synth.chunk_qkv(43, 1, cfg.chunk_tokens, cfg.heads, cfg.head_dim, step, 0)
+        for layer in range(cfg.layers):
+            kv_append_fp8(c8, layer, as16(k), as16(v), [step])
+    c8.v_scale[0, 0, 1, 0, 0] *= 2.0
+    got = chunk_attention_fp8(c8, 0, as16(q), [2], scale)
+    kb, vb = O.valid_keys(c8.base, 0, 0)
+    qr = O.chunk_queries_rotated(cfg, as16(q)[0], 2)
+    c8.v_scale[0, 0, 1, 0, 0] /= 2.0
+    ks = _block_scales(c8.k_scale[0, 0, :3], N)
+    vs = _block_scales(c8.v_scale[0, 0, :3], N)
+    sigma, o = _fp8_attention_sigma(qr[:, 0], kb[:, 0], vb[:, 0], ks[:, 0], vs[:, 0], scale)
+    assert (np.abs(got[0, :, 0] - o) > 6.0 * sigma).any()
 
 
 def test_block_quantiser_tiny_block_clamps_the_inverse():
