@@ -8,6 +8,11 @@ latent frame, chunk of 1 frame, 1 sink + 6 window frames, batch 1), with the
 ring already wrapped (steady state), sink refresh on 1536-wide hidden states
 and motion on 16x64x64 latents.  Inputs are seeded synthetic N(0,1) data.
 
+On one GPU the default run also times, in the same process, the Wan-14B-shaped
+stack at B = 1, 2, 4, 8 (the batch sweep) and the 1.3B shape at 480x832 with
+four streams at staggered positions; each gets its own entry under
+``workloads`` (value, ms_per_step, roofline, clocks).
+
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
 
 Under torchrun each rank runs an independent replica (the path has no
@@ -32,16 +37,20 @@ METRIC = "chunk-attn TFLOP/s + KV HBM GB/s vs roofline; latent frames/s (1.3B/14
 UNIT = "latent frames/s"
 
 WORKLOADS = {
-    # name: cache config + refresh/motion shapes
+    # name: cache config + refresh/motion shapes (+ optional per-stream join steps)
     "wan1.3b-512x512": dict(batch=1, layers=30, heads=12, head_dim=128, frame_h=32, frame_w=32, chunk_frames=1,
                             sink_frames=1, window_frames=6, embed_dim=1536, motion=(16, 64, 64)),
+    # four independent streams at different positions: stream b joins the stream batch at
+    # step join[b], so after the pre-roll the streams sit 0, 2, 6 and 12 frames apart (their
+    # window slots differ: offsets 0, 2, 6, 4 modulo the 8-frame window)
     "wan1.3b-480x832-b4": dict(batch=4, layers=30, heads=12, head_dim=128, frame_h=30, frame_w=52, chunk_frames=2,
-                               sink_frames=1, window_frames=8, embed_dim=1536, motion=(16, 60, 104)),
-    "wan14b-512x512-b1": dict(batch=1, layers=40, heads=40, head_dim=128, frame_h=32, frame_w=32, chunk_frames=1,
-                              sink_frames=1, window_frames=6, embed_dim=5120, motion=(16, 64, 64)),
-    "wan14b-512x512-b8": dict(batch=8, layers=40, heads=40, head_dim=128, frame_h=32, frame_w=32, chunk_frames=1,
-                              sink_frames=1, window_frames=6, embed_dim=5120, motion=(16, 64, 64)),
+                               sink_frames=1, window_frames=8, embed_dim=1536, motion=(16, 60, 104),
+                               join=(0, 1, 3, 6)),
 }
+for _b in (1, 2, 4, 8):   # the batch sweep of the 14B shape
+    WORKLOADS[f"wan14b-512x512-b{_b}"] = dict(batch=_b, layers=40, heads=40, head_dim=128, frame_h=32, frame_w=32,
+                                              chunk_frames=1, sink_frames=1, window_frames=6, embed_dim=5120,
+                                              motion=(16, 64, 64))
 # small-chunk, memory-bound regime: 128x128 video (8x8 latent tokens per frame),
 # 16 independent streams
 WORKLOADS["wan1.3b-128x128-b16"] = dict(batch=16, layers=30, heads=12, head_dim=128, frame_h=8, frame_w=8,
@@ -55,9 +64,13 @@ WORKLOADS["wan1.3b-128x256-b16"] = dict(batch=16, layers=30, heads=12, head_dim=
                                         chunk_frames=1, sink_frames=1, window_frames=6, embed_dim=1536,
                                         motion=(16, 16, 32))
 WORKLOADS["wan1.3b-128x256-b16-fp8"] = dict(WORKLOADS["wan1.3b-128x256-b16"], kv_format="fp8")
+WORKLOADS["wan1.3b-128x128-b16-fp8"] = dict(WORKLOADS["wan1.3b-128x128-b16"], kv_format="fp8")
 WORKLOADS["tiny-stream"] = dict(batch=1, layers=1, heads=2, head_dim=64, frame_h=4, frame_w=4, chunk_frames=1,
                                 sink_frames=1, window_frames=2, embed_dim=64, motion=(16, 4, 4))
 DEFAULT_WORKLOAD = "wan1.3b-512x512"
+# timed beside the default workload on one GPU, each under ``workloads``
+EXTRA_WORKLOADS = ("wan14b-512x512-b1", "wan14b-512x512-b2", "wan14b-512x512-b4", "wan14b-512x512-b8",
+                   "wan1.3b-480x832-b4")
 TAU = 0.9
 
 
@@ -109,13 +122,16 @@ def workload_config(name, w, world):
     n = w["frame_h"] * w["frame_w"]
     slots = w["sink_frames"] + w["window_frames"]
     cache_mb = 2.0 * w["layers"] * w["batch"] * slots * n * w["heads"] * w["head_dim"] * kv_elem(w) / 1e6
-    return {"workload": name, "batch": w["batch"], "layers": w["layers"], "heads": w["heads"],
-            "head_dim": w["head_dim"], "tokens_per_frame": n, "chunk_frames": w["chunk_frames"],
-            "sink_frames": w["sink_frames"], "window_frames": w["window_frames"], "keys_per_stream": slots * n,
-            "queries_per_stream": w["chunk_frames"] * n, "refresh_embed_dim": w["embed_dim"],
-            "motion_latent": list(w["motion"]),
-            "l2": "inputs larger than L2 (per-step caches %.0f MB over %d layers)" % (cache_mb, w["layers"]),
-            "kv_format": w.get("kv_format", "bf16"), "parallelism": f"replicas x{world}"}
+    cfg = {"workload": name, "batch": w["batch"], "layers": w["layers"], "heads": w["heads"],
+           "head_dim": w["head_dim"], "tokens_per_frame": n, "chunk_frames": w["chunk_frames"],
+           "sink_frames": w["sink_frames"], "window_frames": w["window_frames"], "keys_per_stream": slots * n,
+           "queries_per_stream": w["chunk_frames"] * n, "refresh_embed_dim": w["embed_dim"],
+           "motion_latent": list(w["motion"]),
+           "l2": "inputs larger than L2 (per-step caches %.0f MB over %d layers)" % (cache_mb, w["layers"]),
+           "kv_format": w.get("kv_format", "bf16"), "parallelism": f"replicas x{world}"}
+    if "join" in w:
+        cfg["stream_join_steps"] = list(w["join"])
+    return cfg
 
 
 def kv_elem(w):
@@ -129,23 +145,57 @@ def attn_flops(w, keys):
 
 
 def attn_bytes(w, keys):
-    """Bytes one attention kernel launch must move: K and V read once, the rotated queries
-    read, O (bf16) written.  The fp8 cache stores 1-byte codes, reads E4M3 queries, and adds
-    one K and one V scale per 128-token block and head and one scale per query row."""
+    """Bytes one attention kernel launch must move: K and V read once, the raw bf16
+    queries read (the kernel rotates them on load), O (bf16) written.  The fp8 cache
+    stores 1-byte codes and adds one K and one V scale per 128-token block and head."""
     lq = w["chunk_frames"] * w["frame_h"] * w["frame_w"]
     hd = w["heads"] * w["head_dim"]
     e = kv_elem(w)
     total = 0.0
     for k in keys:
-        total += 2.0 * e * k * hd + e * lq * hd + 2.0 * lq * hd
+        total += 2.0 * e * k * hd + 2.0 * lq * hd + 2.0 * lq * hd
         if e == 1:
-            total += 2 * 4.0 * w["heads"] * k / 128 + 4.0 * w["heads"] * lq
+            total += 2 * 4.0 * w["heads"] * k / 128
     return total
 
 
 def steady_keys(w):
     n = w["frame_h"] * w["frame_w"]
     return [(w["sink_frames"] + w["window_frames"]) * n] * w["batch"]
+
+
+def attention_roofline(w, name, kern_us, peaks, peak_src):
+    """Roofline entry of the attention kernel from its own event-timed duration.  The
+    kernel is timed launch by launch in a pass of its own, so its tensor peak is the
+    burst figure (bf16_tflops); the fraction against the sustained figure is reported
+    beside it."""
+    fp8 = w.get("kv_format", "bf16") == "fp8"
+    keys = steady_keys(w)
+    flops = attn_flops(w, keys)
+    abytes = attn_bytes(w, keys)
+    peak, peak_name = peaks["bf16_tflops"], "bf16_tflops (burst)"
+    sustained = peaks.get("bf16_tflops_sustained", peak)
+    if fp8:
+        # E4M3 products: the measured bf16 peak times the nominal fp8 / bf16 ratio (4.5 / 2.25)
+        peak, sustained, peak_name = 2.0 * peak, 2.0 * sustained, "bf16_tflops (burst) x 2 (nominal fp8/bf16 ratio)"
+    hbm = peaks["hbm_gbs"]
+    hbm_bound = abytes / (hbm * 1e9) > flops / (peak * 1e12)
+    t = kern_us / 1e6
+    achieved_tf = flops / t / 1e12
+    achieved_gbs = abytes / t / 1e9
+    r = {"kernel": "chunk_attention_kernel", "bound": "hbm" if hbm_bound else "tensor",
+         "achieved": round(achieved_gbs if hbm_bound else achieved_tf, 2), "peak": hbm if hbm_bound else peak,
+         "unit": "GB/s" if hbm_bound else "TFLOP/s",
+         "frac": round(achieved_gbs / hbm if hbm_bound else achieved_tf / peak, 4),
+         "traffic": profiled_traffic(name),
+         "peak_source": f"{peak_src} " + ("hbm_gbs" if hbm_bound else peak_name),
+         "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": abytes,
+         "avg_launch_us": round(kern_us, 3),
+         "timing": "CUDA events recorded by the library right before and after the kernel's launch "
+                   "(sdv2_cache_time_attention), in a pass of its own"}
+    if not hbm_bound:
+        r["frac_vs_sustained_peak"] = round(achieved_tf / sustained, 4)
+    return r
 
 
 class ClockSampler:
@@ -218,63 +268,75 @@ def dist_setup(args):
     return world, rank, local
 
 
+def stream_frames(w, step_index):
+    """First frame of each stream's chunk at the given global step (-1: not yet joined)."""
+    join = w.get("join", (0,) * w["batch"])
+    tp = w["chunk_frames"]
+    return [(step_index - j) * tp if step_index >= j else -1 for j in join]
+
+
+def preroll_steps(w):
+    """Steps after which every stream's ring has wrapped (every slot valid and reused)."""
+    join = w.get("join", (0,) * w["batch"])
+    slots = w["sink_frames"] + w["window_frames"]
+    return max(join) + (slots + w["chunk_frames"] - 1) // w["chunk_frames"] + 1
+
+
 # ----------------------------------------------------------------------------- our arm
 
-def run_ours(args, w, name):
-    import datetime
+class Runner:
+    """One workload on one GPU: the cache, the input pool and the streamed step."""
 
-    import torch
+    def __init__(self, w, dev, seed, n_inputs):
+        import torch
 
-    import synth
-    from causal_dit_kv_b200 import KVCache, MotionState, binding
+        import synth
+        from causal_dit_kv_b200 import KVCache, MotionState
 
-    world, rank, local = dist_setup(args)
-    torch.cuda.set_device(local)
-    pg = None
-    if world > 1:
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-        pg = dist
-    B, L, H, D = w["batch"], w["layers"], w["heads"], w["head_dim"]
-    N = w["frame_h"] * w["frame_w"]
-    Tp = w["chunk_frames"]
-    Lq = Tp * N
-    E = w["embed_dim"]
-    C, MH, MW = w["motion"]
-    fp8 = w.get("kv_format", "bf16") == "fp8"
-    cache = KVCache(B, L, H, D, w["frame_h"], w["frame_w"], Tp, w["sink_frames"], w["window_frames"], embed_dim=E,
-                    kv_format=w.get("kv_format", "bf16"))
-    mot = MotionState(B, Tp, C, MH, MW, window=4, sigma=2.0, lam=0.9)
-    scale = 1.0 / math.sqrt(D)
-    dev = torch.device("cuda", local)
+        self.w = w
+        self.dev = dev
+        B, L, H, D = w["batch"], w["layers"], w["heads"], w["head_dim"]
+        self.B, self.L = B, L
+        N = w["frame_h"] * w["frame_w"]
+        self.Tp = w["chunk_frames"]
+        self.Lq = self.Tp * N
+        E = w["embed_dim"]
+        C, MH, MW = w["motion"]
+        self.cache = KVCache(B, L, H, D, w["frame_h"], w["frame_w"], self.Tp, w["sink_frames"], w["window_frames"],
+                             embed_dim=E, kv_format=w.get("kv_format", "bf16"))
+        self.mot = MotionState(B, self.Tp, C, MH, MW, window=4, sigma=2.0, lam=0.9)
+        self.scale = 1.0 / math.sqrt(D)
+        # Input pool: two distinct steps' worth of Q/K/V for every layer, drawn on the
+        # device.  Hidden states and latents form one continuous stream per step (a slowly
+        # drifting chunk embedding with rare scene cuts, latents with segment-wise motion).
+        self.n_inputs = n_inputs
+        self.pool = []
+        for p in range(2):
+            qkv = [synth.chunk_qkv_on(dev, seed, B, self.Lq, H, D, p, l) for l in range(L)]
+            self.pool.append(dict(q=[t[0] for t in qkv], k=[t[1] for t in qkv], v=[t[2] for t in qkv]))
+        self.hid_seq = [h.to(dev) for h in synth.drifting_hidden(seed, B, self.Lq, E, n_inputs, drift=0.02,
+                                                                 cut_prob=0.01)]
+        self.lat_seq = [x.to(dev) for x in synth.motion_latents(seed, B, self.Tp, C, MH, MW, n_inputs)]
+        self.out = torch.empty((B, self.Lq, H, D), dtype=torch.bfloat16, device=dev)
+        self.out_slot = torch.empty(B, dtype=torch.int32, device=dev)
+        self.rate = torch.empty(B, dtype=torch.float32, device=dev)
+        self.n_step = 0
+        self.stream = torch.cuda.current_stream(dev)
 
-    # Input pool: two distinct steps' worth of Q/K/V for every layer.  Hidden states and
-    # latents form one continuous stream per step (a slowly drifting chunk embedding
-    # with rare scene cuts, latents with segment-wise motion), as in a live stream.
-    pool = []
-    seed = 2000 + rank
-    n_total = (w["sink_frames"] + w["window_frames"] + 1) + args.warmup + 5 * args.steps + 3
-    for p in range(2):
-        qkv = [synth.chunk_qkv(seed, B, Lq, H, D, p, l) for l in range(L)]
-        pool.append(dict(qkv=qkv))
-    hid_seq = [h.to(dev) for h in synth.drifting_hidden(seed, B, Lq, E, n_total, drift=0.02, cut_prob=0.01)]
-    lat_seq = [x.to(dev) for x in synth.motion_latents(seed, B, Tp, C, MH, MW, n_total)]
-    dev_pool = [dict(q=[t[0].to(dev) for t in p["qkv"]], k=[t[1].to(dev) for t in p["qkv"]],
-                     v=[t[2].to(dev) for t in p["qkv"]]) for p in pool]
-    out = torch.empty((B, Lq, H, D), dtype=torch.bfloat16, device=dev)
-    out_slot = torch.empty(B, dtype=torch.int32, device=dev)
-    rate = torch.empty(B, dtype=torch.float32, device=dev)
-    frame = [0]
-    n_step = [0]
-    stream = torch.cuda.current_stream(dev)
+    def rec(self):
+        import torch
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(self.stream)
+        return e
 
-    def step(inp, ev=None, wait=None, kernel_ev=None):
-        """One streamed chunk through every layer; ev (optional) collects event pairs per call;
-        kernel_ev (optional) collects event pairs around each attention kernel alone; wait
-        (optional) is called with the layer index (L for the refresh/motion inputs) before
-        the calls that read that layer's inputs."""
-        f0 = [frame[0]] * B
-        for l in range(L):
+    def step(self, inp, ev=None, wait=None, kernel_ev=None):
+        """One streamed chunk through every layer; ev (optional) collects event pairs per
+        call; kernel_ev (optional) collects event pairs around each attention kernel alone;
+        wait (optional) is called with the layer index (L for the refresh/motion inputs)
+        before the calls that read that layer's inputs."""
+        f0 = stream_frames(self.w, self.n_step)
+        cache, rec = self.cache, self.rec
+        for l in range(self.L):
             if wait is not None:
                 wait(l)
             if ev is not None:
@@ -286,89 +348,139 @@ def run_ours(args, w, name):
             if kernel_ev is not None:
                 k0, k1 = rec(), rec()                    # recorded once so the CUDA events exist
                 cache.time_attention(k0, k1)
-            cache.chunk_attention(l, inp["q"][l], out, f0, scale)
+            cache.chunk_attention(l, inp["q"][l], self.out, f0, self.scale)
             if kernel_ev is not None:
                 cache.time_attention()
                 kernel_ev.append([k0, k1])
             if ev is not None:
                 ev["attention"][-1].append(rec())
         if wait is not None:
-            wait(L)
+            wait(self.L)
         if ev is not None:
             ev["refresh"].append([rec()])
-        hid, lat = (inp["hid"], inp["lat"]) if "hid" in inp else (hid_seq[n_step[0] % n_total], lat_seq[n_step[0] % n_total])
-        cache.sink_refresh(hid, TAU, f0, out_slot)
+        i = self.n_step % self.n_inputs
+        hid, lat = (inp["hid"], inp["lat"]) if "hid" in inp else (self.hid_seq[i], self.lat_seq[i])
+        cache.sink_refresh(hid, TAU, f0, self.out_slot)
         if ev is not None:
             ev["refresh"][-1].append(rec())
             ev["motion"].append([rec()])
-        mot.noise_rate(lat, rate)
+        self.mot.noise_rate(lat, self.rate)
         if ev is not None:
             ev["motion"][-1].append(rec())
-        frame[0] += Tp
-        n_step[0] += 1
+        self.n_step += 1
 
-    def rec():
-        e = torch.cuda.Event(enable_timing=True)
-        e.record(stream)
-        return e
-
-    # Pre-roll to steady state (ring wrapped, every slot valid), then warm up.
-    for i in range(w["sink_frames"] + w["window_frames"] + 1):
-        step(dev_pool[i % 2])
-    for i in range(args.warmup):
-        step(dev_pool[i % 2])
-    torch.cuda.synchronize()
-
-    # ---- device-resident timing of whole steps (no per-call events: they would
-    # break the overlap of dependent launches)
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    launches0 = binding.sdv2_launch_count()
-    with ClockSampler(local) as clocks:
-        if pg:
-            pg.barrier()
+    def warm(self, warmup):
+        import torch
+        for i in range(preroll_steps(self.w) + warmup):
+            self.step(self.pool[i % 2])
         torch.cuda.synchronize()
-        t0.record(stream)
-        for i in range(args.steps):
-            step(dev_pool[i % 2])
-        t1.record(stream)
-        torch.cuda.synchronize()
-        if pg:
-            pg.barrier()
-    launches = binding.sdv2_launch_count() - launches0
-    ms = t0.elapsed_time(t1)
 
-    # ---- per-call timing: the same steps again with events around every call
-    ev = {k: [] for k in ("append", "attention", "refresh", "motion")}
-    for i in range(args.steps):
-        step(dev_pool[i % 2], ev)
-    torch.cuda.synchronize()
-    call_us = {}
-    for k, pairs in ev.items():
-        call_us[k] = statistics.mean(a.elapsed_time(b) for a, b in pairs) * 1e3
-    # ---- the attention kernel alone: the library records events right around its launch
-    kev = []
-    for i in range(args.steps):
-        step(dev_pool[i % 2], kernel_ev=kev)
-    torch.cuda.synchronize()
-    call_us["attn_kernel"] = statistics.mean(a.elapsed_time(b) for a, b in kev) * 1e3
-    assert cache.check() == 0 and mot.check() == 0, "device status word set"
+    def timed_steps(self, steps, pg=None):
+        """Device time (ms) of `steps` whole steps, no events inside (they would break
+        the overlap of dependent launches); returns (ms, launches, clocks)."""
+        import torch
+
+        from causal_dit_kv_b200 import binding
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        launches0 = binding.sdv2_launch_count()
+        with ClockSampler(self.dev.index or 0) as clocks:
+            if pg:
+                pg.barrier()
+            torch.cuda.synchronize()
+            t0.record(self.stream)
+            for i in range(steps):
+                self.step(self.pool[i % 2])
+            t1.record(self.stream)
+            torch.cuda.synchronize()
+            if pg:
+                pg.barrier()
+        return t0.elapsed_time(t1), binding.sdv2_launch_count() - launches0, clocks.summary()
+
+    def kernel_us(self, steps):
+        """Mean duration of the attention kernel alone (library-recorded events)."""
+        import torch
+        kev = []
+        for i in range(steps):
+            self.step(self.pool[i % 2], kernel_ev=kev)
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in kev) * 1e3
+
+    def call_us(self, steps):
+        import torch
+        ev = {k: [] for k in ("append", "attention", "refresh", "motion")}
+        for i in range(steps):
+            self.step(self.pool[i % 2], ev)
+        torch.cuda.synchronize()
+        return {k: statistics.mean(a.elapsed_time(b) for a, b in pairs) * 1e3 for k, pairs in ev.items()}
+
+    def close(self):
+        self.cache.close()
+        self.mot.close()
+
+
+def measure_extra(name, args, dev, peaks, peak_src):
+    """Value, step time, attention roofline and clocks of one more workload (one GPU).
+    Its hidden states and latents cycle through 8 consecutive chunks of the stream."""
+    import torch
+    w = WORKLOADS[name]
+    run = Runner(w, dev, 2100, n_inputs=8)
+    try:
+        run.warm(args.warmup)
+        ms, launches, clocks = run.timed_steps(args.steps)
+        kern = run.kernel_us(args.steps)
+        assert run.cache.check() == 0 and run.mot.check() == 0, "device status word set"
+    finally:
+        run.close()
+        del run
+        torch.cuda.empty_cache()
+    frames = args.steps * w["batch"] * w["chunk_frames"]
+    return {"value": round(frames / (ms / 1e3), 3), "unit": UNIT, "ms_per_step": round(ms / args.steps, 4),
+            "steps": args.steps, "config": workload_config(name, w, 1),
+            "roofline": attention_roofline(w, name, kern, peaks, peak_src), "gpu_launches": int(launches),
+            "clocks": clocks}
+
+
+def run_ours(args, w, name):
+    import datetime
+
+    import torch
+
+    world, rank, local = dist_setup(args)
+    torch.cuda.set_device(local)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    dev = torch.device("cuda", local)
+    B, L, H, D = w["batch"], w["layers"], w["heads"], w["head_dim"]
+    Tp = w["chunk_frames"]
+    C, MH, MW = w["motion"]
+    run = Runner(w, dev, 2000 + rank, n_inputs=preroll_steps(w) + args.warmup + 5 * args.steps + 3)
+    run.warm(args.warmup)
+
+    ms, launches, clocks = run.timed_steps(args.steps, pg)
+    call_us = run.call_us(args.steps)
+    call_us["attn_kernel"] = run.kernel_us(args.steps)
+    assert run.cache.check() == 0 and run.mot.check() == 0, "device status word set"
 
     # ---- end to end: pinned host inputs copied in, results copied out, every step.  The
     # copies run on their own stream, layer by layer, into one of two staging sets
     # (alternating by step), so step i+1's inputs arrive while step i computes; each
     # layer's calls wait only for that layer's inputs.
+    stream = run.stream
     host_pool = []
-    for i, p in enumerate(pool):
-        host_pool.append(dict(q=[t[0].pin_memory() for t in p["qkv"]], k=[t[1].pin_memory() for t in p["qkv"]],
-                              v=[t[2].pin_memory() for t in p["qkv"]], hid=hid_seq[i].cpu().pin_memory(),
-                              lat=lat_seq[i].cpu().pin_memory()))
-    stages = [dict(q=[torch.empty_like(t) for t in dev_pool[0]["q"]], k=[torch.empty_like(t) for t in dev_pool[0]["k"]],
-                   v=[torch.empty_like(t) for t in dev_pool[0]["v"]], hid=torch.empty_like(hid_seq[0]),
-                   lat=torch.empty_like(lat_seq[0])) for _ in range(2)]
+    for i, p in enumerate(run.pool):
+        host_pool.append(dict(q=[t.cpu().pin_memory() for t in p["q"]], k=[t.cpu().pin_memory() for t in p["k"]],
+                              v=[t.cpu().pin_memory() for t in p["v"]], hid=run.hid_seq[i].cpu().pin_memory(),
+                              lat=run.lat_seq[i].cpu().pin_memory()))
+    stages = [dict(q=[torch.empty_like(t) for t in run.pool[0]["q"]], k=[torch.empty_like(t) for t in run.pool[0]["k"]],
+                   v=[torch.empty_like(t) for t in run.pool[0]["v"]], hid=torch.empty_like(run.hid_seq[0]),
+                   lat=torch.empty_like(run.lat_seq[0])) for _ in range(2)]
     copy_stream = torch.cuda.Stream(dev)
     landed = [[torch.cuda.Event() for _ in range(L + 1)] for _ in range(2)]   # per staging set: layer inputs in
     freed = [torch.cuda.Event() for _ in range(2)]                           # per staging set: last reader done
-    res_out = torch.empty((B, Lq, H, D), dtype=torch.bfloat16).pin_memory()
+    res_out = torch.empty(tuple(run.out.shape), dtype=torch.bfloat16).pin_memory()
     res_rate = torch.empty(B, dtype=torch.float32).pin_memory()
     res_slot = torch.empty(B, dtype=torch.int32).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host_pool[0]["q"] + host_pool[0]["k"] + host_pool[0]["v"])
@@ -386,11 +498,11 @@ def run_ours(args, w, name):
             sg["hid"].copy_(hp["hid"], non_blocking=True)
             sg["lat"].copy_(hp["lat"], non_blocking=True)
             landed[i % 2][L].record(copy_stream)
-        step(sg, wait=lambda l: stream.wait_event(landed[i % 2][l]))
+        run.step(sg, wait=lambda l: stream.wait_event(landed[i % 2][l]))
         freed[i % 2].record(stream)
-        res_out.copy_(out, non_blocking=True)
-        res_rate.copy_(rate, non_blocking=True)
-        res_slot.copy_(out_slot, non_blocking=True)
+        res_out.copy_(run.out, non_blocking=True)
+        res_rate.copy_(run.rate, non_blocking=True)
+        res_slot.copy_(run.out_slot, non_blocking=True)
 
     for i in range(2):
         freed[i].record(stream)
@@ -415,7 +527,7 @@ def run_ours(args, w, name):
     try:
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
-            step(dev_pool[0])
+            run.step(run.pool[0])
         for _ in range(3):
             graph.replay()
         torch.cuda.synchronize()
@@ -432,7 +544,7 @@ def run_ours(args, w, name):
             g1.record(stream)
             torch.cuda.synchronize()
             graph_ms = g0.elapsed_time(g1)
-            assert cache.check() == 0 and mot.check() == 0, "device status word set"
+            assert run.cache.check() == 0 and run.mot.check() == 0, "device status word set"
         except Exception as exc:
             graph_err = f"{type(exc).__name__}: {exc}"[:200]
     del graph
@@ -444,52 +556,35 @@ def run_ours(args, w, name):
     value = frames / (ms / 1e3)
     e2e_value = frames / (e2e_ms / 1e3)
 
+    peaks, peak_src = load_peaks()
+    hbm = peaks["hbm_gbs"]
     keys = steady_keys(w)
     flops = attn_flops(w, keys)
     abytes = attn_bytes(w, keys)
-    attn_avg_s = call_us["attention"] / 1e6                  # whole call: RoPE pass, kernel, split merge
-    kern_avg_s = call_us["attn_kernel"] / 1e6                # chunk_attention_kernel alone
-    peaks, peak_src = load_peaks()
-    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    peak_name = "bf16_tflops_sustained"
-    if fp8:
-        # E4M3 products: the measured bf16 peak times the nominal fp8 / bf16 ratio (4.5 / 2.25)
-        peak, peak_name = 2.0 * peak, "bf16_tflops_sustained x 2 (nominal fp8/bf16 ratio)"
-    hbm = peaks["hbm_gbs"]
+    attn_avg_s = call_us["attention"] / 1e6                  # whole call
+    call_peak = peaks["bf16_tflops"] * (2.0 if kv_elem(w) == 1 else 1.0)
     achieved = flops / attn_avg_s / 1e12
-    k_achieved = flops / kern_avg_s / 1e12
-    # roofline of the attention kernel: the slower of its FLOPs at the bf16 peak and its
-    # bytes at the HBM peak decides the bound
-    hbm_bound = abytes / (hbm * 1e9) > flops / (peak * 1e12)
     kv_gbs = abytes / attn_avg_s / 1e9
-    k_kv_gbs = abytes / kern_avg_s / 1e9
+    Lq, N = run.Lq, w["frame_h"] * w["frame_w"]
+    E = w["embed_dim"]
     kv_chunk = 2.0 * B * Lq * H * D * 2                      # K + V of the chunk, bf16
     append_bytes = kv_chunk + kv_chunk * kv_elem(w) / 2       # read (bf16) + written (bf16 or E4M3 codes)
     refresh_bytes = B * Lq * E * 2 + B * E * 8 * (w["sink_frames"] + 1)
     motion_bytes = B * (Tp + 2) * C * MH * MW * 4             # chunk + previous frame read, last frame written
-    traffic = profiled_traffic(name)
     result = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3" if fp8 else "bf16", "data": "synthetic",
-        "config": workload_config(name, w, world),
-        "roofline": {"kernel": "chunk_attention_kernel", "bound": "hbm" if hbm_bound else "tensor",
-                     "achieved": round(k_kv_gbs if hbm_bound else k_achieved, 2), "peak": hbm if hbm_bound else peak,
-                     "unit": "GB/s" if hbm_bound else "TFLOP/s",
-                     "frac": round(k_kv_gbs / hbm if hbm_bound else k_achieved / peak, 4), "traffic": traffic,
-                     "peak_source": f"{peak_src} " + ("hbm_gbs" if hbm_bound else peak_name),
-                     "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": abytes,
-                     "avg_launch_us": round(kern_avg_s * 1e6, 3),
-                     "timing": "CUDA events recorded by the library right before and after the kernel's launch "
-                               "(sdv2_cache_time_attention), in a pass of its own"},
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3" if kv_elem(w) == 1 else "bf16",
+        "data": "synthetic", "config": workload_config(name, w, world),
+        "roofline": attention_roofline(w, name, call_us["attn_kernel"], peaks, peak_src),
         "rows": {
             "kv_append": {"us": round(call_us["append"], 3), "bytes": append_bytes,
                           "gbs": round(append_bytes / call_us["append"] / 1e3, 1),
                           "frac_hbm": round(append_bytes / call_us["append"] / 1e3 / hbm, 4)},
             "chunk_attention": {"us": round(call_us["attention"], 3), "tflops": round(achieved, 2),
-                                "frac_tensor": round(achieved / peak, 4),
+                                "frac_tensor": round(achieved / call_peak, 4),
                                 "kv_gbs": round(kv_gbs, 1), "frac_hbm": round(kv_gbs / hbm, 4),
-                                "what": "whole sdv2_chunk_attention call: rope_q + kernel + split merge"},
+                                "what": "whole sdv2_chunk_attention call: every kernel it launches"},
             "sink_refresh": {"us": round(call_us["refresh"], 3), "bytes_without_copy": refresh_bytes,
                              "gbs": round(refresh_bytes / call_us["refresh"] / 1e3, 1)},
             "motion_noise_rate": {"us": round(call_us["motion"], 3), "bytes": motion_bytes,
@@ -503,8 +598,13 @@ def run_ours(args, w, name):
                         "what": "one captured step replayed (same slots and positions every replay)"}
                        if not graph_fail else {"unavailable": graph_err or "failed on another rank"}),
         "gpu_launches": int(launches),
-        "clocks": clocks.summary(),
+        "clocks": clocks,
     }
+    run.close()
+    del run, stages, host_pool
+    torch.cuda.empty_cache()
+    if world == 1 and name == DEFAULT_WORKLOAD and not args.no_extra:
+        result["workloads"] = {x: measure_extra(x, args, dev, peaks, peak_src) for x in EXTRA_WORKLOADS}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w)
     if pg:
@@ -516,15 +616,30 @@ def run_ours(args, w, name):
 
 # ----------------------------------------------------------------------------- oracle arms
 
+def blas_threads():
+    """Threads numpy's BLAS uses now (the oracle's matrix products run there)."""
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads") for p in threadpool_info() if p.get("user_api") == "blas"]
+        return max(n) if n else None
+    except Exception:                                   # pragma: no cover
+        return None
+
+
 def oracle_sample(w, threads=None):
     """Time the fp64 oracle on one layer of the workload's step (append + attention of
-    every query of every stream) plus the refresh and motion of the step; returns
-    the step time extrapolated to all layers."""
-    import numpy as np
+    every query of every stream) plus the refresh and motion of the step.  ``threads``
+    limits numpy's BLAS threads (None: its default, every core).  Returns (time of the
+    sample, time of the layer, time of refresh + motion) in seconds."""
+    import contextlib
 
     import oracle as O
     import synth
 
+    limit = contextlib.nullcontext()
+    if threads is not None:
+        from threadpoolctl import threadpool_limits
+        limit = threadpool_limits(limits=threads, user_api="blas")
     B, H, D = w["batch"], w["heads"], w["head_dim"]
     N = w["frame_h"] * w["frame_w"]
     Tp = w["chunk_frames"]
@@ -552,50 +667,72 @@ def oracle_sample(w, threads=None):
     q, k, v = synth.chunk_qkv(5, B, Lq, H, D, pre, 0)
     f0 = [pre * Tp] * B
     x = next(lat).numpy()
-    t0 = time.perf_counter()
-    append(cache, 0, synth.bf16_bits(k), synth.bf16_bits(v), f0)
-    attention(cache, 0, synth.bf16_bits(q), f0, 1.0 / math.sqrt(D))
-    t1 = time.perf_counter()
-    refresh(cache, synth.bf16_bits(hid), TAU, f0)
-    O.motion_noise_rate(mstate, x)
-    t2 = time.perf_counter()
-    layer_s = t1 - t0
-    step_s = layer_s * w["layers"] + (t2 - t1)
-    return step_s, layer_s, t2 - t1
+    with limit:
+        t0 = time.perf_counter()
+        append(cache, 0, synth.bf16_bits(k), synth.bf16_bits(v), f0)
+        attention(cache, 0, synth.bf16_bits(q), f0, 1.0 / math.sqrt(D))
+        t1 = time.perf_counter()
+        refresh(cache, synth.bf16_bits(hid), TAU, f0)
+        O.motion_noise_rate(mstate, x)
+        t2 = time.perf_counter()
+    return t2 - t0, t1 - t0, t2 - t1
 
 
-def cpu_baseline(w):
-    import torch
-    step_s, layer_s, rest_s = oracle_sample(w)
+def _extrapolated_step(w, layer_s, rest_s):
+    return layer_s * w["layers"] + rest_s
+
+
+SAMPLE_TEXT = ("one sample = 1 of the {L} layers (append + attention of every query of every stream, fp64 "
+               "numpy oracle) + the step's sink refresh and motion; full-step time extrapolated as "
+               "{L} x layer + refresh + motion")
+
+
+def cpu_baseline(w, samples=3):
+    """The oracle on this host's cores: `samples` samples with numpy's default BLAS
+    threading, and one with a single BLAS thread."""
+    runs = [oracle_sample(w) for _ in range(samples)]
+    layer_s = statistics.median(r[1] for r in runs)
+    rest_s = statistics.median(r[2] for r in runs)
+    one = oracle_sample(w, threads=1)
     frames = w["batch"] * w["chunk_frames"]
-    return {"value": round(frames / step_s, 5), "unit": UNIT, "cores": torch.get_num_threads(), "kind": "oracle",
-            "sample": f"1 of {w['layers']} layers (append + attention of all queries, fp64 numpy, "
-                      f"{layer_s:.2f} s) + sink refresh and motion ({rest_s:.2f} s); step time = "
-                      f"{w['layers']} x layer + refresh + motion"}
+    step_s = _extrapolated_step(w, layer_s, rest_s)
+    step1 = _extrapolated_step(w, one[1], one[2])
+    return {"value": round(frames / step_s, 5), "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+            "blas_threads": blas_threads(),
+            "single_thread_value": round(frames / step1, 5),
+            "sample": SAMPLE_TEXT.format(L=w["layers"]) + f"; median of {samples} samples with numpy's default "
+                      f"BLAS threads (layer {layer_s:.2f} s), plus one with 1 BLAS thread (layer {one[1]:.2f} s)"}
 
 
 def run_reference(args, w, name):
     world, rank, _ = dist_setup(args)
     if rank != 0:
         return
-    import torch
-    times = []
+    layer, rest, sample = [], [], []
     for i in range(args.warmup + args.steps):
-        step_s, layer_s, rest_s = oracle_sample(w)
+        s, l, r = oracle_sample(w)
         if i >= args.warmup:
-            times.append(step_s)
-    mean_step = statistics.mean(times)
+            sample.append(s)
+            layer.append(l)
+            rest.append(r)
+    step_s = _extrapolated_step(w, statistics.mean(layer), statistics.mean(rest))
+    one = oracle_sample(w, threads=1)
     frames = w["batch"] * w["chunk_frames"]
-    value = frames / mean_step
-    cores = torch.get_num_threads()
-    sample = (f"per step: 1 of {w['layers']} layers (append + attention, fp64 numpy oracle) + refresh + motion, "
-              f"extrapolated to {w['layers']} layers")
+    value = frames / step_s
+    sample_text = SAMPLE_TEXT.format(L=w["layers"]) + (
+        f"; each of the {args.steps} timed steps is one sample with numpy's default BLAS threads "
+        f"({blas_threads()} threads on {os.cpu_count()} cores)")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(mean_step * 1e3, 3),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(statistics.mean(sample) * 1e3, 3),
+        "step_is": "one sample (1 of the layers + refresh + motion); value is over the extrapolated full step",
+        "ms_per_full_step_extrapolated": round(step_s * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(name, w, world), "gpu_launches": 0,
-        "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+                         "blas_threads": blas_threads(),
+                         "single_thread_value": round(frames / _extrapolated_step(w, one[1], one[2]), 5),
+                         "sample": sample_text},
         "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }))
 
@@ -608,6 +745,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the extra workloads timed beside the default one")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -38,11 +38,16 @@
 // accumulator sets on that tile: even KV tiles go to S_0/O_0, odd ones to
 // S_1/O_1, so the softmax of one still overlaps the MMAs of the other; the
 // two partial results are merged in the epilogue.
-// Q: rope_q_kernel rotates the chunk's queries once per call (fp32 RoPE,
-// rounded to bf16) into a scratch buffer; the producer warp TMA-loads the
-// rotated tiles straight into the 128-byte-swizzled K-major layout the MMA
-// reads.
-// fp8 (E4M3) cache (the F8 instantiation, head_dim 128): KV tiles are the
+// Q: RoPE is applied on load.  The producer TMA-loads the chunk's raw bf16
+// query tiles (128-byte-swizzled, the layout the MMA reads) before the kernel
+// waits for the KV append it depends on; the softmax warps, idle until the
+// first scores arrive, rotate their own rows in place in fp32 (rounded to
+// bf16) from a per-CTA table of the temporal (cos, sin), evaluated in fp64 for
+// the chunk frames the CTA's rows span, and the cache's fp32 row and column
+// tables; they fence the writes for the tensor core and release the first MMA.
+// fp8 (E4M3) cache (the F8 instantiation, head_dim 128): the raw queries land in
+// a staging area and each rotated row is coded as E4M3 with its own scale
+// (amax / 448 over the row) into the Q tile.  KV tiles are the
 // 128-token blocks of each valid slot (tile g = block g % n_blk of slot
 // g / n_blk, padding tokens masked), V tiles come from the slot's transposed
 // codes, and Q, K, P and V enter kind::f8f6f4 MMAs (K = 32 per instruction).
@@ -63,7 +68,7 @@ namespace sdv2 {
 
 template <int D, bool F8 = false>
 struct AttnLayout {
-    static constexpr int kElem = F8 ? 1 : 2;          // bytes per element of Q, K, V
+    static constexpr int kElem = F8 ? 1 : 2;          // bytes per element of Q, K, V in the MMA tiles
     static constexpr int kQTile = kBlockM * D * kElem;    // bytes of one Q tile
     static constexpr int kKVTile = kBlockN * D * kElem;   // bytes of one K (or V) tile
     static constexpr int kSub = kBlockM * 128;        // one 64-column (128-byte) sub-tile
@@ -72,10 +77,16 @@ struct AttnLayout {
     static constexpr int kQ = 0;
     static constexpr int kK = kQ + kQTilesPerCta * kQTile;
     static constexpr int kV = kK + kKStages * kKVTile;
-    static constexpr int kBar = kV + kVStages * kKVTile;
+    // raw bf16 query tiles as loaded (fp8: a staging area; bf16: the Q tiles themselves,
+    // rotated in place)
+    static constexpr int kQRaw = F8 ? kV + kVStages * kKVTile : kQ;
+    static constexpr int kQRawTile = kBlockM * D * 2;
+    static constexpr int kTab = F8 ? kQRaw + kQTilesPerCta * kQRawTile : kV + kVStages * kKVTile;
+    static constexpr int kBar = kTab + kAttnTabEntries * 8;
     // barriers
-    static constexpr int kQFull = 0;
-    static constexpr int kKFull = 1;
+    static constexpr int kQFull = 0;                  // raw query tiles landed (TMA)
+    static constexpr int kQReady = 1;                 // rotated query tiles written and fenced (softmax threads)
+    static constexpr int kKFull = 2;
     static constexpr int kKEmpty = kKFull + kKStages;
     static constexpr int kVFull = kKEmpty + kKStages;
     static constexpr int kVEmpty = kVFull + kVStages;
@@ -87,6 +98,7 @@ struct AttnLayout {
     static constexpr int kMisc = kBar + kNumBars * 8;   // tmem base, abort flag
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;      // room to align the base to 1024 bytes
+    static_assert(kAlloc <= 232448, "shared memory of one CTA");
 };
 
 int attention_smem_bytes(int head_dim) {
@@ -104,108 +116,123 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return __all_sync(0xffffffffu, ok);
 }
 
-// RoPE of the chunk's queries: q_rot = rotate(q) at (phase(frame), row, col),
-// fp32 arithmetic, bf16 result.  Block = 64 (token, head) rows of one stream,
-// 4 threads per row, every 4th 16-byte vector of the row per thread (loads
-// first).  grid = (row blocks, streams of the launch).  The temporal angles
-// phase * base^(-j / n_t) of the stream's chunk frames are evaluated in fp64
-// by each block and rounded to fp32, like the row and column tables.
-__global__ void __launch_bounds__(256) rope_q_kernel(const __grid_constant__ AttnParams p, int head_dim) {
-    // Launched right behind the KV append, whose own wait already ordered it after
-    // the producer of q: q can be read at once.  Completing only after the append
-    // (wait at the end) lets the attention kernel wait on this kernel alone.
-    grid_launch_dependents();
-    const int bl = blockIdx.y;
-    __shared__ float2 s_tab[kAttnTabEntries];        // temporal (cos, sin) of this stream's frames
-    for (int e = threadIdx.x; e < p.chunk_frames * p.n_t; e += blockDim.x) {
-        const int fi = e / p.n_t, j = e - fi * p.n_t;
-        const int64_t f = p.f0[bl] + fi;
-        const int64_t ph = p.rope_reset > 0 ? f % p.rope_reset : f;
-        const double a = static_cast<double>(ph) * pow(p.rope_base, -static_cast<double>(j) / static_cast<double>(p.n_t));
-        double sn, cs;
-        sincos(a, &sn, &cs);
-        s_tab[e] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+// Tables of one query row's rotation: the temporal (cos, sin) of its frame in the
+// CTA's shared-memory table (tab_t: pair 0), and the cache's pair-major fp32 row
+// and column tables ([pair][position]), offset to the row's position (h: prow, w:
+// pcol) and to pair 0 of their axis.
+struct RopeRow {
+    const float2 *tab_t;
+    const float2 *h;
+    const float2 *w;
+    int n_t, n_th, frame_h, frame_w;
+};
+
+// (cos, sin) of pair j.  j is the same in every lane at a given step (one thread per
+// row): the temporal entry is a broadcast and the lanes' row / column entries
+// (consecutive tokens) are consecutive in the pair-major tables.  With the axis
+// split known at compile time (NT temporal pairs, NTH temporal + row pairs), j is a
+// constant after unrolling and each load goes straight to its table; otherwise
+// (NT = 0) the address is selected without a branch, so all of a row's loads can
+// still be in flight together.
+template <int NT, int NTH>
+__device__ __forceinline__ float2 rope_cs(const RopeRow &t, int j) {
+    if constexpr (NT > 0) {
+        if (j < NT) return t.tab_t[j];
+        if (j < NTH) return __ldg(t.h + (j - NT) * t.frame_h);
+        return __ldg(t.w + (j - NTH) * t.frame_w);
+    } else {
+        const float2 *ptr = j < t.n_t ? t.tab_t + j
+                                      : (j < t.n_th ? t.h + (j - t.n_t) * t.frame_h : t.w + (j - t.n_th) * t.frame_w);
+        return *ptr;
     }
-    __syncthreads();
-    const int rows = p.lq * p.heads;
-    const int row = blockIdx.x * 64 + (threadIdx.x >> 2);
-    const int sub = threadIdx.x & 3;
-    if (p.lk[bl] <= 0 || row >= rows) {
-        grid_dependency_wait();
-        return;
-    }
-    const int token = row / p.heads;
-    const int fi = token / p.tokens_per_frame;
-    const int n = token - fi * p.tokens_per_frame;
-    const int prow = n / p.frame_w;
-    const int pcol = n - prow * p.frame_w;
-    const int64_t off = (static_cast<int64_t>(p.b_offset + bl) * rows + row) * head_dim;
-    constexpr int kMaxVec = 4;
-    const int nvec = head_dim / 32;
-    uint4 x[kMaxVec];
+}
+
+// Load one 64-column sub-tile row (8 chunks of 16 bytes at the 128-byte-swizzled
+// positions c ^ (r & 7) of the row) and the (cos, sin) of its 32 pairs j0 .. j0 + 31;
+// every load is issued before any use.
+template <int NT, int NTH>
+__device__ __forceinline__ void rope_load(const uint8_t *row, int r, int j0, const RopeRow &t, uint4 (&x)[8],
+                                          float2 (&cs)[32]) {
 #pragma unroll
-    for (int i = 0; i < kMaxVec; ++i)
-        if (i < nvec) x[i] = *reinterpret_cast<const uint4 *>(p.q + off + (sub + 4 * i) * 8);
-    const float2 *tab_t = s_tab + fi * p.n_t;
-    const float2 *tab_h = reinterpret_cast<const float2 *>(p.rope_h) + prow * p.n_h - p.n_t;
-    const float2 *tab_w = reinterpret_cast<const float2 *>(p.rope_w) + pcol * p.n_w - p.n_t - p.n_h;
-    float2 cs[kMaxVec][4];
+    for (int c = 0; c < 8; ++c) x[c] = *reinterpret_cast<const uint4 *>(row + ((c ^ (r & 7)) << 4));
 #pragma unroll
-    for (int i = 0; i < kMaxVec; ++i) {
-        if (i >= nvec) break;
+    for (int q = 0; q < 32; ++q) cs[q] = rope_cs<NT, NTH>(t, j0 + q);
+}
+
+// Pair q of chunk c of a loaded sub-tile row, rotated in fp32.
+__device__ __forceinline__ float2 rope_apply(const uint4 (&x)[8], const float2 (&cs)[32], int c, int q) {
+    const uint32_t w = q == 0 ? x[c].x : (q == 1 ? x[c].y : (q == 2 ? x[c].z : x[c].w));
+    const float x0 = bf16_lo(w), x1 = bf16_hi(w);
+    const float2 k = cs[4 * c + q];
+    return make_float2(x0 * k.x - x1 * k.y, x0 * k.y + x1 * k.x);
+}
+
+// Rotate the 32 pairs of one 64-column sub-tile of row r in place (bf16 in, fp32
+// rotation, bf16 out).
+template <int NT, int NTH>
+__device__ __forceinline__ void rope_subtile_bf16(uint8_t *sub, int r, int j0, const RopeRow &t) {
+    uint8_t *row = sub + r * 128;
+    uint4 x[8];
+    float2 cs[32];
+    rope_load<NT, NTH>(row, r, j0, t, x, cs);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        uint32_t o[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const int j = (sub + 4 * i) * 4 + q;
-            cs[i][q] = *(j < p.n_t ? tab_t + j : (j < p.n_t + p.n_h ? tab_h + j : tab_w + j));
+            const float2 v = rope_apply(x, cs, c, q);
+            o[q] = pack_bf16x2(v.x, v.y);
         }
+        *reinterpret_cast<uint4 *>(row + ((c ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
     }
-    if (p.q_scale == nullptr) {
+}
+
+// fp8 cache (head_dim 128): rotate the raw bf16 row r (two 64-column swizzled
+// sub-tiles at shared address raw) in fp32, code it as E4M3 with the row's own
+// scale amax / 448 into the 128-byte-swizzled E4M3 row of q8 (when `write`), and
+// return the scale.  Two passes over the row (the maximum, then the codes), one
+// sub-tile at a time, keep the register use low.
+template <int NT, int NTH>
+__device__ __forceinline__ float rope_row_e4m3(const uint8_t *raw, uint8_t *q8, int r, bool write, const RopeRow &t) {
+    float am = 0.0f;
+#pragma unroll 1
+    for (int kb = 0; kb < 2; ++kb) {
+        uint4 x[8];
+        float2 cs[32];
+        rope_load<NT, NTH>(raw + kb * (kBlockM * 128) + r * 128, r, kb * 32, t, x, cs);
 #pragma unroll
-        for (int i = 0; i < kMaxVec; ++i) {
-            if (i >= nvec) break;
-            const uint32_t in[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
-            uint32_t o[4];
+        for (int c = 0; c < 8; ++c)
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const float x0 = bf16_lo(in[q]), x1 = bf16_hi(in[q]);
-                o[q] = pack_bf16x2(x0 * cs[i][q].x - x1 * cs[i][q].y, x0 * cs[i][q].y + x1 * cs[i][q].x);
+                const float2 v = rope_apply(x, cs, c, q);
+                am = fmaxf(am, fmaxf(fabsf(v.x), fabsf(v.y)));
             }
-            *reinterpret_cast<uint4 *>(p.q_rot + off + (sub + 4 * i) * 8) = make_uint4(o[0], o[1], o[2], o[3]);
-        }
-    } else {
-        // fp8 cache (head_dim 128): the rotated row is coded as E4M3 with its own scale
-        // amax / 448, amax over the row's 128 channels (the row's 4 threads combine theirs).
-        float r[kMaxVec][8];
-        float am = 0.0f;
-#pragma unroll
-        for (int i = 0; i < kMaxVec; ++i) {
-            const uint32_t in[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float x0 = bf16_lo(in[q]), x1 = bf16_hi(in[q]);
-                r[i][2 * q] = x0 * cs[i][q].x - x1 * cs[i][q].y;
-                r[i][2 * q + 1] = x0 * cs[i][q].y + x1 * cs[i][q].x;
-                am = fmaxf(am, fmaxf(fabsf(r[i][2 * q]), fabsf(r[i][2 * q + 1])));
-            }
-        }
-        const unsigned group = 0xFu << (threadIdx.x & 28u);
-        am = fmaxf(am, __shfl_xor_sync(group, am, 1));
-        am = fmaxf(am, __shfl_xor_sync(group, am, 2));
-        float scale, inv;
-        e4m3_scale_inv(am, scale, inv);
-        uint8_t *q8 = reinterpret_cast<uint8_t *>(p.q_rot);
-#pragma unroll
-        for (int i = 0; i < kMaxVec; ++i) {
-            uint32_t c[2];
-#pragma unroll
-            for (int k = 0; k < 2; ++k)
-                c[k] = pack_e4m3x2(r[i][4 * k] * inv, r[i][4 * k + 1] * inv) |
-                       (pack_e4m3x2(r[i][4 * k + 2] * inv, r[i][4 * k + 3] * inv) << 16);
-            *reinterpret_cast<uint2 *>(q8 + off + (sub + 4 * i) * 8) = make_uint2(c[0], c[1]);
-        }
-        if (sub == 0) p.q_scale[static_cast<int64_t>(p.b_offset + bl) * rows + row] = scale;
     }
-    grid_dependency_wait();
+    float scale, inv;
+    e4m3_scale_inv(am, scale, inv);
+    if (write) {
+#pragma unroll 1
+        for (int kb = 0; kb < 2; ++kb) {
+            uint4 x[8];
+            float2 cs[32];
+            rope_load<NT, NTH>(raw + kb * (kBlockM * 128) + r * 128, r, kb * 32, t, x, cs);
+            // E4M3 chunk e (16 codes, pairs 8e .. 8e + 7) takes raw chunks 2e, 2e + 1 of this sub-tile
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                uint32_t w[4];
+#pragma unroll
+                for (int hlf = 0; hlf < 2; ++hlf) {
+                    const float2 v0 = rope_apply(x, cs, 2 * e + hlf, 0), v1 = rope_apply(x, cs, 2 * e + hlf, 1);
+                    const float2 v2 = rope_apply(x, cs, 2 * e + hlf, 2), v3 = rope_apply(x, cs, 2 * e + hlf, 3);
+                    w[2 * hlf] = pack_e4m3x2(v0.x * inv, v0.y * inv) | (pack_e4m3x2(v1.x * inv, v1.y * inv) << 16);
+                    w[2 * hlf + 1] = pack_e4m3x2(v2.x * inv, v2.y * inv) | (pack_e4m3x2(v3.x * inv, v3.y * inv) << 16);
+                }
+                const int cq = kb * 4 + e;              // E4M3 chunk of the 128-byte row
+                *reinterpret_cast<uint4 *>(q8 + r * 128 + ((cq ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+    }
+    return scale;
 }
 
 // P = 2^(s*scale_log2 - m) for one row of 128 scores (raw fp32 bits in sr),
@@ -347,6 +374,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(&bars[L::kQFull], 1);
+        mbar_init(&bars[L::kQReady], kAttnThreads - 128);
         for (int s = 0; s < L::kKStages; ++s) {
             mbar_init(&bars[L::kKFull + s], 1);
             mbar_init(&bars[L::kKEmpty + s], 1);
@@ -378,8 +406,105 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // Everything above overlaps the previous kernels (dependent launch); the
-    // rotated queries, the cache and the split partials are only touched below.
+
+    // ---- queries: raw tiles by TMA, RoPE on load by the softmax warps.  Neither the
+    // queries nor the cache's row / column tables are written by the kernels this launch
+    // depends on (the KV append), so this overlaps them, before the dependency wait.
+    if (warp == 0 && lane == 0 && n_local > 0) {
+        mbar_arrive_expect_tx(&bars[L::kQFull], n_qt * L::kQRawTile);
+        for (int t = 0; t < n_qt; ++t)
+#pragma unroll
+            for (int kb = 0; kb < D / 64; ++kb)
+                tma_load_4d(smem + L::kQRaw + t * L::kQRawTile + kb * L::kSub, &tmap_q, &bars[L::kQFull], kb * 64, h,
+                            q_row0 + t * kBlockM, bg);
+    }
+    // RoPE on load by the softmax warps (idle until the first scores arrive): thread
+    // (t, row) rotates its own query row (the single-tile mode: sub-tile t of tile 0's row)
+    float q_row_scale = 0.0f;                   // fp8: E4M3 scale of this thread's query row
+    if (warp >= 4 && n_local > 0) {
+        const int t = (warp - 4) >> 2;
+        const int row = ((warp & 3) << 5) + lane;
+        const int qt = dual ? 0 : t;            // query tile of this thread's row
+        const int n_rows = min(p.lq - q_row0, dual ? kBlockM : 2 * kBlockM);
+        const int fi_lo = q_row0 / p.tokens_per_frame;
+        const int fi_hi = (q_row0 + n_rows - 1) / p.tokens_per_frame;
+        // temporal (cos, sin) of the chunk frames this CTA's rows span.  The angle
+        // phase * base^(-j/n_t) is formed and reduced modulo 2 pi in fp64 (an FMA with
+        // the nearest multiple), then sine and cosine are taken in fp32.
+        float2 *tab = reinterpret_cast<float2 *>(smem + L::kTab);
+        const int n_tab = (fi_hi - fi_lo + 1) * p.n_t;           // <= kAttnTabEntries (checked on the host)
+        for (int e = threadIdx.x - 128; e < n_tab; e += kAttnThreads - 128) {
+            const int fi = e / p.n_t, j = e - fi * p.n_t;
+            const int64_t f = p.f0[bl] + fi_lo + fi;
+            const int64_t ph = p.rope_reset > 0 ? f % p.rope_reset : f;
+            const double a = static_cast<double>(ph) * p.omega_t[j];
+            const double turns = rint(a * 0.15915494309189535);  // a / (2 pi), nearest integer
+            const float r = static_cast<float>(fma(-turns, 6.283185307179586, a));
+            float sn, cs;
+            sincosf(r, &sn, &cs);
+            tab[e] = make_float2(cs, sn);
+        }
+        const int token = q_row0 + qt * kBlockM + row;
+        const bool in_chunk = token < p.lq;
+        RopeRow rt;
+        {
+            const int fi = in_chunk ? token / p.tokens_per_frame : fi_lo;
+            const int n = in_chunk ? token - fi * p.tokens_per_frame : 0;
+            const int prow = n / p.frame_w;
+            const int pcol = n - prow * p.frame_w;
+            rt.tab_t = tab + (fi - fi_lo) * p.n_t;
+            rt.h = reinterpret_cast<const float2 *>(p.rope_h) + prow;
+            rt.w = reinterpret_cast<const float2 *>(p.rope_w) + pcol;
+            rt.n_t = p.n_t;
+            rt.n_th = p.n_t + p.n_h;
+            rt.frame_h = p.frame_h;
+            rt.frame_w = p.frame_w;
+        }
+        uint8_t *qtile = smem + L::kQ + qt * L::kQTile;
+        // the default axis split (c - 2 floor(c/3), floor(c/3), floor(c/3)) pairs, c = d/2
+        constexpr int kNt = D / 2 - 2 * (D / 6), kNth = kNt + D / 6;
+        const bool def_split = p.n_t == kNt && p.n_t + p.n_h == kNth;
+        bool ok = true;
+        if (!F8 && D == 128 && def_split) {
+            // sub-tile 1 holds only row and column pairs: rotated while the temporal table
+            // is still being written, then sub-tile 0 after the barrier
+            ok = warp_wait(&bars[L::kQFull], 0, abort_flag, p.status, kStatusSoftmaxWait);
+            if (ok && in_chunk && (!dual || t == 1)) rope_subtile_bf16<kNt, kNth>(qtile + L::kSub, row, 32, rt);
+            named_bar_sync(2, kAttnThreads - 128);
+            if (ok && in_chunk && (!dual || t == 0)) rope_subtile_bf16<kNt, kNth>(qtile, row, 0, rt);
+        } else {
+            named_bar_sync(2, kAttnThreads - 128);
+            ok = warp_wait(&bars[L::kQFull], 0, abort_flag, p.status, kStatusSoftmaxWait);
+            if (ok && in_chunk) {
+                if constexpr (F8) {
+                    // both threads of a row in the single-tile mode need its scale; one writes the codes
+                    const uint8_t *raw = smem + L::kQRaw + qt * L::kQRawTile;
+                    q_row_scale = def_split ? rope_row_e4m3<kNt, kNth>(raw, qtile, row, !dual || t == 0, rt)
+                                            : rope_row_e4m3<0, 0>(raw, qtile, row, !dual || t == 0, rt);
+                } else {
+                    // two-tile mode: the whole row; single-tile mode: thread t takes sub-tile t
+#pragma unroll
+                    for (int kb = 0; kb < D / 64; ++kb) {
+                        if (dual && kb != t) continue;
+                        if (def_split)
+                            rope_subtile_bf16<kNt, kNth>(qtile + kb * L::kSub, row, kb * 32, rt);
+                        else
+                            rope_subtile_bf16<0, 0>(qtile + kb * L::kSub, row, kb * 32, rt);
+                    }
+                }
+            } else if (F8 && ok && (!dual || t == 0)) {
+                // rows past the chunk: E4M3 zeros (the bf16 tiles were zero-filled by the TMA)
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4 *>(qtile + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+            }
+        }
+        fence_proxy_async_shared();             // the tensor core reads these rows next
+        mbar_arrive(&bars[L::kQReady]);
+    }
+
+    // Everything above overlaps the previous kernels (dependent launch); the cache and
+    // the split partials are only touched below.
     grid_dependency_wait();
     grid_launch_dependents();
 
@@ -388,18 +513,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0 && n_local > 0) {
-            // rotated query tiles of this CTA (rows past lq are filled with zeros)
-            mbar_arrive_expect_tx(&bars[L::kQFull], n_qt * L::kQTile);
-            for (int t = 0; t < n_qt; ++t) {
-                if constexpr (F8) {
-                    tma_load_4d(smem + L::kQ + t * L::kQTile, &tmap_q, &bars[L::kQFull], 0, h, q_row0 + t * kBlockM, bg);
-                } else {
-#pragma unroll
-                    for (int kb = 0; kb < D / 64; ++kb)
-                        tma_load_4d(smem + L::kQ + t * L::kQTile + kb * L::kSub, &tmap_q, &bars[L::kQFull], kb * 64,
-                                    h, q_row0 + t * kBlockM, bg);
-                }
-            }
             // K tile `it` and V tile `it` are issued as soon as their own ring slot is free.
             int k_issued = 0, v_issued = 0;
             bool ok = true;
@@ -501,7 +614,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                 b0 + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv, (acc || kk > 0) ? 1u : 0u);
                 }
             };
-            bool ok = mbar_wait(&bars[L::kQFull], 0, abort_flag, p.status, kStatusMmaWait);
+            bool ok = mbar_wait(&bars[L::kQReady], 0, abort_flag, p.status, kStatusMmaWait);
             if (dual) {
                 // KV tile i -> accumulator set i & 1.  Prologue: S_0 = Q K_0^T, S_1 = Q K_1^T.
                 for (int i = 0; ok && i < n_local && i < 2; ++i) {
@@ -615,7 +728,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             float sq = 1.0f, sv_ref = 1.0f;
             int64_t scale_base = 0;
             if constexpr (F8) {
-                sq = valid ? p.q_scale[(static_cast<int64_t>(bg) * p.lq + token) * p.heads + h] : 0.0f;
+                sq = valid ? q_row_scale : 0.0f;
                 scale_base = static_cast<int64_t>(bg) * p.slots * p.scale_slot_stride + h * p.n_blk;
                 sv_ref = 0.0f;
                 for (int i = 0; i < n_local; ++i) {
@@ -845,14 +958,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 // Merge of the KV-split partials: out = sum_s 2^(m_s - m) O_s / sum_s 2^(m_s - m) l_s.
 // Thread = (row, 4 float4 columns) of one (stream, head, query-tile pair) block:
 // consecutive threads take consecutive rows, so every load of a split's column
-// is coalesced.  Every split's (max, sum) and columns are loaded unconditionally
-// (a split CTA without keys writes zeros), so all of a thread's loads are in
-// flight at once; the partials are read once (evict-first loads).
+// is coalesced.  The row maxima of all splits come first (m), then the splits
+// are accumulated in order, four at a time with all their loads in flight (a
+// split CTA without keys wrote zeros and a -inf maximum); the partial columns
+// are read once (evict-first loads).
 template <int D>
 __global__ void __launch_bounds__(256) attention_combine_kernel(const __grid_constant__ AttnParams p) {
     grid_dependency_wait();                         // the split CTAs' partials
     grid_launch_dependents();
     constexpr int kC16 = D / 16;                    // 16-column chunks per row
+    constexpr int kGroup = 4;                       // splits whose loads are in flight together
     const int n_su = p.n_units - p.n_whole;         // split units
     const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int srow = static_cast<int>(idx & 255);
@@ -866,37 +981,41 @@ __global__ void __launch_bounds__(256) attention_combine_kernel(const __grid_con
     const int bg = p.b_offset + p.unit_stream[unit / (p.n_qpairs * p.heads)];
     const int token = qpair * 256 + srow;
     if (token >= p.lq) return;
-    float2 ml[kMaxSplits];
-    float4 u[kMaxSplits][4];
-#pragma unroll
-    for (int s = 0; s < kMaxSplits; ++s) {
-        ml[s] = make_float2(-INFINITY, 0.0f);
-        if (s < p.n_pieces) {
-            const int64_t blk = static_cast<int64_t>(s) * n_su + su;
-            ml[s] = __ldcs(reinterpret_cast<const float2 *>(p.part_ml) + blk * 256 + srow);
-            const float4 *po = reinterpret_cast<const float4 *>(p.part_o) + blk * (D / 4) * 256 + (c16 * 4) * 256 + srow;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) u[s][i] = __ldcs(po + i * 256);
-        }
-    }
+    const int np = p.n_pieces;
+    const float2 *ml_row = reinterpret_cast<const float2 *>(p.part_ml) + static_cast<int64_t>(su) * 256 + srow;
+    const int64_t ml_split = static_cast<int64_t>(n_su) * 256;        // float2 stride between splits
     float m = -INFINITY;
-#pragma unroll
-    for (int s = 0; s < kMaxSplits; ++s) m = fmaxf(m, ml[s].x);
+    for (int s = 0; s < np; ++s) m = fmaxf(m, __ldcg(ml_row + s * ml_split).x);
     float a[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) a[i] = 0.0f;
     float l = 0.0f;
+    for (int s0 = 0; s0 < np; s0 += kGroup) {
+        float2 ml[kGroup];
+        float4 u[kGroup][4];
 #pragma unroll
-    for (int s = 0; s < kMaxSplits; ++s) {
-        if (s < p.n_pieces) {
-            const float w = ml[s].x == -INFINITY ? 0.0f : exp2f(ml[s].x - m);
-            l += w * ml[s].y;
+        for (int g = 0; g < kGroup; ++g) {
+            ml[g] = make_float2(-INFINITY, 0.0f);
+            if (s0 + g < np) {
+                const int64_t blk = static_cast<int64_t>(s0 + g) * n_su + su;
+                ml[g] = __ldcg(ml_row + (s0 + g) * ml_split);
+                const float4 *po = reinterpret_cast<const float4 *>(p.part_o) + blk * (D / 4) * 256 + (c16 * 4) * 256 + srow;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                a[4 * i] += w * u[s][i].x;
-                a[4 * i + 1] += w * u[s][i].y;
-                a[4 * i + 2] += w * u[s][i].z;
-                a[4 * i + 3] += w * u[s][i].w;
+                for (int i = 0; i < 4; ++i) u[g][i] = __ldcs(po + i * 256);
+            }
+        }
+#pragma unroll
+        for (int g = 0; g < kGroup; ++g) {
+            if (s0 + g < np) {
+                const float w = ml[g].x == -INFINITY ? 0.0f : exp2f(ml[g].x - m);
+                l += w * ml[g].y;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    a[4 * i] += w * u[g][i].x;
+                    a[4 * i + 1] += w * u[g][i].y;
+                    a[4 * i + 2] += w * u[g][i].z;
+                    a[4 * i + 3] += w * u[g][i].w;
+                }
             }
         }
     }
@@ -954,7 +1073,7 @@ static cudaError_t launch_attention_d(const AttnParams &p, const CUtensorMap &tq
 
 cudaError_t launch_attention(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
                              const CUtensorMap &tv, int head_dim, cudaStream_t s) {
-    if (p.q_scale != nullptr) return launch_attention_d<128, true>(p, tq, tk, tv, s);
+    if (p.f8) return launch_attention_d<128, true>(p, tq, tk, tv, s);
     if (head_dim == 64) return launch_attention_d<64, false>(p, tq, tk, tv, s);
     return launch_attention_d<128, false>(p, tq, tk, tv, s);
 }
@@ -965,18 +1084,6 @@ cudaError_t launch_combine(const AttnParams &p, int head_dim, cudaStream_t s) {
     const dim3 grid(static_cast<unsigned>((threads + 255) / 256));
     if (head_dim == 64) return launch_dependent(attention_combine_kernel<64>, grid, dim3(256), 0, s, p);
     return launch_dependent(attention_combine_kernel<128>, grid, dim3(256), 0, s, p);
-}
-
-cudaError_t launch_rope_q(const AttnParams &p, int sm_count, cudaStream_t s) {
-    (void)sm_count;
-    int nb = 0;
-    for (int i = 0; i < kMaxBatch; ++i)
-        if (p.lk[i] > 0) nb = i + 1;
-    if (nb == 0) return cudaSuccess;
-    const int head_dim = static_cast<int>(p.n_t + p.n_h + p.n_w) * 2;
-    const int rows = p.lq * p.heads;
-    dim3 grid(static_cast<unsigned>((rows + 63) / 64), static_cast<unsigned>(nb));
-    return launch_dependent(rope_q_kernel, grid, dim3(256), 0, s, p, head_dim);
 }
 
 }  // namespace sdv2

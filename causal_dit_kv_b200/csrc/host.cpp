@@ -75,18 +75,18 @@ struct Geometry {
     bool f8;                 // fp8 (E4M3) block-scaled cache
     int64_t np_tokens;       // fp8: tokens per slot padded to whole 128-token blocks
     int n_blk, scale_slot_stride;
-    uint64_t k_scale, v_scale, scale_layer_stride, q_scale, q_scale_bytes;
+    uint64_t k_scale, v_scale, scale_layer_stride;
     int n_qpairs, lq_pad;
     int refresh_chunks;  // token chunks of the refresh reduction
     int64_t part_rows;  // capacity of the split-KV partial buffer, rows of d floats
     // region offsets
     uint64_t rope_h64, rope_w64, rope_h32, rope_w32;
     uint64_t sink_embed, sink_frame, status;
-    uint64_t scratch, refresh_mean, refresh_counter, q_rot, q_rot_bytes, part_ml, part_o, scratch_end;
+    uint64_t scratch, refresh_mean, refresh_counter, part_ml, part_o, scratch_end;
     uint64_t k, v, layer_stride, total;
 };
 
-constexpr int64_t kPartRowsCap = 196608;  // split-KV partial rows (~100 MB at d = 128)
+constexpr int64_t kPartRowsCap = 98304;   // split-KV partial rows: 384 blocks of 256 (~50 MB at d = 128)
 
 sdv2_status check_config(const sdv2_cache_config *c, sdv2_cache_config *norm) {
     if (!c) return fail(SDV2_E_ARG, "config is NULL");
@@ -117,9 +117,15 @@ sdv2_status check_config(const sdv2_cache_config *c, sdv2_cache_config *norm) {
         return fail(SDV2_E_SHAPE, "rope_pairs must be >= 0 and sum to head_dim/2");
     if (n.rope_pairs[0] < 1 || n.rope_pairs[0] > 64)
         return fail(SDV2_E_SHAPE, "the temporal axis needs 1..64 rotation pairs");
-    if (n.rope_pairs[0] * n.chunk_frames > kAttnTabEntries)
-        return fail(SDV2_E_SHAPE, "chunk_frames * temporal pairs exceeds %d", kAttnTabEntries);
     const int64_t N = static_cast<int64_t>(n.frame_h) * n.frame_w;
+    {
+        // the temporal (cos, sin) of the chunk frames that one attention CTA's 256 query rows
+        // can span are kept in shared memory
+        const int64_t frames = std::min<int64_t>(n.chunk_frames, 255 / N + 2);
+        if (frames * n.rope_pairs[0] > kAttnTabEntries)
+            return fail(SDV2_E_SHAPE, "temporal pairs x chunk frames spanned by 256 queries exceeds %d",
+                        kAttnTabEntries);
+    }
     const int64_t slots = n.sink_frames + n.window_frames;
     const int64_t fe = N * n.heads * n.head_dim;
     const int64_t np_tok = (N + 127) / 128 * 128;
@@ -185,16 +191,6 @@ Geometry geometry(const sdv2_cache_config &c) {
     off = align_up(off + 8ull * c.batch * g.refresh_chunks * (c.embed_dim > 0 ? c.embed_dim : 1), 256);
     g.refresh_counter = off;
     off = align_up(off + 4ull * (kMaxBatch + static_cast<uint64_t>(c.batch) * kRefreshMaxColBlocks), 256);
-    // two buffers of rotated queries, used by alternate attention calls: a call's RoPE
-    // pass may then start before the previous call's attention kernel has finished
-    g.q_rot = off;
-    g.q_rot_bytes = align_up(2ull * c.batch * g.lq * c.heads * c.head_dim, 1024);
-    off = align_up(off + 2 * g.q_rot_bytes, 1024);
-    if (g.f8) {                       // per-row scales of the E4M3 queries, one per query buffer
-        g.q_scale = off;
-        g.q_scale_bytes = align_up(4ull * c.batch * g.lq * c.heads, 256);
-        off = align_up(off + 2 * g.q_scale_bytes, 256);
-    }
     g.part_ml = off;
     off = align_up(off + 8ull * g.part_rows, 256);
     g.part_o = off;
@@ -208,10 +204,12 @@ Geometry geometry(const sdv2_cache_config &c) {
 // query-tile pair) units of at most max_tiles KV tiles each.  Either every
 // unit runs whole (one CTA each), or the units beyond the last complete wave
 // (all of them, when there are fewer units than SMs) are split over the KV
-// range into `pieces` CTAs each and merged afterwards.  Chosen by an estimate
-// of the makespan: whole waves x tiles per unit + waves of pieces x tiles per
-// piece + the merge (a fixed cost plus the partials written and read back),
-// within the partial buffer's capacity.
+// range into `pieces` CTAs each (2 .. kMaxSplits) and merged afterwards.
+// Chosen by an estimate of the makespan, in KV-tile times: each wave of CTAs
+// costs its longest CTA, i.e. a fixed start-up and epilogue (about 1.5 tiles)
+// plus its tiles; the split pieces run in the waves after the whole units;
+// the merge adds a fixed launch and the partials written and read back.
+// Within the partial buffer's capacity.
 struct AttnPlan {
     int64_t whole;
     int pieces;
@@ -221,30 +219,30 @@ AttnPlan plan_attention(const sdv2_cache_config &c, const Geometry &g, int64_t u
                         int sm_count) {
     AttnPlan best{units, 1};
     if (units <= 0 || max_tiles <= 1 || sm_count <= 0) return best;
-    // Cost units: one KV tile of one CTA (~2.5 us on a B200 SM at these sizes).
-    const double tile_us = 2.5;
-    const double merge_us = 3.0;
-    const double bytes_per_us = 6.0e6;   // ~6 TB/s
+    const double tile_us = 2.0;            // one KV tile of one CTA (both query tiles) on a B200 SM
+    const double cta_fixed_us = 3.0;       // CTA start-up (barriers, TMEM, first tiles) and epilogue
+    const double merge_us = 3.0;           // the dependent merge launch
+    const double bytes_per_us = 6.0e6;     // ~6 TB/s for the partials written and read back
     const int64_t cap = g.part_rows / 256;  // partial blocks of 256 rows
     auto waves = [&](int64_t ctas) { return (ctas + sm_count - 1) / sm_count; };
-    double best_cost = static_cast<double>(waves(units) * max_tiles) * tile_us;
+    auto wave_us = [&](int64_t tiles) { return cta_fixed_us + static_cast<double>(tiles) * tile_us; };
+    double best_cost = static_cast<double>(waves(units)) * wave_us(max_tiles);
     const int64_t full = (units / sm_count) * sm_count;   // units that fill whole waves
-    for (int s = 2; s <= kMaxSplits; ++s) {
+    for (int s = 2; s <= kMaxSplits && s <= max_tiles; ++s) {
         const int64_t per = (max_tiles + s - 1) / s;
         for (int tail = 0; tail < 2; ++tail) {
             const int64_t whole = tail ? full : 0;
             if (tail && (full == 0 || full == units)) continue;
             const int64_t rest = units - whole;
             if (rest * s > cap) continue;
-            const double cost = static_cast<double>(whole / sm_count * max_tiles) * tile_us +
-                                static_cast<double>(waves(rest * s) * per) * tile_us + merge_us +
+            const double cost = static_cast<double>(whole / sm_count) * wave_us(max_tiles) +
+                                static_cast<double>(waves(rest * s)) * wave_us(per) + merge_us +
                                 static_cast<double>(rest * s) * 256.0 * (c.head_dim + 2) * 8.0 / bytes_per_us;
             if (cost < best_cost - 1e-9) {
                 best_cost = cost;
                 best = {whole, s};
             }
         }
-        if (per <= 1) break;
     }
     return best;
 }
@@ -281,8 +279,6 @@ struct sdv2_cache {
     int sm_count;
     std::vector<int64_t> next_frame;  // [B][L]
     std::vector<CUtensorMap> tk, tv;  // [L]
-    CUtensorMap tq[2];                // the two rotated-query buffers in scratch: (d, H, Lq, B)
-    uint64_t attention_calls = 0;     // selects the rotated-query buffer
     cudaEvent_t time_start = nullptr;  // measurement hook: events around the attention kernel
     cudaEvent_t time_stop = nullptr;
 };
@@ -407,8 +403,18 @@ sdv2_status sdv2_cache_create(const sdv2_cache_config *cfg, void *dev_buf, size_
             w64[2 * (col * nw + j)] = std::cos(a);
             w64[2 * (col * nw + j) + 1] = std::sin(a);
         }
-    for (size_t i = 0; i < h64.size(); ++i) h32[i] = static_cast<float>(h64[i]);
-    for (size_t i = 0; i < w64.size(); ++i) w32[i] = static_cast<float>(w64[i]);
+    // fp32 copies for the queries, pair-major ([pair][position] (cos, sin)): the attention
+    // kernel rotates one query row per thread, so for a given pair the 32 lanes of a warp
+    // (consecutive tokens, consecutive columns) read consecutive entries
+    for (int r = 0; r < n.frame_h; ++r)
+        for (int j = 0; j < nh; ++j)
+            for (int k = 0; k < 2; ++k)
+                h32[2 * (static_cast<size_t>(j) * n.frame_h + r) + k] = static_cast<float>(h64[2 * (r * nh + j) + k]);
+    for (int col = 0; col < n.frame_w; ++col)
+        for (int j = 0; j < nw; ++j)
+            for (int k = 0; k < 2; ++k)
+                w32[2 * (static_cast<size_t>(j) * n.frame_w + col) + k] =
+                    static_cast<float>(w64[2 * (col * nw + j) + k]);
     std::vector<int64_t> sink_frames(static_cast<size_t>(n.batch) * n.sink_frames, -1);
     struct Up { uint64_t off; const void *src; size_t bytes; } ups[] = {
         {g.rope_h64, h64.data(), h64.size() * 8}, {g.rope_w64, w64.data(), w64.size() * 8},
@@ -468,26 +474,6 @@ sdv2_status sdv2_cache_create(const sdv2_cache_config *cfg, void *dev_buf, size_
             if (r != CUDA_SUCCESS) {
                 delete c;
                 return fail(SDV2_E_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
-            }
-        }
-    }
-    {
-        // rotated queries: bf16 (d, H, Lq, B) in 64-channel boxes, or E4M3 codes in 128-byte boxes
-        const cuuint64_t esz = g.f8 ? 1 : 2;
-        const cuuint64_t qdims[4] = {static_cast<cuuint64_t>(n.head_dim), static_cast<cuuint64_t>(n.heads),
-                                     static_cast<cuuint64_t>(g.lq), static_cast<cuuint64_t>(n.batch)};
-        const cuuint64_t qstrides[3] = {static_cast<cuuint64_t>(n.head_dim) * esz,
-                                        static_cast<cuuint64_t>(n.heads) * n.head_dim * esz,
-                                        static_cast<cuuint64_t>(g.lq) * n.heads * n.head_dim * esz};
-        const cuuint32_t qbox[4] = {g.f8 ? 128u : 64u, 1, static_cast<cuuint32_t>(kBlockM), 1};
-        for (int buf = 0; buf < 2; ++buf) {
-            CUresult r = encode(&c->tq[buf], g.f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
-                                c->base + g.q_rot + buf * g.q_rot_bytes, qdims, qstrides, qbox, estr,
-                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-            if (r != CUDA_SUCCESS) {
-                delete c;
-                return fail(SDV2_E_CUDA, "cuTensorMapEncodeTiled (queries) failed (%d)", static_cast<int>(r));
             }
         }
     }
@@ -612,11 +598,27 @@ sdv2_status sdv2_chunk_attention(sdv2_cache *c, int32_t layer, const void *q, vo
     const int n_t = n.rope_pairs[0];
     const int streams_per_launch = kMaxBatch;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // The caller's un-rotated queries as a TMA tensor (d, H, Lq, B), bf16, in boxes of 64
+    // channels x 128 rows with the 128-byte swizzle of the MMA's Q tiles; the kernel rotates
+    // them on load.  Encoded per call: q is the caller's buffer.
+    CUtensorMap tq;
+    {
+        PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode_fn();
+        if (!encode) return fail(SDV2_E_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+        const cuuint64_t qdims[4] = {static_cast<cuuint64_t>(n.head_dim), static_cast<cuuint64_t>(n.heads),
+                                     static_cast<cuuint64_t>(g.lq), static_cast<cuuint64_t>(n.batch)};
+        const cuuint64_t qstrides[3] = {static_cast<cuuint64_t>(n.head_dim) * 2,
+                                        static_cast<cuuint64_t>(n.heads) * n.head_dim * 2,
+                                        static_cast<cuuint64_t>(g.lq) * n.heads * n.head_dim * 2};
+        const cuuint32_t qbox[4] = {64u, 1, static_cast<cuuint32_t>(kBlockM), 1};
+        const cuuint32_t estr[4] = {1, 1, 1, 1};
+        CUresult r = encode(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(q), qdims, qstrides, qbox,
+                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return fail(SDV2_E_CUDA, "cuTensorMapEncodeTiled (queries) failed (%d)", static_cast<int>(r));
+    }
     AttnParams p;
     std::memset(&p, 0, sizeof(p));
-    p.q = static_cast<const uint16_t *>(q);
-    const int qbuf = static_cast<int>(c->attention_calls & 1);
-    p.q_rot = reinterpret_cast<uint16_t *>(c->base + g.q_rot + qbuf * g.q_rot_bytes);
     p.out = static_cast<uint16_t *>(out);
     p.part_o = reinterpret_cast<float *>(c->base + g.part_o);
     p.part_ml = reinterpret_cast<float *>(c->base + g.part_ml);
@@ -627,6 +629,7 @@ sdv2_status sdv2_chunk_attention(sdv2_cache *c, int32_t layer, const void *q, vo
     p.heads = n.heads;
     p.lq = static_cast<int32_t>(g.lq);
     p.tokens_per_frame = static_cast<int32_t>(g.N);
+    p.frame_h = n.frame_h;
     p.frame_w = n.frame_w;
     p.chunk_frames = n.chunk_frames;
     p.n_t = n_t;
@@ -634,12 +637,12 @@ sdv2_status sdv2_chunk_attention(sdv2_cache *c, int32_t layer, const void *q, vo
     p.n_w = n.rope_pairs[2];
     p.n_qpairs = g.n_qpairs;
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
-    p.rope_base = n.rope_base;
+    for (int j = 0; j < n_t; ++j) p.omega_t[j] = rope_angle(n.rope_base, j, n_t, 1);
     p.rope_reset = n.rope_reset_period;
     if (g.f8) {
         p.k_scale = reinterpret_cast<const float *>(c->base + g.k_scale + g.scale_layer_stride * layer);
         p.v_scale = reinterpret_cast<const float *>(c->base + g.v_scale + g.scale_layer_stride * layer);
-        p.q_scale = reinterpret_cast<float *>(c->base + g.q_scale + qbuf * g.q_scale_bytes);
+        p.f8 = 1;
         p.slots = static_cast<int32_t>(g.slots);
         p.np_tokens = static_cast<int32_t>(g.np_tokens);
         p.n_blk = g.n_blk;
@@ -665,26 +668,24 @@ sdv2_status sdv2_chunk_attention(sdv2_cache *c, int32_t layer, const void *q, vo
         const AttnPlan plan = plan_attention(n, g, p.n_units, max_kv_tiles(g, keys.data() + b0, nb), c->sm_count);
         p.n_whole = static_cast<int32_t>(plan.whole);
         p.n_pieces = plan.pieces;
-        cudaError_t e = launch_rope_q(p, c->sm_count, s);
-        if (e != cudaSuccess) return cuda_fail(e, "rope_q launch");
+        cudaError_t e = cudaSuccess;
         if (c->time_start && b0 == 0) {
             e = cudaEventRecord(c->time_start, s);
             if (e != cudaSuccess) return cuda_fail(e, "chunk_attention start event");
         }
-        e = launch_attention(p, c->tq[qbuf], c->tk[layer], c->tv[layer], n.head_dim, s);
+        e = launch_attention(p, tq, c->tk[layer], c->tv[layer], n.head_dim, s);
         if (e != cudaSuccess) return cuda_fail(e, "chunk_attention launch");
         if (c->time_stop && b0 + streams_per_launch >= n.batch) {
             e = cudaEventRecord(c->time_stop, s);
             if (e != cudaSuccess) return cuda_fail(e, "chunk_attention stop event");
         }
-        g_launches.fetch_add(2);
+        g_launches.fetch_add(1);
         if (p.n_whole < p.n_units) {
             e = launch_combine(p, n.head_dim, s);
             if (e != cudaSuccess) return cuda_fail(e, "attention combine launch");
             g_launches.fetch_add(1);
         }
     }
-    ++c->attention_calls;
     return SDV2_OK;
 }
 

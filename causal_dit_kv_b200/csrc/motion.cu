@@ -14,7 +14,8 @@
 // the slice of the stored previous frame with the chunk's last frame (only
 // this block touches that slice, so no ordering across blocks is needed).
 // The last block of a stream to finish (counted with an atomic ticket) sums
-// the partials in block order and runs the recurrence in fp64.
+// the partials (one warp, lanes over blocks, then a fixed butterfly) and runs
+// the recurrence in fp64.
 #include <cmath>
 
 #include "ptx.cuh"
@@ -22,6 +23,12 @@
 namespace sdv2 {
 
 __global__ void __launch_bounds__(kMotionThreads) motion_kernel(const __grid_constant__ MotionParams p) {
+    // Launched as a dependent of the step's last kernel: the motion state is written only
+    // by this kernel (whose previous launch completed before this step's first kernel), so
+    // the work needs nothing from the kernel before it.  Every thread still waits for that
+    // kernel before it exits, so that this grid completes only after it (later kernels of
+    // the stream rely on that order).
+    grid_launch_dependents();
     const int b = blockIdx.y;
     const int blk = blockIdx.x;
     const int tid = threadIdx.x;
@@ -89,9 +96,26 @@ __global__ void __launch_bounds__(kMotionThreads) motion_kernel(const __grid_con
         is_last = ticket == static_cast<unsigned>(p.n_blocks - 1);
     }
     __syncthreads();
-    if (!is_last || tid != 0) return;
+    if (!is_last || tid >= 32) {
+        grid_dependency_wait();
+        return;
+    }
     __threadfence();
 
+    // The last block's first warp: every lane sums the partials i = lane, lane + 32, ...
+    // of each frame (all loads in flight at once), then a fixed butterfly adds the lanes.
+    double ss_frame[kMotionMaxFrames];
+    for (int t = 0; t < p.chunk_frames; ++t) {
+        const double *part = p.partial + (static_cast<int64_t>(b) * p.chunk_frames + t) * p.n_blocks;
+        double ss = 0.0;
+        for (int i = tid; i < p.n_blocks; i += 32) ss += __ldcg(part + i);
+        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        if (t < kMotionMaxFrames) ss_frame[t] = ss;
+    }
+    if (tid != 0) {
+        grid_dependency_wait();
+        return;
+    }
     double rate = p.rate[b];
     int len = p.hist_len[b];
     int pos = p.hist_pos[b];
@@ -100,10 +124,7 @@ __global__ void __launch_bounds__(kMotionThreads) motion_kernel(const __grid_con
     for (int t = 0; t < p.chunk_frames; ++t) {
         float d_out = -1.0f;
         if (have) {
-            double ss = 0.0;
-            const double *part = p.partial + (static_cast<int64_t>(b) * p.chunk_frames + t) * p.n_blocks;
-            for (int i = 0; i < p.n_blocks; ++i) ss += __ldcg(part + i);
-            const double d = sqrt(ss / static_cast<double>(n));
+            const double d = sqrt(ss_frame[t] / static_cast<double>(n));
             hist[pos] = d;
             pos = (pos + 1) % p.window;
             if (len < p.window) ++len;
@@ -124,12 +145,12 @@ __global__ void __launch_bounds__(kMotionThreads) motion_kernel(const __grid_con
     p.has_prev[b] = 1;
     p.out_rate[b] = static_cast<float>(rate);
     p.counter[b] = 0u;
+    grid_dependency_wait();
 }
 
 cudaError_t launch_motion(const MotionParams &p, cudaStream_t s) {
     dim3 grid(static_cast<unsigned>(p.n_blocks), static_cast<unsigned>(p.batch));
-    motion_kernel<<<grid, kMotionThreads, 0, s>>>(p);
-    return cudaGetLastError();
+    return launch_dependent(motion_kernel, grid, dim3(kMotionThreads), 0, s, p);
 }
 
 }  // namespace sdv2

@@ -308,6 +308,17 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return d;
 }
 
+// Named barrier over `count` threads (every participating warp executes it converged).
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+    asm volatile("barrier.sync.aligned %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Make this thread's generic-proxy writes to shared memory visible to the async proxy
+// (the tensor core's operand reads) once a later barrier orders them.
+__device__ __forceinline__ void fence_proxy_async_shared() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Named barrier over `count` threads that also returns the AND of `pred`
 // over them (every participating warp executes it converged).
 __device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t count, bool pred) {

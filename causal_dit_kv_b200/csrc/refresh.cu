@@ -46,9 +46,15 @@ __device__ __forceinline__ double block_sum_fixed(double v, double *red) {
 }
 
 __global__ void __launch_bounds__(kRefreshThreads) refresh_decide_kernel(const __grid_constant__ RefreshParams p) {
+    // Launched as a dependent of the last layer's attention: the column sums read only
+    // the caller's hidden states and this call's scratch, so they start at once; the
+    // kernel waits for its predecessor before it touches what later kernels read (the
+    // decision), and lets the copy kernel launch early (it waits for this grid).
+    grid_launch_dependents();
     const int b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (!p.active[b]) {
+        grid_dependency_wait();
         if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) p.out_slot[b] = -1;
         return;
     }
@@ -101,6 +107,7 @@ __global__ void __launch_bounds__(kRefreshThreads) refresh_decide_kernel(const _
     // in place of token chunk 0's sums; the last column block of the stream then
     // takes the decision.
     uint32_t *col_counter = p.counter + kMaxBatch + static_cast<int64_t>(b) * kRefreshMaxColBlocks + blockIdx.x;
+    grid_dependency_wait();
     __threadfence();
     __syncthreads();
     if (tid == 0) is_last = atomicAdd(col_counter, 1u) == gridDim.y - 1;
@@ -111,8 +118,14 @@ __global__ void __launch_bounds__(kRefreshThreads) refresh_decide_kernel(const _
     {
         const int c = blockIdx.x * kRefreshCols + tid;
         if (c < p.dim) {
+            // all chunk sums of the column in flight at once, then added in chunk order
+            double v[kRefreshMaxChunks];
+#pragma unroll
+            for (int r = 0; r < kRefreshMaxChunks; ++r)
+                v[r] = r < p.row_chunks ? __ldcg(pb + static_cast<int64_t>(r) * p.dim + c) : 0.0;
             double sum = 0.0;
-            for (int r = 0; r < p.row_chunks; ++r) sum += __ldcg(pb + static_cast<int64_t>(r) * p.dim + c);
+#pragma unroll
+            for (int r = 0; r < kRefreshMaxChunks; ++r) sum += v[r];
             pb[c] = sum / static_cast<double>(p.lq);
         }
     }
@@ -187,6 +200,8 @@ __global__ void __launch_bounds__(kRefreshThreads) refresh_decide_kernel(const _
 }
 
 __global__ void __launch_bounds__(256) refresh_copy_kernel(const __grid_constant__ RefreshParams p) {
+    grid_dependency_wait();                     // the decision, and every earlier kernel's reads of the slots
+    grid_launch_dependents();
     const int b = blockIdx.y;
     if (!p.active[b] || p.fill_count[b] > 0) return;
     const int dst_slot = *reinterpret_cast<volatile const int32_t *>(p.out_slot + b);
@@ -210,15 +225,13 @@ __global__ void __launch_bounds__(256) refresh_copy_kernel(const __grid_constant
 cudaError_t launch_refresh(const RefreshParams &p, int sm_count, cudaStream_t s, int *launches) {
     dim3 g1(static_cast<unsigned>((p.dim + kRefreshCols - 1) / kRefreshCols), static_cast<unsigned>(p.row_chunks),
             static_cast<unsigned>(p.batch));
-    refresh_decide_kernel<<<g1, kRefreshThreads, 0, s>>>(p);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_dependent(refresh_decide_kernel, g1, dim3(kRefreshThreads), 0, s, p);
     if (e != cudaSuccess) return e;
     unsigned blocks = static_cast<unsigned>(sm_count) * 2u / static_cast<unsigned>(p.batch);
     if (blocks < 4) blocks = 4;
     dim3 g2(blocks, static_cast<unsigned>(p.batch));
-    refresh_copy_kernel<<<g2, 256, 0, s>>>(p);
     *launches = 2;
-    return cudaGetLastError();
+    return launch_dependent(refresh_copy_kernel, g2, dim3(256), 0, s, p);
 }
 
 }  // namespace sdv2

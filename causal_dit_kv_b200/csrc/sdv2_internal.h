@@ -15,9 +15,10 @@ constexpr int kMaxBatch = 64;
 // fp64 (cos, sin) entries of the temporal axis carried in one append launch.
 constexpr int kAppendTabEntries = 256;    // 4 KB of kernel parameters (rows of distinct phases)
 constexpr int kAppendMaxFrames = 64;
-// fp32 (cos, sin) entries of the temporal axis carried in one attention launch.
-constexpr int kAttnTabEntries = 256;      // temporal (cos, sin) of one stream's chunk, in shared memory
-constexpr int kMaxSplits = 4;
+// fp32 (cos, sin) entries of the temporal axis that one attention CTA keeps in shared
+// memory: n_t pairs for each chunk frame its (up to 256) query rows span.
+constexpr int kAttnTabEntries = 128;
+constexpr int kMaxSplits = 16;                // KV pieces of one split unit, at most
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits give up after 2 s
 
 // Device status word bits (set with atomicOr, never cleared by kernels).
@@ -54,15 +55,13 @@ struct AppendParams {
 };
 
 struct AttnParams {
-    const uint16_t *q;          // [B][Lq][H][d] as given (not rotated)
-    uint16_t *q_rot;            // [B][Lq][H][d] RoPE(q) in bf16, scratch (read by TMA)
     uint16_t *out;              // [B][Lq][H][d]
     float *part_o;              // [piece][split unit][d/4][256] float4 (split units only)
     float *part_ml;             // [piece][split unit][256] float2 (row max in log2 units, row sum)
-    const float *rope_h;        // [frame_h][n_h][2] fp32
-    const float *rope_w;        // [frame_w][n_w][2]
+    const float *rope_h;        // [n_h][frame_h][2] fp32, pair-major
+    const float *rope_w;        // [n_w][frame_w][2]
     uint32_t *status;
-    int32_t batch, heads, lq, tokens_per_frame, frame_w, chunk_frames;
+    int32_t batch, heads, lq, tokens_per_frame, frame_h, frame_w, chunk_frames;
     int32_t n_t, n_h, n_w;
     int32_t n_qpairs, b_offset;
     // Work units u = (i * heads + h) * n_qpairs + qpair over the launch's active streams
@@ -73,15 +72,16 @@ struct AttnParams {
     uint8_t unit_stream[kMaxBatch];
     float scale_log2;           // softmax_scale * log2(e)
     int32_t lk[kMaxBatch];      // valid keys per stream of this launch (0 = skip)
-    double rope_base;           // RoPE frequency base
+    double omega_t[64];         // temporal frequencies base^(-j / n_t), fp64 (host-computed)
     int32_t rope_reset;         // temporal phase period (0: none)
     int64_t f0[kMaxBatch];      // first frame of each stream's chunk
     // fp8 (E4M3) cache only: KV tiles are 128-token blocks of one slot (slot s, block j at
-    // tile s * n_blk + j), each with its own K and V scale; queries are rounded to E4M3 per row
+    // tile s * n_blk + j), each with its own K and V scale; the kernel rounds each rotated
+    // query row to E4M3 with its own scale
     const float *k_scale;       // this layer: [B][slots][scale_slot_stride]
     const float *v_scale;
-    float *q_scale;             // scratch [B][Lq][H]: scale of each rotated query row
     int32_t slots, np_tokens, n_blk, scale_slot_stride;
+    int32_t f8;                 // 1: fp8 cache (E4M3 queries, keys, values and probabilities)
 };
 
 struct RefreshParams {
@@ -146,11 +146,11 @@ inline cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 bl
 // Launchers (defined next to their kernels).  Each returns the CUDA error
 // of the launch; the host layer turns it into an sdv2_status.
 cudaError_t launch_append(const AppendParams &p, int sm_count, cudaStream_t s);
-// RoPE(q) -> q_rot for the streams of the launch (lk > 0), then the attention kernel.
-cudaError_t launch_rope_q(const AttnParams &p, int sm_count, cudaStream_t s);
 cudaError_t launch_wait_selftest(uint32_t *status, uint64_t limit_ns, cudaStream_t s);
 // Merge of the KV-split partials into out (a dependent launch after the attention kernel).
 cudaError_t launch_combine(const AttnParams &p, int head_dim, cudaStream_t s);
+// Attention of the launch's streams; tq maps the caller's (un-rotated) bf16 queries as
+// (d, H, Lq, B) in boxes of 64 channels x 128 rows, 128-byte swizzle.
 cudaError_t launch_attention(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
                              const CUtensorMap &tv, int head_dim, cudaStream_t s);
 cudaError_t launch_refresh(const RefreshParams &p, int sm_count, cudaStream_t s, int *launches);
@@ -170,5 +170,6 @@ constexpr int kRefreshMaxChunks = 32;     // token chunks the chunk-mean reducti
 constexpr int kRefreshMaxColBlocks = 64;  // 256-column blocks of the refresh reduction (embed_dim <= 16384)
 constexpr int kMotionBlockElems = 2048;   // latent elements per motion block
 constexpr int kMotionThreads = 256;
+constexpr int kMotionMaxFrames = 64;      // chunk_frames of a motion state, at most
 
 }  // namespace sdv2

@@ -133,7 +133,9 @@ sdv2_status sdv2_cache_layout_of(const sdv2_cache_config *cfg, sdv2_cache_layout
  * and uploads the RoPE row/column tables, synchronously (not on the hot
  * path).  Every stream starts empty at frame 0.
  * Limits: head_dim in {64, 128}; batch <= 64; N, H, L, S, W, T' >= 1,
- * W >= T'; sink refresh requires embed_dim >= 1.
+ * W >= T'; sink refresh requires embed_dim >= 1; rope_pairs[0] (temporal
+ * pairs) x min(T', floor(255 / N) + 2) <= 128 (the temporal angles of the
+ * chunk frames that 256 consecutive queries span are kept on chip).
  * Errors: SDV2_E_ARG, SDV2_E_SHAPE, SDV2_E_ALIGN (buffer unaligned or too
  * small), SDV2_E_CUDA. */
 sdv2_status sdv2_cache_create(const sdv2_cache_config *cfg, void *dev_buf, size_t bytes,
@@ -166,11 +168,14 @@ sdv2_status sdv2_kv_append(sdv2_cache *cache, int32_t layer, const void *k, cons
 /* Attention of the chunk's queries over the valid sink + window keys of
  * layer `layer`: out = softmax(softmax_scale * RoPE(q) K^T) V.
  * [A] "深入分析" (KV-cache load per chunk), [Q] "Adaptive sink and RoPE refresh".
- * q:   device bf16 [B][T'*N][H][d], NOT rotated: the call rotates it (fp32,
- *      rounded to bf16 for the tensor cores, into the cache's scratch) at the
- *      same (phase, row, col) as the chunk's keys.  With the fp8 cache each
- *      rotated row is coded as E4M3 with its own scale instead, the products
- *      run on E4M3 operands and the probabilities are coded as E4M3 too.
+ * q:   device bf16 [B][T'*N][H][d], NOT rotated.  RoPE is applied on load:
+ *      the attention kernel reads the raw tiles and rotates each row in fp32
+ *      at the same (phase, row, col) as the chunk's keys, rounded to bf16 in
+ *      shared memory for the tensor cores (q itself is never written).  With
+ *      the fp8 cache each rotated row is coded as E4M3 with its own scale
+ *      instead, the products run on E4M3 operands and the probabilities are
+ *      coded as E4M3 too.  q must stay unchanged until the call's kernels
+ *      have run (stream order).
  * out: device bf16 [B][T'*N][H][d].
  * chunk_first_frame: HOST int64 [B], the frames of this chunk; the chunk must
  *      already be appended to this layer (f0 + T' == frames appended).
@@ -231,8 +236,8 @@ sdv2_status sdv2_cache_selftest_wait(sdv2_cache *cache, uint64_t limit_ns, sdv2_
 /* Measurement hook (no counterpart in the pages): while set, every
  * sdv2_chunk_attention call on this cache records `start` on its stream
  * right before the attention kernel's launch and `stop` right after it, so
- * the time between them is that kernel alone (the query RoPE pass before it
- * and the split merge after it are outside).  Recording events between the
+ * the time between them is that kernel alone (the split merge after it is
+ * outside).  Recording events between the
  * call's launches serialises them; use it in a separate timing pass.  Pass
  * NULL for both to switch it off.  The events are the caller's.
  * Errors: SDV2_E_ARG (only one of the two given). */

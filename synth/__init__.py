@@ -2,8 +2,10 @@
 
 This module draws random numbers and lays them out; it holds none of the
 method's arithmetic (no RoPE, no attention, no cosine, no motion measure).
-Every generator returns CPU torch tensors; callers move them to the GPU or
-view their bits for the oracle.  The recipes mirror the shapes and value
+Every generator returns CPU torch tensors (callers move them to the GPU or
+view their bits for the oracle), except ``chunk_qkv_on``, which draws the same
+distribution directly on a device for benchmark inputs too large to draw on
+the host (its values differ from ``chunk_qkv``'s; no oracle comparison uses it).  The recipes mirror the shapes and value
 distributions of the streamed workloads: Q/K/V ~ N(0, 1) rounded to bf16,
 chunk hidden states around a slowly drifting direction with seeded scene
 cuts, and latent frames whose inter-frame steps follow a seeded piecewise-
@@ -36,6 +38,19 @@ def chunk_qkv(seed: int, batch: int, chunk_tokens: int, heads: int, head_dim: in
     base = (int(seed) * 1_000_003 + int(step) * 7919 + int(layer) * 104_729) & 0x7FFFFFFF
     shape = (batch, chunk_tokens, heads, head_dim)
     return (randn_bf16(base + 1, shape), randn_bf16(base + 2, shape), randn_bf16(base + 3, shape))
+
+
+def chunk_qkv_on(device, seed: int, batch: int, chunk_tokens: int, heads: int, head_dim: int, step: int,
+                 layer: int):
+    """Q, K, V [B][T'*N][H][d] bf16 ~ N(0, 1) drawn on ``device`` with a seeded generator
+    of that device (benchmark inputs only)."""
+    import torch as _t
+    base = (int(seed) * 1_000_003 + int(step) * 7919 + int(layer) * 104_729) & 0x7FFFFFFF
+    g = _t.Generator(device=device)
+    g.manual_seed(base)
+    shape = (3, batch, chunk_tokens, heads, head_dim)
+    x = _t.randn(shape, generator=g, dtype=_t.float32, device=device).to(_t.bfloat16)
+    return x[0], x[1], x[2]
 
 
 def drifting_hidden(seed: int, batch: int, chunk_tokens: int, dim: int, n_chunks: int,

@@ -107,7 +107,7 @@ def test_split_plan(B):
     c2 = B.make_cache_config(1, 30, 12, 128, 32, 32, 1, 1, 6)
     # 48 units (12 heads x 4 query-tile pairs) on 148 SMs: every unit split over the KV range
     whole, pieces = B.sdv2_attention_plan(c2, [7168], 148)
-    assert whole == 0 and 2 <= pieces <= 4 and 48 * pieces <= 148
+    assert whole == 0 and 2 <= pieces <= 16 and 48 * pieces <= 148
     assert B.sdv2_attention_splits(c2, [7168], 148) == pieces
     # 37 heads x 4 pairs = 148 units fill the GPU exactly once: nothing split
     full = B.make_cache_config(1, 1, 37, 128, 32, 32, 1, 1, 6)
@@ -116,10 +116,10 @@ def test_split_plan(B):
     c3 = B.make_cache_config(4, 30, 12, 128, 30, 52, 2, 1, 8)
     whole, pieces = B.sdv2_attention_plan(c3, [14040] * 4, 148)
     assert whole == 4 * 148 and pieces > 1 and (624 - whole) * pieces <= 148
-    # 160 units: one full wave whole, the 12 left split
+    # 160 units: one full wave whole, the 12 left split finely enough to fill one more wave
     c4 = B.make_cache_config(1, 40, 40, 128, 32, 32, 1, 1, 6)
     whole, pieces = B.sdv2_attention_plan(c4, [7168], 148)
-    assert whole == 148 and pieces > 1
+    assert whole == 148 and pieces > 4 and 12 * pieces <= 148
     tiny = B.make_cache_config(1, 1, 2, 64, 4, 4, 1, 1, 2)
     assert B.sdv2_attention_plan(tiny, [48], 148) == (2, 1)     # 2 heads, a single KV tile: nothing to split
     assert B.sdv2_attention_plan(c2, [0], 148) == (0, 1)        # no active stream
@@ -148,7 +148,7 @@ def test_plan_properties_over_random_shapes(B):
         sms = rng.choice([132, 148, 160])
         whole, pieces = B.sdv2_attention_plan(cfg, keys, sms)
         units = sum(1 for k in keys if k > 0) * h * ((tp * n + 255) // 256)
-        assert 1 <= pieces <= 4
+        assert 1 <= pieces <= 16 and pieces <= max(1, max(-(-k // 128) for k in keys))
         assert 0 <= whole <= units
         if pieces == 1:
             assert whole == units                     # nothing split
@@ -166,4 +166,4 @@ def test_fp8_plan_counts_whole_blocks_per_slot(B):
     assert tiles_bf == 110 and tiles_f8 == 117
     for cfg in (bf, f8):
         whole, pieces = B.sdv2_attention_plan(cfg, keys, 148)
-        assert 1 <= pieces <= 4 and 0 <= whole <= 12 * 13
+        assert 1 <= pieces <= 16 and 0 <= whole <= 12 * 13

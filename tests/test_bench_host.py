@@ -83,8 +83,8 @@ def test_fp8_workloads_byte_accounting():
     b16, b8 = bench.attn_bytes(w16, keys), bench.attn_bytes(w8, keys)
     hd, lq = 12 * 128, 1024
     assert b16 == 4 * 7168 * hd + 4 * lq * hd                               # K+V, Q, O in bf16
-    # codes for K, V and Q, bf16 O, one K and one V scale per block and head, one scale per query row
-    assert b8 == 2 * 7168 * hd + lq * hd + 2 * lq * hd + 2 * 4 * 12 * 56 + 4 * 12 * lq
+    # codes for K and V, raw bf16 Q (rotated on load), bf16 O, one K and one V scale per block and head
+    assert b8 == 2 * 7168 * hd + 2 * lq * hd + 2 * lq * hd + 2 * 4 * 12 * 56
     assert bench.attn_flops(w8, keys) == bench.attn_flops(w16, keys)
     assert bench.workload_config("x", w8, 1)["kv_format"] == "fp8"
     assert bench.workload_config("x", w16, 1)["kv_format"] == "bf16"

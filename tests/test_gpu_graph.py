@@ -11,7 +11,7 @@ from causal_dit_kv_b200 import KVCache
 
 pytestmark = pytest.mark.gpu
 
-# two query-tile pairs (one ragged) and a 3-way KV split: rope_q, kernel and merge all captured
+# two query-tile pairs (one ragged) and a 3-way KV split: kernel and merge both captured
 CFG = dict(batch=2, layers=2, heads=3, head_dim=128, frame_h=12, frame_w=15, chunk_frames=2, sink_frames=1,
            window_frames=4)
 
