@@ -72,6 +72,9 @@ DEFAULT_WORKLOAD = "wan1.3b-512x512"
 EXTRA_WORKLOADS = ("wan14b-512x512-b1", "wan14b-512x512-b2", "wan14b-512x512-b4", "wan14b-512x512-b8",
                    "wan1.3b-480x832-b4")
 TAU = 0.9
+# device-side wait (cycles, ~40 us at 1.9 GHz) queued ahead of every call that a timing
+# pass brackets with events
+LEAD_CYCLES = 80_000
 
 
 def load_peaks():
@@ -192,7 +195,8 @@ def attention_roofline(w, name, kern_us, peaks, peak_src):
          "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": abytes,
          "avg_launch_us": round(kern_us, 3),
          "timing": "CUDA events recorded by the library right before and after the kernel's launch "
-                   "(sdv2_cache_time_attention), in a pass of its own"}
+                   "(sdv2_cache_time_attention), in a pass of its own; each launch is preceded on the stream "
+                   "by a short device-side wait so that the events time the kernel, not the host's launch latency"}
     if not hbm_bound:
         r["frac_vs_sustained_peak"] = round(achieved_tf / sustained, 4)
     return r
@@ -329,6 +333,14 @@ class Runner:
         e.record(self.stream)
         return e
 
+    def lead(self):
+        """Keep the GPU busy while the host submits the next timed call: a short device-side
+        wait queued ahead of the start event, so the events time the GPU work of the call
+        and not the host's launch latency (an idle GPU would timestamp the start event
+        before the call's kernels have even been submitted)."""
+        import torch
+        torch.cuda._sleep(LEAD_CYCLES)
+
     def step(self, inp, ev=None, wait=None, kernel_ev=None):
         """One streamed chunk through every layer; ev (optional) collects event pairs per
         call; kernel_ev (optional) collects event pairs around each attention kernel alone;
@@ -340,14 +352,17 @@ class Runner:
             if wait is not None:
                 wait(l)
             if ev is not None:
+                self.lead()
                 ev["append"].append([rec()])
             cache.kv_append(l, inp["k"][l], inp["v"][l], f0)
             if ev is not None:
                 ev["append"][-1].append(rec())
+                self.lead()
                 ev["attention"].append([rec()])
             if kernel_ev is not None:
                 k0, k1 = rec(), rec()                    # recorded once so the CUDA events exist
                 cache.time_attention(k0, k1)
+                self.lead()
             cache.chunk_attention(l, inp["q"][l], self.out, f0, self.scale)
             if kernel_ev is not None:
                 cache.time_attention()
@@ -357,12 +372,14 @@ class Runner:
         if wait is not None:
             wait(self.L)
         if ev is not None:
+            self.lead()
             ev["refresh"].append([rec()])
         i = self.n_step % self.n_inputs
         hid, lat = (inp["hid"], inp["lat"]) if "hid" in inp else (self.hid_seq[i], self.lat_seq[i])
         cache.sink_refresh(hid, TAU, f0, self.out_slot)
         if ev is not None:
             ev["refresh"][-1].append(rec())
+            self.lead()
             ev["motion"].append([rec()])
         self.mot.noise_rate(lat, self.rate)
         if ev is not None:
@@ -589,8 +606,9 @@ def run_ours(args, w, name):
                              "gbs": round(refresh_bytes / call_us["refresh"] / 1e3, 1)},
             "motion_noise_rate": {"us": round(call_us["motion"], 3), "bytes": motion_bytes,
                                   "gbs": round(motion_bytes / call_us["motion"] / 1e3, 1)},
-            "note": "per-call times from a second pass with events around each call (events serialise "
-                    "the dependent launches, so these are upper bounds of the in-step cost)"},
+            "note": "per-call times from a second pass with events around each call, each preceded by a "
+                    "short device-side wait so the events time the GPU work, not the host's launch latency "
+                    "(events serialise the dependent launches, so these are upper bounds of the in-step cost)"},
         "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h)},
         "cuda_graph": ({"value": round(frames / (graph_ms / 1e3), 3), "unit": UNIT,

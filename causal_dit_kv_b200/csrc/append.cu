@@ -43,10 +43,11 @@ __device__ __forceinline__ uint32_t rotate_pair(uint32_t w, double c, double s) 
     return static_cast<uint32_t>(bf16_from_f64_rn(r0)) | (static_cast<uint32_t>(bf16_from_f64_rn(r1)) << 16);
 }
 
-// Block = 32 (token, head) rows of one frame, 4 threads per row; each thread
-// moves every 4th 16-byte vector of its row (4 vectors for d = 128), all
-// loads issued before the rotations and stores.  grid = (row blocks, frames
-// of the launch, {K, V}).
+// K block = 32 (token, head) rows of one frame, 4 threads per row; each thread
+// moves every 4th 16-byte vector of its row (4 vectors for d = 128), all loads
+// issued before the rotations and stores.  V block = 64 rows, 2 threads per row
+// (a copy needs no tables).  grid = (K row blocks, frames of the launch, {K, V});
+// the V blocks past the last 64-row block return at once.
 constexpr int kAppendRowsPerBlock = 32;
 
 __global__ void __launch_bounds__(128) kv_append_kernel(const __grid_constant__ AppendParams p) {
@@ -64,10 +65,32 @@ __global__ void __launch_bounds__(128) kv_append_kernel(const __grid_constant__ 
         __syncthreads();
     }
     const int rows = static_cast<int>(p.frame_elems / p.head_dim);     // N * H
+    const int b = p.src_b[fi];
+    if (is_v) {
+        // V is copied: 2 threads per row, 8 (d = 128) or 4 (d = 64) 16-byte vectors each, all
+        // loads in flight before the stores; twice the rows of a K block, so the V blocks
+        // need half the threads and the whole launch fits one wave of the GPU
+        const int vrow = blockIdx.x * (2 * kAppendRowsPerBlock) + (threadIdx.x >> 1);
+        const int vsub = threadIdx.x & 1;
+        if (vrow >= rows) return;
+        const int64_t vsrc = static_cast<int64_t>(b) * p.chunk_tokens * p.heads * p.head_dim +
+                             static_cast<int64_t>(p.src_i[fi]) * p.frame_elems + static_cast<int64_t>(vrow) * p.head_dim;
+        const int64_t vdst = (static_cast<int64_t>(b) * p.slots + p.dst_slot[fi]) * p.frame_elems +
+                             static_cast<int64_t>(vrow) * p.head_dim;
+        constexpr int kMaxV = 8;
+        const int nv = p.head_dim / 16;              // vectors per thread: 8 (d = 128) or 4 (d = 64)
+        uint4 y[kMaxV];
+#pragma unroll
+        for (int i = 0; i < kMaxV; ++i)
+            if (i < nv) y[i] = ld_nc_v4(p.v_in + vsrc + (vsub + 2 * i) * 8);
+#pragma unroll
+        for (int i = 0; i < kMaxV; ++i)
+            if (i < nv) *reinterpret_cast<uint4 *>(p.v_layer + vdst + (vsub + 2 * i) * 8) = y[i];
+        return;
+    }
     const int row = blockIdx.x * kAppendRowsPerBlock + (threadIdx.x >> 2);
     const int sub = threadIdx.x & 3;
     if (row >= rows) return;
-    const int b = p.src_b[fi];
     const int64_t src = static_cast<int64_t>(b) * p.chunk_tokens * p.heads * p.head_dim +
                         static_cast<int64_t>(p.src_i[fi]) * p.frame_elems + static_cast<int64_t>(row) * p.head_dim;
     const int64_t dst = (static_cast<int64_t>(b) * p.slots + p.dst_slot[fi]) * p.frame_elems +
@@ -75,16 +98,9 @@ __global__ void __launch_bounds__(128) kv_append_kernel(const __grid_constant__ 
     constexpr int kMaxVec = 4;                       // d = 128: 16 vectors per row / 4 threads
     const int nvec = p.head_dim / 32;                // vectors per thread: 4 (d = 128) or 2 (d = 64)
     uint4 x[kMaxVec];
-    const uint16_t *in = is_v ? p.v_in : p.k_in;
 #pragma unroll
     for (int i = 0; i < kMaxVec; ++i)
-        if (i < nvec) x[i] = ld_nc_v4(in + src + (sub + 4 * i) * 8);
-    if (is_v) {
-#pragma unroll
-        for (int i = 0; i < kMaxVec; ++i)
-            if (i < nvec) *reinterpret_cast<uint4 *>(p.v_layer + dst + (sub + 4 * i) * 8) = x[i];
-        return;
-    }
+        if (i < nvec) x[i] = ld_nc_v4(p.k_in + src + (sub + 4 * i) * 8);
     const int n = row / p.heads;                     // token in the frame
     const int prow = n / p.frame_w;
     const int pcol = n - prow * p.frame_w;

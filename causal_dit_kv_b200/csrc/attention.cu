@@ -958,10 +958,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 // Merge of the KV-split partials: out = sum_s 2^(m_s - m) O_s / sum_s 2^(m_s - m) l_s.
 // Thread = (row, 4 float4 columns) of one (stream, head, query-tile pair) block:
 // consecutive threads take consecutive rows, so every load of a split's column
-// is coalesced.  The row maxima of all splits come first (m), then the splits
-// are accumulated in order, four at a time with all their loads in flight (a
-// split CTA without keys wrote zeros and a -inf maximum); the partial columns
-// are read once (evict-first loads).
+// is coalesced.  The splits are merged four at a time with all their loads in
+// flight (a split CTA without keys wrote zeros and a -inf maximum): the group's
+// maximum updates the running one and rescales what was merged before, as in the
+// online softmax; with up to four splits that is one group and no rescale.  The
+// partials are read once (evict-first loads).
 template <int D>
 __global__ void __launch_bounds__(256) attention_combine_kernel(const __grid_constant__ AttnParams p) {
     grid_dependency_wait();                         // the split CTAs' partials
@@ -984,8 +985,7 @@ __global__ void __launch_bounds__(256) attention_combine_kernel(const __grid_con
     const int np = p.n_pieces;
     const float2 *ml_row = reinterpret_cast<const float2 *>(p.part_ml) + static_cast<int64_t>(su) * 256 + srow;
     const int64_t ml_split = static_cast<int64_t>(n_su) * 256;        // float2 stride between splits
-    float m = -INFINITY;
-    for (int s = 0; s < np; ++s) m = fmaxf(m, __ldcg(ml_row + s * ml_split).x);
+    float m = -INFINITY;                            // running maximum over the splits merged so far
     float a[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) a[i] = 0.0f;
@@ -998,16 +998,24 @@ __global__ void __launch_bounds__(256) attention_combine_kernel(const __grid_con
             ml[g] = make_float2(-INFINITY, 0.0f);
             if (s0 + g < np) {
                 const int64_t blk = static_cast<int64_t>(s0 + g) * n_su + su;
-                ml[g] = __ldcg(ml_row + (s0 + g) * ml_split);
+                ml[g] = __ldcs(ml_row + (s0 + g) * ml_split);
                 const float4 *po = reinterpret_cast<const float4 *>(p.part_o) + blk * (D / 4) * 256 + (c16 * 4) * 256 + srow;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) u[g][i] = __ldcs(po + i * 256);
             }
         }
+        float mg = m;
+#pragma unroll
+        for (int g = 0; g < kGroup; ++g) mg = fmaxf(mg, ml[g].x);
+        // rescale what was merged so far to the new maximum (nothing merged yet: factor 0)
+        const float c = m == -INFINITY ? 0.0f : exp2f(m - mg);
+        l *= c;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) a[i] *= c;
 #pragma unroll
         for (int g = 0; g < kGroup; ++g) {
-            if (s0 + g < np) {
-                const float w = ml[g].x == -INFINITY ? 0.0f : exp2f(ml[g].x - m);
+            if (s0 + g < np) {                      // (the slots past the last split hold no data)
+                const float w = ml[g].x == -INFINITY ? 0.0f : exp2f(ml[g].x - mg);
                 l += w * ml[g].y;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
@@ -1018,6 +1026,7 @@ __global__ void __launch_bounds__(256) attention_combine_kernel(const __grid_con
                 }
             }
         }
+        m = mg;
     }
     const float inv = 1.0f / l;
     uint16_t *orow = p.out + ((static_cast<int64_t>(bg) * p.lq + token) * p.heads + h) * D + c16 * 16;
