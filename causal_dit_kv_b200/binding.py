@@ -78,6 +78,7 @@ _SIGNATURES = [
     ("sdv2_attention_splits", c_int32, [POINTER(sdv2_cache_config), POINTER(c_int64), c_int32]),
     ("sdv2_attention_plan", c_int32, [POINTER(sdv2_cache_config), POINTER(c_int64), c_int32, POINTER(c_int32),
                                       POINTER(c_int32)]),
+    ("sdv2_attention_pair_mode", c_int32, [POINTER(sdv2_cache_config), POINTER(c_int64), c_int32]),
     ("sdv2_launch_count", c_uint64, []),
     ("sdv2_last_error", c_char_p, []),
     ("sdv2_version", c_char_p, []),
@@ -274,6 +275,11 @@ def sdv2_valid_slots(frame_end: int, sink_frames: int, window_frames: int):
 def sdv2_attention_splits(cfg: sdv2_cache_config, keys, sm_count: int) -> int:
     arr = (c_int64 * cfg.batch)(*[int(k) for k in keys])
     return int(lib().sdv2_attention_splits(ctypes.byref(cfg), arr, sm_count))
+
+
+def sdv2_attention_pair_mode(cfg: sdv2_cache_config, keys, sm_count: int) -> int:
+    arr = (c_int64 * cfg.batch)(*[int(k) for k in keys])
+    return int(lib().sdv2_attention_pair_mode(ctypes.byref(cfg), arr, sm_count))
 
 
 def sdv2_attention_plan(cfg: sdv2_cache_config, keys, sm_count: int):

@@ -340,9 +340,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    // work unit of this CTA: whole units first, then the pieces of the split ones
+    // work unit of this CTA: whole units first, then the pieces of the split ones; in the
+    // pair mode (single-tile chunks, no split) CTA x takes heads 2k and 2k+1 of one stream
     int unit, split, n_split;
-    if (static_cast<int>(blockIdx.x) < p.n_whole) {
+    int h_pair = -1;                            // pair mode: head of accumulator set 1
+    if (p.pair) {
+        const int hp = (p.heads + 1) >> 1;
+        const int k = blockIdx.x % hp;
+        unit = (blockIdx.x / hp) * p.heads + 2 * k;   // (n_qpairs == 1)
+        if (2 * k + 1 < p.heads) h_pair = 2 * k + 1;
+        split = 0;
+        n_split = 1;
+    } else if (static_cast<int>(blockIdx.x) < p.n_whole) {
         unit = blockIdx.x;
         split = 0;
         n_split = 1;
@@ -367,10 +376,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int per = (n_kv + n_split - 1) / n_split;
     const int kv_begin = split * per;
     const int kv_end = min(n_kv, kv_begin + per);
-    const int n_local = kv_end > kv_begin ? kv_end - kv_begin : 0;
+    const bool paired = h_pair >= 0;            // set t: head (t ? h_pair : h), its own query tile and KV tiles
+    // KV tiles of this CTA, in the order the sets take them: in the pair mode both heads'
+    // tiles interleaved (even: head h, odd: head h_pair), otherwise this piece's range
+    const int n_local = paired ? 2 * n_kv : (kv_end > kv_begin ? kv_end - kv_begin : 0);
     const int q_row0 = qpair * (kBlockM * kQTilesPerCta);
-    const int n_qt = (q_row0 + kBlockM < p.lq) ? 2 : 1;
-    const bool dual = n_qt == 1;                // one query tile: the two accumulator sets split the KV tiles
+    const int n_qt = paired || (q_row0 + kBlockM < p.lq) ? 2 : 1;
+    // the two accumulator sets alternate over the KV tiles when there is one query tile
+    // (both sets on that tile, merged at the end) or in the pair mode (one head each)
+    const bool alt = n_qt == 1 || paired;
+    const bool one_q = n_qt == 1;               // one query tile, two accumulator sets merged in the epilogue
 
     if (threadIdx.x == 0) {
         mbar_init(&bars[L::kQFull], 1);
@@ -415,8 +430,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int t = 0; t < n_qt; ++t)
 #pragma unroll
             for (int kb = 0; kb < D / 64; ++kb)
-                tma_load_4d(smem + L::kQRaw + t * L::kQRawTile + kb * L::kSub, &tmap_q, &bars[L::kQFull], kb * 64, h,
-                            q_row0 + t * kBlockM, bg);
+                tma_load_4d(smem + L::kQRaw + t * L::kQRawTile + kb * L::kSub, &tmap_q, &bars[L::kQFull], kb * 64,
+                            paired && t ? h_pair : h, q_row0 + (paired ? 0 : t * kBlockM), bg);
     }
     // RoPE on load by the softmax warps (idle until the first scores arrive): thread
     // (t, row) rotates its own query row (the single-tile mode: sub-tile t of tile 0's row)
@@ -424,8 +439,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (warp >= 4 && n_local > 0) {
         const int t = (warp - 4) >> 2;
         const int row = ((warp & 3) << 5) + lane;
-        const int qt = dual ? 0 : t;            // query tile of this thread's row
-        const int n_rows = min(p.lq - q_row0, dual ? kBlockM : 2 * kBlockM);
+        const int qt = one_q ? 0 : t;           // query tile of this thread's row
+        const int n_rows = min(p.lq - q_row0, alt ? kBlockM : 2 * kBlockM);
         const int fi_lo = q_row0 / p.tokens_per_frame;
         const int fi_hi = (q_row0 + n_rows - 1) / p.tokens_per_frame;
         // temporal (cos, sin) of the chunk frames this CTA's rows span.  The angle
@@ -444,7 +459,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             sincosf(r, &sn, &cs);
             tab[e] = make_float2(cs, sn);
         }
-        const int token = q_row0 + qt * kBlockM + row;
+        const int token = q_row0 + (paired ? 0 : qt * kBlockM) + row;   // (pair mode: both tiles hold rows 0..)
         const bool in_chunk = token < p.lq;
         RopeRow rt;
         {
@@ -469,9 +484,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             // sub-tile 1 holds only row and column pairs: rotated while the temporal table
             // is still being written, then sub-tile 0 after the barrier
             ok = warp_wait(&bars[L::kQFull], 0, abort_flag, p.status, kStatusSoftmaxWait);
-            if (ok && in_chunk && (!dual || t == 1)) rope_subtile_bf16<kNt, kNth>(qtile + L::kSub, row, 32, rt);
+            if (ok && in_chunk && (!one_q || t == 1)) rope_subtile_bf16<kNt, kNth>(qtile + L::kSub, row, 32, rt);
             named_bar_sync(2, kAttnThreads - 128);
-            if (ok && in_chunk && (!dual || t == 0)) rope_subtile_bf16<kNt, kNth>(qtile, row, 0, rt);
+            if (ok && in_chunk && (!one_q || t == 0)) rope_subtile_bf16<kNt, kNth>(qtile, row, 0, rt);
         } else {
             named_bar_sync(2, kAttnThreads - 128);
             ok = warp_wait(&bars[L::kQFull], 0, abort_flag, p.status, kStatusSoftmaxWait);
@@ -479,20 +494,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 if constexpr (F8) {
                     // both threads of a row in the single-tile mode need its scale; one writes the codes
                     const uint8_t *raw = smem + L::kQRaw + qt * L::kQRawTile;
-                    q_row_scale = def_split ? rope_row_e4m3<kNt, kNth>(raw, qtile, row, !dual || t == 0, rt)
-                                            : rope_row_e4m3<0, 0>(raw, qtile, row, !dual || t == 0, rt);
+                    q_row_scale = def_split ? rope_row_e4m3<kNt, kNth>(raw, qtile, row, !one_q || t == 0, rt)
+                                            : rope_row_e4m3<0, 0>(raw, qtile, row, !one_q || t == 0, rt);
                 } else {
                     // two-tile mode: the whole row; single-tile mode: thread t takes sub-tile t
 #pragma unroll
                     for (int kb = 0; kb < D / 64; ++kb) {
-                        if (dual && kb != t) continue;
+                        if (one_q && kb != t) continue;
                         if (def_split)
                             rope_subtile_bf16<kNt, kNth>(qtile + kb * L::kSub, row, kb * 32, rt);
                         else
                             rope_subtile_bf16<0, 0>(qtile + kb * L::kSub, row, kb * 32, rt);
                     }
                 }
-            } else if (F8 && ok && (!dual || t == 0)) {
+            } else if (F8 && ok && (!one_q || t == 0)) {
                 // rows past the chunk: E4M3 zeros (the bf16 tiles were zero-filled by the TMA)
 #pragma unroll
                 for (int c = 0; c < 8; ++c)
@@ -530,10 +545,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         tma_load_4d(smem + L::kK + st * L::kKVTile, &tmap_k, &bars[L::kKFull + st], 0, h,
                                     sl * p.np_tokens + (g - sl * p.n_blk) * kBlockN, bg);
                     } else {
+                        // (pair mode: sequence tile i is tile i / 2 of head h or h_pair)
+                        const int hk = paired && (k_issued & 1) ? h_pair : h;
+                        const int tk = paired ? k_issued >> 1 : kv_begin + k_issued;
 #pragma unroll
                         for (int kb = 0; kb < D / 64; ++kb)
                             tma_load_4d(smem + L::kK + st * L::kKVTile + kb * L::kSub, &tmap_k, &bars[L::kKFull + st],
-                                        kb * 64, h, (kv_begin + k_issued) * kBlockN, bg);
+                                        kb * 64, hk, tk * kBlockN, bg);
                     }
                     ++k_issued;
                 }
@@ -549,10 +567,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     tma_load_5d(smem + L::kV + st * L::kKVTile, &tmap_v, &bars[L::kVFull + st],
                                 (g - sl * p.n_blk) * kBlockN, 0, h, sl, bg);
                 } else {
+                    const int hv = paired && (v_issued & 1) ? h_pair : h;
+                    const int tv = paired ? v_issued >> 1 : kv_begin + v_issued;
 #pragma unroll
                     for (int kb = 0; kb < D / 64; ++kb)
                         tma_load_4d(smem + L::kV + st * L::kKVTile + kb * L::kSub, &tmap_v, &bars[L::kVFull + st],
-                                    kb * 64, h, (kv_begin + v_issued) * kBlockN, bg);
+                                    kb * 64, hv, tv * kBlockN, bg);
                 }
                 ++v_issued;
             }
@@ -586,7 +606,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const uint64_t dk = smem_desc_sw128(smem_addr(smem + L::kK), 16, 1024);
             const uint64_t dv = smem_desc_sw128(smem_addr(smem + L::kV), F8 ? 16 : L::kSub, 1024);
             auto issue_qk = [&](int t, int st) {
-                const uint64_t a0 = dq + static_cast<uint64_t>((dual ? 0 : t) * (L::kQTile >> 4));
+                const uint64_t a0 = dq + static_cast<uint64_t>((one_q ? 0 : t) * (L::kQTile >> 4));
                 const uint64_t b0 = dk + static_cast<uint64_t>(st * (L::kKVTile >> 4));
                 if constexpr (F8) {
 #pragma unroll
@@ -615,7 +635,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
             };
             bool ok = mbar_wait(&bars[L::kQReady], 0, abort_flag, p.status, kStatusMmaWait);
-            if (dual) {
+            if (alt) {
                 // KV tile i -> accumulator set i & 1.  Prologue: S_0 = Q K_0^T, S_1 = Q K_1^T.
                 for (int i = 0; ok && i < n_local && i < 2; ++i) {
                     ok = mbar_wait(&bars[L::kKFull + i % L::kKStages], (i / L::kKStages) & 1, abort_flag, p.status,
@@ -713,11 +733,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int t = (warp - 4) >> 2;               // query tile of this warpgroup
         const int row = ((warp & 3) << 5) + lane;    // TMEM lane == query row in the tile
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) << 5) << 16;
-        if (t < n_qt || dual) {
+        if (t < n_qt || alt) {
             // in the single-tile mode, tile 1's warps take the odd KV tiles of tile 0's rows
-            const int token = q_row0 + (dual ? 0 : t) * kBlockM + row;
+            const int token = q_row0 + (alt ? 0 : t) * kBlockM + row;
+            const int hs = paired && t ? h_pair : h;   // head of this set's rows
             const bool valid = token < p.lq;
-            const int n_mine = dual ? (n_local + 1 - t) / 2 : n_local;
+            const int n_mine = alt ? (n_local + 1 - t) / 2 : n_local;
             float m_run = -INFINITY;   // running max of scale*log2(e)*s
             float l_run = 0.0f;
             bool ok = true;
@@ -729,7 +750,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             int64_t scale_base = 0;
             if constexpr (F8) {
                 sq = valid ? q_row_scale : 0.0f;
-                scale_base = static_cast<int64_t>(bg) * p.slots * p.scale_slot_stride + h * p.n_blk;
+                scale_base = static_cast<int64_t>(bg) * p.slots * p.scale_slot_stride + hs * p.n_blk;
                 sv_ref = 0.0f;
                 for (int i = 0; i < n_local; ++i) {
                     const int g = kv_begin + i, sl = g / p.n_blk;
@@ -738,7 +759,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 sv_ref = fmaxf(sv_ref, 1e-30f);
             }
             for (int it = 0; it < n_mine; ++it) {
-                const int g = kv_begin + (dual ? 2 * it + t : it);   // KV tile of this iteration
+                // KV tile of this iteration (pair mode: tile `it` of this set's own head)
+                const int g = kv_begin + (paired ? it : (alt ? 2 * it + t : it));
                 float c_t = p.scale_log2, r_t = 1.0f;
                 int valid_cols;
                 if constexpr (F8) {
@@ -812,7 +834,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 mbar_arrive(&bars[L::kPFull + t]);
             }
 
-            if (dual) {
+            if (one_q) {
                 // ---- single-tile epilogue: merge the two accumulator sets of the row; thread
                 // (t, row) produces output columns [t d/2, (t+1) d/2)
                 const int n0 = (n_local + 1) / 2, n1 = n_local / 2;
@@ -886,7 +908,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 if (n_split == 1) {
                     if (ok) {
                         const float inv = svr / l_run;
-                        uint16_t *orow = p.out + ((static_cast<int64_t>(bg) * p.lq + token) * p.heads + h) * D;
+                        uint16_t *orow = p.out + ((static_cast<int64_t>(bg) * p.lq + token) * p.heads + hs) * D;
 #pragma unroll
                         for (int cb = 0; cb < D / 32; ++cb) {
                             uint32_t r[32];
@@ -964,7 +986,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 // online softmax; with up to four splits that is one group and no rescale.  The
 // partials are read once (evict-first loads).
 template <int D>
-__global__ void __launch_bounds__(256) attention_combine_kernel(const __grid_constant__ AttnParams p) {
+__global__ void __launch_bounds__(256, 3) attention_combine_kernel(const __grid_constant__ AttnParams p) {
     grid_dependency_wait();                         // the split CTAs' partials
     grid_launch_dependents();
     constexpr int kC16 = D / 16;                    // 16-column chunks per row
@@ -991,19 +1013,11 @@ __global__ void __launch_bounds__(256) attention_combine_kernel(const __grid_con
     for (int i = 0; i < 16; ++i) a[i] = 0.0f;
     float l = 0.0f;
     for (int s0 = 0; s0 < np; s0 += kGroup) {
+        // the group's (max, sum) first, then its columns split by split
         float2 ml[kGroup];
-        float4 u[kGroup][4];
 #pragma unroll
-        for (int g = 0; g < kGroup; ++g) {
-            ml[g] = make_float2(-INFINITY, 0.0f);
-            if (s0 + g < np) {
-                const int64_t blk = static_cast<int64_t>(s0 + g) * n_su + su;
-                ml[g] = __ldcs(ml_row + (s0 + g) * ml_split);
-                const float4 *po = reinterpret_cast<const float4 *>(p.part_o) + blk * (D / 4) * 256 + (c16 * 4) * 256 + srow;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) u[g][i] = __ldcs(po + i * 256);
-            }
-        }
+        for (int g = 0; g < kGroup; ++g)
+            ml[g] = s0 + g < np ? __ldcs(ml_row + (s0 + g) * ml_split) : make_float2(-INFINITY, 0.0f);
         float mg = m;
 #pragma unroll
         for (int g = 0; g < kGroup; ++g) mg = fmaxf(mg, ml[g].x);
@@ -1015,14 +1029,17 @@ __global__ void __launch_bounds__(256) attention_combine_kernel(const __grid_con
 #pragma unroll
         for (int g = 0; g < kGroup; ++g) {
             if (s0 + g < np) {                      // (the slots past the last split hold no data)
+                const int64_t blk = static_cast<int64_t>(s0 + g) * n_su + su;
+                const float4 *po = reinterpret_cast<const float4 *>(p.part_o) + blk * (D / 4) * 256 + (c16 * 4) * 256 + srow;
                 const float w = ml[g].x == -INFINITY ? 0.0f : exp2f(ml[g].x - mg);
                 l += w * ml[g].y;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    a[4 * i] += w * u[g][i].x;
-                    a[4 * i + 1] += w * u[g][i].y;
-                    a[4 * i + 2] += w * u[g][i].z;
-                    a[4 * i + 3] += w * u[g][i].w;
+                    const float4 u = __ldcs(po + i * 256);
+                    a[4 * i] += w * u.x;
+                    a[4 * i + 1] += w * u.y;
+                    a[4 * i + 2] += w * u.z;
+                    a[4 * i + 3] += w * u.w;
                 }
             }
         }
@@ -1075,7 +1092,9 @@ static cudaError_t launch_attention_d(const AttnParams &p, const CUtensorMap &tq
         configured = true;
     }
     if (p.n_units == 0) return cudaSuccess;
-    dim3 grid(static_cast<unsigned>(p.n_whole + (p.n_units - p.n_whole) * p.n_pieces));
+    // pair mode: one CTA per (stream, pair of heads); otherwise whole units, then pieces
+    dim3 grid(static_cast<unsigned>(p.pair ? p.n_units / p.heads * ((p.heads + 1) / 2)
+                                           : p.n_whole + (p.n_units - p.n_whole) * p.n_pieces));
     return launch_dependent(chunk_attention_kernel<D, F8>, grid, dim3(kAttnThreads), static_cast<size_t>(smem), s, p,
                             tq, tk, tv);
 }

@@ -247,6 +247,14 @@ AttnPlan plan_attention(const sdv2_cache_config &c, const Geometry &g, int64_t u
     return best;
 }
 
+// Pair mode of the attention launch: with chunks of one query tile (bf16 cache) and more
+// (stream, head) units than SMs, a CTA takes two heads of one stream, one accumulator set
+// and query tile each, their KV tiles interleaved; half the CTAs, each start-up shared by
+// two heads, and the two softmax / MMA chains of a CTA still overlap.
+bool use_pair_mode(const Geometry &g, const sdv2_cache_config &c, int64_t units, int sm_count) {
+    return !g.f8 && g.n_qpairs == 1 && g.lq <= kBlockM && c.heads >= 2 && sm_count > 0 && units > sm_count;
+}
+
 // KV tiles of the longest stream: 128-key runs of its valid prefix, or for the fp8 cache
 // the 128-token blocks of each valid slot.
 int64_t max_kv_tiles(const Geometry &g, const int64_t *keys, int n) {
@@ -665,9 +673,16 @@ sdv2_status sdv2_chunk_attention(sdv2_cache *c, int32_t layer, const void *q, vo
         }
         if (!any) continue;
         p.n_units = n_active * n.heads * g.n_qpairs;
-        const AttnPlan plan = plan_attention(n, g, p.n_units, max_kv_tiles(g, keys.data() + b0, nb), c->sm_count);
-        p.n_whole = static_cast<int32_t>(plan.whole);
-        p.n_pieces = plan.pieces;
+        if (use_pair_mode(g, n, p.n_units, c->sm_count)) {
+            p.pair = 1;
+            p.n_whole = p.n_units;
+            p.n_pieces = 1;
+        } else {
+            p.pair = 0;
+            const AttnPlan plan = plan_attention(n, g, p.n_units, max_kv_tiles(g, keys.data() + b0, nb), c->sm_count);
+            p.n_whole = static_cast<int32_t>(plan.whole);
+            p.n_pieces = plan.pieces;
+        }
         cudaError_t e = cudaSuccess;
         if (c->time_start && b0 == 0) {
             e = cudaEventRecord(c->time_start, s);
@@ -1012,6 +1027,16 @@ void sdv2_valid_slots(int64_t frame_end, int32_t sink_frames, int32_t window_fra
     if (window_valid) *window_valid = wv;
 }
 
+int32_t sdv2_attention_pair_mode(const sdv2_cache_config *cfg, const int64_t *keys, int32_t sm_count) {
+    sdv2_cache_config n;
+    if (check_config(cfg, &n) != SDV2_OK || !keys) return -1;
+    const Geometry g = geometry(n);
+    int64_t active = 0;
+    for (int b = 0; b < std::min(n.batch, kMaxBatch); ++b)
+        if (keys[b] > 0) ++active;
+    return use_pair_mode(g, n, active * n.heads * g.n_qpairs, sm_count) ? 1 : 0;
+}
+
 int32_t sdv2_attention_splits(const sdv2_cache_config *cfg, const int64_t *keys, int32_t sm_count) {
     int32_t whole = 0, pieces = 0;
     if (sdv2_attention_plan(cfg, keys, sm_count, &whole, &pieces) != SDV2_OK) return -1;
@@ -1028,8 +1053,13 @@ sdv2_status sdv2_attention_plan(const sdv2_cache_config *cfg, const int64_t *key
     int active = 0;
     for (int b = 0; b < std::min(n.batch, kMaxBatch); ++b)
         if (keys[b] > 0) ++active;
-    const AttnPlan plan = plan_attention(n, g, static_cast<int64_t>(active) * n.heads * g.n_qpairs,
-                                         max_kv_tiles(g, keys, std::min(n.batch, kMaxBatch)), sm_count);
+    const int64_t units = static_cast<int64_t>(active) * n.heads * g.n_qpairs;
+    if (use_pair_mode(g, n, units, sm_count)) {     // pair mode: every unit whole
+        *whole_units = static_cast<int32_t>(units);
+        *pieces = 1;
+        return SDV2_OK;
+    }
+    const AttnPlan plan = plan_attention(n, g, units, max_kv_tiles(g, keys, std::min(n.batch, kMaxBatch)), sm_count);
     *whole_units = static_cast<int32_t>(plan.whole);
     *pieces = plan.pieces;
     return SDV2_OK;

@@ -97,7 +97,22 @@ def test_small_chunk_many_streams():
     cfg = dict(batch=16, layers=1, heads=12, head_dim=128, frame_h=8, frame_w=8, chunk_frames=1, sink_frames=1,
                window_frames=6)
     ps = PairedStream(seed=1012, **cfg)
+    from causal_dit_kv_b200 import binding as B
+    assert B.sdv2_attention_pair_mode(ps.gpu.cfg, [448] * 16, 148) == 1     # 192 single-tile units: pair mode
     _stream_and_check(ps, 9, check_every=4, active_fn=lambda s: set(range(15)) if s < 3 else set(range(16)))
+
+
+def test_pair_mode_odd_heads_staggered_streams():
+    """Pair mode with an odd head count (the last head of every stream runs alone, both
+    accumulator sets on its one query tile), d = 64, 60 tokens per frame (a ragged query
+    tile and ragged key tiles) and streams joining at different steps, so their key
+    counts differ while the two heads of a CTA always share one."""
+    from causal_dit_kv_b200 import binding as B
+    cfg = dict(batch=12, layers=2, heads=13, head_dim=64, frame_h=6, frame_w=10, chunk_frames=1, sink_frames=1,
+               window_frames=3)
+    ps = PairedStream(seed=1013, **cfg)
+    assert B.sdv2_attention_pair_mode(ps.gpu.cfg, [240] * 12, 148) == 1     # 156 units
+    _stream_and_check(ps, 8, active_fn=lambda s: {b for b in range(12) if s >= b % 4})
 
 
 def test_many_heads_unsplit_path():
