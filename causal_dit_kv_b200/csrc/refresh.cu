@@ -14,10 +14,10 @@
 // sums in chunk order, divides by the token count, computes the dot products
 // and norms in fp64, takes the decision, updates the sink embedding and the
 // sink-frame record, and writes out_slot[b].
-// Kernel 2, grid (blocks, B): if out_slot[b] >= 0, copies slot last_slot[b]
-// to slot out_slot[b] in every layer, K and V (for the fp8 cache: K and V
-// codes and their block scales), as 16-byte vectors; otherwise the blocks
-// return at once.
+// Kernel 2, two blocks per SM: for every stream b with out_slot[b] >= 0, copies
+// slot last_slot[b] to slot out_slot[b] in every layer, K and V (for the fp8
+// cache: K and V codes and their block scales), as 16-byte vectors spread over
+// all blocks; streams without a refresh are skipped.
 #include <cmath>
 
 #include "ptx.cuh"
@@ -202,22 +202,37 @@ __global__ void __launch_bounds__(kRefreshThreads) refresh_decide_kernel(const _
 __global__ void __launch_bounds__(256) refresh_copy_kernel(const __grid_constant__ RefreshParams p) {
     grid_dependency_wait();                     // the decision, and every earlier kernel's reads of the slots
     grid_launch_dependents();
-    const int b = blockIdx.y;
-    if (!p.active[b] || p.fill_count[b] > 0) return;
-    const int dst_slot = *reinterpret_cast<volatile const int32_t *>(p.out_slot + b);
-    if (dst_slot < 0) return;
-    const int src_slot = p.last_slot[b];
-    for (int r = 0; r < p.n_copy; ++r) {
-        const int64_t vec_per_slot = p.copy_slot_bytes[r] / 16;
-        const int64_t total = static_cast<int64_t>(p.layers) * vec_per_slot;
-        for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < total;
-             g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-            const int64_t layer = g / vec_per_slot;
-            const int64_t vec = g - layer * vec_per_slot;
-            uint8_t *lb = p.copy_base[r] + layer * p.copy_layer_bytes[r] +
-                          static_cast<int64_t>(b) * p.slots * p.copy_slot_bytes[r];
-            const uint4 x = *reinterpret_cast<const uint4 *>(lb + src_slot * p.copy_slot_bytes[r] + vec * 16);
-            *reinterpret_cast<uint4 *>(lb + dst_slot * p.copy_slot_bytes[r] + vec * 16) = x;
+    // Every block takes a share of every refreshed stream's copy (streams whose decision
+    // was "no refresh" cost one load of out_slot), four 16-byte vectors in flight per thread.
+    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    for (int b = 0; b < p.batch; ++b) {
+        if (!p.active[b] || p.fill_count[b] > 0) continue;
+        const int dst_slot = *reinterpret_cast<volatile const int32_t *>(p.out_slot + b);
+        if (dst_slot < 0) continue;
+        const int src_slot = p.last_slot[b];
+        for (int r = 0; r < p.n_copy; ++r) {
+            const int64_t vec_per_slot = p.copy_slot_bytes[r] / 16;
+            const int64_t total = static_cast<int64_t>(p.layers) * vec_per_slot;
+            for (int64_t g0 = gid; g0 < total; g0 += 4 * nthreads) {
+                uint4 x[4];
+                uint4 *dst[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int64_t g = g0 + u * nthreads;
+                    if (g < total) {
+                        const int64_t layer = g / vec_per_slot;
+                        const int64_t vec = g - layer * vec_per_slot;
+                        uint8_t *lb = p.copy_base[r] + layer * p.copy_layer_bytes[r] +
+                                      static_cast<int64_t>(b) * p.slots * p.copy_slot_bytes[r];
+                        x[u] = *reinterpret_cast<const uint4 *>(lb + src_slot * p.copy_slot_bytes[r] + vec * 16);
+                        dst[u] = reinterpret_cast<uint4 *>(lb + dst_slot * p.copy_slot_bytes[r] + vec * 16);
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (g0 + u * nthreads < total) *dst[u] = x[u];
+            }
         }
     }
 }
@@ -227,9 +242,7 @@ cudaError_t launch_refresh(const RefreshParams &p, int sm_count, cudaStream_t s,
             static_cast<unsigned>(p.batch));
     cudaError_t e = launch_dependent(refresh_decide_kernel, g1, dim3(kRefreshThreads), 0, s, p);
     if (e != cudaSuccess) return e;
-    unsigned blocks = static_cast<unsigned>(sm_count) * 2u / static_cast<unsigned>(p.batch);
-    if (blocks < 4) blocks = 4;
-    dim3 g2(blocks, static_cast<unsigned>(p.batch));
+    dim3 g2(static_cast<unsigned>(sm_count > 0 ? 2 * sm_count : 296));
     *launches = 2;
     return launch_dependent(refresh_copy_kernel, g2, dim3(256), 0, s, p);
 }
