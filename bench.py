@@ -65,12 +65,15 @@ WORKLOADS["wan1.3b-128x256-b16"] = dict(batch=16, layers=30, heads=12, head_dim=
                                         motion=(16, 16, 32))
 WORKLOADS["wan1.3b-128x256-b16-fp8"] = dict(WORKLOADS["wan1.3b-128x256-b16"], kv_format="fp8")
 WORKLOADS["wan1.3b-128x128-b16-fp8"] = dict(WORKLOADS["wan1.3b-128x128-b16"], kv_format="fp8")
+# the small-chunk shapes with the append fused into the attention (sdv2_append_attention)
+WORKLOADS["wan1.3b-128x128-b16-fused"] = dict(WORKLOADS["wan1.3b-128x128-b16"], fused=True)
+WORKLOADS["wan1.3b-128x256-b16-fused"] = dict(WORKLOADS["wan1.3b-128x256-b16"], fused=True)
 WORKLOADS["tiny-stream"] = dict(batch=1, layers=1, heads=2, head_dim=64, frame_h=4, frame_w=4, chunk_frames=1,
                                 sink_frames=1, window_frames=2, embed_dim=64, motion=(16, 4, 4))
 DEFAULT_WORKLOAD = "wan1.3b-512x512"
 # timed beside the default workload on one GPU, each under ``workloads``
 EXTRA_WORKLOADS = ("wan14b-512x512-b1", "wan14b-512x512-b2", "wan14b-512x512-b4", "wan14b-512x512-b8",
-                   "wan1.3b-480x832-b4")
+                   "wan1.3b-480x832-b4", "wan1.3b-128x128-b16", "wan1.3b-128x128-b16-fused")
 TAU = 0.9
 # device-side wait (cycles, ~40 us at 1.9 GHz) queued ahead of every call that a timing
 # pass brackets with events
@@ -134,6 +137,8 @@ def workload_config(name, w, world):
            "kv_format": w.get("kv_format", "bf16"), "parallelism": f"replicas x{world}"}
     if "join" in w:
         cfg["stream_join_steps"] = list(w["join"])
+    if w.get("fused"):
+        cfg["append"] = "fused into the attention (sdv2_append_attention)"
     return cfg
 
 
@@ -150,7 +155,9 @@ def attn_flops(w, keys):
 def attn_bytes(w, keys):
     """Bytes one attention kernel launch must move: K and V read once, the raw bf16
     queries read (the kernel rotates them on load), O (bf16) written.  The fp8 cache
-    stores 1-byte codes and adds one K and one V scale per 128-token block and head."""
+    stores 1-byte codes and adds one K and one V scale per 128-token block and head.
+    With the append fused in, the chunk's own K and V (part of the keys read once, from
+    the caller's buffers) are also written to their ring slots."""
     lq = w["chunk_frames"] * w["frame_h"] * w["frame_w"]
     hd = w["heads"] * w["head_dim"]
     e = kv_elem(w)
@@ -159,6 +166,8 @@ def attn_bytes(w, keys):
         total += 2.0 * e * k * hd + 2.0 * lq * hd + 2.0 * lq * hd
         if e == 1:
             total += 2 * 4.0 * w["heads"] * k / 128
+        if w.get("fused"):
+            total += 2.0 * 2.0 * lq * hd
     return total
 
 
@@ -186,7 +195,8 @@ def attention_roofline(w, name, kern_us, peaks, peak_src):
     t = kern_us / 1e6
     achieved_tf = flops / t / 1e12
     achieved_gbs = abytes / t / 1e9
-    r = {"kernel": "chunk_attention_kernel", "bound": "hbm" if hbm_bound else "tensor",
+    r = {"kernel": "chunk_attention_kernel" + ("<fused append>" if w.get("fused") else ""),
+         "bound": "hbm" if hbm_bound else "tensor",
          "achieved": round(achieved_gbs if hbm_bound else achieved_tf, 2), "peak": hbm if hbm_bound else peak,
          "unit": "GB/s" if hbm_bound else "TFLOP/s",
          "frac": round(achieved_gbs / hbm if hbm_bound else achieved_tf / peak, 4),
@@ -348,22 +358,28 @@ class Runner:
         before the calls that read that layer's inputs."""
         f0 = stream_frames(self.w, self.n_step)
         cache, rec = self.cache, self.rec
+        fused = self.w.get("fused", False)
         for l in range(self.L):
             if wait is not None:
                 wait(l)
-            if ev is not None:
+            if ev is not None and not fused:
                 self.lead()
                 ev["append"].append([rec()])
-            cache.kv_append(l, inp["k"][l], inp["v"][l], f0)
+            if not fused:
+                cache.kv_append(l, inp["k"][l], inp["v"][l], f0)
             if ev is not None:
-                ev["append"][-1].append(rec())
+                if not fused:
+                    ev["append"][-1].append(rec())
                 self.lead()
                 ev["attention"].append([rec()])
             if kernel_ev is not None:
                 k0, k1 = rec(), rec()                    # recorded once so the CUDA events exist
                 cache.time_attention(k0, k1)
                 self.lead()
-            cache.chunk_attention(l, inp["q"][l], self.out, f0, self.scale)
+            if fused:
+                cache.append_attention(l, inp["q"][l], inp["k"][l], inp["v"][l], self.out, f0, self.scale)
+            else:
+                cache.chunk_attention(l, inp["q"][l], self.out, f0, self.scale)
             if kernel_ev is not None:
                 cache.time_attention()
                 kernel_ev.append([k0, k1])
@@ -428,7 +444,8 @@ class Runner:
         for i in range(steps):
             self.step(self.pool[i % 2], ev)
         torch.cuda.synchronize()
-        return {k: statistics.mean(a.elapsed_time(b) for a, b in pairs) * 1e3 for k, pairs in ev.items()}
+        return {k: (statistics.mean(a.elapsed_time(b) for a, b in pairs) * 1e3 if pairs else None)
+                for k, pairs in ev.items()}
 
     def close(self):
         self.cache.close()
@@ -595,13 +612,17 @@ def run_ours(args, w, name):
         "data": "synthetic", "config": workload_config(name, w, world),
         "roofline": attention_roofline(w, name, call_us["attn_kernel"], peaks, peak_src),
         "rows": {
-            "kv_append": {"us": round(call_us["append"], 3), "bytes": append_bytes,
-                          "gbs": round(append_bytes / call_us["append"] / 1e3, 1),
-                          "frac_hbm": round(append_bytes / call_us["append"] / 1e3 / hbm, 4)},
+            "kv_append": ({"us": round(call_us["append"], 3), "bytes": append_bytes,
+                           "gbs": round(append_bytes / call_us["append"] / 1e3, 1),
+                           "frac_hbm": round(append_bytes / call_us["append"] / 1e3 / hbm, 4)}
+                          if call_us["append"] is not None else
+                          {"fused": "into the attention call (sdv2_append_attention)"}),
             "chunk_attention": {"us": round(call_us["attention"], 3), "tflops": round(achieved, 2),
                                 "frac_tensor": round(achieved / call_peak, 4),
                                 "kv_gbs": round(kv_gbs, 1), "frac_hbm": round(kv_gbs / hbm, 4),
-                                "what": "whole sdv2_chunk_attention call: every kernel it launches"},
+                                "what": ("whole sdv2_append_attention call (append fused in): every kernel it "
+                                         "launches" if w.get("fused") else
+                                         "whole sdv2_chunk_attention call: every kernel it launches")},
             "sink_refresh": {"us": round(call_us["refresh"], 3), "bytes_without_copy": refresh_bytes,
                              "gbs": round(refresh_bytes / call_us["refresh"] / 1e3, 1)},
             "motion_noise_rate": {"us": round(call_us["motion"], 3), "bytes": motion_bytes,

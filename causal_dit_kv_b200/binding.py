@@ -60,6 +60,8 @@ _SIGNATURES = [
     ("sdv2_cache_destroy", c_int32, [c_void_p]),
     ("sdv2_kv_append", c_int32, [c_void_p, c_int32, c_void_p, c_void_p, POINTER(c_int64), c_void_p]),
     ("sdv2_chunk_attention", c_int32, [c_void_p, c_int32, c_void_p, c_void_p, POINTER(c_int64), c_float, c_void_p]),
+    ("sdv2_append_attention", c_int32,
+     [c_void_p, c_int32, c_void_p, c_void_p, c_void_p, c_void_p, POINTER(c_int64), c_float, c_void_p]),
     ("sdv2_sink_refresh", c_int32, [c_void_p, c_void_p, c_float, POINTER(c_int64), c_void_p, c_void_p]),
     ("sdv2_cache_query", c_int32, [c_void_p, c_int32, c_int32, POINTER(c_int64), POINTER(c_int32), POINTER(c_int32)]),
     ("sdv2_cache_layout_get", c_int32, [c_void_p, POINTER(sdv2_cache_layout)]),
@@ -79,6 +81,7 @@ _SIGNATURES = [
     ("sdv2_attention_plan", c_int32, [POINTER(sdv2_cache_config), POINTER(c_int64), c_int32, POINTER(c_int32),
                                       POINTER(c_int32)]),
     ("sdv2_attention_pair_mode", c_int32, [POINTER(sdv2_cache_config), POINTER(c_int64), c_int32]),
+    ("sdv2_append_attention_mode", c_int32, [POINTER(sdv2_cache_config), POINTER(c_int64), c_int32]),
     ("sdv2_launch_count", c_uint64, []),
     ("sdv2_last_error", c_char_p, []),
     ("sdv2_version", c_char_p, []),
@@ -191,6 +194,13 @@ def sdv2_chunk_attention(cache: int, layer: int, q, out, chunk_first_frame, soft
                                       float(softmax_scale), _stream(stream)), "sdv2_chunk_attention")
 
 
+def sdv2_append_attention(cache: int, layer: int, q, k, v, out, chunk_first_frame, softmax_scale: float, batch: int,
+                          stream=None) -> None:
+    _check(lib().sdv2_append_attention(cache, layer, _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                       _frames(chunk_first_frame, batch), float(softmax_scale), _stream(stream)),
+           "sdv2_append_attention")
+
+
 def sdv2_sink_refresh(cache: int, hidden, tau: float, chunk_first_frame, out_slot, batch: int, stream=None) -> None:
     _check(lib().sdv2_sink_refresh(cache, _ptr(hidden), float(tau), _frames(chunk_first_frame, batch), _ptr(out_slot),
                                    _stream(stream)), "sdv2_sink_refresh")
@@ -280,6 +290,12 @@ def sdv2_attention_splits(cfg: sdv2_cache_config, keys, sm_count: int) -> int:
 def sdv2_attention_pair_mode(cfg: sdv2_cache_config, keys, sm_count: int) -> int:
     arr = (c_int64 * cfg.batch)(*[int(k) for k in keys])
     return int(lib().sdv2_attention_pair_mode(ctypes.byref(cfg), arr, sm_count))
+
+
+def sdv2_append_attention_mode(cfg: sdv2_cache_config, chunk_first_frame, sm_count: int) -> int:
+    """0: two launches, 1: fused kernel, 2: fused kernel in the pair mode (-1: bad argument)."""
+    arr = (c_int64 * cfg.batch)(*[int(f) for f in chunk_first_frame])
+    return int(lib().sdv2_append_attention_mode(ctypes.byref(cfg), arr, sm_count))
 
 
 def sdv2_attention_plan(cfg: sdv2_cache_config, keys, sm_count: int):

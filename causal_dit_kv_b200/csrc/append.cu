@@ -16,33 +16,6 @@
 
 namespace sdv2 {
 
-__device__ __forceinline__ uint16_t bf16_from_f64_rn(double x) {
-    uint16_t r;
-    asm("cvt.rn.bf16.f64 %0, %1;" : "=h"(r) : "d"(x));
-    return r;
-}
-
-__device__ __forceinline__ uint4 ld_nc_v4(const uint16_t *p) {
-    uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
-}
-
-__device__ __forceinline__ double bf16_to_f64(uint32_t bits16) {
-    return static_cast<double>(__uint_as_float(bits16 << 16));
-}
-
-// Rotate one packed pair (lo = dim 2j, hi = dim 2j+1) by (c, s).
-__device__ __forceinline__ uint32_t rotate_pair(uint32_t w, double c, double s) {
-    const double x0 = bf16_to_f64(w & 0xFFFFu);
-    const double x1 = bf16_to_f64(w >> 16);
-    const double r0 = __dsub_rn(__dmul_rn(x0, c), __dmul_rn(x1, s));
-    const double r1 = __dadd_rn(__dmul_rn(x0, s), __dmul_rn(x1, c));
-    return static_cast<uint32_t>(bf16_from_f64_rn(r0)) | (static_cast<uint32_t>(bf16_from_f64_rn(r1)) << 16);
-}
-
 // K block = 32 (token, head) rows of one frame, 4 threads per row; each thread
 // moves every 4th 16-byte vector of its row (4 vectors for d = 128), all loads
 // issued before the rotations and stores.  V block = 64 rows, 2 threads per row

@@ -61,12 +61,13 @@
 // Every wait is bounded (2 s), after which the CTA records an error in the
 // device status word and unwinds; TMEM is always released.
 #include <cmath>
+#include <type_traits>
 
 #include "ptx.cuh"
 
 namespace sdv2 {
 
-template <int D, bool F8 = false>
+template <int D, bool F8 = false, bool FUSE = false>
 struct AttnLayout {
     static constexpr int kElem = F8 ? 1 : 2;          // bytes per element of Q, K, V in the MMA tiles
     static constexpr int kQTile = kBlockM * D * kElem;    // bytes of one Q tile
@@ -82,6 +83,12 @@ struct AttnLayout {
     static constexpr int kQRaw = F8 ? kV + kVStages * kKVTile : kQ;
     static constexpr int kQRawTile = kBlockM * D * 2;
     static constexpr int kTab = F8 ? kQRaw + kQTilesPerCta * kQRawTile : kV + kVStages * kKVTile;
+    // fused append: fp64 (cos, sin) for the keys (temporal entries of the chunk's frames,
+    // then the cache's row table and column table) in V stage 2, which no tile uses before
+    // the assembled tiles are built (the producer loads it only after kAsm)
+    static constexpr int kTab64 = kV + 2 * kKVTile;
+    static constexpr int kTabHW = kTab64 + kFuseTabSmem * 16;
+    static_assert(!FUSE || kFuseTabSmem * 16 + fuse_tab_hw_bytes(D) <= kKVTile, "key tables fit V stage 2");
     static constexpr int kBar = kTab + kAttnTabEntries * 8;
     // barriers
     static constexpr int kQFull = 0;                  // raw query tiles landed (TMA)
@@ -94,8 +101,10 @@ struct AttnLayout {
     static constexpr int kPFull = kSFull + 2;
     static constexpr int kOFull = kPFull + 2;
     static constexpr int kDrain = kOFull + 2;
-    static constexpr int kNumBars = kDrain + 1;
-    static constexpr int kMisc = kBar + kNumBars * 8;   // tmem base, abort flag
+    static constexpr int kAsm = kDrain + 1;           // fused append: assembled tiles written (one arrival per warp 2..11)
+    static constexpr int kTabReady = kAsm + 1;        // fused append: fp64 key tables in shared memory
+    static constexpr int kNumBars = kAsm + (FUSE ? 2 : 0);
+    static constexpr int kMisc = kBar + kNumBars * 8;   // tmem base, abort flag, assembly work counter
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;      // room to align the base to 1024 bytes
     static_assert(kAlloc <= 232448, "shared memory of one CTA");
@@ -326,12 +335,238 @@ __device__ __forceinline__ void merge_sets(uint32_t o0, uint32_t o1, bool has1, 
     for (int i = 0; i < 32; ++i) r0[i] = __float_as_uint(w0 * __uint_as_float(r0[i]) + w1 * __uint_as_float(r1[i]));
 }
 
-template <int D, bool F8>
+// Fused append: TMA of the 8-row groups `groups` of an assembled tile (bit q: rows
+// 8q .. 8q + 7), as runs: consecutive groups whose rows are consecutive in the tensor go
+// together, each run in boxes of 64, 32, 16, 8 rows, largest first (maps[i]: boxes of
+// 64 >> i rows x 64 channels; row_of(q): the tensor row of group q's first row).  A load
+// lands in the tile at dst (a box of rows starting at tile row 8q goes to byte 1024 q of
+// each 128-byte-swizzled sub-tile, where a whole-tile load puts those rows); a store
+// (store = true) writes the tile's rows to the tensor instead.
+template <int D, typename L, typename RowOf>
+__device__ __forceinline__ void move_row_groups(uint8_t *dst, const CUtensorMap *maps, uint64_t *bar, uint32_t groups,
+                                                int hh, int bg, RowOf row_of, bool store) {
+    int q = 0;
+    while (q < 16) {
+        if (!((groups >> q) & 1u)) {
+            ++q;
+            continue;
+        }
+        const int row0 = row_of(q);
+        int e = q + 1;                                // the run: groups q .. e - 1
+        while (e < 16 && ((groups >> e) & 1u) && row_of(e) == row0 + 8 * (e - q)) ++e;
+        for (int g = q; g < e;) {
+            const int left = e - g;                   // groups left in the run
+            const int i = left >= 8 ? 0 : (left >= 4 ? 1 : (left >= 2 ? 2 : 3));
+            const int row = row0 + 8 * (g - q);
+#pragma unroll
+            for (int kb = 0; kb < D / 64; ++kb) {
+                if (store)
+                    tma_store_4d(&maps[i], dst + kb * L::kSub + g * 1024, kb * 64, hh, row, bg);
+                else
+                    tma_load_4d(dst + kb * L::kSub + g * 1024, &maps[i], bar, kb * 64, hh, row, bg);
+            }
+            g += 8 >> i;
+        }
+        q = e;
+    }
+}
+
+// Fused append, the rows of the assembled tiles that straddle slots (the "part" 8-row
+// groups mp0, mp1 of tiles g0, g1; rare: only where a slot boundary is not a multiple of
+// 8 rows).  They are cut into slots of kRowsPerIter rows, dealt round-robin to warps
+// 2 .. 11 (wi = warp - 2); in a slot kLanes lanes share a row and lane c takes pairs c,
+// c + kLanes, c + 2 kLanes, c + 3 kLanes (one 32-bit word of K and of V each), so a
+// row's loads are contiguous words and neighbouring lanes read neighbouring entries of
+// the shared-memory tables (no bank conflicts).  A warp issues the loads of up to kBatch
+// slots at once, then rotates and stores them.  A row of one of the chunk's frames is
+// read from the caller's k / v (keys rotated pair by pair with the append's fp64 rule),
+// written to its ring slot and to the tile; another valid row is read from the cache;
+// rows past the valid prefix are zero (masked, and finite under the zero
+// probabilities).  Words land at the 128-byte-swizzled positions a TMA load gives them.
+template <int D, typename L>
+__device__ __forceinline__ void build_part_groups(uint8_t *smem, uint64_t *bars, const AttnParams &p,
+                                                  const FuseParams &f, int bg, int lk, int h, int h_pair, bool paired,
+                                                  int g0, int g1, uint32_t mp0, uint32_t mp1,
+                                                  const int (&ns)[kFuseMaxFrames], int wi, int lane,
+                                                  volatile uint32_t *abort_flag, bool &have_tab) {
+    constexpr int kLanes = D / 8;                     // lanes per row (4 pairs each)
+    constexpr int kRowsPerIter = 32 / kLanes;         // rows of one slot
+    constexpr int kIters = 8 / kRowsPerIter;          // slots of an 8-row group
+    constexpr int kWarps = (kAttnThreads - 64) / 32;  // warps 2 .. 11
+    constexpr int kBatch = 4;                         // slots of one warp whose loads are in flight together
+    const int c0 = __popc(mp0);
+    const int n_slots = kIters * (c0 + __popc(mp1));
+    if (wi >= n_slots) return;
+    const int c = lane % kLanes;
+    const int rr = lane / kLanes;
+    const int N = p.tokens_per_frame;
+    const int n_t = p.n_t, n_th = p.n_t + p.n_h, n_h = p.n_h, n_w = p.n_w, fw = p.frame_w;
+    const int64_t row_elems = static_cast<int64_t>(p.heads) * D;
+    const int64_t cache_row0 = static_cast<int64_t>(bg) * f.slots * N;   // first key row of this stream
+    const int64_t in_row0 = static_cast<int64_t>(bg) * p.lq;
+    const double2 *tab_t = reinterpret_cast<const double2 *>(smem + L::kTab64);
+    const double2 *tab_h = reinterpret_cast<const double2 *>(smem + L::kTabHW);
+    const double2 *tab_w = tab_h + p.frame_h * n_h;
+    for (int s0 = wi; s0 < n_slots; s0 += kWarps * kBatch) {
+        uint32_t xk[kBatch][4], xv[kBatch][4];
+        int fi[kBatch], nn[kBatch], rw[kBatch];       // chunk frame (-1: not the chunk's, -2: no slot); token; tile row | tile << 8
+        int64_t dst[kBatch];                          // element offset of this lane's row in the layer (pair 0)
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            const int s = s0 + b * kWarps;
+            fi[b] = -2;
+            nn[b] = 0;
+            rw[b] = 0;
+            dst[b] = 0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) xk[b][q] = xv[b][q] = 0u;
+            if (s < n_slots) {
+                const int a = s < kIters * c0 ? 0 : 1;
+                const int sa = a ? s - kIters * c0 : s;
+                uint32_t m = a ? mp1 : mp0;
+                for (int k = sa / kIters; k > 0; --k) m &= m - 1u;
+                const int r = (__ffs(m) - 1) * 8 + (sa % kIters) * kRowsPerIter + rr;
+                const int kr = (a ? g1 : g0) * kBlockN + r;
+                const int hs = paired && a == 1 ? h_pair : h;
+                rw[b] = r | (a << 8);
+                fi[b] = -1;
+                if (kr < lk) {
+                    const int sl = kr / N;
+                    const int n = kr - sl * N;
+#pragma unroll
+                    for (int i = 0; i < kFuseMaxFrames; ++i)
+                        if (ns[i] == sl) fi[b] = i;
+                    nn[b] = n;
+                    dst[b] = (cache_row0 + kr) * row_elems + hs * D;
+                    const int64_t src =
+                        fi[b] >= 0 ? (in_row0 + static_cast<int64_t>(fi[b]) * N + n) * row_elems + hs * D : dst[b];
+                    const uint32_t *ks = reinterpret_cast<const uint32_t *>((fi[b] >= 0 ? f.k_in : f.k_layer) + src);
+                    const uint32_t *vs = reinterpret_cast<const uint32_t *>((fi[b] >= 0 ? f.v_in : f.v_layer) + src);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        xk[b][q] = ld_nc_u32(ks + c + kLanes * q);
+                        xv[b][q] = ld_nc_u32(vs + c + kLanes * q);
+                    }
+                }
+            }
+        }
+        if (!have_tab) {                              // the key tables, once
+            have_tab = warp_wait(&bars[L::kTabReady], 0, abort_flag, p.status, kStatusSoftmaxWait);
+            if (!have_tab) return;
+        }
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            if (fi[b] == -2) continue;
+            const int r = rw[b] & 0xFF, a = rw[b] >> 8;
+            uint8_t *krow = smem + L::kK + a * L::kKVTile + r * 128;
+            uint8_t *vrow = smem + L::kV + a * L::kKVTile + r * 128;
+            const int prow = nn[b] / fw;
+            const int pcol = nn[b] - prow * fw;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int j = c + kLanes * q;         // pair: dims 2j, 2j + 1
+                uint32_t wk = xk[b][q];
+                if (fi[b] >= 0) {
+                    const double2 cs = j < n_t ? tab_t[fi[b] * n_t + j]
+                                               : (j < n_th ? tab_h[prow * n_h + (j - n_t)] : tab_w[pcol * n_w + (j - n_th)]);
+                    wk = rotate_pair(wk, cs.x, cs.y);
+                    reinterpret_cast<uint32_t *>(f.k_layer + dst[b])[j] = wk;
+                    reinterpret_cast<uint32_t *>(f.v_layer + dst[b])[j] = xv[b][q];
+                }
+                // 128-byte-swizzled position of pair j: sub-tile j / 32, 16-byte chunk (j % 32) / 4
+                const int off = (j >> 5) * L::kSub + ((((j & 31) >> 2) ^ (r & 7)) << 4) + ((j & 3) << 2);
+                *reinterpret_cast<uint32_t *>(krow + off) = wk;
+                *reinterpret_cast<uint32_t *>(vrow + off) = xv[b][q];
+            }
+        }
+    }
+}
+
+// Fused append, the "full" 8-row groups mf0, mf1 of the assembled tiles (eight
+// consecutive tokens of one chunk frame each): their un-rotated keys and values came by
+// TMA from the caller's k / v into the tiles; once a tile's loads have landed (its kKFull
+// phase), the keys are rotated in place, pair by pair with the append's fp64 rule.  Rows
+// are dealt round-robin to warps 2 .. 11 in slots of kRowsPerIter rows; lane c of a row
+// takes pairs c + kLanes q (32-bit words of the swizzled row; neighbouring table entries).
+// The producer writes these rows to their ring slots by TMA after kAsm.
+template <int D, typename L>
+__device__ __forceinline__ void rotate_full_groups(uint8_t *smem, uint64_t *bars, const AttnParams &p, int g0, int g1,
+                                                   uint32_t mf0, uint32_t mf1, const int (&ns)[kFuseMaxFrames], int wi,
+                                                   int lane, volatile uint32_t *abort_flag, bool &have_tab) {
+    constexpr int kLanes = D / 8;
+    constexpr int kRowsPerIter = 32 / kLanes;
+    constexpr int kIters = 8 / kRowsPerIter;
+    constexpr int kWarps = (kAttnThreads - 64) / 32;
+    const int c0 = __popc(mf0);
+    const int n_slots = kIters * (c0 + __popc(mf1));
+    if (wi >= n_slots) return;
+    const int c = lane % kLanes;
+    const int rr = lane / kLanes;
+    const int N = p.tokens_per_frame;
+    const int n_t = p.n_t, n_th = p.n_t + p.n_h, n_h = p.n_h, n_w = p.n_w, fw = p.frame_w;
+    const double2 *tab_t = reinterpret_cast<const double2 *>(smem + L::kTab64);
+    const double2 *tab_h = reinterpret_cast<const double2 *>(smem + L::kTabHW);
+    const double2 *tab_w = tab_h + p.frame_h * n_h;
+    if (!have_tab) {
+        have_tab = warp_wait(&bars[L::kTabReady], 0, abort_flag, p.status, kStatusSoftmaxWait);
+        if (!have_tab) return;
+    }
+    uint32_t landed = 0u;                             // tiles whose loads this warp has seen land
+    for (int s = wi; s < n_slots; s += kWarps) {
+        const int a = s < kIters * c0 ? 0 : 1;
+        if (!((landed >> a) & 1u)) {
+            if (!warp_wait(&bars[L::kKFull + a], 0, abort_flag, p.status, kStatusSoftmaxWait)) return;
+            landed |= 1u << a;
+        }
+        const int sa = a ? s - kIters * c0 : s;
+        uint32_t m = a ? mf1 : mf0;
+        for (int k = sa / kIters; k > 0; --k) m &= m - 1u;
+        const int r = (__ffs(m) - 1) * 8 + (sa % kIters) * kRowsPerIter + rr;
+        const int kr = (a ? g1 : g0) * kBlockN + r;
+        const int sl = kr / N;
+        const int n = kr - sl * N;
+        int fi = 0;
+#pragma unroll
+        for (int i = 0; i < kFuseMaxFrames; ++i)
+            if (ns[i] == sl) fi = i;
+        const int prow = n / fw;
+        const int pcol = n - prow * fw;
+        uint8_t *krow = smem + L::kK + a * L::kKVTile + r * 128;
+        uint32_t w[4];
+        int off[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int j = c + kLanes * q;
+            off[q] = (j >> 5) * L::kSub + ((((j & 31) >> 2) ^ (r & 7)) << 4) + ((j & 3) << 2);
+            w[q] = *reinterpret_cast<const uint32_t *>(krow + off[q]);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int j = c + kLanes * q;
+            const double2 cs = j < n_t ? tab_t[fi * n_t + j]
+                                       : (j < n_th ? tab_h[prow * n_h + (j - n_t)] : tab_w[pcol * n_w + (j - n_th)]);
+            *reinterpret_cast<uint32_t *>(krow + off[q]) = rotate_pair(w[q], cs.x, cs.y);
+        }
+    }
+}
+
+// Fused append: a warp's writes to the assembled tiles are done; fence them for the
+// tensor core and the TMA stores, then one arrival on kAsm (warps 2 .. 11).
+template <typename L>
+__device__ __forceinline__ void assembled(uint64_t *bars, int lane) {
+    fence_proxy_async_shared();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars[L::kAsm]);
+}
+
+template <int D, bool F8, bool FUSE>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     chunk_attention_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
-                           const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v) {
-    using L = AttnLayout<D, F8>;
+                           const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+                           const __grid_constant__ std::conditional_t<FUSE, FuseParams, FuseNone> f) {
+    using L = AttnLayout<D, F8, FUSE>;
     static_assert(!F8 || D == 128, "the fp8 cache is built for head_dim 128");
+    static_assert(!(F8 && FUSE), "the fused append is built for the bf16 cache");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBar);
@@ -386,6 +621,53 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // (both sets on that tile, merged at the end) or in the pair mode (one head each)
     const bool alt = n_qt == 1 || paired;
     const bool one_q = n_qt == 1;               // one query tile, two accumulator sets merged in the epilogue
+    // Fused append: the KV tiles of this CTA's range that hold the chunk's own rows (a0 < a1;
+    // pair mode: the stream's one such tile, for both heads) are assembled in shared memory
+    // and taken first; n_asm local tiles (K and V stages 0 .. n_asm - 1) come that way.
+    int n_asm = 0, na = 0, a0 = -1, a1 = -1;
+    int ns[kFuseMaxFrames];                     // fused append: ring slots of the chunk's frames (-1: none),
+    int phs[kFuseMaxFrames];                    // their temporal phases,
+    uint32_t mf0 = 0u, mf1 = 0u, mp0 = 0u, mp1 = 0u;   // and the full / part 8-row groups of the assembled tiles
+    if constexpr (FUSE) {
+        const int t0 = f.asm_tile[bl][0], t1 = f.asm_tile[bl][1];
+#pragma unroll
+        for (int i = 0; i < kFuseMaxFrames; ++i) {
+            ns[i] = i < p.chunk_frames ? f.new_slot[bl][i] : -1;
+            phs[i] = i < p.chunk_frames ? f.phase[bl][i] : 0;
+        }
+        if (paired) {
+            a0 = t0;
+            na = 1;
+            n_asm = 2;
+        } else {
+            if (t0 >= kv_begin && t0 < kv_end) a0 = t0;
+            if (t1 >= kv_begin && t1 < kv_end) (a0 < 0 ? a0 : a1) = t1;
+            na = (a0 >= 0) + (a1 >= 0);
+            n_asm = na;
+        }
+        if (n_asm > 0) {
+            const int e = a0 == t0 ? 0 : 1;
+            mf0 = f.grp_full[bl][e];
+            mp0 = f.grp_part[bl][e];
+        }
+        if (n_asm > 1) {
+            mf1 = paired ? mf0 : f.grp_full[bl][1];
+            mp1 = paired ? mp0 : f.grp_part[bl][1];
+        }
+    }
+    // KV tile of the i-th position of a head's sequence: the assembled tiles, then the rest
+    // of the range in order (the plain attention: the range in order)
+    auto tile_at = [&](int i) -> int {
+        if constexpr (!FUSE) {
+            return kv_begin + i;
+        } else {
+            if (i < na) return i == 0 ? a0 : a1;
+            int g = kv_begin + i - na;
+            if (a0 >= 0 && a0 <= g) ++g;
+            if (a1 >= 0 && a1 <= g) ++g;
+            return g;
+        }
+    };
 
     if (threadIdx.x == 0) {
         mbar_init(&bars[L::kQFull], 1);
@@ -404,6 +686,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_init(&bars[L::kOFull + t], 1);
         }
         mbar_init(&bars[L::kDrain], 1);
+        if constexpr (FUSE) {
+            mbar_init(&bars[L::kAsm], (kAttnThreads - 64) / 32);
+            mbar_init(&bars[L::kTabReady], 1);
+            *reinterpret_cast<int *>(smem + L::kMisc + 8) = 0;
+        }
         *abort_flag = 0u;
         fence_barrier_init();
     }
@@ -411,6 +698,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tma_prefetch_desc(&tmap_q);
         tma_prefetch_desc(&tmap_k);
         tma_prefetch_desc(&tmap_v);
+    }
+    if constexpr (FUSE) {
+        // the fused append's descriptors (cache and chunk K / V, four box heights each)
+        if (warp == 0 && lane < 4 * kFuseBoxes && n_asm > 0) {
+            const int i = lane % kFuseBoxes;
+            const CUtensorMap *m = lane < kFuseBoxes       ? &f.tmap_kc[i]
+                                   : lane < 2 * kFuseBoxes ? &f.tmap_vc[i]
+                                   : lane < 3 * kFuseBoxes ? &f.tmap_ki[i]
+                                                           : &f.tmap_vi[i];
+            tma_prefetch_desc(m);
+        }
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -425,6 +723,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // ---- queries: raw tiles by TMA, RoPE on load by the softmax warps.  Neither the
     // queries nor the cache's row / column tables are written by the kernels this launch
     // depends on (the KV append), so this overlaps them, before the dependency wait.
+    // The fused launch has no append before it: its inputs may come from the kernel just
+    // before, so it waits first.
+    if constexpr (FUSE) {
+        grid_dependency_wait();
+        grid_launch_dependents();
+    }
     if (warp == 0 && lane == 0 && n_local > 0) {
         mbar_arrive_expect_tx(&bars[L::kQFull], n_qt * L::kQRawTile);
         for (int t = 0; t < n_qt; ++t)
@@ -432,11 +736,75 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             for (int kb = 0; kb < D / 64; ++kb)
                 tma_load_4d(smem + L::kQRaw + t * L::kQRawTile + kb * L::kSub, &tmap_q, &bars[L::kQFull], kb * 64,
                             paired && t ? h_pair : h, q_row0 + (paired ? 0 : t * kBlockM), bg);
+        if constexpr (FUSE) {
+            if (n_asm > 0) {
+                // the fp64 tables of the keys the CTA rotates: the temporal (cos, sin) rows of the
+                // chunk's phases (T' n_t <= kFuseTabSmem entries), the cache's row and column tables
+                const uint32_t tb = static_cast<uint32_t>(p.n_t) * 16u;
+                const uint32_t hb = static_cast<uint32_t>(p.frame_h * p.n_h) * 16u;
+                const uint32_t wb = static_cast<uint32_t>(p.frame_w * p.n_w) * 16u;   // (checked on the host)
+                mbar_arrive_expect_tx(&bars[L::kTabReady], p.chunk_frames * tb + hb + wb);
+#pragma unroll
+                for (int i = 0; i < kFuseMaxFrames; ++i)
+                    if (i < p.chunk_frames)
+                        bulk_load(smem + L::kTab64 + i * tb, f.rope_t + static_cast<int64_t>(phs[i]) * p.n_t * 2, tb,
+                                  &bars[L::kTabReady]);
+                if (hb > 0) bulk_load(smem + L::kTabHW, f.rope_h, hb, &bars[L::kTabReady]);
+                if (wb > 0) bulk_load(smem + L::kTabHW + hb, f.rope_w, wb, &bars[L::kTabReady]);
+                // the assembled tiles (K and V stages 0 .. n_asm - 1): the cache's rows in the
+                // 8-row groups without the chunk's rows, the caller's rows in the full groups
+                // (the part groups are built by the CTA's warps)
+                const int N = p.tokens_per_frame;
+                // every K before any V: the keys are rotated, and the first products taken,
+                // before the values are needed
+                for (int u = 0; u < 2 * n_asm; ++u) {
+                    const bool is_v = u >= n_asm;
+                    const int i = is_v ? u - n_asm : u;
+                    const int hi = paired && i == 1 ? h_pair : h;
+                    const int ti = i == 0 || paired ? a0 : a1;
+                    const uint32_t mf = i ? mf1 : mf0, mp = i ? mp1 : mp0;
+                    const uint32_t old = ~(mf | mp) & 0xFFFFu;
+                    const uint32_t bytes = static_cast<uint32_t>(__popc(old) + __popc(mf)) * 8u * 128u * (D / 64);
+                    auto cache_row = [&](int q) { return ti * kBlockN + 8 * q; };
+                    auto chunk_token = [&](int q) {           // first row of a full group: its chunk token
+                        const int kr = ti * kBlockN + 8 * q, sl = kr / N;
+                        int fi = 0;
+#pragma unroll
+                        for (int e = 0; e < kFuseMaxFrames; ++e)
+                            if (ns[e] == sl) fi = e;
+                        return fi * N + (kr - sl * N);
+                    };
+                    uint8_t *tile = smem + (is_v ? L::kV : L::kK) + i * L::kKVTile;
+                    uint64_t *bar = &bars[(is_v ? L::kVFull : L::kKFull) + i];
+                    mbar_arrive_expect_tx(bar, bytes);
+                    move_row_groups<D, L>(tile, is_v ? f.tmap_vc : f.tmap_kc, bar, old, hi, bg, cache_row, false);
+                    move_row_groups<D, L>(tile, is_v ? f.tmap_vi : f.tmap_ki, bar, mf, hi, bg, chunk_token, false);
+                }
+            }
+        }
+    }
+    // Fused append: warps 2 and 3 start on the assembled tiles at once.
+    bool have_tab = false;
+    if constexpr (FUSE) {
+        if ((warp == 2 || warp == 3) && n_asm > 0) {
+            build_part_groups<D, L>(smem, bars, p, f, bg, lk, h, h_pair, paired, a0, paired ? a0 : a1, mp0, mp1, ns,
+                                    warp - 2, lane, abort_flag, have_tab);
+            rotate_full_groups<D, L>(smem, bars, p, a0, paired ? a0 : a1, mf0, mf1, ns, warp - 2, lane, abort_flag,
+                                     have_tab);
+            assembled<L>(bars, lane);
+        }
     }
     // RoPE on load by the softmax warps (idle until the first scores arrive): thread
     // (t, row) rotates its own query row (the single-tile mode: sub-tile t of tile 0's row)
     float q_row_scale = 0.0f;                   // fp8: E4M3 scale of this thread's query row
     if (warp >= 4 && n_local > 0) {
+        if constexpr (FUSE) {
+            // fused append: the straddling rows first (their loads in flight while the query
+            // tiles land); the full groups' keys after the query rotation
+            if (n_asm > 0)
+                build_part_groups<D, L>(smem, bars, p, f, bg, lk, h, h_pair, paired, a0, paired ? a0 : a1, mp0, mp1, ns,
+                                        warp - 2, lane, abort_flag, have_tab);
+        }
         const int t = (warp - 4) >> 2;
         const int row = ((warp & 3) << 5) + lane;
         const int qt = one_q ? 0 : t;           // query tile of this thread's row
@@ -452,7 +820,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const int fi = e / p.n_t, j = e - fi * p.n_t;
             const int64_t f = p.f0[bl] + fi_lo + fi;
             const int64_t ph = p.rope_reset > 0 ? f % p.rope_reset : f;
-            const double a = static_cast<double>(ph) * p.omega_t[j];
+            const double a = static_cast<double>(ph) * __ldg(p.omega_t + j);
             const double turns = rint(a * 0.15915494309189535);  // a / (2 pi), nearest integer
             const float r = static_cast<float>(fma(-turns, 6.283185307179586, a));
             float sn, cs;
@@ -516,21 +884,57 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         fence_proxy_async_shared();             // the tensor core reads these rows next
         mbar_arrive(&bars[L::kQReady]);
+        if constexpr (FUSE) {
+            if (n_asm > 0) {
+                rotate_full_groups<D, L>(smem, bars, p, a0, paired ? a0 : a1, mf0, mf1, ns, warp - 2, lane, abort_flag,
+                                         have_tab);
+                assembled<L>(bars, lane);
+            }
+        }
     }
 
     // Everything above overlaps the previous kernels (dependent launch); the cache and
     // the split partials are only touched below.
-    grid_dependency_wait();
-    grid_launch_dependents();
+    if constexpr (!FUSE) {
+        grid_dependency_wait();
+        grid_launch_dependents();
+    }
 
     if (warp < 4) {
       regs_dec<80>();
       if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0 && n_local > 0) {
-            // K tile `it` and V tile `it` are issued as soon as their own ring slot is free.
-            int k_issued = 0, v_issued = 0;
+            // K tile `it` and V tile `it` are issued as soon as their own ring slot is free
+            // (fused append: the first n_asm were issued with the queries).
+            int k_issued = n_asm, v_issued = n_asm;
             bool ok = true;
+            bool stores_reading = false;                 // fused append: TMA stores still reading stages < n_asm
+            bool stored = false;
+            if constexpr (FUSE) {
+                // nothing goes into V stage 2 (the key tables) before the assembled tiles are
+                // built; then the chunk's full groups, keys rotated in place, values as loaded
+                // (their stages' kVFull), go to their ring slots
+                if (n_asm > 0) ok = mbar_wait(&bars[L::kAsm], 0, abort_flag, p.status, kStatusTmaWait);
+                if (n_asm > 0 && (mf0 | mf1) != 0u) {
+                    for (int i = 0; ok && i < n_asm; ++i)
+                        ok = mbar_wait(&bars[L::kVFull + i], 0, abort_flag, p.status, kStatusTmaWait);
+                    if (ok) {
+                        for (int i = 0; i < n_asm; ++i) {
+                            const int hi = paired && i == 1 ? h_pair : h;
+                            const int ti = i == 0 || paired ? a0 : a1;
+                            const uint32_t mf = i ? mf1 : mf0;
+                            auto cache_row = [&](int q) { return ti * kBlockN + 8 * q; };
+                            move_row_groups<D, L>(smem + L::kK + i * L::kKVTile, f.tmap_kc, nullptr, mf, hi, bg,
+                                                  cache_row, true);
+                            move_row_groups<D, L>(smem + L::kV + i * L::kKVTile, f.tmap_vc, nullptr, mf, hi, bg,
+                                                  cache_row, true);
+                        }
+                        bulk_commit_group();
+                        stores_reading = stored = true;
+                    }
+                }
+            }
             while (ok && v_issued < n_local) {
                 if (k_issued < n_local && k_issued <= v_issued + 1) {
                     const int st = k_issued % L::kKStages;
@@ -539,15 +943,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&bars[L::kKFull + st], L::kKVTile);
+                    if (stores_reading && st < n_asm) {     // (the stage is an assembled tile's)
+                        bulk_wait_group_read0();
+                        stores_reading = false;
+                    }
                     if constexpr (F8) {
+                        mbar_arrive_expect_tx(&bars[L::kKFull + st], L::kKVTile);
                         const int g = kv_begin + k_issued, sl = g / p.n_blk;
                         tma_load_4d(smem + L::kK + st * L::kKVTile, &tmap_k, &bars[L::kKFull + st], 0, h,
                                     sl * p.np_tokens + (g - sl * p.n_blk) * kBlockN, bg);
                     } else {
                         // (pair mode: sequence tile i is tile i / 2 of head h or h_pair)
                         const int hk = paired && (k_issued & 1) ? h_pair : h;
-                        const int tk = paired ? k_issued >> 1 : kv_begin + k_issued;
+                        const int tk = paired ? tile_at(k_issued >> 1) : tile_at(k_issued);
+                        mbar_arrive_expect_tx(&bars[L::kKFull + st], L::kKVTile);
 #pragma unroll
                         for (int kb = 0; kb < D / 64; ++kb)
                             tma_load_4d(smem + L::kK + st * L::kKVTile + kb * L::kSub, &tmap_k, &bars[L::kKFull + st],
@@ -561,14 +970,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     ok = false;
                     break;
                 }
-                mbar_arrive_expect_tx(&bars[L::kVFull + st], L::kKVTile);
+                if (stores_reading && st < n_asm) {
+                    bulk_wait_group_read0();
+                    stores_reading = false;
+                }
                 if constexpr (F8) {
+                    mbar_arrive_expect_tx(&bars[L::kVFull + st], L::kKVTile);
                     const int g = kv_begin + v_issued, sl = g / p.n_blk;
                     tma_load_5d(smem + L::kV + st * L::kKVTile, &tmap_v, &bars[L::kVFull + st],
                                 (g - sl * p.n_blk) * kBlockN, 0, h, sl, bg);
                 } else {
                     const int hv = paired && (v_issued & 1) ? h_pair : h;
-                    const int tv = paired ? v_issued >> 1 : kv_begin + v_issued;
+                    const int tv = paired ? tile_at(v_issued >> 1) : tile_at(v_issued);
+                    mbar_arrive_expect_tx(&bars[L::kVFull + st], L::kKVTile);
 #pragma unroll
                     for (int kb = 0; kb < D / 64; ++kb)
                         tma_load_4d(smem + L::kV + st * L::kKVTile + kb * L::kSub, &tmap_v, &bars[L::kVFull + st],
@@ -589,7 +1003,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     while (!mbar_try_wait(&bars[L::kVFull + i % L::kVStages], (i / L::kVStages) & 1))
                         if (global_timer_ns() - t0 > kWaitLimitNs) break;
                 }
+                if constexpr (FUSE) {
+                    if (n_asm > 0)
+                        while (!mbar_try_wait(&bars[L::kTabReady], 0))
+                            if (global_timer_ns() - t0 > kWaitLimitNs) break;
+                }
             }
+            if (stored) bulk_wait_group0();              // the ring-slot writes are complete before the CTA ends
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
@@ -635,6 +1055,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
             };
             bool ok = mbar_wait(&bars[L::kQReady], 0, abort_flag, p.status, kStatusMmaWait);
+            if constexpr (FUSE) {
+                // the chunk's rows of the first n_asm tiles (their other rows come by TMA)
+                if (ok && n_asm > 0) ok = mbar_wait(&bars[L::kAsm], 0, abort_flag, p.status, kStatusMmaWait);
+            }
             if (alt) {
                 // KV tile i -> accumulator set i & 1.  Prologue: S_0 = Q K_0^T, S_1 = Q K_1^T.
                 for (int i = 0; ok && i < n_local && i < 2; ++i) {
@@ -758,19 +1182,36 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
                 sv_ref = fmaxf(sv_ref, 1e-30f);
             }
+            // bf16: the one iteration of this set whose KV tile is the valid prefix's ragged
+            // last tile (keys past lk masked), found once: the tile's position in the CTA's
+            // tile order (the inverse of tile_at), then the set's iteration of that position
+            int rag_it = -1;
+            const int rag_cols = lk - (n_kv - 1) * kBlockN;
+            if constexpr (!F8) {
+                const int gl = n_kv - 1;
+                int pos = -1;
+                if (rag_cols < kBlockN && gl >= kv_begin && gl < kv_end) {
+                    if (gl == a0)
+                        pos = 0;
+                    else if (gl == a1)
+                        pos = 1;
+                    else
+                        pos = gl - kv_begin + na - (a0 >= 0 && a0 < gl) - (a1 >= 0 && a1 < gl);
+                }
+                if (pos >= 0) rag_it = paired || !alt ? pos : ((pos & 1) == t ? pos >> 1 : -1);
+            }
             for (int it = 0; it < n_mine; ++it) {
-                // KV tile of this iteration (pair mode: tile `it` of this set's own head)
-                const int g = kv_begin + (paired ? it : (alt ? 2 * it + t : it));
                 float c_t = p.scale_log2, r_t = 1.0f;
                 int valid_cols;
                 if constexpr (F8) {
+                    const int g = kv_begin + (alt ? 2 * it + t : it);      // KV tile of this iteration
                     const int sl = g / p.n_blk;
                     const int64_t si = scale_base + sl * (p.scale_slot_stride - p.n_blk) + g;
                     c_t = fmaxf(p.scale_log2 * sq * p.k_scale[si], 1e-30f);
                     r_t = p.v_scale[si] / sv_ref;
                     valid_cols = p.tokens_per_frame - (g - sl * p.n_blk) * kBlockN;
                 } else {
-                    valid_cols = lk - g * kBlockN;
+                    valid_cols = it == rag_it ? rag_cols : kBlockN;
                 }
                 if (!warp_wait(&bars[L::kSFull + t], it & 1, abort_flag, p.status, kStatusSoftmaxWait)) {
                     ok = false;
@@ -1080,14 +1521,14 @@ cudaError_t launch_wait_selftest(uint32_t *status, uint64_t limit_ns, cudaStream
     return cudaGetLastError();
 }
 
-template <int D, bool F8>
-static cudaError_t launch_attention_d(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
+template <int D, bool F8, bool FUSE, typename FP>
+static cudaError_t launch_attention_d(const AttnParams &p, const FP &f, const CUtensorMap &tq, const CUtensorMap &tk,
                                       const CUtensorMap &tv, cudaStream_t s) {
     static bool configured = false;
-    const int smem = AttnLayout<D, F8>::kAlloc;
+    const int smem = AttnLayout<D, F8, FUSE>::kAlloc;
     if (!configured) {
-        cudaError_t e =
-            cudaFuncSetAttribute(chunk_attention_kernel<D, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        cudaError_t e = cudaFuncSetAttribute(chunk_attention_kernel<D, F8, FUSE>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         configured = true;
     }
@@ -1095,15 +1536,22 @@ static cudaError_t launch_attention_d(const AttnParams &p, const CUtensorMap &tq
     // pair mode: one CTA per (stream, pair of heads); otherwise whole units, then pieces
     dim3 grid(static_cast<unsigned>(p.pair ? p.n_units / p.heads * ((p.heads + 1) / 2)
                                            : p.n_whole + (p.n_units - p.n_whole) * p.n_pieces));
-    return launch_dependent(chunk_attention_kernel<D, F8>, grid, dim3(kAttnThreads), static_cast<size_t>(smem), s, p,
-                            tq, tk, tv);
+    return launch_dependent(chunk_attention_kernel<D, F8, FUSE>, grid, dim3(kAttnThreads), static_cast<size_t>(smem),
+                            s, p, tq, tk, tv, f);
 }
 
 cudaError_t launch_attention(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
                              const CUtensorMap &tv, int head_dim, cudaStream_t s) {
-    if (p.f8) return launch_attention_d<128, true>(p, tq, tk, tv, s);
-    if (head_dim == 64) return launch_attention_d<64, false>(p, tq, tk, tv, s);
-    return launch_attention_d<128, false>(p, tq, tk, tv, s);
+    const FuseNone none{0};
+    if (p.f8) return launch_attention_d<128, true, false>(p, none, tq, tk, tv, s);
+    if (head_dim == 64) return launch_attention_d<64, false, false>(p, none, tq, tk, tv, s);
+    return launch_attention_d<128, false, false>(p, none, tq, tk, tv, s);
+}
+
+cudaError_t launch_append_attention(const AttnParams &p, const FuseParams &f, const CUtensorMap &tq,
+                                    const CUtensorMap &tk, const CUtensorMap &tv, int head_dim, cudaStream_t s) {
+    if (head_dim == 64) return launch_attention_d<64, false, true>(p, f, tq, tk, tv, s);
+    return launch_attention_d<128, false, true>(p, f, tq, tk, tv, s);
 }
 
 cudaError_t launch_combine(const AttnParams &p, int head_dim, cudaStream_t s) {

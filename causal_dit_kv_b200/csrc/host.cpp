@@ -14,6 +14,7 @@
 #include <cstdio>
 #include <cstring>
 #include <atomic>
+#include <memory>
 #include <string>
 #include <vector>
 
@@ -81,6 +82,9 @@ struct Geometry {
     int64_t part_rows;  // capacity of the split-KV partial buffer, rows of d floats
     // region offsets
     uint64_t rope_h64, rope_w64, rope_h32, rope_w32;
+    uint64_t omega;          // [n_t] fp64 temporal frequencies (query rotation)
+    uint64_t rope_t64;       // [n_phase][n_t] fp64 (cos, sin) of the temporal pairs (fused append, bf16 cache)
+    int64_t n_phase;
     uint64_t sink_embed, sink_frame, status;
     uint64_t scratch, refresh_mean, refresh_counter, part_ml, part_o, scratch_end;
     uint64_t k, v, layer_stride, total;
@@ -174,6 +178,11 @@ Geometry geometry(const sdv2_cache_config &c) {
     off = align_up(off + 8ull * c.frame_h * c.rope_pairs[1], 256);
     g.rope_w32 = off;
     off = align_up(off + 8ull * c.frame_w * c.rope_pairs[2], 256);
+    g.omega = off;
+    off = align_up(off + 8ull * c.rope_pairs[0], 256);
+    g.n_phase = g.f8 ? 0 : std::min<int64_t>(c.rope_reset_period > 0 ? c.rope_reset_period : kFusePhaseCap, kFusePhaseCap);
+    g.rope_t64 = off;
+    off = align_up(off + 16ull * g.n_phase * c.rope_pairs[0], 256);
     g.sink_embed = off;
     off = align_up(off + 8ull * c.batch * c.sink_frames * (c.embed_dim > 0 ? c.embed_dim : 1), 256);
     g.sink_frame = off;
@@ -287,6 +296,7 @@ struct sdv2_cache {
     int sm_count;
     std::vector<int64_t> next_frame;  // [B][L]
     std::vector<CUtensorMap> tk, tv;  // [L]
+    std::vector<CUtensorMap> tkh, tvh;  // [L][kFuseBoxes] bf16 cache: the same maps in boxes of 64, 32, 16, 8 rows (fused append)
     cudaEvent_t time_start = nullptr;  // measurement hook: events around the attention kernel
     cudaEvent_t time_stop = nullptr;
 };
@@ -329,6 +339,258 @@ sdv2_status check_stream_frames(const sdv2_cache *c, int32_t layer, const int64_
         }
     }
     *active_out = active;
+    return SDV2_OK;
+}
+
+// KV tiles of one stream that hold rows of its chunk's own frames (ascending), for the
+// fused append: rows [slot * N, slot * N + N) of each chunk frame's ring slot, 128 keys
+// per tile.  Returns their number (it may exceed `cap`; only `cap` are stored).
+int chunk_tiles(const sdv2_cache_config &n, const Geometry &g, int64_t f0, int32_t *tiles, int cap) {
+    int cnt = 0;
+    for (int i = 0; i < n.chunk_frames; ++i) {
+        const int64_t sl = slot_of(f0 + i, n.sink_frames, n.window_frames);
+        for (int64_t t = sl * g.N / kBlockN; t <= (sl * g.N + g.N - 1) / kBlockN; ++t) {
+            bool seen = false;
+            for (int e = 0; e < std::min(cnt, cap); ++e) seen = seen || tiles[e] == t;
+            if (seen) continue;
+            if (cnt < cap) {
+                int e = cnt;                      // insertion keeps them ascending
+                while (e > 0 && tiles[e - 1] > t) {
+                    tiles[e] = tiles[e - 1];
+                    --e;
+                }
+                tiles[e] = static_cast<int32_t>(t);
+            }
+            ++cnt;
+        }
+    }
+    return cnt;
+}
+
+// The 8-row groups of KV tile t of one stream (lk valid keys, chunk frame i in ring slot
+// slots[i]) that hold rows of the chunk's own frames: *full gets the groups whose eight
+// rows are consecutive tokens of one chunk frame (the fused kernel moves them by TMA),
+// *part the others (built row by row).  Bit q: rows 8q .. 8q + 7 of the tile.
+void chunk_groups(const sdv2_cache_config &n, const Geometry &g, const int32_t *slots, int64_t lk, int64_t t,
+                  uint32_t *full, uint32_t *part) {
+    *full = *part = 0u;
+    for (int q = 0; q < kBlockN / 8; ++q) {
+        const int64_t kr0 = t * kBlockN + 8 * q;
+        bool any = false, whole = true;
+        for (int k = 0; k < 8; ++k) {
+            const int64_t kr = kr0 + k;
+            if (kr >= lk) {
+                whole = false;
+                continue;
+            }
+            const int64_t sl = kr / g.N;
+            bool is_new = false;
+            for (int i = 0; i < n.chunk_frames; ++i) is_new = is_new || slots[i] == sl;
+            any = any || is_new;
+            whole = whole && is_new && sl == kr0 / g.N;
+        }
+        if (any) *(whole ? full : part) |= 1u << q;
+    }
+}
+
+// Whether sdv2_append_attention runs the fused kernel for these chunk positions: bf16
+// cache, at most two query tiles per stream (one CTA, or its KV pieces, per stream and
+// head), at most kFuseMaxFrames chunk frames whose temporal tables fit the CTA's
+// kFuseTabSmem entries and whose phases lie in the cache's phase table, row and column
+// tables that fit fuse_tab_hw_bytes(head_dim), and at most
+// kFuseMaxAsmTiles KV tiles per stream holding the chunk's rows.  0: the append and the attention run as two launches; 1: fused;
+// 2: fused, pair mode (one tile per stream and more (stream, head) units than SMs).
+int fuse_mode(const sdv2_cache_config &n, const Geometry &g, const int64_t *f0, int sm_count) {
+    if (g.f8 || g.n_qpairs != 1 || n.chunk_frames > kFuseMaxFrames ||
+        n.chunk_frames * n.rope_pairs[0] > kFuseTabSmem ||
+        (static_cast<int64_t>(n.frame_h) * n.rope_pairs[1] + static_cast<int64_t>(n.frame_w) * n.rope_pairs[2]) * 16 >
+            fuse_tab_hw_bytes(n.head_dim))
+        return 0;
+    bool one_tile = true;
+    int64_t active = 0;
+    for (int b = 0; b < n.batch; ++b) {
+        if (f0[b] < 0) continue;
+        ++active;
+        for (int i = 0; i < n.chunk_frames; ++i)
+            if (phase_of(f0[b] + i, n.rope_reset_period) >= g.n_phase) return 0;   // beyond the cache's phase table
+        int32_t t[kFuseMaxAsmTiles];
+        const int cnt = chunk_tiles(n, g, f0[b], t, kFuseMaxAsmTiles);
+        if (cnt > kFuseMaxAsmTiles) return 0;
+        one_tile = one_tile && cnt == 1;
+    }
+    return one_tile && use_pair_mode(g, n, active * n.heads * g.n_qpairs, sm_count) ? 2 : 1;
+}
+
+// One attention call over the streams with chunk_first_frame >= 0 (the caller checked
+// the arguments and the stream positions).  With k and v given, the chunk's KV append
+// is fused in (fuse_mode != 0).
+sdv2_status run_attention(sdv2_cache *c, int32_t layer, const void *q, void *out, const int64_t *chunk_first_frame,
+                          float softmax_scale, cudaStream_t s, const void *k, const void *v) {
+    const sdv2_cache_config &n = c->cfg;
+    const Geometry &g = c->g;
+    const bool fuse = k != nullptr;
+    std::vector<int64_t> keys(n.batch, 0);
+    for (int b = 0; b < n.batch; ++b) {
+        if (chunk_first_frame[b] < 0) continue;
+        int32_t sv, wv;
+        valid_counts(chunk_first_frame[b] + n.chunk_frames, n.sink_frames, n.window_frames, &sv, &wv);
+        keys[b] = static_cast<int64_t>(sv + wv) * g.N;
+    }
+    const int n_t = n.rope_pairs[0];
+    // The caller's un-rotated queries as a TMA tensor (d, H, Lq, B), bf16, in boxes of 64
+    // channels x 128 rows with the 128-byte swizzle of the MMA's Q tiles; the kernel rotates
+    // them on load.  Encoded per call: q is the caller's buffer.
+    CUtensorMap tq;
+    {
+        PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode_fn();
+        if (!encode) return fail(SDV2_E_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+        const cuuint64_t qdims[4] = {static_cast<cuuint64_t>(n.head_dim), static_cast<cuuint64_t>(n.heads),
+                                     static_cast<cuuint64_t>(g.lq), static_cast<cuuint64_t>(n.batch)};
+        const cuuint64_t qstrides[3] = {static_cast<cuuint64_t>(n.head_dim) * 2,
+                                        static_cast<cuuint64_t>(n.heads) * n.head_dim * 2,
+                                        static_cast<cuuint64_t>(g.lq) * n.heads * n.head_dim * 2};
+        const cuuint32_t qbox[4] = {64u, 1, static_cast<cuuint32_t>(kBlockM), 1};
+        const cuuint32_t estr[4] = {1, 1, 1, 1};
+        CUresult r = encode(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(q), qdims, qstrides, qbox,
+                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return fail(SDV2_E_CUDA, "cuTensorMapEncodeTiled (queries) failed (%d)", static_cast<int>(r));
+    }
+    AttnParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.out = static_cast<uint16_t *>(out);
+    p.part_o = reinterpret_cast<float *>(c->base + g.part_o);
+    p.part_ml = reinterpret_cast<float *>(c->base + g.part_ml);
+    p.rope_h = reinterpret_cast<const float *>(c->base + g.rope_h32);
+    p.rope_w = reinterpret_cast<const float *>(c->base + g.rope_w32);
+    p.status = reinterpret_cast<uint32_t *>(c->base + g.status);
+    p.batch = n.batch;
+    p.heads = n.heads;
+    p.lq = static_cast<int32_t>(g.lq);
+    p.tokens_per_frame = static_cast<int32_t>(g.N);
+    p.frame_h = n.frame_h;
+    p.frame_w = n.frame_w;
+    p.chunk_frames = n.chunk_frames;
+    p.n_t = n_t;
+    p.n_h = n.rope_pairs[1];
+    p.n_w = n.rope_pairs[2];
+    p.n_qpairs = g.n_qpairs;
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.omega_t = reinterpret_cast<const double *>(c->base + g.omega);
+    p.rope_reset = n.rope_reset_period;
+    if (g.f8) {
+        p.k_scale = reinterpret_cast<const float *>(c->base + g.k_scale + g.scale_layer_stride * layer);
+        p.v_scale = reinterpret_cast<const float *>(c->base + g.v_scale + g.scale_layer_stride * layer);
+        p.f8 = 1;
+        p.slots = static_cast<int32_t>(g.slots);
+        p.np_tokens = static_cast<int32_t>(g.np_tokens);
+        p.n_blk = g.n_blk;
+        p.scale_slot_stride = g.scale_slot_stride;
+    }
+    std::unique_ptr<FuseParams> fp;
+    if (fuse) {
+        fp.reset(new FuseParams());
+        std::memset(fp.get(), 0, sizeof(FuseParams));
+        fp->k_in = static_cast<const uint16_t *>(k);
+        fp->v_in = static_cast<const uint16_t *>(v);
+        fp->k_layer = reinterpret_cast<uint16_t *>(c->base + g.k + g.layer_stride * layer);
+        fp->v_layer = reinterpret_cast<uint16_t *>(c->base + g.v + g.layer_stride * layer);
+        fp->rope_h = reinterpret_cast<const double *>(c->base + g.rope_h64);
+        fp->rope_w = reinterpret_cast<const double *>(c->base + g.rope_w64);
+        fp->rope_t = reinterpret_cast<const double *>(c->base + g.rope_t64);
+        fp->slots = static_cast<int32_t>(g.slots);
+        for (int i = 0; i < kFuseBoxes; ++i) {
+            fp->tmap_kc[i] = c->tkh[static_cast<size_t>(layer) * kFuseBoxes + i];
+            fp->tmap_vc[i] = c->tvh[static_cast<size_t>(layer) * kFuseBoxes + i];
+        }
+        // the caller's k and v as TMA tensors (d, H, T'N, B), bf16, boxes of 64 channels x
+        // (64 >> i) rows, 128-byte swizzle (the tiles' layout); encoded per call: k and v are
+        // the caller's
+        PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode_fn();
+        const cuuint64_t dims[4] = {static_cast<cuuint64_t>(n.head_dim), static_cast<cuuint64_t>(n.heads),
+                                    static_cast<cuuint64_t>(g.lq), static_cast<cuuint64_t>(n.batch)};
+        const cuuint64_t strides[3] = {static_cast<cuuint64_t>(n.head_dim) * 2,
+                                       static_cast<cuuint64_t>(n.heads) * n.head_dim * 2,
+                                       static_cast<cuuint64_t>(g.lq) * n.heads * n.head_dim * 2};
+        const cuuint32_t estr[4] = {1, 1, 1, 1};
+        for (int kv = 0; kv < 2; ++kv)
+            for (int i = 0; i < kFuseBoxes; ++i) {
+                const cuuint32_t box[4] = {64u, 1, static_cast<cuuint32_t>(64 >> i), 1};
+                CUresult r = encode(kv ? &fp->tmap_vi[i] : &fp->tmap_ki[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                                    const_cast<void *>(kv ? v : k), dims, strides, box, estr,
+                                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                if (r != CUDA_SUCCESS)
+                    return fail(SDV2_E_CUDA, "cuTensorMapEncodeTiled (chunk k / v) failed (%d)", static_cast<int>(r));
+            }
+    }
+    for (int b0 = 0; b0 < n.batch; b0 += kMaxBatch) {
+        const int nb = std::min(kMaxBatch, n.batch - b0);     // the launch's streams: b0 .. b0 + nb - 1
+        if (fuse)
+            for (int bl = 0; bl < nb; ++bl) {
+                const int64_t f0 = chunk_first_frame[b0 + bl];
+                if (f0 < 0) continue;
+                for (int i = 0; i < n.chunk_frames; ++i) {
+                    fp->new_slot[bl][i] = slot_of(f0 + i, n.sink_frames, n.window_frames);
+                    fp->phase[bl][i] = static_cast<int32_t>(phase_of(f0 + i, n.rope_reset_period));
+                }
+                int32_t t[kFuseMaxAsmTiles] = {-1, -1};
+                chunk_tiles(n, g, f0, t, kFuseMaxAsmTiles);
+                for (int e = 0; e < kFuseMaxAsmTiles; ++e) {
+                    fp->asm_tile[bl][e] = t[e];
+                    fp->grp_full[bl][e] = fp->grp_part[bl][e] = 0u;
+                    if (t[e] >= 0)
+                        chunk_groups(n, g, fp->new_slot[bl], keys[b0 + bl], t[e], &fp->grp_full[bl][e],
+                                     &fp->grp_part[bl][e]);
+                }
+            }
+        p.b_offset = b0;
+        bool any = false, one_tile = true;
+        int n_active = 0;
+        for (int bl = 0; bl < kMaxBatch; ++bl) p.lk[bl] = 0;
+        for (int bl = 0; bl < nb; ++bl) {
+            const int b = b0 + bl;
+            p.lk[bl] = static_cast<int32_t>(keys[b]);
+            p.f0[bl] = chunk_first_frame[b];
+            if (keys[b] > 0) {
+                any = true;
+                p.unit_stream[n_active++] = static_cast<uint8_t>(bl);
+                if (fuse) one_tile = one_tile && fp->asm_tile[bl][1] < 0;
+            }
+        }
+        if (!any) continue;
+        p.n_units = n_active * n.heads * g.n_qpairs;
+        // (the fused pair mode takes the one assembled tile of each stream for both heads)
+        if (use_pair_mode(g, n, p.n_units, c->sm_count) && (!fuse || one_tile)) {
+            p.pair = 1;
+            p.n_whole = p.n_units;
+            p.n_pieces = 1;
+        } else {
+            p.pair = 0;
+            const AttnPlan plan =
+                plan_attention(n, g, p.n_units, max_kv_tiles(g, keys.data() + b0, nb), c->sm_count);
+            p.n_whole = static_cast<int32_t>(plan.whole);
+            p.n_pieces = plan.pieces;
+        }
+        cudaError_t e = cudaSuccess;
+        if (c->time_start && b0 == 0) {
+            e = cudaEventRecord(c->time_start, s);
+            if (e != cudaSuccess) return cuda_fail(e, "chunk_attention start event");
+        }
+        e = fuse ? launch_append_attention(p, *fp, tq, c->tk[layer], c->tv[layer], n.head_dim, s)
+                 : launch_attention(p, tq, c->tk[layer], c->tv[layer], n.head_dim, s);
+        if (e != cudaSuccess) return cuda_fail(e, fuse ? "append_attention launch" : "chunk_attention launch");
+        if (c->time_stop && b0 + kMaxBatch >= n.batch) {
+            e = cudaEventRecord(c->time_stop, s);
+            if (e != cudaSuccess) return cuda_fail(e, "chunk_attention stop event");
+        }
+        g_launches.fetch_add(1);
+        if (p.n_whole < p.n_units) {
+            e = launch_combine(p, n.head_dim, s);
+            if (e != cudaSuccess) return cuda_fail(e, "attention combine launch");
+            g_launches.fetch_add(1);
+        }
+    }
     return SDV2_OK;
 }
 
@@ -424,9 +686,22 @@ sdv2_status sdv2_cache_create(const sdv2_cache_config *cfg, void *dev_buf, size_
                 w32[2 * (static_cast<size_t>(j) * n.frame_w + col) + k] =
                     static_cast<float>(w64[2 * (col * nw + j) + k]);
     std::vector<int64_t> sink_frames(static_cast<size_t>(n.batch) * n.sink_frames, -1);
+    // temporal frequencies (the queries' angles are formed on the device), and the fp64
+    // (cos, sin) of every temporal pair at phases 0 .. n_phase - 1 (the fused append
+    // rotates keys with these, the same values the append's per-call table carries)
+    const int nt = n.rope_pairs[0];
+    std::vector<double> omega(nt), t64(2ull * g.n_phase * nt);
+    for (int j = 0; j < nt; ++j) omega[j] = rope_angle(n.rope_base, j, nt, 1);
+    for (int64_t ph = 0; ph < g.n_phase; ++ph)
+        for (int j = 0; j < nt; ++j) {
+            const double a = rope_angle(n.rope_base, j, nt, ph);
+            t64[2 * (ph * nt + j)] = std::cos(a);
+            t64[2 * (ph * nt + j) + 1] = std::sin(a);
+        }
     struct Up { uint64_t off; const void *src; size_t bytes; } ups[] = {
         {g.rope_h64, h64.data(), h64.size() * 8}, {g.rope_w64, w64.data(), w64.size() * 8},
         {g.rope_h32, h32.data(), h32.size() * 4}, {g.rope_w32, w32.data(), w32.size() * 4},
+        {g.omega, omega.data(), omega.size() * 8}, {g.rope_t64, t64.data(), t64.size() * 8},
         {g.sink_frame, sink_frames.data(), sink_frames.size() * 8}};
     for (const Up &u : ups) {
         if (u.bytes == 0) continue;
@@ -441,6 +716,8 @@ sdv2_status sdv2_cache_create(const sdv2_cache_config *cfg, void *dev_buf, size_
     // (Np, d, H, slots, B), boxes of 128 bytes x 128 rows.
     c->tk.resize(n.layers);
     c->tv.resize(n.layers);
+    c->tkh.resize(g.f8 ? 0 : static_cast<size_t>(n.layers) * kFuseBoxes);
+    c->tvh.resize(g.f8 ? 0 : static_cast<size_t>(n.layers) * kFuseBoxes);
     const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     for (int l = 0; l < n.layers; ++l) {
         for (int kv = 0; kv < 2; ++kv) {
@@ -456,6 +733,13 @@ sdv2_status sdv2_cache_create(const sdv2_cache_config *cfg, void *dev_buf, size_
                 r = encode(kv ? &c->tv[l] : &c->tk[l], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, ptr, dims, strides, box,
                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                for (int i = 0; r == CUDA_SUCCESS && i < kFuseBoxes; ++i) {
+                    const cuuint32_t boxh[4] = {64, 1, static_cast<cuuint32_t>(64 >> i), 1};
+                    CUtensorMap *m = &(kv ? c->tvh : c->tkh)[static_cast<size_t>(l) * kFuseBoxes + i];
+                    r = encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, ptr, dims, strides, boxh, estr,
+                               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                }
             } else if (kv == 0) {
                 const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(n.heads),
                                             static_cast<cuuint64_t>(g.slots * g.np_tokens),
@@ -594,113 +878,32 @@ sdv2_status sdv2_chunk_attention(sdv2_cache *c, int32_t layer, const void *q, vo
     if (st != SDV2_OK) return st;
     if ((st = check_device(c->device)) != SDV2_OK) return st;
     if (active == 0) return SDV2_OK;
-    const sdv2_cache_config &n = c->cfg;
-    const Geometry &g = c->g;
-    std::vector<int64_t> keys(n.batch, 0);
-    for (int b = 0; b < n.batch; ++b) {
-        if (chunk_first_frame[b] < 0) continue;
-        int32_t sv, wv;
-        valid_counts(chunk_first_frame[b] + n.chunk_frames, n.sink_frames, n.window_frames, &sv, &wv);
-        keys[b] = static_cast<int64_t>(sv + wv) * g.N;
+    return run_attention(c, layer, q, out, chunk_first_frame, softmax_scale, reinterpret_cast<cudaStream_t>(stream),
+                         nullptr, nullptr);
+}
+
+sdv2_status sdv2_append_attention(sdv2_cache *c, int32_t layer, const void *q, const void *k, const void *v,
+                                  void *out, const int64_t *chunk_first_frame, float softmax_scale,
+                                  sdv2_stream stream) {
+    if (!c || !q || !k || !v || !out) return fail(SDV2_E_ARG, "NULL argument");
+    if (layer < 0 || layer >= c->cfg.layers) return fail(SDV2_E_ARG, "layer %d out of range", layer);
+    if (!(softmax_scale > 0.0f) || !std::isfinite(softmax_scale)) return fail(SDV2_E_ARG, "softmax_scale must be > 0");
+    if (!aligned16(q) || !aligned16(out) || !aligned16(k) || !aligned16(v))
+        return fail(SDV2_E_ALIGN, "q, k, v and out must be 16-byte aligned");
+    int active = 0;
+    sdv2_status st = check_stream_frames(c, layer, chunk_first_frame, false, &active);
+    if (st != SDV2_OK) return st;
+    if ((st = check_device(c->device)) != SDV2_OK) return st;
+    if (active == 0) return SDV2_OK;
+    if (fuse_mode(c->cfg, c->g, chunk_first_frame, c->sm_count) == 0) {
+        // not covered by the fused kernel: the append, then the attention (same results)
+        if ((st = sdv2_kv_append(c, layer, k, v, chunk_first_frame, stream)) != SDV2_OK) return st;
+        return sdv2_chunk_attention(c, layer, q, out, chunk_first_frame, softmax_scale, stream);
     }
-    const int n_t = n.rope_pairs[0];
-    const int streams_per_launch = kMaxBatch;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // The caller's un-rotated queries as a TMA tensor (d, H, Lq, B), bf16, in boxes of 64
-    // channels x 128 rows with the 128-byte swizzle of the MMA's Q tiles; the kernel rotates
-    // them on load.  Encoded per call: q is the caller's buffer.
-    CUtensorMap tq;
-    {
-        PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode_fn();
-        if (!encode) return fail(SDV2_E_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-        const cuuint64_t qdims[4] = {static_cast<cuuint64_t>(n.head_dim), static_cast<cuuint64_t>(n.heads),
-                                     static_cast<cuuint64_t>(g.lq), static_cast<cuuint64_t>(n.batch)};
-        const cuuint64_t qstrides[3] = {static_cast<cuuint64_t>(n.head_dim) * 2,
-                                        static_cast<cuuint64_t>(n.heads) * n.head_dim * 2,
-                                        static_cast<cuuint64_t>(g.lq) * n.heads * n.head_dim * 2};
-        const cuuint32_t qbox[4] = {64u, 1, static_cast<cuuint32_t>(kBlockM), 1};
-        const cuuint32_t estr[4] = {1, 1, 1, 1};
-        CUresult r = encode(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(q), qdims, qstrides, qbox,
-                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) return fail(SDV2_E_CUDA, "cuTensorMapEncodeTiled (queries) failed (%d)", static_cast<int>(r));
-    }
-    AttnParams p;
-    std::memset(&p, 0, sizeof(p));
-    p.out = static_cast<uint16_t *>(out);
-    p.part_o = reinterpret_cast<float *>(c->base + g.part_o);
-    p.part_ml = reinterpret_cast<float *>(c->base + g.part_ml);
-    p.rope_h = reinterpret_cast<const float *>(c->base + g.rope_h32);
-    p.rope_w = reinterpret_cast<const float *>(c->base + g.rope_w32);
-    p.status = reinterpret_cast<uint32_t *>(c->base + g.status);
-    p.batch = n.batch;
-    p.heads = n.heads;
-    p.lq = static_cast<int32_t>(g.lq);
-    p.tokens_per_frame = static_cast<int32_t>(g.N);
-    p.frame_h = n.frame_h;
-    p.frame_w = n.frame_w;
-    p.chunk_frames = n.chunk_frames;
-    p.n_t = n_t;
-    p.n_h = n.rope_pairs[1];
-    p.n_w = n.rope_pairs[2];
-    p.n_qpairs = g.n_qpairs;
-    p.scale_log2 = softmax_scale * 1.4426950408889634f;
-    for (int j = 0; j < n_t; ++j) p.omega_t[j] = rope_angle(n.rope_base, j, n_t, 1);
-    p.rope_reset = n.rope_reset_period;
-    if (g.f8) {
-        p.k_scale = reinterpret_cast<const float *>(c->base + g.k_scale + g.scale_layer_stride * layer);
-        p.v_scale = reinterpret_cast<const float *>(c->base + g.v_scale + g.scale_layer_stride * layer);
-        p.f8 = 1;
-        p.slots = static_cast<int32_t>(g.slots);
-        p.np_tokens = static_cast<int32_t>(g.np_tokens);
-        p.n_blk = g.n_blk;
-        p.scale_slot_stride = g.scale_slot_stride;
-    }
-    for (int b0 = 0; b0 < n.batch; b0 += streams_per_launch) {
-        const int nb = std::min(streams_per_launch, n.batch - b0);
-        p.b_offset = b0;
-        bool any = false;
-        int n_active = 0;
-        for (int bl = 0; bl < kMaxBatch; ++bl) p.lk[bl] = 0;
-        for (int bl = 0; bl < nb; ++bl) {
-            const int b = b0 + bl;
-            p.lk[bl] = static_cast<int32_t>(keys[b]);
-            p.f0[bl] = chunk_first_frame[b];
-            if (keys[b] > 0) {
-                any = true;
-                p.unit_stream[n_active++] = static_cast<uint8_t>(bl);
-            }
-        }
-        if (!any) continue;
-        p.n_units = n_active * n.heads * g.n_qpairs;
-        if (use_pair_mode(g, n, p.n_units, c->sm_count)) {
-            p.pair = 1;
-            p.n_whole = p.n_units;
-            p.n_pieces = 1;
-        } else {
-            p.pair = 0;
-            const AttnPlan plan = plan_attention(n, g, p.n_units, max_kv_tiles(g, keys.data() + b0, nb), c->sm_count);
-            p.n_whole = static_cast<int32_t>(plan.whole);
-            p.n_pieces = plan.pieces;
-        }
-        cudaError_t e = cudaSuccess;
-        if (c->time_start && b0 == 0) {
-            e = cudaEventRecord(c->time_start, s);
-            if (e != cudaSuccess) return cuda_fail(e, "chunk_attention start event");
-        }
-        e = launch_attention(p, tq, c->tk[layer], c->tv[layer], n.head_dim, s);
-        if (e != cudaSuccess) return cuda_fail(e, "chunk_attention launch");
-        if (c->time_stop && b0 + streams_per_launch >= n.batch) {
-            e = cudaEventRecord(c->time_stop, s);
-            if (e != cudaSuccess) return cuda_fail(e, "chunk_attention stop event");
-        }
-        g_launches.fetch_add(1);
-        if (p.n_whole < p.n_units) {
-            e = launch_combine(p, n.head_dim, s);
-            if (e != cudaSuccess) return cuda_fail(e, "attention combine launch");
-            g_launches.fetch_add(1);
-        }
-    }
+    st = run_attention(c, layer, q, out, chunk_first_frame, softmax_scale, reinterpret_cast<cudaStream_t>(stream), k, v);
+    if (st != SDV2_OK) return st;
+    for (int b = 0; b < c->cfg.batch; ++b)
+        if (chunk_first_frame[b] >= 0) c->next_frame[static_cast<size_t>(b) * c->cfg.layers + layer] += c->cfg.chunk_frames;
     return SDV2_OK;
 }
 
@@ -1035,6 +1238,12 @@ int32_t sdv2_attention_pair_mode(const sdv2_cache_config *cfg, const int64_t *ke
     for (int b = 0; b < std::min(n.batch, kMaxBatch); ++b)
         if (keys[b] > 0) ++active;
     return use_pair_mode(g, n, active * n.heads * g.n_qpairs, sm_count) ? 1 : 0;
+}
+
+int32_t sdv2_append_attention_mode(const sdv2_cache_config *cfg, const int64_t *chunk_first_frame, int32_t sm_count) {
+    sdv2_cache_config n;
+    if (check_config(cfg, &n) != SDV2_OK || !chunk_first_frame) return -1;
+    return fuse_mode(n, geometry(n), chunk_first_frame, sm_count);
 }
 
 int32_t sdv2_attention_splits(const sdv2_cache_config *cfg, const int64_t *keys, int32_t sm_count) {

@@ -106,6 +106,32 @@ __device__ __forceinline__ void tma_load_5d(void *smem_dst, const CUtensorMap *m
         : "memory");
 }
 
+// 4-D tile store shared -> global (bulk-group completion).  The shared-memory source
+// was written by the generic proxy: the writers fence it (fence_proxy_async_shared)
+// before the issuing thread learns of them.  Coordinates must not be negative.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, const void *smem_src, int c0, int c1, int c2,
+                                             int c3) {
+    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_addr(smem_src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until the committed bulk stores have read their shared-memory sources.
+__device__ __forceinline__ void bulk_wait_group_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Wait until the committed bulk stores are complete.
+__device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Untiled bulk copy global -> shared of `bytes` bytes, completion counted in bytes on
+// `bar`.  Both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void *smem_dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
@@ -362,5 +388,43 @@ __device__ __forceinline__ void e4m3_scale_inv(float amax, float &scale, float &
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// ---- key rotation (the cache's rounding rule, shared by the append and the fused
+// append + attention kernel): each pair is rotated in fp64 with separately rounded
+// products and sums (no FMA) and rounded once to bf16, nearest even.
+__device__ __forceinline__ uint16_t bf16_from_f64_rn(double x) {
+    uint16_t r;
+    asm("cvt.rn.bf16.f64 %0, %1;" : "=h"(r) : "d"(x));
+    return r;
+}
+
+__device__ __forceinline__ double bf16_to_f64(uint32_t bits16) {
+    return static_cast<double>(__uint_as_float(bits16 << 16));
+}
+
+// Rotate one packed pair (lo = dim 2j, hi = dim 2j+1) by (c, s).
+__device__ __forceinline__ uint32_t rotate_pair(uint32_t w, double c, double s) {
+    const double x0 = bf16_to_f64(w & 0xFFFFu);
+    const double x1 = bf16_to_f64(w >> 16);
+    const double r0 = __dsub_rn(__dmul_rn(x0, c), __dmul_rn(x1, s));
+    const double r1 = __dadd_rn(__dmul_rn(x0, s), __dmul_rn(x1, c));
+    return static_cast<uint32_t>(bf16_from_f64_rn(r0)) | (static_cast<uint32_t>(bf16_from_f64_rn(r1)) << 16);
+}
+
+// 4-byte load that bypasses L1 allocation (data read once).
+__device__ __forceinline__ uint32_t ld_nc_u32(const uint32_t *p) {
+    uint32_t r;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(r) : "l"(p));
+    return r;
+}
+
+// 16-byte load that bypasses L1 allocation (data read once).
+__device__ __forceinline__ uint4 ld_nc_v4(const uint16_t *p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
 
 }  // namespace sdv2

@@ -75,7 +75,7 @@ struct AttnParams {
     uint8_t unit_stream[kMaxBatch];
     float scale_log2;           // softmax_scale * log2(e)
     int32_t lk[kMaxBatch];      // valid keys per stream of this launch (0 = skip)
-    double omega_t[64];         // temporal frequencies base^(-j / n_t), fp64 (host-computed)
+    const double *omega_t;      // [n_t] temporal frequencies base^(-j / n_t), fp64 (in the cache buffer)
     int32_t rope_reset;         // temporal phase period (0: none)
     int64_t f0[kMaxBatch];      // first frame of each stream's chunk
     // fp8 (E4M3) cache only: KV tiles are 128-token blocks of one slot (slot s, block j at
@@ -85,6 +85,54 @@ struct AttnParams {
     const float *v_scale;
     int32_t slots, np_tokens, n_blk, scale_slot_stride;
     int32_t f8;                 // 1: fp8 cache (E4M3 queries, keys, values and probabilities)
+};
+
+// Append fused into the attention (bf16 cache, chunks of at most two query tiles):
+// the CTA that reads a KV tile holding rows of the chunk's own frames brings those rows
+// from the caller's k / v into the tile instead (by TMA, or row by row where an 8-row
+// group straddles slots), rotates the keys there by the append's rule and writes the
+// rows to their ring slots (by TMA); the tile's other rows come from the cache.  Such
+// "assembled" tiles go first in each CTA's tile order; every other tile comes by TMA as
+// in the plain attention.
+constexpr int kFuseMaxFrames = 4;          // chunk frames, at most
+constexpr int kFuseMaxAsmTiles = 2;        // assembled KV tiles of one stream, at most
+constexpr int kFuseTabSmem = 48;           // fp64 temporal (cos, sin) entries a CTA keeps: T' * n_t, at most
+// fp64 row and column tables a CTA keeps, (frame_h n_h + frame_w n_w) 16 B, at most: one
+// KV tile's shared memory (128 x head_dim bf16) less 1 KB for the temporal entries
+constexpr int fuse_tab_hw_bytes(int head_dim) { return 256 * head_dim - 1024; }
+constexpr int kFusePhaseCap = 4096;        // temporal phases in the cache's fp64 (cos, sin) table for the fused append
+
+constexpr int kFuseBoxes = 4;              // TMA box heights of the fused append: 64, 32, 16, 8 rows
+
+struct FuseParams {
+    // this layer's K and V, and the caller's k and v as (d, H, T'N, B), as tensor maps in
+    // boxes of 64 channels x (64 >> i) rows: runs of whole 8-row groups of an assembled tile
+    // move by TMA in a few boxes each
+    CUtensorMap tmap_kc[kFuseBoxes];
+    CUtensorMap tmap_vc[kFuseBoxes];
+    CUtensorMap tmap_ki[kFuseBoxes];
+    CUtensorMap tmap_vi[kFuseBoxes];
+    const uint16_t *k_in;       // [B][T'N][H][d] (caller's, un-rotated)
+    const uint16_t *v_in;
+    uint16_t *k_layer;          // [B][slots][N][H][d] of this layer
+    uint16_t *v_layer;
+    const double *rope_h;       // [frame_h][n_h][2] fp64 (cos, sin)
+    const double *rope_w;       // [frame_w][n_w][2]
+    const double *rope_t;       // [phase][n_t][2] fp64 (cos, sin) of the temporal pairs (phases < kFusePhaseCap)
+    int32_t slots;
+    int32_t new_slot[kMaxBatch][kFuseMaxFrames];       // ring slot of chunk frame i of each stream
+    int32_t phase[kMaxBatch][kFuseMaxFrames];          // temporal phase of chunk frame i of each stream
+    int32_t asm_tile[kMaxBatch][kFuseMaxAsmTiles];     // KV tiles holding the chunk's rows (-1: none), ascending
+    // 8-row groups of those tiles (bit q: rows 8q .. 8q + 7) that hold the chunk's rows:
+    // full = all eight are consecutive tokens of one chunk frame (TMA in, keys rotated in
+    // place, TMA out); part = the others (built row by row)
+    uint32_t grp_full[kMaxBatch][kFuseMaxAsmTiles];
+    uint32_t grp_part[kMaxBatch][kFuseMaxAsmTiles];
+};
+
+// The non-fused attention instantiations take this in place of FuseParams.
+struct FuseNone {
+    int32_t unused;
 };
 
 struct RefreshParams {
@@ -156,6 +204,9 @@ cudaError_t launch_combine(const AttnParams &p, int head_dim, cudaStream_t s);
 // (d, H, Lq, B) in boxes of 64 channels x 128 rows, 128-byte swizzle.
 cudaError_t launch_attention(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
                              const CUtensorMap &tv, int head_dim, cudaStream_t s);
+// The same launch with the chunk's KV append fused in (bf16 cache, FuseParams above).
+cudaError_t launch_append_attention(const AttnParams &p, const FuseParams &f, const CUtensorMap &tq,
+                                    const CUtensorMap &tk, const CUtensorMap &tv, int head_dim, cudaStream_t s);
 cudaError_t launch_refresh(const RefreshParams &p, int sm_count, cudaStream_t s, int *launches);
 cudaError_t launch_motion(const MotionParams &p, cudaStream_t s);
 // Same kernel with partial/counter in the library's static device array.

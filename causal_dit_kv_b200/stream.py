@@ -50,6 +50,14 @@ class KVCache:
         scale = 1.0 / math.sqrt(self.head_dim) if softmax_scale is None else softmax_scale
         B.sdv2_chunk_attention(self.handle, layer, q, out, chunk_first_frame, scale, self.batch, stream)
 
+    def append_attention(self, layer, q, k, v, out, chunk_first_frame, softmax_scale=None, stream=None):
+        """kv_append then chunk_attention of the same chunk, fused into one launch where it applies."""
+        scale = 1.0 / math.sqrt(self.head_dim) if softmax_scale is None else softmax_scale
+        B.sdv2_append_attention(self.handle, layer, q, k, v, out, chunk_first_frame, scale, self.batch, stream)
+
+    def append_attention_mode(self, chunk_first_frame, sm_count):
+        return B.sdv2_append_attention_mode(self.cfg, chunk_first_frame, sm_count)
+
     def time_attention(self, start=None, stop=None):
         """Record torch.cuda.Event start/stop (enable_timing=True, already recorded once so
         that they exist) around the attention kernel of the following chunk_attention

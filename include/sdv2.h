@@ -4,6 +4,7 @@
  *
  * The path, one latent chunk of T' frames per stream per step:
  *   for every DiT layer l:  sdv2_kv_append(l)  then  sdv2_chunk_attention(l)
+ *                           (or both at once: sdv2_append_attention(l))
  *   once per step:          sdv2_sink_refresh, sdv2_motion_noise_rate
  *
  * Sources (page title, section):
@@ -190,6 +191,34 @@ sdv2_status sdv2_chunk_attention(sdv2_cache *cache, int32_t layer, const void *q
                                  const int64_t *chunk_first_frame, float softmax_scale,
                                  sdv2_stream stream);
 
+/* The KV append fused into the chunk attention: the same results as
+ * sdv2_kv_append(layer, k, v) followed by sdv2_chunk_attention(layer, q, out)
+ * (the cache bit for bit; out within the attention's fp32 accumulation, the
+ * keys being taken in another order), in one launch where it applies.
+ * [A] "深入分析" (each chunk loads the long KV cache but computes only on
+ * the current input: the chunk's own K/V should not make a second trip),
+ * [Q] "Adaptive sink and RoPE refresh".
+ * q, k, v: device bf16 [B][T'*N][H][d] as for the two calls; out as for
+ *      sdv2_chunk_attention.  chunk_first_frame as for sdv2_kv_append (the
+ *      chunk is NOT yet appended); the call appends it.
+ * Fused (bf16 cache, T'*N <= 256, T' <= 4, T' * temporal pairs <= 48, the
+ * chunk's temporal phases below 4096 (the cache keeps their fp64 (cos, sin)),
+ * 16 * (frame_h * row pairs + frame_w * column pairs) <= 256 * head_dim - 1024,
+ * and the chunk's
+ * rows of every stream within at most two 128-key tiles of its valid slot
+ * prefix; see sdv2_append_attention_mode): the attention CTA that reads a KV
+ * tile holding the chunk's rows builds those rows in shared memory from k and v
+ * (keys rotated exactly as sdv2_kv_append rotates them), writes them to their
+ * ring slots and feeds the same values to the tensor cores; the rest of the
+ * cache comes by TMA as usual.  The chunk's K/V are read from k / v once
+ * and never read back from the cache.  Otherwise the call makes the two calls.
+ * Unlike sdv2_chunk_attention, the fused launch waits for the previous kernel
+ * in the stream before reading q (q, k, v may come from it).
+ * Errors: SDV2_E_ARG, SDV2_E_ALIGN, SDV2_E_STATE (wrong f0), SDV2_E_CUDA. */
+sdv2_status sdv2_append_attention(sdv2_cache *cache, int32_t layer, const void *q, const void *k,
+                                  const void *v, void *out, const int64_t *chunk_first_frame,
+                                  float softmax_scale, sdv2_stream stream);
+
 /* Adaptive sink refresh, after the chunk was appended to every layer.
  * [Q] "Adaptive sink and RoPE refresh".
  * hidden: device bf16 [B][T'*N][D] (D = embed_dim); the chunk embedding is
@@ -234,8 +263,9 @@ sdv2_status sdv2_cache_check(sdv2_cache *cache);
 sdv2_status sdv2_cache_selftest_wait(sdv2_cache *cache, uint64_t limit_ns, sdv2_stream stream);
 
 /* Measurement hook (no counterpart in the pages): while set, every
- * sdv2_chunk_attention call on this cache records `start` on its stream
- * right before the attention kernel's launch and `stop` right after it, so
+ * sdv2_chunk_attention call (and fused sdv2_append_attention call) on this
+ * cache records `start` on its stream right before the attention kernel's
+ * launch and `stop` right after it, so
  * the time between them is that kernel alone (the split merge after it is
  * outside).  Recording events between the
  * call's launches serialises them; use it in a separate timing pass.  Pass
@@ -339,6 +369,13 @@ int32_t sdv2_attention_splits(const sdv2_cache_config *cfg, const int64_t *keys,
  * half as many CTAs start and the two heads' softmax and tensor-core work overlap.
  * Host-side, no device needed. */
 int32_t sdv2_attention_pair_mode(const sdv2_cache_config *cfg, const int64_t *keys, int32_t sm_count);
+/* How sdv2_append_attention runs chunks starting at chunk_first_frame[0..batch-1]
+ * (negative: stream skipped) on a GPU with sm_count SMs: 0 as two launches (the
+ * append, then the attention), 1 as the fused kernel, 2 as the fused kernel in
+ * the pair mode (one KV tile per stream holds the chunk's rows); -1 on a bad
+ * argument.  Host-side, no device needed. */
+int32_t sdv2_append_attention_mode(const sdv2_cache_config *cfg, const int64_t *chunk_first_frame,
+                                   int32_t sm_count);
 
 /* Kernels launched by this library in this process so far. */
 uint64_t sdv2_launch_count(void);

@@ -51,6 +51,16 @@ class PairedStream:
         want = O.chunk_attention(self.ora, layer, synth.bf16_bits(q), f0, f32(scale), rows=rows)
         return out, want
 
+    def append_attention(self, layer, f0, q, k, v, rows=None):
+        """The fused call on the GPU; the oracle's append, then its attention."""
+        c = self.cfg
+        out = torch.zeros((c.batch, c.chunk_tokens, c.heads, c.head_dim), dtype=torch.bfloat16, device="cuda")
+        scale = 1.0 / math.sqrt(c.head_dim)
+        self.gpu.append_attention(layer, q.cuda(), k.cuda(), v.cuda(), out, f0, scale)
+        O.kv_append(self.ora, layer, synth.bf16_bits(k), synth.bf16_bits(v), f0)
+        want = O.chunk_attention(self.ora, layer, synth.bf16_bits(q), f0, f32(scale), rows=rows)
+        return out, want
+
     def advance(self, active=None):
         """Next chunk's first frames (negative for streams not in ``active``)."""
         c = self.cfg

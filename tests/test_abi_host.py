@@ -133,6 +133,77 @@ def test_split_plan(B):
     assert B.sdv2_attention_plan(c2, [0], 148) == (0, 1)        # no active stream
 
 
+def _fuse_mode_model(cfg, f0s, sms):
+    """The fused append + attention rule restated: bf16 cache, at most 256 queries, at most 4
+    chunk frames whose temporal pairs fit 48 entries and whose phases are below 4096 (the cache's
+    fp64 phase table), fp64 row and column tables within 256 head_dim - 1024 bytes, the chunk's rows of every
+    stream within at
+    most two 128-key tiles of its slot-major prefix; pair mode when every stream has one such
+    tile, chunks of at most 128 queries, at least two heads and more (stream, head) units than SMs."""
+    n = cfg.frame_h * cfg.frame_w
+    c2 = cfg.head_dim // 2
+    tp, nt = cfg.chunk_frames, (cfg.rope_pairs[0] if any(cfg.rope_pairs) else c2 - 2 * (c2 // 3))
+    nh = cfg.rope_pairs[1] if any(cfg.rope_pairs) else c2 // 3
+    nw = cfg.rope_pairs[2] if any(cfg.rope_pairs) else c2 // 3
+    if cfg.kv_format != 0 or tp * n > 256 or tp > 4 or tp * nt > 48 or 16 * (cfg.frame_h * nh + cfg.frame_w * nw) > 256 * cfg.head_dim - 1024:
+        return 0
+    reset = cfg.rope_reset_period
+    n_phase = min(reset if reset > 0 else 4096, 4096)     # the cache's precomputed temporal phases
+    one, active = True, 0
+    for f0 in f0s:
+        if f0 < 0:
+            continue
+        active += 1
+        if any(O.rope_phase(f0 + i, reset) >= n_phase for i in range(tp)):
+            return 0
+        tiles = set()
+        for i in range(tp):
+            s = O.slot_of_frame(f0 + i, cfg.sink_frames, cfg.window_frames)
+            tiles |= set(range(s * n // 128, (s * n + n - 1) // 128 + 1))
+        if len(tiles) > 2:
+            return 0
+        one = one and len(tiles) == 1
+    pair = one and tp * n <= 128 and cfg.heads >= 2 and active * cfg.heads > sms
+    return 2 if pair else 1
+
+
+def test_append_attention_mode(B):
+    small = B.make_cache_config(16, 1, 12, 128, 8, 8, 1, 1, 6)
+    assert B.sdv2_append_attention_mode(small, [5] * 16, 148) == 2          # 192 units, one tile each
+    assert B.sdv2_append_attention_mode(small, [5] * 12 + [-1] * 4, 148) == 1
+    assert B.sdv2_append_attention_mode(B.make_cache_config(16, 1, 12, 128, 8, 8, 1, 1, 6, kv_format="fp8"),
+                                        [5] * 16, 148) == 0
+    assert B.sdv2_append_attention_mode(B.make_cache_config(1, 1, 12, 128, 32, 32, 1, 1, 6), [3], 148) == 0
+    straddle = B.make_cache_config(16, 1, 12, 128, 8, 12, 1, 2, 4)         # 96 tokens per frame
+    assert B.sdv2_append_attention_mode(straddle, [1] * 16, 148) == 1       # rows 96..191: two tiles
+    assert B.sdv2_append_attention_mode(straddle, [0] * 16, 148) == 2       # rows 0..95: one tile, pair mode
+    two = B.make_cache_config(1, 1, 2, 64, 8, 12, 2, 1, 4)                  # T' = 2, 192 queries
+    assert B.sdv2_append_attention_mode(two, [0], 148) == 1
+    assert B.sdv2_append_attention_mode(two, [4], 148) == 0                 # slots 4 and 1: three tiles
+    assert B.sdv2_append_attention_mode(B.make_cache_config(1, 1, 2, 128, 8, 8, 3, 1, 6), [0], 148) == 0  # 3 x 22 pairs
+    assert B.sdv2_append_attention_mode(B.make_cache_config(1, 1, 2, 128, 4, 4, 3, 1, 6, rope_pairs=(10, 27, 27)),
+                                        [0], 148) == 1
+    assert B.sdv2_append_attention_mode(B.make_cache_config(1, 1, 2, 128, 1, 128, 1, 1, 6), [0], 148) == 0  # 128 x 21 x 16 B
+    assert B.sdv2_append_attention_mode(small, [4095] * 16, 148) == 2                 # no reset: phase table 0 .. 4095
+    assert B.sdv2_append_attention_mode(small, [4096] + [5] * 15, 148) == 0
+    assert B.sdv2_append_attention_mode(B.make_cache_config(16, 1, 12, 128, 8, 8, 1, 1, 6, rope_reset_period=9000),
+                                        [8999] * 16, 148) == 0                         # phase 8999 > 4095
+    assert B.sdv2_append_attention_mode(B.make_cache_config(16, 1, 12, 128, 8, 8, 1, 1, 6, rope_reset_period=300),
+                                        [10 ** 6] * 16, 148) == 2
+    import random
+    rng = random.Random(5)
+    for _ in range(400):
+        b, h, d = rng.randint(1, 24), rng.choice([1, 2, 7, 12, 13]), rng.choice([64, 128])
+        fh, fw, tp = rng.randint(1, 12), rng.choice([rng.randint(1, 16), rng.randint(60, 200)]), rng.randint(1, 5)
+        s_, w = rng.randint(1, 3), rng.randint(tp, 8)
+        cfg = B.make_cache_config(b, 1, h, d, fh, fw, tp, s_, w, rope_reset_period=rng.choice([0, 0, 7, 5000]))
+        if B.lib().sdv2_cache_bytes(cfg) == 0:
+            continue                                                        # (a config the library rejects)
+        f0s = [rng.choice([-1, rng.randint(0, 40), rng.randint(4000, 4200)]) for _ in range(b)]
+        sms = rng.choice([16, 148])
+        assert B.sdv2_append_attention_mode(cfg, f0s, sms) == _fuse_mode_model(cfg, f0s, sms), (b, h, d, fh, fw, tp)
+
+
 def test_null_handles_are_rejected_without_a_device(B):
     import ctypes
     lib = B.lib()

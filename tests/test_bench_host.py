@@ -89,3 +89,17 @@ def test_fp8_workloads_byte_accounting():
     assert bench.workload_config("x", w8, 1)["kv_format"] == "fp8"
     assert bench.workload_config("x", w16, 1)["kv_format"] == "bf16"
     assert bench.kv_elem(w8) == 1 and bench.kv_elem(w16) == 2
+
+
+def test_fused_workloads_byte_accounting():
+    import bench
+    plain, fused = bench.WORKLOADS["wan1.3b-128x128-b16"], bench.WORKLOADS["wan1.3b-128x128-b16-fused"]
+    keys = bench.steady_keys(plain)
+    assert keys == [448] * 16
+    hd, lq = 12 * 128, 64
+    # the fused launch also writes the chunk's K and V (bf16) to their ring slots
+    assert bench.attn_bytes(fused, keys) == bench.attn_bytes(plain, keys) + 16 * 4 * lq * hd
+    assert bench.attn_flops(fused, keys) == bench.attn_flops(plain, keys)
+    assert "fused" in bench.workload_config("x", fused, 1)["append"]
+    assert "append" not in bench.workload_config("x", plain, 1)
+    assert "wan1.3b-128x128-b16-fused" in bench.EXTRA_WORKLOADS
