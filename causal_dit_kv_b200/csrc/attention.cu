@@ -948,9 +948,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         stores_reading = false;
                     }
                     if constexpr (F8) {
+                        // (pair mode: sequence tile i is tile i / 2 of head h or h_pair)
+                        const int hk = paired && (k_issued & 1) ? h_pair : h;
                         mbar_arrive_expect_tx(&bars[L::kKFull + st], L::kKVTile);
-                        const int g = kv_begin + k_issued, sl = g / p.n_blk;
-                        tma_load_4d(smem + L::kK + st * L::kKVTile, &tmap_k, &bars[L::kKFull + st], 0, h,
+                        const int g = paired ? k_issued >> 1 : kv_begin + k_issued, sl = g / p.n_blk;
+                        tma_load_4d(smem + L::kK + st * L::kKVTile, &tmap_k, &bars[L::kKFull + st], 0, hk,
                                     sl * p.np_tokens + (g - sl * p.n_blk) * kBlockN, bg);
                     } else {
                         // (pair mode: sequence tile i is tile i / 2 of head h or h_pair)
@@ -975,10 +977,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     stores_reading = false;
                 }
                 if constexpr (F8) {
+                    const int hv = paired && (v_issued & 1) ? h_pair : h;
                     mbar_arrive_expect_tx(&bars[L::kVFull + st], L::kKVTile);
-                    const int g = kv_begin + v_issued, sl = g / p.n_blk;
+                    const int g = paired ? v_issued >> 1 : kv_begin + v_issued, sl = g / p.n_blk;
                     tma_load_5d(smem + L::kV + st * L::kKVTile, &tmap_v, &bars[L::kVFull + st],
-                                (g - sl * p.n_blk) * kBlockN, 0, h, sl, bg);
+                                (g - sl * p.n_blk) * kBlockN, 0, hv, sl, bg);
                 } else {
                     const int hv = paired && (v_issued & 1) ? h_pair : h;
                     const int tv = paired ? tile_at(v_issued >> 1) : tile_at(v_issued);
@@ -1176,7 +1179,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 sq = valid ? q_row_scale : 0.0f;
                 scale_base = static_cast<int64_t>(bg) * p.slots * p.scale_slot_stride + hs * p.n_blk;
                 sv_ref = 0.0f;
-                for (int i = 0; i < n_local; ++i) {
+                // this set's tiles (pair mode: all of its own head's; otherwise the CTA's range,
+                // which both sets of a single query tile share)
+                for (int i = 0; i < (paired ? n_kv : n_local); ++i) {
                     const int g = kv_begin + i, sl = g / p.n_blk;
                     sv_ref = fmaxf(sv_ref, p.v_scale[scale_base + sl * (p.scale_slot_stride - p.n_blk) + g]);
                 }
@@ -1204,7 +1209,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 float c_t = p.scale_log2, r_t = 1.0f;
                 int valid_cols;
                 if constexpr (F8) {
-                    const int g = kv_begin + (alt ? 2 * it + t : it);      // KV tile of this iteration
+                    const int g = kv_begin + (paired ? it : (alt ? 2 * it + t : it));   // KV tile of this iteration
                     const int sl = g / p.n_blk;
                     const int64_t si = scale_base + sl * (p.scale_slot_stride - p.n_blk) + g;
                     c_t = fmaxf(p.scale_log2 * sq * p.k_scale[si], 1e-30f);

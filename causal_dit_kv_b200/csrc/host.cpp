@@ -256,12 +256,12 @@ AttnPlan plan_attention(const sdv2_cache_config &c, const Geometry &g, int64_t u
     return best;
 }
 
-// Pair mode of the attention launch: with chunks of one query tile (bf16 cache) and more
-// (stream, head) units than SMs, a CTA takes two heads of one stream, one accumulator set
-// and query tile each, their KV tiles interleaved; half the CTAs, each start-up shared by
-// two heads, and the two softmax / MMA chains of a CTA still overlap.
+// Pair mode of the attention launch: with chunks of one query tile and more (stream, head)
+// units than SMs, a CTA takes two heads of one stream, one accumulator set and query tile
+// each, their KV tiles interleaved; half the CTAs, each start-up shared by two heads, and
+// the two softmax / MMA chains of a CTA still overlap.  (Both cache formats.)
 bool use_pair_mode(const Geometry &g, const sdv2_cache_config &c, int64_t units, int sm_count) {
-    return !g.f8 && g.n_qpairs == 1 && g.lq <= kBlockM && c.heads >= 2 && sm_count > 0 && units > sm_count;
+    return g.n_qpairs == 1 && g.lq <= kBlockM && c.heads >= 2 && sm_count > 0 && units > sm_count;
 }
 
 // KV tiles of the longest stream: 128-key runs of its valid prefix, or for the fp8 cache

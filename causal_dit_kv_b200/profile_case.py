@@ -3,8 +3,9 @@
     python -m causal_dit_kv_b200.profile_case --kernel attention [--workload wan1.3b-512x512]
 
 Sets up one layer of the named workload's cache at steady state (ring full)
-with a handful of appends, then runs the requested call once; the ncu
-capture selects the kernel with -k.  Device memory stays well under 1 GB.
+with a handful of appends, then runs the requested call once (append_attention:
+the next chunk's append fused into its attention); the ncu capture selects the
+kernel with -k.  Device memory stays well under 1 GB.
 """
 from __future__ import annotations
 
@@ -36,7 +37,8 @@ def main():
     from causal_dit_kv_b200 import KVCache, MotionState
 
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kernel", choices=["attention", "append", "refresh", "motion"], default="attention")
+    ap.add_argument("--kernel", choices=["attention", "append", "append_attention", "refresh", "motion"],
+                    default="attention")
     ap.add_argument("--workload", choices=sorted(SHAPES), default="wan1.3b-512x512")
     ap.add_argument("--repeat", type=int, default=1)
     a = ap.parse_args()
@@ -60,6 +62,10 @@ def main():
     if a.kernel == "attention":
         for _ in range(a.repeat):
             cache.chunk_attention(0, q, out, f0, 1.0 / math.sqrt(D))
+    elif a.kernel == "append_attention":
+        for _ in range(a.repeat):
+            cache.append_attention(0, q, k, v, out, [frame] * B, 1.0 / math.sqrt(D))
+            frame += Tp
     elif a.kernel == "append":
         for _ in range(a.repeat):
             cache.kv_append(0, k, v, [frame] * B)

@@ -120,13 +120,13 @@ def test_split_plan(B):
     c4 = B.make_cache_config(1, 40, 40, 128, 32, 32, 1, 1, 6)
     whole, pieces = B.sdv2_attention_plan(c4, [7168], 148)
     assert whole == 148 and pieces > 4 and 12 * pieces <= 148
-    # pair mode: chunks of one query tile with more (stream, head) units than SMs, bf16 only
+    # pair mode: chunks of one query tile with more (stream, head) units than SMs
     small = B.make_cache_config(16, 1, 12, 128, 8, 8, 1, 1, 6)
     assert B.sdv2_attention_pair_mode(small, [448] * 16, 148) == 1
     assert B.sdv2_attention_plan(small, [448] * 16, 148) == (192, 1)
     assert B.sdv2_attention_pair_mode(small, [448] * 12 + [0] * 4, 148) == 0          # 144 units fit one wave
     assert B.sdv2_attention_pair_mode(B.make_cache_config(16, 1, 12, 128, 8, 8, 1, 1, 6, kv_format="fp8"),
-                                      [448] * 16, 148) == 0
+                                      [448] * 16, 148) == 1                           # both cache formats
     assert B.sdv2_attention_pair_mode(c2, [7168], 148) == 0                           # 1024 queries
     tiny = B.make_cache_config(1, 1, 2, 64, 4, 4, 1, 1, 2)
     assert B.sdv2_attention_plan(tiny, [48], 148) == (2, 1)     # 2 heads, a single KV tile: nothing to split

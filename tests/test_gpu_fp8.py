@@ -112,9 +112,14 @@ def _check_out(pair, out, want, layer, f0, q_bits, rows=None):
     assert float(np.concatenate([r.ravel() for r in ratios]).mean()) < 1.2
 
 
-@pytest.mark.parametrize("case", ["ragged_single_tile", "two_tiles", "multi_frame_chunks"])
+@pytest.mark.parametrize("case", ["ragged_single_tile", "two_tiles", "multi_frame_chunks", "pair_mode"])
 def test_fp8_stream_parity(case):
     cfg = {
+        # 64 tokens per frame (one ragged block per slot), 13 heads x 12 streams = 156 units
+        # on 148 SMs: the pair mode (heads 2k and 2k + 1 of a stream in one CTA, the last
+        # head of each stream alone), streams joining at different steps
+        "pair_mode": dict(batch=12, layers=1, heads=13, head_dim=128, frame_h=8, frame_w=8, chunk_frames=1,
+                          sink_frames=1, window_frames=3),
         # N = 150: two blocks per slot, the second of 22 tokens; one query tile (both accumulator sets)
         "ragged_single_tile": dict(batch=2, layers=1, heads=2, head_dim=128, frame_h=10, frame_w=15, chunk_frames=1,
                                    sink_frames=1, window_frames=3, rope_reset_period=4),
@@ -126,8 +131,12 @@ def test_fp8_stream_parity(case):
                                    sink_frames=2, window_frames=4),
     }[case]
     pair = Fp8Pair(seed=3001, **cfg)
+    if case == "pair_mode":
+        from causal_dit_kv_b200 import binding as B
+        assert B.sdv2_attention_pair_mode(pair.gpu.cfg, [256] * 12, 148) == 1
     for step in range(7):
-        active = None if case != "multi_frame_chunks" else [b for b in range(3) if step >= b]
+        active = None if case not in ("multi_frame_chunks", "pair_mode") else \
+            [b for b in range(pair.cfg.batch) if step >= b % 3]
         f0 = pair.step_frames(active)
         for layer in range(pair.cfg.layers):
             out, want = pair.run_layer(step, layer, f0)
