@@ -69,7 +69,7 @@ struct AttnParams {
     // n_units) are split over the KV range into n_pieces CTAs each and merged by
     // attention_combine_kernel.
     int32_t n_units, n_whole, n_pieces;
-    // 1: pair mode (bf16, chunks of one query tile, nothing split): CTA x takes heads 2k and
+    // 1: pair mode (chunks of one query tile, nothing split): CTA x takes heads 2k and
     // 2k + 1 of stream unit_stream[x / ceil(H / 2)], one accumulator set and query tile each
     int32_t pair;
     uint8_t unit_stream[kMaxBatch];

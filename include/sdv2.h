@@ -363,7 +363,7 @@ sdv2_status sdv2_attention_plan(const sdv2_cache_config *cfg, const int64_t *key
  * argument. */
 int32_t sdv2_attention_splits(const sdv2_cache_config *cfg, const int64_t *keys, int32_t sm_count);
 /* 1 if sdv2_chunk_attention would run that launch in the pair mode, 0 if not, -1
- * on a bad argument.  Pair mode (bf16 cache, chunks of at most 128 queries, more
+ * on a bad argument.  Pair mode (either cache format, chunks of at most 128 queries, more
  * (stream, head) units than SMs): one CTA takes heads 2k and 2k+1 of a stream,
  * each on its own query tile and accumulator set, their KV tiles interleaved, so
  * half as many CTAs start and the two heads' softmax and tensor-core work overlap.
