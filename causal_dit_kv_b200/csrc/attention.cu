@@ -783,28 +783,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
         }
     }
-    // Fused append: warps 2 and 3 start on the assembled tiles at once.
     bool have_tab = false;
-    if constexpr (FUSE) {
-        if ((warp == 2 || warp == 3) && n_asm > 0) {
-            build_part_groups<D, L>(smem, bars, p, f, bg, lk, h, h_pair, paired, a0, paired ? a0 : a1, mp0, mp1, ns,
-                                    warp - 2, lane, abort_flag, have_tab);
-            rotate_full_groups<D, L>(smem, bars, p, a0, paired ? a0 : a1, mf0, mf1, ns, warp - 2, lane, abort_flag,
-                                     have_tab);
-            assembled<L>(bars, lane);
-        }
-    }
     // RoPE on load by the softmax warps (idle until the first scores arrive): thread
     // (t, row) rotates its own query row (the single-tile mode: sub-tile t of tile 0's row)
     float q_row_scale = 0.0f;                   // fp8: E4M3 scale of this thread's query row
     if (warp >= 4 && n_local > 0) {
-        if constexpr (FUSE) {
-            // fused append: the straddling rows first (their loads in flight while the query
-            // tiles land); the full groups' keys after the query rotation
-            if (n_asm > 0)
-                build_part_groups<D, L>(smem, bars, p, f, bg, lk, h, h_pair, paired, a0, paired ? a0 : a1, mp0, mp1, ns,
-                                        warp - 2, lane, abort_flag, have_tab);
-        }
         const int t = (warp - 4) >> 2;
         const int row = ((warp & 3) << 5) + lane;
         const int qt = one_q ? 0 : t;           // query tile of this thread's row
@@ -884,12 +867,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         fence_proxy_async_shared();             // the tensor core reads these rows next
         mbar_arrive(&bars[L::kQReady]);
-        if constexpr (FUSE) {
-            if (n_asm > 0) {
-                rotate_full_groups<D, L>(smem, bars, p, a0, paired ? a0 : a1, mf0, mf1, ns, warp - 2, lane, abort_flag,
-                                         have_tab);
-                assembled<L>(bars, lane);
-            }
+    }
+    // Fused append: warps 2 and 3 at once, the softmax warps after the query rotation, build
+    // the assembled tiles' chunk rows, all from this one place in the code (one copy of it
+    // in the instruction cache)
+    if constexpr (FUSE) {
+        if (warp >= 2 && n_asm > 0) {
+            build_part_groups<D, L>(smem, bars, p, f, bg, lk, h, h_pair, paired, a0, paired ? a0 : a1, mp0, mp1, ns,
+                                    warp - 2, lane, abort_flag, have_tab);
+            rotate_full_groups<D, L>(smem, bars, p, a0, paired ? a0 : a1, mf0, mf1, ns, warp - 2, lane, abort_flag,
+                                     have_tab);
+            assembled<L>(bars, lane);
         }
     }
 
