@@ -335,16 +335,15 @@ __device__ __forceinline__ void merge_sets(uint32_t o0, uint32_t o1, bool has1, 
     for (int i = 0; i < 32; ++i) r0[i] = __float_as_uint(w0 * __uint_as_float(r0[i]) + w1 * __uint_as_float(r1[i]));
 }
 
-// Fused append: TMA of the 8-row groups `groups` of an assembled tile (bit q: rows
+// Fused append: TMA loads of the 8-row groups `groups` of an assembled tile (bit q: rows
 // 8q .. 8q + 7), as runs: consecutive groups whose rows are consecutive in the tensor go
 // together, each run in boxes of 64, 32, 16, 8 rows, largest first (maps[i]: boxes of
-// 64 >> i rows x 64 channels; row_of(q): the tensor row of group q's first row).  A load
-// lands in the tile at dst (a box of rows starting at tile row 8q goes to byte 1024 q of
-// each 128-byte-swizzled sub-tile, where a whole-tile load puts those rows); a store
-// (store = true) writes the tile's rows to the tensor instead.
+// 64 >> i rows x 64 channels; row_of(q): the tensor row of group q's first row).  A box
+// of rows starting at tile row 8q lands at byte 1024 q of each 128-byte-swizzled sub-tile
+// of the tile at dst, where a whole-tile load puts those rows.
 template <int D, typename L, typename RowOf>
-__device__ __forceinline__ void move_row_groups(uint8_t *dst, const CUtensorMap *maps, uint64_t *bar, uint32_t groups,
-                                                int hh, int bg, RowOf row_of, bool store) {
+__device__ __forceinline__ void load_row_groups(uint8_t *dst, const CUtensorMap *maps, uint64_t *bar, uint32_t groups,
+                                                int hh, int bg, RowOf row_of) {
     int q = 0;
     while (q < 16) {
         if (!((groups >> q) & 1u)) {
@@ -359,12 +358,8 @@ __device__ __forceinline__ void move_row_groups(uint8_t *dst, const CUtensorMap 
             const int i = left >= 8 ? 0 : (left >= 4 ? 1 : (left >= 2 ? 2 : 3));
             const int row = row0 + 8 * (g - q);
 #pragma unroll
-            for (int kb = 0; kb < D / 64; ++kb) {
-                if (store)
-                    tma_store_4d(&maps[i], dst + kb * L::kSub + g * 1024, kb * 64, hh, row, bg);
-                else
-                    tma_load_4d(dst + kb * L::kSub + g * 1024, &maps[i], bar, kb * 64, hh, row, bg);
-            }
+            for (int kb = 0; kb < D / 64; ++kb)
+                tma_load_4d(dst + kb * L::kSub + g * 1024, &maps[i], bar, kb * 64, hh, row, bg);
             g += 8 >> i;
         }
         q = e;
@@ -484,19 +479,23 @@ __device__ __forceinline__ void build_part_groups(uint8_t *smem, uint64_t *bars,
 
 // Fused append, the "full" 8-row groups mf0, mf1 of the assembled tiles (eight
 // consecutive tokens of one chunk frame each): their un-rotated keys and values came by
-// TMA from the caller's k / v into the tiles; once a tile's loads have landed (its kKFull
-// phase), the keys are rotated in place, pair by pair with the append's fp64 rule.  Rows
-// are dealt round-robin to warps 2 .. 11 in slots of kRowsPerIter rows; lane c of a row
-// takes pairs c + kLanes q (32-bit words of the swizzled row; neighbouring table entries).
-// The producer writes these rows to their ring slots by TMA after kAsm.
+// TMA from the caller's k / v into the tiles; once a tile's key loads have landed (its
+// kKFull phase), the keys are rotated in place, pair by pair with the append's fp64
+// rule, and written from registers to their ring slots; the values go to their ring
+// slots straight from the caller's v (loaded before the wait, so that latency is hidden).
+// Rows are dealt round-robin to warps 2 .. 11 in slots of kRowsPerIter rows, kBatch slots
+// of a warp at a time; lane c of a row takes pairs c + kLanes q (32-bit words of the
+// swizzled row; neighbouring table entries; contiguous global words).
 template <int D, typename L>
-__device__ __forceinline__ void rotate_full_groups(uint8_t *smem, uint64_t *bars, const AttnParams &p, int g0, int g1,
-                                                   uint32_t mf0, uint32_t mf1, const int (&ns)[kFuseMaxFrames], int wi,
-                                                   int lane, volatile uint32_t *abort_flag, bool &have_tab) {
+__device__ __forceinline__ void rotate_full_groups(uint8_t *smem, uint64_t *bars, const AttnParams &p,
+                                                   const FuseParams &f, int bg, int h, int h_pair, bool paired, int g0,
+                                                   int g1, uint32_t mf0, uint32_t mf1, const int (&ns)[kFuseMaxFrames],
+                                                   int wi, int lane, volatile uint32_t *abort_flag, bool &have_tab) {
     constexpr int kLanes = D / 8;
     constexpr int kRowsPerIter = 32 / kLanes;
     constexpr int kIters = 8 / kRowsPerIter;
     constexpr int kWarps = (kAttnThreads - 64) / 32;
+    constexpr int kBatch = 4;
     const int c0 = __popc(mf0);
     const int n_slots = kIters * (c0 + __popc(mf1));
     if (wi >= n_slots) return;
@@ -504,48 +503,77 @@ __device__ __forceinline__ void rotate_full_groups(uint8_t *smem, uint64_t *bars
     const int rr = lane / kLanes;
     const int N = p.tokens_per_frame;
     const int n_t = p.n_t, n_th = p.n_t + p.n_h, n_h = p.n_h, n_w = p.n_w, fw = p.frame_w;
+    const int64_t row_elems = static_cast<int64_t>(p.heads) * D;
     const double2 *tab_t = reinterpret_cast<const double2 *>(smem + L::kTab64);
     const double2 *tab_h = reinterpret_cast<const double2 *>(smem + L::kTabHW);
     const double2 *tab_w = tab_h + p.frame_h * n_h;
-    if (!have_tab) {
-        have_tab = warp_wait(&bars[L::kTabReady], 0, abort_flag, p.status, kStatusSoftmaxWait);
-        if (!have_tab) return;
-    }
-    uint32_t landed = 0u;                             // tiles whose loads this warp has seen land
-    for (int s = wi; s < n_slots; s += kWarps) {
-        const int a = s < kIters * c0 ? 0 : 1;
-        if (!((landed >> a) & 1u)) {
-            if (!warp_wait(&bars[L::kKFull + a], 0, abort_flag, p.status, kStatusSoftmaxWait)) return;
-            landed |= 1u << a;
+    uint32_t landed = 0u;                             // tiles whose key loads this warp has seen land
+    for (int s0 = wi; s0 < n_slots; s0 += kWarps * kBatch) {
+        uint32_t xv[kBatch][4];
+        int rw[kBatch], pos[kBatch];                  // tile row | tile << 8 | chunk frame << 12; row, col packed
+        int64_t dst[kBatch];                          // element offset of this lane's row in the layer (-1: no slot)
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            const int s = s0 + b * kWarps;
+            dst[b] = -1;
+            rw[b] = pos[b] = 0;
+            if (s >= n_slots) continue;
+            const int a = s < kIters * c0 ? 0 : 1;
+            const int sa = a ? s - kIters * c0 : s;
+            uint32_t m = a ? mf1 : mf0;
+            for (int k = sa / kIters; k > 0; --k) m &= m - 1u;
+            const int r = (__ffs(m) - 1) * 8 + (sa % kIters) * kRowsPerIter + rr;
+            const int kr = (a ? g1 : g0) * kBlockN + r;
+            const int sl = kr / N;
+            const int n = kr - sl * N;
+            int fi = 0;
+#pragma unroll
+            for (int i = 0; i < kFuseMaxFrames; ++i)
+                if (ns[i] == sl) fi = i;
+            const int prow = n / fw;
+            const int hs = paired && a == 1 ? h_pair : h;
+            rw[b] = r | (a << 8) | (fi << 12);
+            pos[b] = (prow << 16) | (n - prow * fw);
+            dst[b] = (static_cast<int64_t>(bg) * f.slots * N + kr) * row_elems + hs * D;
+            const uint32_t *vs = reinterpret_cast<const uint32_t *>(
+                f.v_in + (static_cast<int64_t>(bg) * p.lq + static_cast<int64_t>(fi) * N + n) * row_elems + hs * D);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) xv[b][q] = ld_nc_u32(vs + c + kLanes * q);
         }
-        const int sa = a ? s - kIters * c0 : s;
-        uint32_t m = a ? mf1 : mf0;
-        for (int k = sa / kIters; k > 0; --k) m &= m - 1u;
-        const int r = (__ffs(m) - 1) * 8 + (sa % kIters) * kRowsPerIter + rr;
-        const int kr = (a ? g1 : g0) * kBlockN + r;
-        const int sl = kr / N;
-        const int n = kr - sl * N;
-        int fi = 0;
-#pragma unroll
-        for (int i = 0; i < kFuseMaxFrames; ++i)
-            if (ns[i] == sl) fi = i;
-        const int prow = n / fw;
-        const int pcol = n - prow * fw;
-        uint8_t *krow = smem + L::kK + a * L::kKVTile + r * 128;
-        uint32_t w[4];
-        int off[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int j = c + kLanes * q;
-            off[q] = (j >> 5) * L::kSub + ((((j & 31) >> 2) ^ (r & 7)) << 4) + ((j & 3) << 2);
-            w[q] = *reinterpret_cast<const uint32_t *>(krow + off[q]);
+        if (!have_tab) {
+            have_tab = warp_wait(&bars[L::kTabReady], 0, abort_flag, p.status, kStatusSoftmaxWait);
+            if (!have_tab) return;
         }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int j = c + kLanes * q;
-            const double2 cs = j < n_t ? tab_t[fi * n_t + j]
-                                       : (j < n_th ? tab_h[prow * n_h + (j - n_t)] : tab_w[pcol * n_w + (j - n_th)]);
-            *reinterpret_cast<uint32_t *>(krow + off[q]) = rotate_pair(w[q], cs.x, cs.y);
+        for (int b = 0; b < kBatch; ++b) {
+            if (dst[b] < 0) continue;
+            const int r = rw[b] & 0xFF, a = (rw[b] >> 8) & 0xF, fi = rw[b] >> 12;
+            if (!((landed >> a) & 1u)) {
+                if (!warp_wait(&bars[L::kKFull + a], 0, abort_flag, p.status, kStatusSoftmaxWait)) return;
+                landed |= 1u << a;
+            }
+            const int prow = pos[b] >> 16, pcol = pos[b] & 0xFFFF;
+            uint8_t *krow = smem + L::kK + a * L::kKVTile + r * 128;
+            uint32_t *kdst = reinterpret_cast<uint32_t *>(f.k_layer + dst[b]);
+            uint32_t *vdst = reinterpret_cast<uint32_t *>(f.v_layer + dst[b]);
+            uint32_t w[4];
+            int off[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int j = c + kLanes * q;
+                off[q] = (j >> 5) * L::kSub + ((((j & 31) >> 2) ^ (r & 7)) << 4) + ((j & 3) << 2);
+                w[q] = *reinterpret_cast<const uint32_t *>(krow + off[q]);
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int j = c + kLanes * q;
+                const double2 cs = j < n_t ? tab_t[fi * n_t + j]
+                                           : (j < n_th ? tab_h[prow * n_h + (j - n_t)] : tab_w[pcol * n_w + (j - n_th)]);
+                const uint32_t wr = rotate_pair(w[q], cs.x, cs.y);
+                *reinterpret_cast<uint32_t *>(krow + off[q]) = wr;
+                kdst[j] = wr;
+                vdst[j] = xv[b][q];
+            }
         }
     }
 }
@@ -777,8 +805,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     uint8_t *tile = smem + (is_v ? L::kV : L::kK) + i * L::kKVTile;
                     uint64_t *bar = &bars[(is_v ? L::kVFull : L::kKFull) + i];
                     mbar_arrive_expect_tx(bar, bytes);
-                    move_row_groups<D, L>(tile, is_v ? f.tmap_vc : f.tmap_kc, bar, old, hi, bg, cache_row, false);
-                    move_row_groups<D, L>(tile, is_v ? f.tmap_vi : f.tmap_ki, bar, mf, hi, bg, chunk_token, false);
+                    load_row_groups<D, L>(tile, is_v ? f.tmap_vc : f.tmap_kc, bar, old, hi, bg, cache_row);
+                    load_row_groups<D, L>(tile, is_v ? f.tmap_vi : f.tmap_ki, bar, mf, hi, bg, chunk_token);
                 }
             }
         }
@@ -875,8 +903,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (warp >= 2 && n_asm > 0) {
             build_part_groups<D, L>(smem, bars, p, f, bg, lk, h, h_pair, paired, a0, paired ? a0 : a1, mp0, mp1, ns,
                                     warp - 2, lane, abort_flag, have_tab);
-            rotate_full_groups<D, L>(smem, bars, p, a0, paired ? a0 : a1, mf0, mf1, ns, warp - 2, lane, abort_flag,
-                                     have_tab);
+            rotate_full_groups<D, L>(smem, bars, p, f, bg, h, h_pair, paired, a0, paired ? a0 : a1, mf0, mf1, ns,
+                                     warp - 2, lane, abort_flag, have_tab);
             assembled<L>(bars, lane);
         }
     }
@@ -897,31 +925,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             // (fused append: the first n_asm were issued with the queries).
             int k_issued = n_asm, v_issued = n_asm;
             bool ok = true;
-            bool stores_reading = false;                 // fused append: TMA stores still reading stages < n_asm
-            bool stored = false;
             if constexpr (FUSE) {
-                // nothing goes into V stage 2 (the key tables) before the assembled tiles are
-                // built; then the chunk's full groups, keys rotated in place, values as loaded
-                // (their stages' kVFull), go to their ring slots
+                // nothing goes into V stage 2 (the key tables) before the assembled tiles are built
                 if (n_asm > 0) ok = mbar_wait(&bars[L::kAsm], 0, abort_flag, p.status, kStatusTmaWait);
-                if (n_asm > 0 && (mf0 | mf1) != 0u) {
-                    for (int i = 0; ok && i < n_asm; ++i)
-                        ok = mbar_wait(&bars[L::kVFull + i], 0, abort_flag, p.status, kStatusTmaWait);
-                    if (ok) {
-                        for (int i = 0; i < n_asm; ++i) {
-                            const int hi = paired && i == 1 ? h_pair : h;
-                            const int ti = i == 0 || paired ? a0 : a1;
-                            const uint32_t mf = i ? mf1 : mf0;
-                            auto cache_row = [&](int q) { return ti * kBlockN + 8 * q; };
-                            move_row_groups<D, L>(smem + L::kK + i * L::kKVTile, f.tmap_kc, nullptr, mf, hi, bg,
-                                                  cache_row, true);
-                            move_row_groups<D, L>(smem + L::kV + i * L::kKVTile, f.tmap_vc, nullptr, mf, hi, bg,
-                                                  cache_row, true);
-                        }
-                        bulk_commit_group();
-                        stores_reading = stored = true;
-                    }
-                }
             }
             while (ok && v_issued < n_local) {
                 if (k_issued < n_local && k_issued <= v_issued + 1) {
@@ -930,10 +936,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     if (!mbar_wait(&bars[L::kKEmpty + st], ph ^ 1u, abort_flag, p.status, kStatusTmaWait)) {
                         ok = false;
                         break;
-                    }
-                    if (stores_reading && st < n_asm) {     // (the stage is an assembled tile's)
-                        bulk_wait_group_read0();
-                        stores_reading = false;
                     }
                     if constexpr (F8) {
                         // (pair mode: sequence tile i is tile i / 2 of head h or h_pair)
@@ -959,10 +961,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 if (!mbar_wait(&bars[L::kVEmpty + st], ph ^ 1u, abort_flag, p.status, kStatusTmaWait)) {
                     ok = false;
                     break;
-                }
-                if (stores_reading && st < n_asm) {
-                    bulk_wait_group_read0();
-                    stores_reading = false;
                 }
                 if constexpr (F8) {
                     const int hv = paired && (v_issued & 1) ? h_pair : h;
@@ -1000,7 +998,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                             if (global_timer_ns() - t0 > kWaitLimitNs) break;
                 }
             }
-            if (stored) bulk_wait_group0();              // the ring-slot writes are complete before the CTA ends
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer

@@ -91,7 +91,8 @@ struct AttnParams {
 // the CTA that reads a KV tile holding rows of the chunk's own frames brings those rows
 // from the caller's k / v into the tile instead (by TMA, or row by row where an 8-row
 // group straddles slots), rotates the keys there by the append's rule and writes the
-// rows to their ring slots (by TMA); the tile's other rows come from the cache.  Such
+// rows to their ring slots (keys from the rotating threads' registers, values copied
+// from v); the tile's other rows come from the cache.  Such
 // "assembled" tiles go first in each CTA's tile order; every other tile comes by TMA as
 // in the plain attention.
 constexpr int kFuseMaxFrames = 4;          // chunk frames, at most
