@@ -579,7 +579,7 @@ __device__ __forceinline__ void rotate_full_groups(uint8_t *smem, uint64_t *bars
 }
 
 // Fused append: a warp's writes to the assembled tiles are done; fence them for the
-// tensor core and the TMA stores, then one arrival on kAsm (warps 2 .. 11).
+// tensor core, then one arrival on kAsm (warps 2 .. 11).
 template <typename L>
 __device__ __forceinline__ void assembled(uint64_t *bars, int lane) {
     fence_proxy_async_shared();
