@@ -155,17 +155,19 @@ def attn_flops(w, keys):
 def attn_bytes(w, keys):
     """Bytes one attention kernel launch must move: K and V read once, the raw bf16
     queries read (the kernel rotates them on load), O (bf16) written.  The fp8 cache
-    stores 1-byte codes and adds one K and one V scale per 128-token block and head.
+    stores 1-byte codes and adds one K and one V scale per block of up to 128 tokens of a
+    slot and head (frames of 64 tokens: one block per slot; their padding is not read).
     With the append fused in, the chunk's own K and V (part of the keys read once, from
     the caller's buffers) are also written to their ring slots."""
-    lq = w["chunk_frames"] * w["frame_h"] * w["frame_w"]
+    n = w["frame_h"] * w["frame_w"]
+    lq = w["chunk_frames"] * n
     hd = w["heads"] * w["head_dim"]
     e = kv_elem(w)
     total = 0.0
     for k in keys:
         total += 2.0 * e * k * hd + 2.0 * lq * hd + 2.0 * lq * hd
         if e == 1:
-            total += 2 * 4.0 * w["heads"] * k / 128
+            total += 2 * 4.0 * w["heads"] * (k // n) * -(-n // 128)
         if w.get("fused"):
             total += 2.0 * 2.0 * lq * hd
     return total

@@ -51,10 +51,13 @@
 // 128-token blocks of each valid slot (tile g = block g % n_blk of slot
 // g / n_blk, padding tokens masked), V tiles come from the slot's transposed
 // codes, and Q, K, P and V enter kind::f8f6f4 MMAs (K = 32 per instruction).
-// Each tile's K scale and the query row's scale fold into the softmax scale of
-// that tile; each tile's V scale divided by the CTA's largest V scale
-// multiplies P before its E4M3 coding, and the epilogue multiplies O back by
-// that largest scale.  P takes columns [0, 32) of S_t.
+// Slots of 64 tokens are packed two to a tile instead (tile g: slots 2g and
+// 2g + 1): K rows 0..63 and 64..127 come from the two slots, and the V tile is
+// two 64-byte-swizzled halves, one per slot, read by the PV MMAs as keys 0..63
+// and 64..127.  Each tile's (each half's) K scale and the query row's scale
+// fold into the softmax scale of its columns; its V scale divided by the CTA's
+// largest V scale multiplies P before its E4M3 coding, and the epilogue
+// multiplies O back by that largest scale.  P takes columns [0, 32) of S_t.
 // KV splits: each split CTA writes its unnormalised O, row max and row sum;
 // attention_combine_kernel (a dependent launch) merges them over the whole
 // GPU.
@@ -281,17 +284,20 @@ __device__ __forceinline__ float softmax_exp_store(const uint32_t (&sr)[kBlockN 
 // [0, 32) of the row's S region; r = (this tile's V scale) / (the CTA's
 // largest V scale) folds the tile's V scale into P, so one O accumulates
 // tiles of different scales.
+template <bool PK>
 __device__ __forceinline__ float softmax_exp_store_f8(const uint32_t (&sr)[kBlockN / 32][32], float c, float neg_m,
-                                                      float r, uint32_t s_tmem) {
+                                                      float r, float r_hi, uint32_t s_tmem) {
     const uint64_t scale2 = f2_pack(c, c);
     const uint64_t negm2 = f2_pack(neg_m, neg_m);
-    const uint64_t r2 = f2_pack(r, r);
     const uint64_t zero2 = f2_pack(0.0f, 0.0f);
     uint64_t acc[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[i] = 0ull;
 #pragma unroll
     for (int cb = 0; cb < kBlockN / 32; ++cb) {
+        // columns 64 .. 127 at their own V ratio (a tile of two 64-token slots)
+        const float rc = PK && cb >= kBlockN / 64 ? r_hi : r;
+        const uint64_t r2 = f2_pack(rc, rc);
         uint32_t pk[8];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -587,7 +593,7 @@ __device__ __forceinline__ void assembled(uint64_t *bars, int lane) {
     if (lane == 0) mbar_arrive(&bars[L::kAsm]);
 }
 
-template <int D, bool F8, bool FUSE>
+template <int D, bool F8, bool FUSE, bool PK>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     chunk_attention_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmap_q,
                            const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
@@ -595,6 +601,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     using L = AttnLayout<D, F8, FUSE>;
     static_assert(!F8 || D == 128, "the fp8 cache is built for head_dim 128");
     static_assert(!(F8 && FUSE), "the fused append is built for the bf16 cache");
+    static_assert(!PK || F8, "two slots per KV tile: the fp8 cache's 64-token slots");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBar);
@@ -634,8 +641,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (lk <= 0) return;                        // (active streams only; uniform per CTA)
 
     // KV tiles: 128-key runs of the valid prefix (bf16), or the 128-token blocks of each
-    // valid slot (fp8: tile g is block g % n_blk of slot g / n_blk)
-    const int n_kv = F8 ? (lk / p.tokens_per_frame) * p.n_blk : (lk + kBlockN - 1) / kBlockN;
+    // valid slot (fp8: tile g is block g % n_blk of slot g / n_blk; 64-token slots: slots
+    // 2g and 2g + 1)
+    const int n_vslots = F8 ? lk / p.tokens_per_frame : 0;
+    const int n_kv = F8 ? (PK ? (n_vslots + 1) >> 1 : n_vslots * p.n_blk) : (lk + kBlockN - 1) / kBlockN;
     const int per = (n_kv + n_split - 1) / n_split;
     const int kv_begin = split * per;
     const int kv_end = min(n_kv, kv_begin + per);
@@ -942,8 +951,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         const int hk = paired && (k_issued & 1) ? h_pair : h;
                         mbar_arrive_expect_tx(&bars[L::kKFull + st], L::kKVTile);
                         const int g = paired ? k_issued >> 1 : kv_begin + k_issued, sl = g / p.n_blk;
-                        tma_load_4d(smem + L::kK + st * L::kKVTile, &tmap_k, &bars[L::kKFull + st], 0, hk,
-                                    sl * p.np_tokens + (g - sl * p.n_blk) * kBlockN, bg);
+                        if constexpr (PK) {
+                            // rows 64 .. 127 from slot 2g + 1, or past the ring (zero-filled, masked)
+                            const int s1 = 2 * g + 1 < n_vslots ? 2 * g + 1 : p.slots;
+                            tma_load_4d(smem + L::kK + st * L::kKVTile, &tmap_k, &bars[L::kKFull + st], 0, hk,
+                                        2 * g * p.np_tokens, bg);
+                            tma_load_4d(smem + L::kK + st * L::kKVTile + L::kKVTile / 2, &tmap_k,
+                                        &bars[L::kKFull + st], 0, hk, s1 * p.np_tokens, bg);
+                        } else {
+                            tma_load_4d(smem + L::kK + st * L::kKVTile, &tmap_k, &bars[L::kKFull + st], 0, hk,
+                                        sl * p.np_tokens + (g - sl * p.n_blk) * kBlockN, bg);
+                        }
                     } else {
                         // (pair mode: sequence tile i is tile i / 2 of head h or h_pair)
                         const int hk = paired && (k_issued & 1) ? h_pair : h;
@@ -966,8 +984,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     const int hv = paired && (v_issued & 1) ? h_pair : h;
                     mbar_arrive_expect_tx(&bars[L::kVFull + st], L::kKVTile);
                     const int g = paired ? v_issued >> 1 : kv_begin + v_issued, sl = g / p.n_blk;
-                    tma_load_5d(smem + L::kV + st * L::kKVTile, &tmap_v, &bars[L::kVFull + st],
-                                (g - sl * p.n_blk) * kBlockN, 0, hv, sl, bg);
+                    if constexpr (PK) {
+                        // two 64-key halves (128 channel rows of 64 bytes each), one per slot
+                        const int s1 = 2 * g + 1 < n_vslots ? 2 * g + 1 : p.slots;
+                        tma_load_5d(smem + L::kV + st * L::kKVTile, &tmap_v, &bars[L::kVFull + st], 0, 0, hv, 2 * g,
+                                    bg);
+                        tma_load_5d(smem + L::kV + st * L::kKVTile + L::kKVTile / 2, &tmap_v, &bars[L::kVFull + st],
+                                    0, 0, hv, s1, bg);
+                    } else {
+                        tma_load_5d(smem + L::kV + st * L::kKVTile, &tmap_v, &bars[L::kVFull + st],
+                                    (g - sl * p.n_blk) * kBlockN, 0, hv, sl, bg);
+                    }
                 } else {
                     const int hv = paired && (v_issued & 1) ? h_pair : h;
                     const int tv = paired ? tile_at(v_issued >> 1) : tile_at(v_issued);
@@ -1031,10 +1058,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             auto issue_pv = [&](int t, int st, bool acc) {
                 const uint64_t b0 = dv + static_cast<uint64_t>(st * (L::kKVTile >> 4));
                 if constexpr (F8) {
+                    if constexpr (PK) {
+                        // 64-token slots: the V tile's two halves, 128 rows of 64 bytes each;
+                        // keys 32 kk .. 32 kk + 31 are half kk / 2, byte 32 (kk % 2) of its rows
+                        const uint64_t b1 = smem_desc_sw64(smem_addr(smem + L::kV), 16, 512) +
+                                            static_cast<uint64_t>(st * (L::kKVTile >> 4));
 #pragma unroll
-                    for (int kk = 0; kk < kBlockN / 32; ++kk)
-                        umma_ts_f8(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, b0 + kk * 2, idesc_pv,
-                                   (acc || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < kBlockN / 32; ++kk)
+                            umma_ts_f8(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
+                                       b1 + static_cast<uint64_t>((kk >> 1) * (L::kKVTile >> 5) + (kk & 1) * 2),
+                                       idesc_pv, (acc || kk > 0) ? 1u : 0u);
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < kBlockN / 32; ++kk)
+                            umma_ts_f8(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, b0 + kk * 2, idesc_pv,
+                                       (acc || kk > 0) ? 1u : 0u);
+                    }
                 } else {
 #pragma unroll
                     for (int kk = 0; kk < kBlockN / 16; ++kk)
@@ -1168,7 +1207,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 // which both sets of a single query tile share)
                 for (int i = 0; i < (paired ? n_kv : n_local); ++i) {
                     const int g = kv_begin + i, sl = g / p.n_blk;
-                    sv_ref = fmaxf(sv_ref, p.v_scale[scale_base + sl * (p.scale_slot_stride - p.n_blk) + g]);
+                    if constexpr (PK) {
+                        // (one block per slot: the scale of slot s at scale_base + s * stride)
+                        sv_ref = fmaxf(sv_ref, p.v_scale[scale_base + 2 * g * p.scale_slot_stride]);
+                        if (2 * g + 1 < n_vslots)
+                            sv_ref = fmaxf(sv_ref, p.v_scale[scale_base + (2 * g + 1) * p.scale_slot_stride]);
+                    } else {
+                        sv_ref = fmaxf(sv_ref, p.v_scale[scale_base + sl * (p.scale_slot_stride - p.n_blk) + g]);
+                    }
                 }
                 sv_ref = fmaxf(sv_ref, 1e-30f);
             }
@@ -1192,14 +1238,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             for (int it = 0; it < n_mine; ++it) {
                 float c_t = p.scale_log2, r_t = 1.0f;
+                float c_h = 0.0f, r_h = 0.0f;           // two slots per tile: scales of columns 64 .. 127
                 int valid_cols;
                 if constexpr (F8) {
                     const int g = kv_begin + (paired ? it : (alt ? 2 * it + t : it));   // KV tile of this iteration
                     const int sl = g / p.n_blk;
-                    const int64_t si = scale_base + sl * (p.scale_slot_stride - p.n_blk) + g;
-                    c_t = fmaxf(p.scale_log2 * sq * p.k_scale[si], 1e-30f);
-                    r_t = p.v_scale[si] / sv_ref;
-                    valid_cols = p.tokens_per_frame - (g - sl * p.n_blk) * kBlockN;
+                    if constexpr (PK) {
+                        const int64_t si = scale_base + static_cast<int64_t>(2 * g) * p.scale_slot_stride;
+                        c_t = fmaxf(p.scale_log2 * sq * p.k_scale[si], 1e-30f);
+                        r_t = p.v_scale[si] / sv_ref;
+                        valid_cols = 2 * g + 1 < n_vslots ? kBlockN : kBlockN / 2;
+                        c_h = c_t;
+                        r_h = r_t;
+                        if (valid_cols == kBlockN) {
+                            const int64_t sj = si + p.scale_slot_stride;
+                            c_h = fmaxf(p.scale_log2 * sq * p.k_scale[sj], 1e-30f);
+                            r_h = p.v_scale[sj] / sv_ref;
+                        }
+                    } else {
+                        const int64_t si = scale_base + sl * (p.scale_slot_stride - p.n_blk) + g;
+                        c_t = fmaxf(p.scale_log2 * sq * p.k_scale[si], 1e-30f);
+                        r_t = p.v_scale[si] / sv_ref;
+                        valid_cols = p.tokens_per_frame - (g - sl * p.n_blk) * kBlockN;
+                    }
                 } else {
                     valid_cols = it == rag_it ? rag_cols : kBlockN;
                 }
@@ -1231,8 +1292,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         m = fmax3(m, __uint_as_float(sr[cb][i]), __uint_as_float(sr[cb][i + 1]));
                     m4[cb] = fmaxf(m, __uint_as_float(sr[cb][31]));
                 }
-                const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-                const float m_tile = mx * c_t;
+                if (PK && c_h != c_t) {
+                    // fp8, a tile of two slots: the half with the smaller scale is brought to
+                    // the larger one (a factor below 1, so nothing overflows), so that one
+                    // scale serves the whole row below; a positive factor keeps the maxima
+                    const int lo = c_h > c_t ? 0 : 1;       // the half scaled down
+                    const float k = lo ? c_h / c_t : c_t / c_h;
+#pragma unroll
+                    for (int cb = 0; cb < kBlockN / 32; ++cb) {
+                        if (cb / (kBlockN / 64) != lo) continue;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) sr[cb][i] = __float_as_uint(__uint_as_float(sr[cb][i]) * k);
+                        m4[cb] *= k;
+                    }
+                    c_t = fmaxf(c_t, c_h);
+                }
+                const float m_tile = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c_t;
                 bool rescale = false;
                 float alpha = 1.0f;
                 if (it == 0) {
@@ -1244,7 +1319,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     m_run = m_tile;
                 }
                 if constexpr (F8)
-                    l_run += softmax_exp_store_f8(sr, c_t, -m_run, r_t, s_tmem);
+                    l_run += softmax_exp_store_f8<PK>(sr, c_t, -m_run, r_t, r_h, s_tmem);
                 else
                     l_run += softmax_exp_store(sr, c_t, -m_run, s_tmem);
                 // O_t is idle here (PV(t, it-1) completed before S(t, it) was signalled and
@@ -1511,13 +1586,13 @@ cudaError_t launch_wait_selftest(uint32_t *status, uint64_t limit_ns, cudaStream
     return cudaGetLastError();
 }
 
-template <int D, bool F8, bool FUSE, typename FP>
+template <int D, bool F8, bool FUSE, bool PK, typename FP>
 static cudaError_t launch_attention_d(const AttnParams &p, const FP &f, const CUtensorMap &tq, const CUtensorMap &tk,
                                       const CUtensorMap &tv, cudaStream_t s) {
     static bool configured = false;
     const int smem = AttnLayout<D, F8, FUSE>::kAlloc;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(chunk_attention_kernel<D, F8, FUSE>,
+        cudaError_t e = cudaFuncSetAttribute(chunk_attention_kernel<D, F8, FUSE, PK>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         configured = true;
@@ -1526,22 +1601,24 @@ static cudaError_t launch_attention_d(const AttnParams &p, const FP &f, const CU
     // pair mode: one CTA per (stream, pair of heads); otherwise whole units, then pieces
     dim3 grid(static_cast<unsigned>(p.pair ? p.n_units / p.heads * ((p.heads + 1) / 2)
                                            : p.n_whole + (p.n_units - p.n_whole) * p.n_pieces));
-    return launch_dependent(chunk_attention_kernel<D, F8, FUSE>, grid, dim3(kAttnThreads), static_cast<size_t>(smem),
+    return launch_dependent(chunk_attention_kernel<D, F8, FUSE, PK>, grid, dim3(kAttnThreads), static_cast<size_t>(smem),
                             s, p, tq, tk, tv, f);
 }
 
 cudaError_t launch_attention(const AttnParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
                              const CUtensorMap &tv, int head_dim, cudaStream_t s) {
     const FuseNone none{0};
-    if (p.f8) return launch_attention_d<128, true, false>(p, none, tq, tk, tv, s);
-    if (head_dim == 64) return launch_attention_d<64, false, false>(p, none, tq, tk, tv, s);
-    return launch_attention_d<128, false, false>(p, none, tq, tk, tv, s);
+    if (p.f8)
+        return p.pack2 ? launch_attention_d<128, true, false, true>(p, none, tq, tk, tv, s)
+                       : launch_attention_d<128, true, false, false>(p, none, tq, tk, tv, s);
+    if (head_dim == 64) return launch_attention_d<64, false, false, false>(p, none, tq, tk, tv, s);
+    return launch_attention_d<128, false, false, false>(p, none, tq, tk, tv, s);
 }
 
 cudaError_t launch_append_attention(const AttnParams &p, const FuseParams &f, const CUtensorMap &tq,
                                     const CUtensorMap &tk, const CUtensorMap &tv, int head_dim, cudaStream_t s) {
-    if (head_dim == 64) return launch_attention_d<64, false, true>(p, f, tq, tk, tv, s);
-    return launch_attention_d<128, false, true>(p, f, tq, tk, tv, s);
+    if (head_dim == 64) return launch_attention_d<64, false, true, false>(p, f, tq, tk, tv, s);
+    return launch_attention_d<128, false, true, false>(p, f, tq, tk, tv, s);
 }
 
 cudaError_t launch_combine(const AttnParams &p, int head_dim, cudaStream_t s) {

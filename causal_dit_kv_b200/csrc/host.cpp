@@ -76,6 +76,7 @@ struct Geometry {
     bool f8;                 // fp8 (E4M3) block-scaled cache
     int64_t np_tokens;       // fp8: tokens per slot padded to whole 128-token blocks
     int n_blk, scale_slot_stride;
+    bool pack2;              // fp8 with 64-token slots: two slots per KV tile (no padding read)
     uint64_t k_scale, v_scale, scale_layer_stride;
     int n_qpairs, lq_pad;
     int refresh_chunks;  // token chunks of the refresh reduction
@@ -151,6 +152,7 @@ Geometry geometry(const sdv2_cache_config &c) {
     g.np_tokens = (g.N + kBlockN - 1) / kBlockN * kBlockN;
     g.n_blk = static_cast<int>(g.np_tokens / kBlockN);
     g.scale_slot_stride = (c.heads * g.n_blk + 3) / 4 * 4;
+    g.pack2 = g.f8 && g.N == kBlockN / 2;
     g.n_qpairs = static_cast<int>((g.lq + kBlockM * kQTilesPerCta - 1) / (kBlockM * kQTilesPerCta));
     g.lq_pad = g.n_qpairs * kBlockM * kQTilesPerCta;
     // partial blocks (256 rows each) for the split units of one launch
@@ -265,12 +267,14 @@ bool use_pair_mode(const Geometry &g, const sdv2_cache_config &c, int64_t units,
 }
 
 // KV tiles of the longest stream: 128-key runs of its valid prefix, or for the fp8 cache
-// the 128-token blocks of each valid slot.
+// the 128-token blocks of each valid slot (64-token slots: pairs of slots).
 int64_t max_kv_tiles(const Geometry &g, const int64_t *keys, int n) {
     int64_t m = 0;
     for (int b = 0; b < n; ++b)
         if (keys[b] > 0)
-            m = std::max<int64_t>(m, g.f8 ? keys[b] / g.N * g.n_blk : (keys[b] + kBlockN - 1) / kBlockN);
+            m = std::max<int64_t>(m, !g.f8    ? (keys[b] + kBlockN - 1) / kBlockN
+                                     : g.pack2 ? (keys[b] / g.N + 1) / 2
+                                               : keys[b] / g.N * g.n_blk);
     return m;
 }
 
@@ -486,6 +490,7 @@ sdv2_status run_attention(sdv2_cache *c, int32_t layer, const void *q, void *out
         p.np_tokens = static_cast<int32_t>(g.np_tokens);
         p.n_blk = g.n_blk;
         p.scale_slot_stride = g.scale_slot_stride;
+        p.pack2 = g.pack2 ? 1 : 0;
     }
     std::unique_ptr<FuseParams> fp;
     if (fuse) {
@@ -713,7 +718,9 @@ sdv2_status sdv2_cache_create(const sdv2_cache_config *cfg, void *dev_buf, size_
     }
     // One TMA descriptor per layer for K and for V.  bf16: dims (d, H, slots*N, B), boxes of
     // 64 channels x 128 keys.  fp8: K codes (d, H, slots*Np, B) and transposed V codes
-    // (Np, d, H, slots, B), boxes of 128 bytes x 128 rows.
+    // (Np, d, H, slots, B), boxes of 128 bytes x 128 rows; with 64-token slots (two per KV
+    // tile) boxes of 64 K rows, and of 64 V bytes (one slot's keys) x 128 rows, 64-byte
+    // swizzled.
     c->tk.resize(n.layers);
     c->tv.resize(n.layers);
     c->tkh.resize(g.f8 ? 0 : static_cast<size_t>(n.layers) * kFuseBoxes);
@@ -746,7 +753,7 @@ sdv2_status sdv2_cache_create(const sdv2_cache_config *cfg, void *dev_buf, size_
                                             static_cast<cuuint64_t>(n.batch)};
                 const cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(n.heads) * 128,
                                                static_cast<cuuint64_t>(g.slots * g.np_tokens * n.heads) * 128};
-                const cuuint32_t box[4] = {128, 1, static_cast<cuuint32_t>(kBlockN), 1};
+                const cuuint32_t box[4] = {128, 1, static_cast<cuuint32_t>(g.pack2 ? kBlockN / 2 : kBlockN), 1};
                 r = encode(&c->tk[l], CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, ptr, dims, strides, box, estr,
                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -758,10 +765,12 @@ sdv2_status sdv2_cache_create(const sdv2_cache_config *cfg, void *dev_buf, size_
                                                static_cast<cuuint64_t>(g.np_tokens) * 128,
                                                static_cast<cuuint64_t>(g.np_tokens) * 128 * n.heads,
                                                static_cast<cuuint64_t>(g.np_tokens) * 128 * n.heads * g.slots};
-                const cuuint32_t box[5] = {static_cast<cuuint32_t>(kBlockN), 128, 1, 1, 1};
+                const cuuint32_t box[5] = {static_cast<cuuint32_t>(g.pack2 ? kBlockN / 2 : kBlockN), 128, 1, 1, 1};
+                // (64-token slots: 64-byte L2 fills, so that a row's padding half is not read)
                 r = encode(&c->tv[l], CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, ptr, dims, strides, box, estr,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                           CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           g.pack2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                           g.pack2 ? CU_TENSOR_MAP_L2_PROMOTION_L2_64B : CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
             }
             if (r != CUDA_SUCCESS) {
                 delete c;

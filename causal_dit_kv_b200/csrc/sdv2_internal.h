@@ -85,6 +85,10 @@ struct AttnParams {
     const float *v_scale;
     int32_t slots, np_tokens, n_blk, scale_slot_stride;
     int32_t f8;                 // 1: fp8 cache (E4M3 queries, keys, values and probabilities)
+    // fp8 with 64-token slots: tile g packs slots 2g and 2g + 1 (64 keys each, the second
+    // absent past the valid slots), so no padding token is read; the K map's boxes are 64
+    // rows, the V map's 64 keys (64-byte swizzle)
+    int32_t pack2;
 };
 
 // Append fused into the attention (bf16 cache, chunks of at most two query tiles):

@@ -26,6 +26,9 @@ SHAPES = {
     "wan1.3b-128x256-b16-fp8": dict(batch=16, layers=30, heads=12, head_dim=128, frame_h=8, frame_w=16,
                                     chunk_frames=1, sink_frames=1, window_frames=6, embed_dim=1536,
                                     motion=(16, 16, 32), kv_format="fp8"),
+    "wan1.3b-128x128-b16-fp8": dict(batch=16, layers=30, heads=12, head_dim=128, frame_h=8, frame_w=8,
+                                    chunk_frames=1, sink_frames=1, window_frames=6, embed_dim=1536,
+                                    motion=(16, 16, 16), kv_format="fp8"),
     "wan14b-512x512-b1": dict(batch=1, layers=40, heads=40, head_dim=128, frame_h=32, frame_w=32, chunk_frames=1,
                               sink_frames=1, window_frames=6, embed_dim=5120, motion=(16, 64, 64)),
 }

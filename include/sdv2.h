@@ -97,7 +97,9 @@ typedef struct {
  *   transposed per slot, [B][S+W][H][d][Np], so both tensor-core operands are
  *   K-major; padding tokens hold code 0.  The attention rounds each rotated
  *   query row to E4M3 with its own scale and the probabilities to E4M3 before
- *   the products (fp32 accumulation).  Requires head_dim 128. */
+ *   the products (fp32 accumulation).  With N = 64 (one half-full block per
+ *   slot) the attention reads no padding: it takes two slots per 128-key tile,
+ *   each half with its own scales.  Requires head_dim 128. */
 enum { SDV2_KV_BF16 = 0, SDV2_KV_FP8_E4M3 = 1 };
 
 typedef struct sdv2_cache sdv2_cache;

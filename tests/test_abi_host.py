@@ -246,3 +246,28 @@ def test_fp8_plan_counts_whole_blocks_per_slot(B):
     for cfg in (bf, f8):
         whole, pieces = B.sdv2_attention_plan(cfg, keys, 148)
         assert 1 <= pieces <= 16 and 0 <= whole <= 12 * 13
+
+
+def test_fp8_plan_packs_64_token_slots_two_to_a_tile(B):
+    # 8 x 8 = 64 tokens per frame: the fp8 kernel packs slots 2g and 2g + 1 into KV tile g,
+    # so its plan counts ceil(slots / 2) tiles, as the bf16 plan counts ceil(64 slots / 128)
+    import random
+    rng = random.Random(5)
+    for _ in range(200):
+        b, h = rng.randint(1, 4), rng.choice([1, 2, 3, 12])
+        s_, w = rng.randint(1, 3), rng.randint(1, 9)
+        bf = B.make_cache_config(b, 1, h, 128, 8, 8, 1, s_, w)
+        f8 = B.make_cache_config(b, 1, h, 128, 8, 8, 1, s_, w, kv_format="fp8")
+        keys = [rng.choice([0, 64 * rng.randint(1, s_ + w)]) for _ in range(b)]
+        if not any(keys):
+            continue
+        sms = rng.choice([16, 148])
+        assert B.sdv2_attention_plan(f8, keys, sms) == B.sdv2_attention_plan(bf, keys, sms), (b, h, s_, w, keys)
+        whole, pieces = B.sdv2_attention_plan(f8, keys, sms)
+        assert pieces <= max(1, (max(keys) // 64 + 1) // 2)
+    # one stream, two heads, five slots: three tiles, three pieces (five without the packing)
+    f8 = B.make_cache_config(1, 1, 2, 128, 8, 8, 1, 1, 4, kv_format="fp8")
+    assert B.sdv2_attention_plan(f8, [5 * 64], 148) == (0, 3)
+    # 96-token slots are not packed: one padded block per slot, five tiles
+    f8 = B.make_cache_config(1, 1, 2, 128, 8, 12, 1, 1, 4, kv_format="fp8")
+    assert B.sdv2_attention_plan(f8, [5 * 96], 148)[1] == 5

@@ -89,6 +89,11 @@ def test_fp8_workloads_byte_accounting():
     assert bench.workload_config("x", w8, 1)["kv_format"] == "fp8"
     assert bench.workload_config("x", w16, 1)["kv_format"] == "bf16"
     assert bench.kv_elem(w8) == 1 and bench.kv_elem(w16) == 2
+    # 64-token frames: 7 slots of one (half-full) block each, 7 K and 7 V scales per head
+    s8 = bench.WORKLOADS["wan1.3b-128x128-b16-fp8"]
+    ks = bench.steady_keys(s8)
+    assert ks == [448] * 16
+    assert bench.attn_bytes(s8, ks) == 16 * (2 * 448 * hd + 2 * 64 * hd + 2 * 64 * hd + 2 * 4 * 12 * 7)
 
 
 def test_fused_workloads_byte_accounting():

@@ -62,9 +62,16 @@ class Fp8Pair:
                 f0.append(-1)
         return f0
 
-    def run_layer(self, step, layer, f0, rows=None):
+    def run_layer(self, step, layer, f0, rows=None, gains=None):
+        """gains: optional (k factors, v factors), one power of two per chunk frame (exact
+        in bf16), so that the slots' block scales differ by those factors."""
         c = self.cfg
         q, k, v = synth.chunk_qkv(self.seed, c.batch, c.chunk_tokens, c.heads, c.head_dim, step, layer)
+        if gains is not None:
+            n = c.tokens_per_frame
+            for x, fac in zip((k, v), gains):
+                for i, a in enumerate(fac):
+                    x[:, i * n:(i + 1) * n] *= a
         self.q_bits = synth.bf16_bits(q)
         self.gpu.kv_append(layer, k.cuda(), v.cuda(), f0)
         kv_append_fp8(self.ora, layer, synth.bf16_bits(k), synth.bf16_bits(v), f0)
@@ -142,6 +149,39 @@ def test_fp8_stream_parity(case):
             out, want = pair.run_layer(step, layer, f0)
             assert all(pair.cache_equal(layer)), (step, layer, pair.cache_equal(layer))
             _check_out(pair, out, want, layer, f0, pair.q_bits)
+    assert pair.gpu.check() == 0
+
+
+@pytest.mark.parametrize("case", ["split_one_frame", "two_frames_staggered"])
+def test_fp8_packed_slots_with_unequal_scales(case):
+    """64-token slots, two to a KV tile: keys and values of each frame scaled by their own
+    power of two (block scales up to 4x apart for K and for V), so a tile's two halves
+    need their own K and V scales (a CPU emulation of the kernel's arithmetic on the first
+    case puts its error at 0.65 of the bound, and at 14x the bound with the halves' K
+    scales swapped); rings filling up (a tile's second slot absent while the valid slot
+    count is odd), KV splits, T' = 2 with a phase reset.  The keys are scaled down, not
+    up: much larger logits make rows so peaked that the probabilities' E4M3 rounding
+    leaves the error model above (a relative error per element)."""
+    from causal_dit_kv_b200 import binding as B
+    cfg = {
+        # 2 units, up to 5 slots: 3 tiles, split into 3 pieces once the ring is full
+        "split_one_frame": dict(batch=1, layers=1, heads=2, head_dim=128, frame_h=8, frame_w=8, chunk_frames=1,
+                                sink_frames=1, window_frames=4),
+        "two_frames_staggered": dict(batch=2, layers=1, heads=3, head_dim=128, frame_h=8, frame_w=8,
+                                     chunk_frames=2, sink_frames=1, window_frames=4, rope_reset_period=3),
+    }[case]
+    pair = Fp8Pair(seed=3004, **cfg)
+    if case == "split_one_frame":
+        assert B.sdv2_attention_plan(pair.gpu.cfg, [5 * 64], 148) == (0, 3)
+    tp = cfg["chunk_frames"]
+    for step in range(7):
+        active = None if case == "split_one_frame" else [b for b in range(pair.cfg.batch) if step >= b]
+        f0 = pair.step_frames(active)
+        gk = [2.0 ** ((step * tp + i) % 3 - 2) for i in range(tp)]
+        gv = [2.0 ** (((step * tp + i) * 2) % 3 - 1) for i in range(tp)]
+        out, want = pair.run_layer(step, 0, f0, gains=(gk, gv))
+        assert all(pair.cache_equal(0)), (step, pair.cache_equal(0))
+        _check_out(pair, out, want, 0, f0, pair.q_bits)
     assert pair.gpu.check() == 0
 
 
