@@ -25,7 +25,8 @@ constexpr int kAppendRowsPerBlock = 32;
 
 __global__ void __launch_bounds__(128) kv_append_kernel(const __grid_constant__ AppendParams p) {
     // The previous kernel in the stream may still be running (dependent launch):
-    // wait for it, then let the next one (the queries' RoPE) start alongside.
+    // wait for it, then let the next one (the attention kernel, whose set-up and query
+    // rotation need nothing this kernel writes) start alongside.
     grid_dependency_wait();
     grid_launch_dependents();
     const int fi = blockIdx.y;

@@ -107,7 +107,7 @@ struct AttnLayout {
     static constexpr int kAsm = kDrain + 1;           // fused append: assembled tiles written (one arrival per warp 2..11)
     static constexpr int kTabReady = kAsm + 1;        // fused append: fp64 key tables in shared memory
     static constexpr int kNumBars = kAsm + (FUSE ? 2 : 0);
-    static constexpr int kMisc = kBar + kNumBars * 8;   // tmem base, abort flag, assembly work counter
+    static constexpr int kMisc = kBar + kNumBars * 8;   // tmem base, abort flag, a spare word (zeroed by the fused launch)
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;      // room to align the base to 1024 bytes
     static_assert(kAlloc <= 232448, "shared memory of one CTA");

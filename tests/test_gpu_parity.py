@@ -213,8 +213,9 @@ def test_full_size_14b_sampled():
 @pytest.mark.parametrize("splits", ["split", "unsplit"])
 def test_back_to_back_attention_calls(splits):
     """Several attention calls on the same appended chunk in a row (and on
-    alternating layers) give the same, correct output: a call's query RoPE pass
-    never overwrites queries an earlier call is still reading."""
+    alternating layers) give the same, correct output: a call's split partials
+    and its in-kernel query rotation never disturb what an earlier call, still
+    running or being merged, reads."""
     if splits == "split":
         cfg = dict(batch=1, layers=2, heads=12, head_dim=128, frame_h=32, frame_w=32, chunk_frames=1,
                    sink_frames=1, window_frames=6)
